@@ -1,0 +1,207 @@
+"""CPU oracle for dynamic block-sparse attention -- TEST INFRASTRUCTURE ONLY.
+
+Only tests/, __graft_entry__.smoke() and bench.py's cpu_baseline/reference legs
+may import this package.  It wraps the plain fp64 C oracle (bsa_oracle.c) with
+numpy marshalling and shares no code with the CUDA library.
+
+Parity pins (tests/test_oracle_pins.py) hold every function here to closed
+forms, invariants, brute force and independent library routines.  The one
+reading that no pin can fix is recorded as "parity unpinned": the exact form of
+P' and of the top-p rule beyond the prose of "Competition Domains Matter" s3
+(its Eq. 1-3 are lost in the page text).
+"""
+import ctypes
+import math
+import os
+
+import numpy as np
+
+from . import build as _build
+
+TEXT_KEEP = 1
+FRAME0_DENSE = 2
+
+
+class OracleLayout(ctypes.Structure):
+    """Problem geometry, mirrored field by field from the caller's config."""
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "batch", "heads", "seq_len", "seq_pad", "head_dim", "q_block", "k_block",
+        "text_len", "tokens_per_frame", "num_frames")]
+
+    @classmethod
+    def from_dict(cls, d):
+        return cls(*[int(d[n]) for n, _ in cls._fields_])
+
+    @property
+    def cq(self):
+        return self.seq_pad // self.q_block
+
+    @property
+    def ck(self):
+        return self.seq_pad // self.k_block
+
+
+class Oracle:
+    """ctypes binding of one build of bsa_oracle.c (the default build, or a
+    deliberately mutated copy used by the pin-sensitivity tests)."""
+
+    def __init__(self, path=None):
+        path = path or _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.POINTER
+        lp = P(OracleLayout)
+        vp = ctypes.c_void_p
+        L.ora_block_count.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        L.ora_block_count.restype = ctypes.c_int
+        L.ora_frame0_qblocks.argtypes = [lp, P(ctypes.c_int), P(ctypes.c_int)]
+        L.ora_text_kblocks.argtypes = [lp]
+        L.ora_text_kblocks.restype = ctypes.c_int
+        L.ora_pool.argtypes = [lp, vp, ctypes.c_int, vp]
+        L.ora_scores.argtypes = [lp, vp, vp, vp]
+        L.ora_entropy.argtypes = [lp, vp, ctypes.c_double, vp, vp]
+        L.ora_topp.argtypes = [lp, vp, vp, vp, vp]
+        L.ora_overrides.argtypes = [lp, ctypes.c_uint32, vp]
+        L.ora_lists.argtypes = [lp, vp, vp, vp]
+        L.ora_attention.argtypes = [lp, vp, vp, vp, vp, ctypes.c_double, ctypes.c_long,
+                                    vp, vp, vp]
+        L.ora_num_threads.restype = ctypes.c_int
+        self.lib = L
+
+    def num_threads(self):
+        return self.lib.ora_num_threads()
+
+    def block_count(self, seq_len, block, idx):
+        return self.lib.ora_block_count(seq_len, block, idx)
+
+    def frame0_qblocks(self, L):
+        L = _layout(L)
+        a, b = ctypes.c_int(), ctypes.c_int()
+        self.lib.ora_frame0_qblocks(ctypes.byref(L), ctypes.byref(a), ctypes.byref(b))
+        return a.value, b.value
+
+    def text_kblocks(self, L):
+        L = _layout(L)
+        return self.lib.ora_text_kblocks(ctypes.byref(L))
+
+    def pool(self, L, x, block):
+        """Block centroids, fp32 [B,H,C,D]."""
+        L = _layout(L)
+        x = _u16(x)
+        out = np.empty((L.batch, L.heads, L.seq_pad // block, L.head_dim), np.float32)
+        self.lib.ora_pool(ctypes.byref(L), _ptr(x), block, _ptr(out))
+        return out
+
+    def scores(self, L, qc, kc):
+        """Cluster-size-weighted softmax P', fp32 [B,H,C_q,C_k]."""
+        L = _layout(L)
+        qc = np.ascontiguousarray(qc, np.float32)
+        kc = np.ascontiguousarray(kc, np.float32)
+        out = np.empty((L.batch, L.heads, L.cq, L.ck), np.float32)
+        self.lib.ora_scores(ctypes.byref(L), _ptr(qc), _ptr(kc), _ptr(out))
+        return out
+
+    def entropy(self, L, probs, eps=1e-8):
+        """Per-head entropy and entropy / ln C_k, fp64 [B,H] each."""
+        L = _layout(L)
+        probs = np.ascontiguousarray(probs, np.float32)
+        H = np.empty((L.batch, L.heads), np.float64)
+        Hn = np.empty((L.batch, L.heads), np.float64)
+        self.lib.ora_entropy(ctypes.byref(L), _ptr(probs), float(eps), _ptr(H), _ptr(Hn))
+        return H, Hn
+
+    def topp(self, L, probs, top_p):
+        """Per-row top-p block mask (u8 [B,H,C_q,C_k]) and k* per row (int32 [B,H,C_q])."""
+        L = _layout(L)
+        probs = np.ascontiguousarray(probs, np.float32)
+        tp = np.ascontiguousarray(np.broadcast_to(np.asarray(top_p, np.float32), (L.heads,)))
+        mask = np.empty((L.batch, L.heads, L.cq, L.ck), np.uint8)
+        kstar = np.empty((L.batch, L.heads, L.cq), np.int32)
+        self.lib.ora_topp(ctypes.byref(L), _ptr(probs), _ptr(tp), _ptr(mask), _ptr(kstar))
+        return mask, kstar
+
+    def overrides(self, L, flags, mask):
+        """Text-keep and frame-0-dense overrides applied to a copy of mask."""
+        L = _layout(L)
+        m = np.ascontiguousarray(mask, np.uint8).copy()
+        self.lib.ora_overrides(ctypes.byref(L), int(flags), _ptr(m))
+        return m
+
+    def lists(self, L, mask):
+        """Ascending selected key blocks per query block (-1 padded) and their counts."""
+        L = _layout(L)
+        mask = np.ascontiguousarray(mask, np.uint8)
+        idx = np.empty((L.batch, L.heads, L.cq, L.ck), np.int32)
+        cnt = np.empty((L.batch, L.heads, L.cq), np.int32)
+        self.lib.ora_lists(ctypes.byref(L), _ptr(mask), _ptr(idx), _ptr(cnt))
+        return idx, cnt
+
+    def attention(self, L, q, k, v, mask=None, scale=None, rows=None):
+        """Exact softmax attention over the selected blocks (mask None = dense).
+
+        rows: optional flat query-block ids (b*H*C_q + h*C_q + i).  Returns
+        out fp32 [nrows, q_block, D] and lse fp32 [nrows, q_block]; with rows
+        None the leading axis covers every query block in (b, h, i) order.
+        """
+        L = _layout(L)
+        q, k, v = _u16(q), _u16(k), _u16(v)
+        if scale is None:
+            scale = 1.0 / math.sqrt(L.head_dim)
+        m = None if mask is None else np.ascontiguousarray(mask, np.uint8)
+        if rows is None:
+            n = L.batch * L.heads * L.cq
+            r = None
+        else:
+            r = np.ascontiguousarray(rows, np.int64)
+            n = r.shape[0]
+        out = np.empty((n, L.q_block, L.head_dim), np.float32)
+        lse = np.empty((n, L.q_block), np.float32)
+        self.lib.ora_attention(ctypes.byref(L), _ptr(q), _ptr(k), _ptr(v), _ptr(m),
+                               float(scale), n, _ptr(r), _ptr(out), _ptr(lse))
+        return out, lse
+
+    def select(self, L, q, k, top_p, flags, eps=1e-8):
+        """The whole selection stage: centroids, P', entropy, top-p, overrides, lists."""
+        L = _layout(L)
+        qc = self.pool(L, q, L.q_block)
+        kc = self.pool(L, k, L.k_block)
+        probs = self.scores(L, qc, kc)
+        H, Hn = self.entropy(L, probs, eps)
+        tmask, kstar = self.topp(L, probs, top_p)
+        m = self.overrides(L, flags, tmask)
+        idx, cnt = self.lists(L, m)
+        return dict(q_centroids=qc, k_centroids=kc, probs=probs, entropy=H, entropy_norm=Hn,
+                    topp_mask=tmask, mask=m, kstar=kstar, kv_index=idx, kv_count=cnt)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(x):
+    x = np.ascontiguousarray(x)
+    if x.dtype != np.uint16:
+        raise TypeError("oracle inputs are raw bf16 bit patterns (uint16)")
+    return x
+
+
+def _layout(L):
+    return L if isinstance(L, OracleLayout) else OracleLayout.from_dict(L)
+
+
+_DEFAULT = None
+
+
+def default():
+    """The oracle built from bsa_oracle.c as committed."""
+    global _DEFAULT
+    if _DEFAULT is None:
+        _DEFAULT = Oracle()
+    return _DEFAULT
+
+
+def __getattr__(name):
+    # module-level shortcuts: oracle.pool(...), oracle.scores(...), ...
+    if name in ("num_threads", "block_count", "frame0_qblocks", "text_kblocks", "pool",
+                "scores", "entropy", "topp", "overrides", "lists", "attention", "select"):
+        return getattr(default(), name)
+    raise AttributeError(name)

@@ -1,0 +1,339 @@
+/*
+ * bsa_oracle.c -- the CPU oracle for dynamic block-sparse attention.
+ *
+ * TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only tests/, __graft_entry__.smoke()
+ * and the cpu_baseline / reference legs of bench.py may load this library.
+ * The CUDA library shares no code, header, table or helper with this file.
+ *
+ * It is deliberately plain and slow: fp64 arithmetic throughout, the steps
+ * taken in the order the pages state them, no blocking, no fusion, no
+ * reordering.  OpenMP only spreads independent rows over host cores; it never
+ * changes the order of any sum.
+ *
+ * Sources restated here (pages by title, with section):
+ *  [p1] "Attention matrix view: make only frame-0 query rows dense"
+ *       s1 token packing, s2 dense vs sparse rows, s4 block-level mask
+ *       override (frame-0 query-block range), s6 before/after masks,
+ *       s7 "always keep text/global blocks".
+ *  [p3] "Competition Domains Matter: Selective Head Globalization for
+ *       Training-Free Sparse Attention in Video Diffusion Transformers"
+ *       s3 setup: centroids with cluster sizes n_i, n_j and the
+ *       cluster-size-weighted softmax P' (Eq. 1, rows sum to one);
+ *       per-head entropy H_h (Eq. 3) and its normalisation by log C_k;
+ *       domain 1 "per-row local" top-p (Eq. 2).
+ *  [p5] "AB-Attention: accurate block-sparse attention for video diffusion"
+ *       TL;DR: exact attention computed only on the selected K/V blocks.
+ *
+ * Readings taken where the pages are silent or garbled (the equations of
+ * [p3] are lost in the extracted text):
+ *  - a cluster is one contiguous fixed-size block, centroid = mean over the
+ *    block's valid tokens, n = its valid-token count;
+ *  - P'[i,j] = n_j exp(s_ij) / sum_j' n_j' exp(s_ij'), s_ij = qc_i.kc_j/sqrt(D);
+ *  - natural log; entropy mean over all C_q rows;
+ *  - top-p = smallest prefix of the row in (P' desc, j asc) order whose
+ *    fp64 running sum of the fp32 values reaches p, the cut entry included;
+ *    every block if the row never reaches p;
+ *  - text keep sets key columns j < ceil(text_len / k_block);
+ *  - the frame-0 override sets every column of query blocks
+ *    text_len / q_block .. (text_len + tokens_per_frame - 1) / q_block;
+ *  - keys at positions >= seq_len are excluded; padded query rows give 0
+ *    output and -inf log-sum-exp.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+    int32_t batch, heads, seq_len, seq_pad, head_dim, q_block, k_block;
+    int32_t text_len, tokens_per_frame, num_frames;
+} ora_layout;
+
+enum { ORA_TEXT_KEEP = 1u, ORA_FRAME0_DENSE = 2u };
+
+/* bf16 bit pattern -> exact double (a bf16 is the top half of an fp32). */
+static double bf16_val(uint16_t h)
+{
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Number of tokens of block `idx` that lie before seq_len ([p3] s3: n_i, n_j). */
+int ora_block_count(int seq_len, int block, int idx)
+{
+    long v = (long)seq_len - (long)idx * block;
+    if (v < 0) return 0;
+    return v > block ? block : (int)v;
+}
+
+/* [p1] s4: first and last query block that overlaps frame 0. */
+void ora_frame0_qblocks(const ora_layout *L, int *first, int *last)
+{
+    int start = L->text_len;
+    int end = L->text_len + L->tokens_per_frame;   /* exclusive */
+    *first = start / L->q_block;
+    *last = (end - 1) / L->q_block;
+}
+
+/* [p1] s7: number of key blocks that hold text tokens. */
+int ora_text_kblocks(const ora_layout *L)
+{
+    return (L->text_len + L->k_block - 1) / L->k_block;
+}
+
+/*
+ * Centroid of every block ([p3] s3 centroids q_{h,i}, k_{h,j}):
+ * mean over the block's valid tokens, summed in fp64 in ascending token
+ * order, stored as fp32.  x is bf16 [B,H,seq_pad,D]; out is fp32 [B,H,C,D].
+ */
+void ora_pool(const ora_layout *L, const uint16_t *x, int block, float *out)
+{
+    const int D = L->head_dim, C = L->seq_pad / block;
+    const long BH = (long)L->batch * L->heads;
+    #pragma omp parallel for schedule(static)
+    for (long r = 0; r < BH * C; ++r) {
+        long bh = r / C;
+        int i = (int)(r % C);
+        int n = ora_block_count(L->seq_len, block, i);
+        const uint16_t *base = x + (bh * L->seq_pad + (long)i * block) * D;
+        for (int d = 0; d < D; ++d) {
+            double s = 0.0;
+            for (int t = 0; t < n; ++t) s += bf16_val(base[(long)t * D + d]);
+            out[r * D + d] = (float)(n > 0 ? s / n : 0.0);
+        }
+    }
+}
+
+/*
+ * Cluster-size-weighted softmax ([p3] s3, Eq. 1):
+ *   s_ij  = (qc_i . kc_j) / sqrt(D)
+ *   P'_ij = n_j exp(s_ij) / sum_j' n_j' exp(s_ij')
+ * evaluated in fp64 with the max of (s_ij + ln n_j) subtracted first, stored
+ * as fp32 [B,H,C_q,C_k].
+ */
+void ora_scores(const ora_layout *L, const float *qc, const float *kc, float *probs)
+{
+    const int D = L->head_dim;
+    const int Cq = L->seq_pad / L->q_block, Ck = L->seq_pad / L->k_block;
+    const long BH = (long)L->batch * L->heads;
+    const double inv_sqrt_d = 1.0 / sqrt((double)D);
+    #pragma omp parallel
+    {
+        double *logit = (double *)malloc(sizeof(double) * Ck);
+        #pragma omp for schedule(static)
+        for (long r = 0; r < BH * Cq; ++r) {
+            long bh = r / Cq;
+            const float *qi = qc + r * D;
+            double m = -INFINITY;
+            for (int j = 0; j < Ck; ++j) {
+                const float *kj = kc + (bh * Ck + j) * D;
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d) dot += (double)qi[d] * (double)kj[d];
+                int nj = ora_block_count(L->seq_len, L->k_block, j);
+                logit[j] = nj > 0 ? dot * inv_sqrt_d + log((double)nj) : -INFINITY;
+                if (logit[j] > m) m = logit[j];
+            }
+            double z = 0.0;
+            for (int j = 0; j < Ck; ++j) z += exp(logit[j] - m);
+            for (int j = 0; j < Ck; ++j) probs[r * Ck + j] = (float)(exp(logit[j] - m) / z);
+        }
+        free(logit);
+    }
+}
+
+/*
+ * Per-head entropy ([p3] s3, Eq. 3): H_h = (1/C_q) sum_i ( -sum_j P' ln(P' + eps) ),
+ * in fp64 over the fp32 P'.  Also H_h / ln C_k.  Outputs fp64 [B,H].
+ */
+void ora_entropy(const ora_layout *L, const float *probs, double eps, double *H, double *H_norm)
+{
+    const int Cq = L->seq_pad / L->q_block, Ck = L->seq_pad / L->k_block;
+    const long BH = (long)L->batch * L->heads;
+    for (long bh = 0; bh < BH; ++bh) {
+        double acc = 0.0;
+        for (int i = 0; i < Cq; ++i) {
+            const float *row = probs + (bh * Cq + i) * (long)Ck;
+            double h = 0.0;
+            for (int j = 0; j < Ck; ++j) h -= (double)row[j] * log((double)row[j] + eps);
+            acc += h;
+        }
+        H[bh] = acc / Cq;
+        if (H_norm) H_norm[bh] = H[bh] / log((double)Ck);
+    }
+}
+
+/* Order used by the top-p rule: larger P' first, then the lower block index. */
+typedef struct { float p; int j; } ora_entry;
+
+static int ora_entry_cmp(const void *a, const void *b)
+{
+    const ora_entry *x = (const ora_entry *)a, *y = (const ora_entry *)b;
+    if (x->p > y->p) return -1;
+    if (x->p < y->p) return 1;
+    return (x->j > y->j) - (x->j < y->j);
+}
+
+/*
+ * Per-row local top-p ([p3] domain 1 "Per-row local", Eq. 2): row (b,h,i)
+ * keeps the first k* entries of its (P' desc, j asc) order, with
+ * k* = min{k : c_k >= p_h}, c_k the fp64 running sum of the first k fp32
+ * values, or every entry when no k qualifies.  Writes mask u8 [B,H,C_q,C_k]
+ * (0/1) and, when kstar is not NULL, k* per row (int32 [B,H,C_q]).
+ */
+void ora_topp(const ora_layout *L, const float *probs, const float *top_p,
+              uint8_t *mask, int32_t *kstar)
+{
+    const int Cq = L->seq_pad / L->q_block, Ck = L->seq_pad / L->k_block;
+    const long BH = (long)L->batch * L->heads;
+    if (Ck <= 0 || Cq <= 0) return;
+    #pragma omp parallel
+    {
+        ora_entry *e = (ora_entry *)malloc(sizeof(ora_entry) * Ck);
+        #pragma omp for schedule(static)
+        for (long r = 0; r < BH * Cq; ++r) {
+            int h = (int)((r / Cq) % L->heads);
+            const float *row = probs + r * Ck;
+            for (int j = 0; j < Ck; ++j) { e[j].p = row[j]; e[j].j = j; }
+            qsort(e, (size_t)Ck, sizeof(ora_entry), ora_entry_cmp);
+            double p = (double)top_p[h], c = 0.0;
+            int k = Ck;
+            for (int t = 0; t < Ck; ++t) {
+                c += (double)e[t].p;
+                if (c >= p) { k = t + 1; break; }
+            }
+            uint8_t *m = mask + r * Ck;
+            memset(m, 0, (size_t)Ck);
+            for (int t = 0; t < k; ++t) m[e[t].j] = 1;
+            if (kstar) kstar[r] = k;
+        }
+        free(e);
+    }
+}
+
+/*
+ * Overrides on the block mask:
+ *  - text keep ([p1] s7 "always keep text/global blocks"): every query row
+ *    keeps every key block that holds a text token;
+ *  - frame-0 dense ([p1] s4 and s6 "After"): every key block of the query
+ *    blocks that overlap frame 0.
+ */
+void ora_overrides(const ora_layout *L, uint32_t flags, uint8_t *mask)
+{
+    const int Cq = L->seq_pad / L->q_block, Ck = L->seq_pad / L->k_block;
+    const long BH = (long)L->batch * L->heads;
+    int tk = ora_text_kblocks(L);
+    if (tk > Ck) tk = Ck;
+    int f0 = 0, f1 = -1;
+    if (L->tokens_per_frame > 0 && L->num_frames > 0) ora_frame0_qblocks(L, &f0, &f1);
+    if (f1 > Cq - 1) f1 = Cq - 1;
+    for (long bh = 0; bh < BH; ++bh) {
+        for (int i = 0; i < Cq; ++i) {
+            uint8_t *m = mask + (bh * Cq + i) * (long)Ck;
+            if (flags & ORA_TEXT_KEEP)
+                for (int j = 0; j < tk; ++j) m[j] = 1;
+            if ((flags & ORA_FRAME0_DENSE) && i >= f0 && i <= f1)
+                for (int j = 0; j < Ck; ++j) m[j] = 1;
+        }
+    }
+}
+
+/* Compacted lists: ascending selected key blocks per query block, and their count. */
+void ora_lists(const ora_layout *L, const uint8_t *mask, int32_t *kv_index, int32_t *kv_count)
+{
+    const int Cq = L->seq_pad / L->q_block, Ck = L->seq_pad / L->k_block;
+    const long rows = (long)L->batch * L->heads * Cq;
+    for (long r = 0; r < rows; ++r) {
+        int c = 0;
+        for (int j = 0; j < Ck; ++j)
+            if (mask[r * Ck + j]) kv_index[r * Ck + c++] = j;
+        for (int t = c; t < Ck; ++t) kv_index[r * Ck + t] = -1;
+        kv_count[r] = c;
+    }
+}
+
+/*
+ * Exact softmax attention over the selected key blocks only
+ * ([p1] s2: dense rows attend to all K/V, sparse rows to the selected K/V;
+ *  [p5] TL;DR: exact attention on the selected blocks).
+ * For each valid query t of query block i:
+ *   U = { u : u in key block j, mask[i][j] = 1, u < seq_len }
+ *   s_u = scale * (Q_t . K_u), two-pass softmax with the exact max,
+ *   O_t = sum_u softmax_u V_u, lse_t = m + ln sum_u exp(s_u - m),
+ * all in fp64, stored as fp32.  mask == NULL means every block (dense).
+ * Only the query blocks listed in `qrows` (flat b*H*C_q + h*C_q + i) are
+ * computed; qrows == NULL means all of them.  out is fp32 [nrows, q_block, D]
+ * and lse fp32 [nrows, q_block] (indexed by position in the row list).
+ */
+void ora_attention(const ora_layout *L, const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                   const uint8_t *mask, double scale, long nrows, const int64_t *qrows,
+                   float *out, float *lse)
+{
+    const int D = L->head_dim, bq = L->q_block, bk = L->k_block;
+    const int Cq = L->seq_pad / bq, Ck = L->seq_pad / bk;
+    const long total = qrows ? nrows : (long)L->batch * L->heads * Cq;
+    #pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * L->seq_pad);
+        int *u_of = (int *)malloc(sizeof(int) * L->seq_pad);
+        double *acc = (double *)malloc(sizeof(double) * D);
+        #pragma omp for schedule(dynamic, 1)
+        for (long n = 0; n < total; ++n) {
+            long r = qrows ? (long)qrows[n] : n;
+            long bh = r / Cq;
+            int i = (int)(r % Cq);
+            const uint16_t *Kb = k + bh * L->seq_pad * (long)D;
+            const uint16_t *Vb = v + bh * L->seq_pad * (long)D;
+            /* the selected keys, ascending */
+            int nu = 0;
+            for (int j = 0; j < Ck; ++j) {
+                if (mask && !mask[r * Ck + j]) continue;
+                int cnt = ora_block_count(L->seq_len, bk, j);
+                for (int t = 0; t < cnt; ++t) u_of[nu++] = j * bk + t;
+            }
+            for (int tq = 0; tq < bq; ++tq) {
+                long t = (long)i * bq + tq;
+                float *o = out + (n * bq + tq) * (long)D;
+                const uint16_t *Qt = q + (bh * L->seq_pad + t) * D;
+                if (t >= L->seq_len || nu == 0) {
+                    for (int d = 0; d < D; ++d) o[d] = 0.0f;
+                    if (lse) lse[n * bq + tq] = -INFINITY;
+                    continue;
+                }
+                double m = -INFINITY;
+                for (int a = 0; a < nu; ++a) {
+                    const uint16_t *Ku = Kb + (long)u_of[a] * D;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += bf16_val(Qt[d]) * bf16_val(Ku[d]);
+                    s[a] = dot * scale;
+                    if (s[a] > m) m = s[a];
+                }
+                double z = 0.0;
+                for (int d = 0; d < D; ++d) acc[d] = 0.0;
+                for (int a = 0; a < nu; ++a) {
+                    double e = exp(s[a] - m);
+                    const uint16_t *Vu = Vb + (long)u_of[a] * D;
+                    z += e;
+                    for (int d = 0; d < D; ++d) acc[d] += e * bf16_val(Vu[d]);
+                }
+                for (int d = 0; d < D; ++d) o[d] = (float)(acc[d] / z);
+                if (lse) lse[n * bq + tq] = (float)(m + log(z));
+            }
+        }
+        free(s);
+        free(u_of);
+        free(acc);
+    }
+}
+
+/* Threads OpenMP will use (reported next to oracle timings). */
+int ora_num_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,62 @@
+"""Pin sensitivity: plant plausible slips in copies of the oracle (on the CPU)
+and check that the pins in test_oracle_pins.py catch every one of them.
+
+A slip that no pin caught would mean the oracle could be wrong in that way
+without any test noticing.
+"""
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+from oracle import build as obuild
+from tests import test_oracle_pins as pins
+
+# (name, exact source text, replacement)
+MUTATIONS = [
+    ("drop n_j weight", "dot * inv_sqrt_d + log((double)nj)", "dot * inv_sqrt_d"),
+    ("scale 1/D instead of 1/sqrt(D)", "1.0 / sqrt((double)D)", "1.0 / (double)D"),
+    ("entropy sign", "h -= (double)row[j]", "h += (double)row[j]"),
+    ("entropy mean over C_k", "H[bh] = acc / Cq;", "H[bh] = acc / Ck;"),
+    ("frame-0 last block off by one", "*last = (end - 1) / L->q_block;", "*last = end / L->q_block;"),
+    ("frame-0 first block rounded up", "*first = start / L->q_block;",
+     "*first = (start + L->q_block - 1) / L->q_block;"),
+    ("cut entry excluded", "if (c >= p)", "if (c > p)"),
+    ("ties to the higher index", "return (x->j > y->j) - (x->j < y->j);",
+     "return (x->j < y->j) - (x->j > y->j);"),
+    ("ascending order", "if (x->p > y->p) return -1;", "if (x->p > y->p) return 1;"),
+    ("pool divides by block size", "s / n : 0.0", "s / block : 0.0"),
+    ("text blocks floored", "(L->text_len + L->k_block - 1) / L->k_block", "L->text_len / L->k_block"),
+    ("padded keys attended", "int cnt = ora_block_count(L->seq_len, bk, j);", "int cnt = bk;"),
+    ("attention scale dropped", "s[a] = dot * scale;", "s[a] = dot;"),
+    ("lse without log", "(float)(m + log(z))", "(float)(m + z)"),
+    ("text keep on query rows", "for (int j = 0; j < tk; ++j) m[j] = 1;",
+     "for (int j = 0; j < tk && i < tk; ++j) m[j] = 1;"),
+]
+
+
+def _build_variant(src, tmpdir, tag):
+    path = os.path.join(tmpdir, "mut_%s.c" % tag)
+    with open(path, "w") as f:
+        f.write(src)
+    lib = os.path.join(tmpdir, "libmut_%s.so" % tag)
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-shared", "-fPIC",
+                    path, "-o", lib, "-lm"], check=True, capture_output=True)
+    return oracle.Oracle(lib)
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_planted_slip(name, old, new):
+    src = open(obuild.SRC).read()
+    assert src.count(old) == 1, "mutation anchor not unique: %r" % old
+    with tempfile.TemporaryDirectory() as d:
+        ora = _build_variant(src.replace(old, new), d, "x")
+        caught = []
+        for check in pins.ALL_CHECKS:
+            try:
+                check(ora)
+            except (AssertionError, ValueError, FloatingPointError):
+                caught.append(check.__name__)
+        assert caught, "no pin caught the planted slip: " + name

@@ -1,0 +1,395 @@
+"""Pins that hold the CPU oracle to something other than itself.
+
+Each check compares the oracle with a closed form, an invariant the pages
+state, a brute-force search, or an independent library routine, so that a
+plausible slip in the oracle (a dropped n_j, a wrong scale, a sign, an
+off-by-one block range, an excluded cut entry, an unmasked padded key) fails at
+least one of them.  tests/test_oracle_mutations.py plants such slips in copies
+of the oracle and checks that these pins catch them.
+
+Sources: "Attention matrix view: make only frame-0 query rows dense" (s1, s2,
+s4, s6, s7); "Competition Domains Matter: Selective Head Globalization ..." s3
+(centroids, cluster-size-weighted softmax P' whose rows sum to one, per-head
+entropy normalised by log C_k, per-row local top-p); "AB-Attention: accurate
+block-sparse attention for video diffusion" TL;DR (exact attention on the
+selected blocks).
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_45_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def lay(seq_len, seq_pad, D=4, bq=4, bk=4, heads=1, batch=1, text_len=0, tpf=0, frames=0):
+    return dict(batch=batch, heads=heads, seq_len=seq_len, seq_pad=seq_pad, head_dim=D,
+                q_block=bq, k_block=bk, text_len=text_len, tokens_per_frame=tpf,
+                num_frames=frames)
+
+
+def bits(x):
+    return synth.f32_to_bf16_bits(np.asarray(x, np.float32))
+
+
+def val(h):
+    return synth.bf16_bits_to_f32(h).astype(np.float64)
+
+
+# --------------------------------------------------------------------------- layout
+
+def check_geometry(ora):
+    g = json.load(open(os.path.join(GOLDEN, "geometry.json")))
+    for name, w in synth.WORKLOADS.items():
+        e = g[name]
+        L = w.layout()
+        assert w.seq_len == e["seq_len"] and w.seq_pad == e["seq_pad"], name
+        cq, ck = w.seq_pad // w.q_block, w.seq_pad // w.k_block
+        assert (cq, ck) == (e["cq"], e["ck"]), name
+        assert ora.block_count(w.seq_len, w.q_block, cq - 1) == e["last_q_valid"], name
+        assert ora.block_count(w.seq_len, w.k_block, ck - 1) == e["last_k_valid"], name
+        assert ora.text_kblocks(L) == e["text_kblocks"], name
+        assert list(ora.frame0_qblocks(L)) == e["frame0_q"], name
+        # density forced by the overrides alone (empty top-p mask)
+        if w.batch * w.heads * cq * ck <= 2_000_000:
+            Ls = dict(L, heads=1, batch=1)
+            m = ora.overrides(Ls, 3, np.zeros((1, 1, cq, ck), np.uint8))
+            assert abs(m.mean() - e["forced_density"]) < 1e-4, name
+
+
+def test_geometry_matches_hand_values(ora):
+    check_geometry(ora)
+
+
+# --------------------------------------------------------------------------- pooling
+
+def check_pooling(ora):
+    rng = np.random.default_rng(5)
+    # constant per block -> centroid equals the constant, padded rows ignored
+    L = lay(seq_len=10, seq_pad=12, D=4, bq=4, bk=4)
+    x = np.zeros((1, 1, 12, 4), np.float32)
+    consts = [1.5, -2.25, 0.375]
+    for i, c in enumerate(consts):
+        x[0, 0, 4 * i:4 * i + 4] = c
+    x[0, 0, 10:] = 1000.0          # padding rows hold garbage; n_2 = 2 valid tokens
+    c = ora.pool(L, bits(x), 4)
+    assert np.array_equal(c[0, 0], np.array([[v] * 4 for v in consts], np.float32))
+    # mean over valid tokens only = independent numpy mean
+    x = rng.standard_normal((2, 3, 40, 8)).astype(np.float32)
+    L = lay(seq_len=37, seq_pad=40, D=8, bq=8, bk=8, heads=3, batch=2)
+    hb = bits(x)
+    c = ora.pool(L, hb, 8)
+    xv = val(hb)
+    for i in range(5):
+        ref = xv[:, :, 8 * i:min(8 * i + 8, 37)].mean(axis=2)
+        np.testing.assert_allclose(c[:, :, i], ref, rtol=1e-6, atol=1e-7)
+    # token order inside a block does not matter
+    perm = np.concatenate([rng.permutation(8) + 8 * i for i in range(4)] + [np.arange(32, 40)])
+    c2 = ora.pool(L, hb[:, :, perm], 8)
+    np.testing.assert_allclose(c2, c, rtol=1e-6, atol=1e-7)
+
+
+def test_pooling(ora):
+    check_pooling(ora)
+
+
+# --------------------------------------------------------------------------- P'
+
+def check_scores(ora):
+    # closed form: D=4 (sqrt D = 2), qc = (2,0,0,0), kc_0 = (ln 3,0,0,0), kc_1 = 0
+    # -> s = (ln 3, 0); with n = (4, 4): P' = (3/4, 1/4); with n = (4, 2): (6/7, 1/7)
+    for seq_len, expect in ((8, (0.75, 0.25)), (6, (6 / 7, 1 / 7))):
+        L = lay(seq_len=seq_len, seq_pad=8, D=4, bq=4, bk=4)
+        qc = np.zeros((1, 1, 2, 4), np.float32)
+        qc[..., 0] = 2.0
+        kc = np.zeros((1, 1, 2, 4), np.float32)
+        kc[0, 0, 0, 0] = math.log(3.0)
+        P = ora.scores(L, qc, kc)
+        np.testing.assert_allclose(P[0, 0, 0], expect, rtol=2e-7)
+    # a sign check: a negative logit lowers the weight
+    L = lay(seq_len=8, seq_pad=8, D=4)
+    qc = np.zeros((1, 1, 2, 4), np.float32)
+    qc[..., 0] = 2.0
+    kc = np.zeros((1, 1, 2, 4), np.float32)
+    kc[0, 0, 0, 0] = -math.log(3.0)
+    P = ora.scores(L, qc, kc)
+    np.testing.assert_allclose(P[0, 0, 0], (0.25, 0.75), rtol=2e-7)
+    # Q = 0: P'_ij = n_j / seq_len (the n_j weight, through a partial last block)
+    L = lay(seq_len=21, seq_pad=24, D=8, bq=8, bk=4, heads=2)
+    rng = np.random.default_rng(1)
+    kc = rng.standard_normal((1, 2, 6, 8)).astype(np.float32)
+    qc = np.zeros((1, 2, 3, 8), np.float32)
+    P = ora.scores(L, qc, kc)
+    n = np.array([4, 4, 4, 4, 4, 1], np.float64)
+    np.testing.assert_allclose(P, np.broadcast_to(n / 21.0, P.shape), rtol=1e-6)
+    # all blocks full: P' is the plain softmax of the centroid logits (torch, fp64)
+    L = lay(seq_len=48, seq_pad=48, D=16, bq=8, bk=6, heads=3, batch=2)
+    qc = rng.standard_normal((2, 3, 6, 16)).astype(np.float32) * 2
+    kc = rng.standard_normal((2, 3, 8, 16)).astype(np.float32) * 2
+    P = ora.scores(L, qc, kc)
+    ref = torch.softmax(torch.from_numpy(qc).double() @ torch.from_numpy(kc).double().transpose(-1, -2)
+                        / 4.0, dim=-1).numpy()
+    np.testing.assert_allclose(P, ref, rtol=1e-6, atol=1e-9)
+    # rows sum to one ("Competition Domains Matter" s3)
+    w = synth.WORKLOADS["tiny"]
+    x = synth.generate(w, ("q", "k"))
+    L = w.layout()
+    P = ora.scores(L, ora.pool(L, x["q"], w.q_block), ora.pool(L, x["k"], w.k_block))
+    np.testing.assert_allclose(P.astype(np.float64).sum(-1), 1.0, atol=1e-6)
+    assert (P >= 0).all()
+
+
+def test_scores(ora):
+    check_scores(ora)
+
+
+# --------------------------------------------------------------------------- entropy
+
+def check_entropy(ora):
+    eps = 1e-8
+    # uniform rows: H = ln C_k (up to C_k * eps), normalised entropy 1
+    for ck in (2, 5, 64):
+        L = lay(seq_len=4 * ck, seq_pad=4 * ck, D=4, bq=4 * ck, bk=4, heads=1)
+        P = np.full((1, 1, 1, ck), 1.0 / ck, np.float32)
+        H, Hn = ora.entropy(L, P, eps)
+        assert abs(H[0, 0] - math.log(ck)) < 1e-6 + ck * eps
+        assert abs(Hn[0, 0] - 1.0) < 1e-6
+    # one-hot rows: H ~ 0; a two-way even split: ln 2; the mean runs over rows
+    L = lay(seq_len=8, seq_pad=8, D=4, bq=4, bk=2, heads=1)
+    P = np.zeros((1, 1, 2, 4), np.float32)
+    P[0, 0, 0, 2] = 1.0
+    P[0, 0, 1, :2] = 0.5
+    H, Hn = ora.entropy(L, P, eps)
+    assert abs(H[0, 0] - math.log(2.0) / 2) < 1e-7
+    assert abs(Hn[0, 0] - math.log(2.0) / 2 / math.log(4)) < 1e-7
+    # Q = 0 closed form: -sum_j (n_j/S) ln(n_j/S + eps)
+    L = lay(seq_len=21, seq_pad=24, D=8, bq=8, bk=4, heads=1)
+    kc = np.random.default_rng(2).standard_normal((1, 1, 6, 8)).astype(np.float32)
+    P = ora.scores(L, np.zeros((1, 1, 3, 8), np.float32), kc)
+    H, _ = ora.entropy(L, P, eps)
+    p = np.array([4, 4, 4, 4, 4, 1]) / 21.0
+    assert abs(H[0, 0] - float(-(p * np.log(p + eps)).sum())) < 1e-6
+    # bounds 0 <= H <= ln C_k on real inputs
+    w = synth.WORKLOADS["tiny"]
+    x = synth.generate(w, ("q", "k"))
+    L = w.layout()
+    P = ora.scores(L, ora.pool(L, x["q"], w.q_block), ora.pool(L, x["k"], w.k_block))
+    H, Hn = ora.entropy(L, P, eps)
+    assert (H >= -1e-6).all() and (H <= math.log(P.shape[-1]) + 1e-6).all()
+
+
+def test_entropy(ora):
+    check_entropy(ora)
+
+
+# --------------------------------------------------------------------------- top-p
+
+def brute_topp(row, p):
+    """Smallest subset with mass >= p; among those the heaviest, then lowest indices."""
+    n = len(row)
+    r64 = row.astype(np.float64)
+    for k in range(1, n + 1):
+        best = None
+        for sub in itertools.combinations(range(n), k):
+            m = float(sum(r64[list(sub)]))
+            if m >= p:
+                key = (-m, sub)
+                if best is None or key < best:
+                    best = key
+        if best is not None:
+            return set(best[1])
+    return set(range(n))
+
+
+def check_topp(ora):
+    rng = np.random.default_rng(3)
+    for ck in (3, 5, 8):
+        L = lay(seq_len=4 * ck, seq_pad=4 * ck, D=4, bq=4, bk=4, heads=1)
+        for trial in range(40):
+            row = rng.dirichlet(np.full(ck, 0.7)).astype(np.float32)
+            if trial % 5 == 0:                    # exact ties, resolved to lower j
+                row[rng.integers(ck)] = row[rng.integers(ck)]
+            p = float(np.float32(rng.uniform(0.05, 0.99)))
+            P = np.broadcast_to(row, (1, 1, ck, ck)).copy()
+            m, kstar = ora.topp(L, P, p)
+            got = set(np.nonzero(m[0, 0, 0])[0].tolist())
+            exp = brute_topp(row, np.float64(np.float32(p)))
+            if len(got) != len(exp) or abs(row[list(got)].astype(np.float64).sum()
+                                           - row[list(exp)].astype(np.float64).sum()) > 0:
+                raise AssertionError((row, p, got, exp))
+            assert kstar[0, 0, 0] == len(got)
+    # the cut entry is included: (1/2, 1/4, 1/8, 1/8) with p = 3/4 keeps 2 blocks
+    L = lay(seq_len=16, seq_pad=16, D=4, bq=16, bk=4)
+    P = np.array([[[[0.125, 0.5, 0.125, 0.25]]]], np.float32)
+    for p, expect in ((0.75, {1, 3}), (0.7, {1, 3}), (0.76, {0, 1, 3}), (0.5, {1}),
+                      (1e-6, {1}), (1.0, {0, 1, 2, 3}), (1.5, {0, 1, 2, 3})):
+        m, _ = ora.topp(L, P, p)
+        assert set(np.nonzero(m[0, 0, 0])[0].tolist()) == expect, p
+    # ties at the cut go to the lower block index
+    P = np.array([[[[0.25, 0.25, 0.25, 0.25]]]], np.float32)
+    m, _ = ora.topp(L, P, 0.5)
+    assert set(np.nonzero(m[0, 0, 0])[0].tolist()) == {0, 1}
+    # per-head p is used per head
+    L = lay(seq_len=16, seq_pad=16, D=4, bq=16, bk=4, heads=2)
+    P = np.array([[[[0.125, 0.5, 0.125, 0.25]], [[0.125, 0.5, 0.125, 0.25]]]], np.float32)
+    m, k = ora.topp(L, P, [0.5, 0.8])
+    assert k[0, 0, 0] == 1 and k[0, 1, 0] == 3
+
+
+def test_topp(ora):
+    check_topp(ora)
+
+
+# --------------------------------------------------------------------------- overrides + lists
+
+def check_overrides_lists(ora):
+    w = synth.WORKLOADS["small"]
+    L = w.layout()
+    cq = ck = 65
+    rng = np.random.default_rng(4)
+    base = (rng.random((1, 1, cq, ck)) < 0.1).astype(np.uint8)
+    Ls = dict(L, heads=1)
+    m = ora.overrides(Ls, 3, base)
+    f0, f1 = 4, 16                                   # golden frame-0 range
+    assert (m[0, 0, f0:f1 + 1] == 1).all()
+    assert (m[0, 0, :, :4] == 1).all()               # text key blocks 0..3
+    rest = np.ones((cq, ck), bool)
+    rest[f0:f1 + 1] = False
+    rest[:, :4] = False
+    assert np.array_equal(m[0, 0][rest], base[0, 0][rest])
+    assert np.array_equal(ora.overrides(Ls, 0, base), base)
+    m1 = ora.overrides(Ls, 1, base)
+    assert (m1[0, 0, :, :4] == 1).all() and np.array_equal(m1[0, 0, :, 4:], base[0, 0, :, 4:])
+    # a text prefix that ends inside a key block still keeps that block, and a
+    # frame 0 that starts and ends inside query blocks densifies both of them
+    Lt = lay(seq_len=100 + 3 * 50, seq_pad=256, D=4, bq=64, bk=32, text_len=100, tpf=50,
+             frames=3)
+    assert ora.text_kblocks(Lt) == 4 and ora.frame0_qblocks(Lt) == (1, 2)
+    mt = ora.overrides(Lt, 3, np.zeros((1, 1, 4, 8), np.uint8))
+    expect = np.zeros((4, 8), np.uint8)
+    expect[:, :4] = 1
+    expect[1:3] = 1
+    assert np.array_equal(mt[0, 0], expect)
+    idx, cnt = ora.lists(Ls, m)
+    assert np.array_equal(cnt, m.sum(-1))
+    for i in range(cq):
+        sel = idx[0, 0, i, :cnt[0, 0, i]]
+        assert np.array_equal(sel, np.nonzero(m[0, 0, i])[0])
+        assert (idx[0, 0, i, cnt[0, 0, i]:] == -1).all()
+
+
+def test_overrides_and_lists(ora):
+    check_overrides_lists(ora)
+
+
+# --------------------------------------------------------------------------- attention
+
+def np_dense(q, k, v, S, scale):
+    """Matrix-form softmax(QK^T * scale)V over the first S keys (fp64, numpy)."""
+    s = (q @ k[..., :S, :].swapaxes(-1, -2)) * scale
+    m = s.max(-1, keepdims=True)
+    e = np.exp(s - m)
+    z = e.sum(-1, keepdims=True)
+    return (e / z) @ v[..., :S, :], (m + np.log(z))[..., 0]
+
+
+def check_attention(ora):
+    rng = np.random.default_rng(6)
+    # all blocks selected == independent matrix-form dense attention (and torch SDPA)
+    S, Sp, D = 45, 48, 16
+    L = lay(seq_len=S, seq_pad=Sp, D=D, bq=8, bk=16, heads=2, batch=1)
+    q = bits(rng.standard_normal((1, 2, Sp, D)) * 1.5)
+    k = bits(rng.standard_normal((1, 2, Sp, D)) * 1.5)
+    v = bits(rng.standard_normal((1, 2, Sp, D)))
+    q[:, :, S:] = bits(np.full((1, 2, Sp - S, D), 7.0))     # garbage in padded rows
+    k[:, :, S:] = bits(np.full((1, 2, Sp - S, D), 50.0))
+    v[:, :, S:] = bits(np.full((1, 2, Sp - S, D), -1e4))
+    out, lse = ora.attention(L, q, k, v, None, 0.25)
+    out = out.reshape(1, 2, Sp, D)
+    lse = lse.reshape(1, 2, Sp)
+    ref, rl = np_dense(val(q), val(k), val(v), S, 0.25)
+    np.testing.assert_allclose(out[:, :, :S], ref[:, :, :S], rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(lse[:, :, :S], rl[:, :, :S], rtol=1e-6, atol=1e-6)
+    assert (out[:, :, S:] == 0).all() and np.isneginf(lse[:, :, S:]).all()
+    t = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(val(q)[:, :, :S]), torch.from_numpy(val(k)[:, :, :S]),
+        torch.from_numpy(val(v)[:, :, :S]), scale=0.25).numpy()
+    np.testing.assert_allclose(out[:, :, :S], t, rtol=1e-5, atol=1e-6)
+    # a mask with all ones == dense
+    full = np.ones((1, 2, 6, 3), np.uint8)
+    o2, _ = ora.attention(L, q, k, v, full, 0.25)
+    np.testing.assert_array_equal(o2.reshape(out.shape), out)
+    # one selected block == softmax over that block alone; the last block is partial
+    for j in range(3):
+        m = np.zeros((1, 2, 6, 3), np.uint8)
+        m[..., j] = 1
+        o3, _ = ora.attention(L, q, k, v, m, 0.25)
+        o3 = o3.reshape(out.shape)
+        hi = min(16 * j + 16, S)
+        ref_j, _ = np_dense(val(q), val(k)[:, :, 16 * j:hi], val(v)[:, :, 16 * j:hi], hi - 16 * j, 0.25)
+        np.testing.assert_allclose(o3[:, :, :S], ref_j[:, :, :S], rtol=1e-5, atol=1e-6)
+    # per-row masks: row block i sees exactly its own key set
+    m = (rng.random((1, 2, 6, 3)) < 0.5).astype(np.uint8)
+    m[..., 0] = 1
+    o4, _ = ora.attention(L, q, k, v, m, 0.25)
+    o4 = o4.reshape(1, 2, 6, 8, D)
+    for h in range(2):
+        for i in range(6):
+            keys = np.concatenate([np.arange(16 * j, min(16 * j + 16, S)) for j in range(3)
+                                   if m[0, h, i, j]])
+            qq = val(q)[0, h, 8 * i:8 * i + 8]
+            ref_i, _ = np_dense(qq, val(k)[0, h][keys], val(v)[0, h][keys], len(keys), 0.25)
+            valid = min(8, S - 8 * i)
+            np.testing.assert_allclose(o4[0, h, i, :valid], ref_i[:valid], rtol=1e-5, atol=1e-6)
+    # shift invariance: adding w to every key adds Q_t.w to every score of row t
+    Sq = 32
+    L2 = lay(seq_len=Sq, seq_pad=Sq, D=8, bq=8, bk=8)
+    qi = rng.integers(-3, 4, (1, 1, Sq, 8)).astype(np.float32) / 4
+    ki = rng.integers(-4, 5, (1, 1, Sq, 8)).astype(np.float32)
+    vi = rng.integers(-8, 9, (1, 1, Sq, 8)).astype(np.float32)
+    wv = rng.integers(-3, 4, (8,)).astype(np.float32)
+    a, _ = ora.attention(L2, bits(qi), bits(ki), bits(vi), None, 0.5)
+    b, _ = ora.attention(L2, bits(qi), bits(ki + wv), bits(vi), None, 0.5)
+    np.testing.assert_allclose(a, b, rtol=1e-9, atol=1e-9)
+    # linearity in V
+    v2 = rng.integers(-8, 9, (1, 1, Sq, 8)).astype(np.float32)
+    c, _ = ora.attention(L2, bits(qi), bits(ki), bits(v2), None, 0.5)
+    d, _ = ora.attention(L2, bits(qi), bits(ki), bits(vi + v2), None, 0.5)
+    np.testing.assert_allclose(a + c, d, rtol=1e-5, atol=1e-5)
+
+
+def test_attention(ora):
+    check_attention(ora)
+
+
+def check_pipeline(ora):
+    """Frame-0 rows of the sparse pipeline equal the dense rows ("Attention matrix
+    view" s2); the reported density equals the mask popcount."""
+    w = synth.WORKLOADS["tiny"]
+    x = synth.generate(w)
+    L = w.layout()
+    sel = ora.select(L, x["q"], x["k"], w.top_p, w.flags)
+    assert np.array_equal(sel["kv_count"], sel["mask"].sum(-1))
+    assert sel["kv_count"].min() >= 1
+    sp, _ = ora.attention(L, x["q"], x["k"], x["v"], sel["mask"])
+    dn, _ = ora.attention(L, x["q"], x["k"], x["v"], None)
+    cq = w.seq_pad // w.q_block
+    sp = sp.reshape(w.batch, w.heads, cq, w.q_block, w.head_dim)
+    dn = dn.reshape(sp.shape)
+    f0, f1 = ora.frame0_qblocks(L)
+    np.testing.assert_array_equal(sp[:, :, f0:f1 + 1], dn[:, :, f0:f1 + 1])
+    assert not np.allclose(sp, dn)      # the sparse rows really are sparse
+
+
+def test_pipeline_invariants(ora):
+    check_pipeline(ora)
+
+
+ALL_CHECKS = [check_geometry, check_pooling, check_scores, check_entropy, check_topp,
+              check_overrides_lists, check_attention, check_pipeline]
