@@ -1,0 +1,419 @@
+"""Benchmark of the dynamic block-sparse attention path on B200.
+
+One step = one pass of the whole path over one batch: bsa_block_scores
+(centroids + P'), bsa_build_mask (top-p, text keep, frame-0 override, entropy,
+lists) and bsa_attention_fwd (exact attention over the selected blocks), on
+seeded synthetic inputs already resident in HBM.  Default workload: the
+HunyuanVideo-shaped sequence (B=1, H=24, D=128, 119,056 tokens, per-head top-p
+calibrated to 90 % skipped key blocks).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-e2e] [--no-cpu-baseline]
+
+Prints ONE JSON line on rank 0.  `value` is the computed attention TFLOP/s of
+the whole step (selected block pairs x 4*bq*bk*D FLOP / step time) summed over
+ranks; `ms_per_step` is the step time (max over ranks).  With torchrun
+(N > 1) every rank runs an independent copy of the workload (the path shards
+by head with no collective; weak scaling).  `--impl reference` times the CPU
+oracle on a bounded sample of the same workload (rank 0 only).
+"""
+import argparse
+import json
+import math
+import os
+import signal
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "block-sparse attn ms/call and computed TFLOP/s (% of B200 BF16 peak) at ~90% sparsity"
+UNIT = "TFLOP/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="hunyuan")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    return ap.parse_args()
+
+
+def load_top_p(w):
+    if w.top_p is not None:
+        return [float(w.top_p)] * w.heads
+    cal = json.load(open(os.path.join(ROOT, "tests", "golden", "top_p_calibrated.json")))
+    return [float(x) for x in cal[w.name]["top_p"]]
+
+
+def measured_peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except OSError:
+        return None
+
+
+def flops_per_pair(w):
+    return 4.0 * w.q_block * w.k_block * w.head_dim
+
+
+# ---------------------------------------------------------------- CPU oracle legs
+
+def oracle_sample(w, x, top_p, budget_s=20.0):
+    """Time the oracle (as it stands) on a bounded sample of the workload.
+
+    Selection for one head (pool, P', entropy, top-p, overrides, lists) plus
+    sparse attention for query blocks of that head, taken in a seeded random
+    order until about budget_s of attention work is done.  Returns computed
+    attention TFLOP/s over the sampled blocks, the sample description and the
+    thread count.
+    """
+    import oracle
+    ora = oracle.default()
+    L1 = dict(w.layout(), heads=1, batch=1)
+    q1, k1, v1 = x["q"][:1, :1], x["k"][:1, :1], x["v"][:1, :1]
+    t0 = time.perf_counter()
+    sel = ora.select(L1, q1, k1, top_p[:1], w.flags)
+    t_sel = time.perf_counter() - t0
+    cq = w.seq_pad // w.q_block
+    order = np.random.default_rng(0).permutation(cq)
+    chunk = max(1, ora.num_threads())     # the oracle spreads query blocks over its threads
+    done, pairs, t_attn = [], 0, 0.0
+    for c0 in range(0, cq, chunk):
+        rows = order[c0:c0 + chunk].astype(np.int64)
+        t1 = time.perf_counter()
+        ora.attention(L1, q1, k1, v1, sel["mask"], rows=rows)
+        t_attn += time.perf_counter() - t1
+        done.extend(int(i) for i in rows)
+        pairs += int(sel["kv_count"][0, 0, rows].sum())
+        if t_attn >= budget_s:
+            break
+    fl = pairs * flops_per_pair(w)
+    # the sampled blocks' share of one head's selection time is charged pro rata
+    t_total = t_attn + t_sel * len(done) / cq
+    return dict(tflops=fl / t_total / 1e12, seconds=t_total, blocks=len(done), pairs=pairs,
+                threads=ora.num_threads(), t_select_head=t_sel)
+
+
+def reference_arm(args, w):
+    """--impl reference: the CPU oracle as the reference arm (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from block_sparse_attention_45_b200 import synth
+    top_p = load_top_p(w)
+    x = synth.generate(w, heads=[0])
+    per = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(w, x, top_p, budget_s=per)
+    vals, secs, desc = [], 0.0, None
+    for _ in range(args.steps):
+        r = oracle_sample(w, x, top_p, budget_s=per)
+        vals.append(r["tflops"])
+        secs += r["seconds"]
+        desc = r
+    v = float(np.mean(vals))
+    sample = ("oracle on head 0 of %s: selection for the head + exact sparse attention for %d "
+              "random query blocks (%d selected block pairs) per step" % (w.name, desc["blocks"],
+                                                                          desc["pairs"]))
+    line = dict(metric=METRIC, value=v, unit=UNIT, n_gpus=args.gpus, steps=args.steps,
+                warmup=args.warmup, ms_per_step=secs / args.steps * 1e3, higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="f64", data="synthetic", impl="reference",
+                config=dict(workload=w.name, **{k: v for k, v in w.layout().items()}),
+                cpu_baseline=dict(value=v, unit=UNIT, cores=desc["threads"], kind="oracle",
+                                  sample=sample),
+                e2e=dict(value=v, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.send_signal(signal.SIGTERM)
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [s.strip() for s in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i] == "Active"})
+        sm = [r[0] for r in rows]
+        return dict(sm_mhz=float(np.median(sm)), sm_max_mhz=max(r[1] for r in rows),
+                    samples=len(rows), reasons=reasons)
+
+
+# ---------------------------------------------------------------- our arm
+
+def our_arm(args, w):
+    import torch
+    import torch.distributed as dist
+    from block_sparse_attention_45_b200 import binding as bsa
+    from block_sparse_attention_45_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    top_p = load_top_p(w)
+    x = synth.generate(w)
+    host = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) for k, v in x.items()}
+    q, k, v = (host[n].to(dev) for n in ("q", "k", "v"))
+    B, H, Sp, D = w.batch, w.heads, w.seq_pad, w.head_dim
+    Cq, Ck = Sp // w.q_block, Sp // w.k_block
+    f32 = dict(dtype=torch.float32, device=dev)
+    qc = torch.empty((B, H, Cq, D), **f32)
+    kc = torch.empty((B, H, Ck, D), **f32)
+    probs = torch.empty((B, H, Cq, Ck), **f32)
+    mask = torch.empty((B, H, Cq, Ck), dtype=torch.uint8, device=dev)
+    kv_index = torch.empty((B, H, Cq, Ck), dtype=torch.int32, device=dev)
+    kv_count = torch.empty((B, H, Cq), dtype=torch.int32, device=dev)
+    ent = torch.empty((B, H), **f32)
+    ent_n = torch.empty((B, H), **f32)
+    ws = torch.empty(bsa.workspace_bytes(w), dtype=torch.uint8, device=dev)
+    out = torch.empty((B, H, Sp, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, Sp), **f32)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def step(qq, kk, vv, marks=None):
+        if marks is not None:
+            marks[0].record(stream)
+        bsa.block_scores(w, qq, kk, qc, kc, probs, stream=stream)
+        if marks is not None:
+            marks[1].record(stream)
+        bsa.build_mask(w, probs, top_p, w.flags, 1e-8, mask, kv_index, kv_count, ent, ent_n, ws,
+                       stream=stream)
+        if marks is not None:
+            marks[2].record(stream)
+        bsa.attention_fwd(w, qq, kk, vv, kv_index, kv_count, None, out, lse, err, stream=stream)
+        if marks is not None:
+            marks[3].record(stream)
+
+    launches_per_step = 5   # pool, score, mask, entropy reduce, attention
+    for _ in range(max(3, args.warmup)):
+        step(q, k, v)
+    torch.cuda.synchronize(dev)
+    assert int(err.item()) == 0, "device error flag %d" % int(err.item())
+    pairs = int(kv_count.sum().item())
+    density = pairs / float(B * H * Cq * Ck)
+    step_flops = pairs * flops_per_pair(w)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    marks = [[ev() for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    t_start, t_end = ev(), ev()
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(q, k, v, marks[s])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    ms_total = t_start.elapsed_time(t_end)
+    ms_attn = [m[2].elapsed_time(m[3]) for m in marks]
+    ms_scores = [m[0].elapsed_time(m[1]) for m in marks]
+    ms_mask = [m[1].elapsed_time(m[2]) for m in marks]
+    if world > 1:
+        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    value = world * step_flops / (ms_step * 1e-3) / 1e12
+
+    # end to end through the C ABI: pinned host inputs -> device, path, output -> host
+    e2e = None
+    if not args.no_e2e:
+        pin = {n: host[n].pin_memory() for n in ("q", "k", "v")}
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        ent_h = torch.empty(ent.shape, dtype=ent.dtype).pin_memory()
+        qd, kd, vd = (torch.empty_like(q) for _ in range(3))
+
+        def e2e_step():
+            qd.copy_(pin["q"], non_blocking=True)
+            kd.copy_(pin["k"], non_blocking=True)
+            vd.copy_(pin["v"], non_blocking=True)
+            step(qd, kd, vd)
+            out_h.copy_(out, non_blocking=True)
+            ent_h.copy_(ent, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        ms_e2e = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        ms_e2e /= args.steps
+        h2d = sum(pin[n].numel() * pin[n].element_size() for n in pin)
+        d2h = out_h.numel() * out_h.element_size() + ent_h.numel() * ent_h.element_size()
+        e2e = dict(value=world * step_flops / (ms_e2e * 1e-3) / 1e12, unit=UNIT,
+                   ms_per_step=ms_e2e, h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h))
+
+    # the dense path (all key blocks) for context: not part of the step
+    dense = None
+    if not args.no_dense:
+        for _ in range(2):
+            bsa.dense_fwd(w, q, k, v, None, out, lse, stream=stream)
+        a, b = ev(), ev()
+        a.record(stream)
+        nd = max(1, min(3, args.steps))
+        for _ in range(nd):
+            bsa.dense_fwd(w, q, k, v, None, out, lse, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        dms = a.elapsed_time(b) / nd
+        dflops = B * H * Cq * Ck * flops_per_pair(w)
+        dense = dict(ms=dms, tflops=dflops / (dms * 1e-3) / 1e12)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks = measured_peaks()
+    attn_ms = float(np.mean(ms_attn))
+    achieved = step_flops / (attn_ms * 1e-3) / 1e12
+    if peaks:
+        peak, peak_note = peaks["bf16_tflops_sustained"], "measured sustained (MEASURED_PEAKS.json)"
+        burst = peaks["bf16_tflops"]
+        hbm = peaks["hbm_gbs"]
+    else:
+        peak, peak_note, burst, hbm = 1400.0, "fallback sustained", 1590.0, 6650.0
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(prof):
+        try:
+            t = json.load(open(prof)).get(w.name)
+            if t and t.get("kernel_sha") == kernel_sha():
+                traffic = t["bytes_per_launch"]
+        except (OSError, ValueError, KeyError):
+            traffic = None
+    # scoring and mask: algorithmic bytes (read Q, K once; write centroids, P'; read P',
+    # write mask, lists, counts) over their measured durations
+    bytes_scores = 2 * B * H * w.seq_len * D * 2 + 4 * B * H * (Cq + Ck) * D + 4 * B * H * Cq * Ck
+    bytes_mask = 4 * B * H * Cq * Ck + B * H * Cq * Ck + 4 * pairs + 4 * B * H * Cq
+    line = dict(
+        metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
+        ms_per_step=ms_step, higher_is_better=True, scaling="weak", vs_baseline=None,
+        dtype="bf16", data="synthetic (seeded clustered Gaussian Q/K, N(0,1) V; per-head top-p "
+                             "calibrated on the CPU oracle)",
+        config=dict(workload=w.name, batch=B, heads=H, seq_len=w.seq_len, seq_pad=Sp, head_dim=D,
+                    q_block=w.q_block, k_block=w.k_block, text_len=w.text_len,
+                    frames=w.num_frames, latent=[w.latent_h, w.latent_w],
+                    density=density, skipped=1 - density, selected_pairs=pairs,
+                    computed_tflop_per_step=step_flops / 1e12,
+                    dense_equiv_tflop=4.0 * B * H * w.seq_len ** 2 * D / 1e12,
+                    parallelism="replicas, one independent problem per GPU" if world > 1 else "1 GPU",
+                    l2="inputs (Q, K, V = %.2f GB) larger than the 126 MB L2; no flush" %
+                       (3 * B * H * Sp * D * 2 / 1e9)),
+        attention=dict(ms=attn_ms, tflops=achieved, dense_equiv_tflops=4.0 * B * H * w.seq_len ** 2
+                       * D / (attn_ms * 1e-3) / 1e12, frac_of_burst=achieved / burst),
+        scores=dict(ms=float(np.mean(ms_scores)), gbs=bytes_scores / (np.mean(ms_scores) * 1e-3) / 1e9,
+                    frac_hbm=bytes_scores / (np.mean(ms_scores) * 1e-3) / 1e9 / hbm),
+        mask=dict(ms=float(np.mean(ms_mask)), gbs=bytes_mask / (np.mean(ms_mask) * 1e-3) / 1e9,
+                  frac_hbm=bytes_mask / (np.mean(ms_mask) * 1e-3) / 1e9 / hbm),
+        dense=dense,
+        roofline=dict(bound="tensor", kernel="attn_kernel", achieved=achieved, peak=peak,
+                      unit="TFLOP/s", frac=achieved / peak, peak_source=peak_note,
+                      traffic=traffic, flop_per_launch=step_flops,
+                      flop_per_unit=flops_per_pair(w), units_per_launch=pairs),
+        gpu_launches=launches_per_step * args.steps,
+        clocks=clk,
+        e2e=e2e,
+    )
+    if not args.no_cpu_baseline and world == 1:
+        r = oracle_sample(w, {n: x[n] for n in ("q", "k", "v")}, top_p, budget_s=20.0)
+        line["cpu_baseline"] = dict(
+            value=r["tflops"], unit=UNIT, cores=r["threads"], kind="oracle",
+            sample="oracle on head 0: selection for the head + exact sparse attention for %d random "
+                   "query blocks (%d selected block pairs), %.1f s" % (r["blocks"], r["pairs"],
+                                                                       r["seconds"]))
+    print(json.dumps(line), flush=True)
+
+
+def kernel_sha():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("attention.cu", "ptx.cuh"):
+        h.update(open(os.path.join(ROOT, "block_sparse_attention_45_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def main():
+    args = parse()
+    from block_sparse_attention_45_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        reference_arm(args, w)
+    else:
+        our_arm(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,238 @@
+"""ctypes binding of libbsa.so (include/bsa.h): argument marshalling only.
+
+Every step of the computation runs in the CUDA kernels behind the C ABI; this
+module only checks tensor metadata, allocates outputs with torch (device
+memory is plumbing) and passes raw pointers plus the current CUDA stream.
+There is no CPU fallback: if the library is missing, every call raises.
+"""
+import ctypes
+import math
+import os
+import re
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libbsa.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "bsa.h")
+
+BSA_OK = 0
+BSA_ERR_INVALID_ARG = 1
+BSA_ERR_UNSUPPORTED = 2
+BSA_ERR_LAUNCH = 3
+BSA_ERR_DRIVER = 4
+TEXT_KEEP = 1
+FRAME0_DENSE = 2
+DEVERR_BAD_INDEX = 1
+DEVERR_BAD_COUNT = 2
+DEVERR_TIMEOUT = 4
+
+LAYOUT_FIELDS = ("batch", "heads", "seq_len", "seq_pad", "head_dim", "q_block", "k_block",
+                 "text_len", "tokens_per_frame", "num_frames")
+
+
+class BsaLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in LAYOUT_FIELDS]
+
+
+class BsaError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__("%s failed: %s" % (fn, status_string(status)))
+
+
+_LIB = None
+
+
+def load():
+    """Load libbsa.so (raises if it was not built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libbsa.so is not built; run `python -m block_sparse_attention_45_b200.build` "
+                               "(there is no CPU fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        lp = ctypes.POINTER(BsaLayout)
+        vp = ctypes.c_void_p
+        L.bsa_block_scores.argtypes = [lp, vp, vp, vp, vp, vp, vp]
+        L.bsa_block_scores.restype = ctypes.c_int
+        L.bsa_build_mask_workspace_bytes.argtypes = [lp]
+        L.bsa_build_mask_workspace_bytes.restype = ctypes.c_size_t
+        L.bsa_build_mask.argtypes = [lp, vp, vp, ctypes.c_uint32, ctypes.c_float, vp, vp, vp, vp,
+                                     vp, vp, vp]
+        L.bsa_build_mask.restype = ctypes.c_int
+        L.bsa_attention_fwd.argtypes = [lp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp]
+        L.bsa_attention_fwd.restype = ctypes.c_int
+        L.bsa_dense_fwd.argtypes = [lp, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp]
+        L.bsa_dense_fwd.restype = ctypes.c_int
+        L.bsa_status_string.argtypes = [ctypes.c_int]
+        L.bsa_status_string.restype = ctypes.c_char_p
+        L.bsa_version.restype = ctypes.c_int
+        _LIB = L
+    return _LIB
+
+
+def declared_symbols():
+    """Function names declared in include/bsa.h."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(bsa_[a-z_0-9]+)\s*\(",
+                                 text, re.M)))
+
+
+def status_string(status):
+    return load().bsa_status_string(int(status)).decode()
+
+
+def make_layout(layout):
+    if isinstance(layout, BsaLayout):
+        return layout
+    if hasattr(layout, "layout"):
+        layout = layout.layout()
+    return BsaLayout(*[int(layout[n]) for n in LAYOUT_FIELDS])
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn, rc):
+    if rc != BSA_OK:
+        raise BsaError(fn, rc)
+
+
+def _need(t, name, dtype, shape):
+    if t.dtype != dtype:
+        raise TypeError("%s: expected %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s: expected shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+
+
+def dims(L):
+    L = make_layout(L)
+    return dict(B=L.batch, H=L.heads, S=L.seq_len, Sp=L.seq_pad, D=L.head_dim,
+                Cq=L.seq_pad // L.q_block, Ck=L.seq_pad // L.k_block)
+
+
+def block_scores(layout, q, k, q_centroids=None, k_centroids=None, probs=None, stream=None):
+    """bsa_block_scores: returns (q_centroids, k_centroids, probs)."""
+    L = make_layout(layout)
+    d = dims(L)
+    qkv = (d["B"], d["H"], d["Sp"], d["D"])
+    _need(q, "q", torch.bfloat16, qkv)
+    _need(k, "k", torch.bfloat16, qkv)
+    dev = q.device
+    if q_centroids is None:
+        q_centroids = torch.empty((d["B"], d["H"], d["Cq"], d["D"]), dtype=torch.float32, device=dev)
+    if k_centroids is None:
+        k_centroids = torch.empty((d["B"], d["H"], d["Ck"], d["D"]), dtype=torch.float32, device=dev)
+    if probs is None:
+        probs = torch.empty((d["B"], d["H"], d["Cq"], d["Ck"]), dtype=torch.float32, device=dev)
+    _need(q_centroids, "q_centroids", torch.float32, (d["B"], d["H"], d["Cq"], d["D"]))
+    _need(k_centroids, "k_centroids", torch.float32, (d["B"], d["H"], d["Ck"], d["D"]))
+    _need(probs, "probs", torch.float32, (d["B"], d["H"], d["Cq"], d["Ck"]))
+    rc = load().bsa_block_scores(ctypes.byref(L), _ptr(q), _ptr(k), _ptr(q_centroids),
+                                 _ptr(k_centroids), _ptr(probs), _stream(stream))
+    _check("bsa_block_scores", rc)
+    return q_centroids, k_centroids, probs
+
+
+def workspace_bytes(layout):
+    L = make_layout(layout)
+    return int(load().bsa_build_mask_workspace_bytes(ctypes.byref(L)))
+
+
+def build_mask(layout, probs, top_p, flags, eps=1e-8, mask=None, kv_index=None, kv_count=None,
+               entropy=None, entropy_norm=None, workspace=None, with_mask=True,
+               with_entropy=True, stream=None):
+    """bsa_build_mask: returns dict(mask, kv_index, kv_count, entropy, entropy_norm)."""
+    L = make_layout(layout)
+    d = dims(L)
+    _need(probs, "probs", torch.float32, (d["B"], d["H"], d["Cq"], d["Ck"]))
+    dev = probs.device
+    tp = (ctypes.c_float * d["H"])(*[float(x) for x in
+                                     (list(top_p) if hasattr(top_p, "__len__") else [top_p] * d["H"])])
+    if len(tp) != d["H"]:
+        raise ValueError("top_p needs one value per head")
+    if mask is None and with_mask:
+        mask = torch.empty((d["B"], d["H"], d["Cq"], d["Ck"]), dtype=torch.uint8, device=dev)
+    if kv_index is None:
+        kv_index = torch.empty((d["B"], d["H"], d["Cq"], d["Ck"]), dtype=torch.int32, device=dev)
+    if kv_count is None:
+        kv_count = torch.empty((d["B"], d["H"], d["Cq"]), dtype=torch.int32, device=dev)
+    if with_entropy:
+        if entropy is None:
+            entropy = torch.empty((d["B"], d["H"]), dtype=torch.float32, device=dev)
+        if entropy_norm is None:
+            entropy_norm = torch.empty((d["B"], d["H"]), dtype=torch.float32, device=dev)
+        if workspace is None:
+            workspace = torch.empty(workspace_bytes(L), dtype=torch.uint8, device=dev)
+    rc = load().bsa_build_mask(ctypes.byref(L), _ptr(probs), ctypes.cast(tp, ctypes.c_void_p),
+                               int(flags), float(eps), _ptr(mask), _ptr(kv_index), _ptr(kv_count),
+                               _ptr(entropy), _ptr(entropy_norm), _ptr(workspace), _stream(stream))
+    _check("bsa_build_mask", rc)
+    return dict(mask=mask, kv_index=kv_index, kv_count=kv_count, entropy=entropy,
+                entropy_norm=entropy_norm)
+
+
+def attention_fwd(layout, q, k, v, kv_index, kv_count, softmax_scale=None, out=None, lse=None,
+                  err_flag=None, with_lse=True, stream=None):
+    """bsa_attention_fwd: returns (out, lse)."""
+    L = make_layout(layout)
+    d = dims(L)
+    qkv = (d["B"], d["H"], d["Sp"], d["D"])
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, qkv)
+    _need(kv_index, "kv_index", torch.int32, (d["B"], d["H"], d["Cq"], d["Ck"]))
+    _need(kv_count, "kv_count", torch.int32, (d["B"], d["H"], d["Cq"]))
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d["D"])
+    if out is None:
+        out = torch.empty(qkv, dtype=torch.bfloat16, device=q.device)
+    if lse is None and with_lse:
+        lse = torch.empty((d["B"], d["H"], d["Sp"]), dtype=torch.float32, device=q.device)
+    rc = load().bsa_attention_fwd(ctypes.byref(L), _ptr(q), _ptr(k), _ptr(v), _ptr(kv_index),
+                                  _ptr(kv_count), float(softmax_scale), _ptr(out), _ptr(lse),
+                                  _ptr(err_flag), _stream(stream))
+    _check("bsa_attention_fwd", rc)
+    return out, lse
+
+
+def dense_fwd(layout, q, k, v, softmax_scale=None, out=None, lse=None, err_flag=None,
+              with_lse=True, stream=None):
+    """bsa_dense_fwd: returns (out, lse)."""
+    L = make_layout(layout)
+    d = dims(L)
+    qkv = (d["B"], d["H"], d["Sp"], d["D"])
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, qkv)
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d["D"])
+    if out is None:
+        out = torch.empty(qkv, dtype=torch.bfloat16, device=q.device)
+    if lse is None and with_lse:
+        lse = torch.empty((d["B"], d["H"], d["Sp"]), dtype=torch.float32, device=q.device)
+    rc = load().bsa_dense_fwd(ctypes.byref(L), _ptr(q), _ptr(k), _ptr(v), float(softmax_scale),
+                              _ptr(out), _ptr(lse), _ptr(err_flag), _stream(stream))
+    _check("bsa_dense_fwd", rc)
+    return out, lse
+
+
+def sparse_attention(layout, q, k, v, top_p, flags, eps=1e-8, softmax_scale=None, stream=None):
+    """The whole path: scores -> mask -> block-sparse attention.  Returns a dict."""
+    qc, kc, probs = block_scores(layout, q, k, stream=stream)
+    sel = build_mask(layout, probs, top_p, flags, eps, stream=stream)
+    out, lse = attention_fwd(layout, q, k, v, sel["kv_index"], sel["kv_count"], softmax_scale,
+                             stream=stream)
+    sel.update(q_centroids=qc, k_centroids=kc, probs=probs, out=out, lse=lse)
+    return sel

@@ -1,0 +1,168 @@
+// api.cu -- the C ABI: host-side validation, geometry, dispatch to the kernels.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "bsa.h"
+#include "internal.h"
+
+namespace bsa {
+
+Geometry make_geometry(const bsa_layout &L) {
+    Geometry g;
+    g.B = L.batch;
+    g.H = L.heads;
+    g.S = L.seq_len;
+    g.S_pad = L.seq_pad;
+    g.D = L.head_dim;
+    g.bq = L.q_block;
+    g.bk = L.k_block;
+    g.Cq = L.seq_pad / L.q_block;
+    g.Ck = L.seq_pad / L.k_block;
+    // "Attention matrix view ..." s7: key blocks that hold a text token.
+    g.text_kblocks = (L.text_len + L.k_block - 1) / L.k_block;
+    if (g.text_kblocks > g.Ck) g.text_kblocks = g.Ck;
+    // "Attention matrix view ..." s4: query blocks that overlap frame 0.
+    if (L.tokens_per_frame > 0 && L.num_frames > 0) {
+        g.f0_first = L.text_len / L.q_block;
+        g.f0_last = (L.text_len + L.tokens_per_frame - 1) / L.q_block;
+        if (g.f0_last > g.Cq - 1) g.f0_last = g.Cq - 1;
+    } else {
+        g.f0_first = 0;
+        g.f0_last = -1;
+    }
+    return g;
+}
+
+}  // namespace bsa
+
+namespace {
+
+using bsa::Geometry;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_layout(const bsa_layout *L) {
+    if (!L) return BSA_ERR_INVALID_ARG;
+    if (L->batch < 1 || L->heads < 1 || L->seq_len < 1 || L->seq_pad < L->seq_len)
+        return BSA_ERR_INVALID_ARG;
+    if (L->heads > bsa::kMaxHeads) return BSA_ERR_UNSUPPORTED;
+    if (L->head_dim != 64 && L->head_dim != 128) return BSA_ERR_UNSUPPORTED;
+    if ((L->q_block != 64 && L->q_block != 128) || (L->k_block != 64 && L->k_block != 128))
+        return BSA_ERR_UNSUPPORTED;
+    const int big = L->q_block > L->k_block ? L->q_block : L->k_block;
+    const int small = L->q_block < L->k_block ? L->q_block : L->k_block;
+    if (L->seq_pad % big != 0) return BSA_ERR_INVALID_ARG;
+    if (L->seq_pad - L->seq_len >= small) return BSA_ERR_INVALID_ARG;  // a block with no token
+    if (L->text_len < 0 || L->tokens_per_frame < 0 || L->num_frames < 0) return BSA_ERR_INVALID_ARG;
+    const long long covered =
+        static_cast<long long>(L->text_len) + static_cast<long long>(L->num_frames) * L->tokens_per_frame;
+    if (covered > L->seq_len) return BSA_ERR_INVALID_ARG;
+    const long long elems = static_cast<long long>(L->batch) * L->heads * L->seq_pad;
+    if (elems > (1ll << 40)) return BSA_ERR_UNSUPPORTED;
+    if (static_cast<long long>(L->batch) * L->heads * (L->seq_pad / L->q_block) > 0x7FFFFFFFll)
+        return BSA_ERR_UNSUPPORTED;
+    return BSA_OK;
+}
+
+int launch_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_LAUNCH; }
+
+}  // namespace
+
+extern "C" {
+
+int bsa_version(void) { return 100; }
+
+const char *bsa_status_string(int status) {
+    switch (status) {
+        case BSA_OK: return "BSA_OK";
+        case BSA_ERR_INVALID_ARG: return "BSA_ERR_INVALID_ARG";
+        case BSA_ERR_UNSUPPORTED: return "BSA_ERR_UNSUPPORTED";
+        case BSA_ERR_LAUNCH: return "BSA_ERR_LAUNCH";
+        case BSA_ERR_DRIVER: return "BSA_ERR_DRIVER";
+        default: return "BSA_ERR_UNKNOWN";
+    }
+}
+
+int bsa_block_scores(const bsa_layout *layout, const void *q, const void *k, float *q_centroids,
+                     float *k_centroids, float *probs, void *stream) {
+    int rc = check_layout(layout);
+    if (rc != BSA_OK) return rc;
+    if (!q || !k || !q_centroids || !k_centroids || !probs) return BSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(q_centroids, 16) || !aligned(k_centroids, 16) ||
+        !aligned(probs, 16))
+        return BSA_ERR_INVALID_ARG;
+    const Geometry g = bsa::make_geometry(*layout);
+    if (g.Ck > bsa::kMaxScoreCk) return BSA_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = launch_status(bsa::launch_pool(g, q, k, q_centroids, k_centroids, st));
+    if (rc != BSA_OK) return rc;
+    return launch_status(bsa::launch_scores(g, q_centroids, k_centroids, probs, st));
+}
+
+size_t bsa_build_mask_workspace_bytes(const bsa_layout *layout) {
+    if (check_layout(layout) != BSA_OK) return 0;
+    const size_t rows = static_cast<size_t>(layout->batch) * layout->heads *
+                        (layout->seq_pad / layout->q_block);
+    return ((rows * sizeof(float) + 255) / 256) * 256;
+}
+
+int bsa_build_mask(const bsa_layout *layout, const float *probs, const float *top_p, uint32_t flags,
+                   float eps, uint8_t *mask, int32_t *kv_index, int32_t *kv_count, float *entropy,
+                   float *entropy_norm, void *workspace, void *stream) {
+    int rc = check_layout(layout);
+    if (rc != BSA_OK) return rc;
+    if (!probs || !top_p || !kv_index || !kv_count) return BSA_ERR_INVALID_ARG;
+    if (flags & ~static_cast<uint32_t>(BSA_TEXT_KEEP | BSA_FRAME0_DENSE)) return BSA_ERR_INVALID_ARG;
+    if (!aligned(probs, 4) || !aligned(kv_index, 4) || !aligned(kv_count, 4)) return BSA_ERR_INVALID_ARG;
+    const bool want_entropy = entropy || entropy_norm;
+    if (want_entropy && (!workspace || !aligned(workspace, 16))) return BSA_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || !isfinite(eps)) return BSA_ERR_INVALID_ARG;
+    const Geometry g = bsa::make_geometry(*layout);
+    if (g.Ck > bsa::kMaxMaskCk) return BSA_ERR_UNSUPPORTED;
+    bsa::TopP tp;
+    memset(&tp, 0, sizeof tp);
+    for (int h = 0; h < g.H; ++h) {
+        if (isnan(top_p[h])) return BSA_ERR_INVALID_ARG;
+        tp.p[h] = top_p[h];
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float *row_ent = want_entropy ? static_cast<float *>(workspace) : nullptr;
+    rc = launch_status(bsa::launch_mask(g, probs, tp, flags, eps, mask, kv_index, kv_count, row_ent, st));
+    if (rc != BSA_OK || !want_entropy) return rc;
+    return launch_status(bsa::launch_entropy_reduce(g, row_ent, entropy, entropy_norm, st));
+}
+
+int bsa_attention_fwd(const bsa_layout *layout, const void *q, const void *k, const void *v,
+                      const int32_t *kv_index, const int32_t *kv_count, float softmax_scale,
+                      void *out, float *lse, int32_t *err_flag, void *stream) {
+    int rc = check_layout(layout);
+    if (rc != BSA_OK) return rc;
+    if (!q || !k || !v || !out || !kv_index || !kv_count) return BSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+        return BSA_ERR_INVALID_ARG;
+    if (!aligned(kv_index, 4) || !aligned(kv_count, 4) || (lse && !aligned(lse, 4)) ||
+        (err_flag && !aligned(err_flag, 4)))
+        return BSA_ERR_INVALID_ARG;
+    if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return BSA_ERR_INVALID_ARG;
+    const Geometry g = bsa::make_geometry(*layout);
+    return bsa::launch_attention(g, q, k, v, kv_index, kv_count, softmax_scale, out, lse, err_flag,
+                                 static_cast<cudaStream_t>(stream));
+}
+
+int bsa_dense_fwd(const bsa_layout *layout, const void *q, const void *k, const void *v,
+                  float softmax_scale, void *out, float *lse, int32_t *err_flag, void *stream) {
+    int rc = check_layout(layout);
+    if (rc != BSA_OK) return rc;
+    if (!q || !k || !v || !out) return BSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+        return BSA_ERR_INVALID_ARG;
+    if ((lse && !aligned(lse, 4)) || (err_flag && !aligned(err_flag, 4))) return BSA_ERR_INVALID_ARG;
+    if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return BSA_ERR_INVALID_ARG;
+    const Geometry g = bsa::make_geometry(*layout);
+    return bsa::launch_attention(g, q, k, v, nullptr, nullptr, softmax_scale, out, lse, err_flag,
+                                 static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

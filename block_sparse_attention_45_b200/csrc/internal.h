@@ -1,0 +1,43 @@
+// internal.h -- launchers shared between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "bsa.h"
+
+namespace bsa {
+
+constexpr int kMaxHeads = 256;
+constexpr int kMaxScoreCk = 2048;  // bsa_block_scores
+constexpr int kMaxMaskCk = 2048;   // bsa_build_mask
+
+struct Geometry {
+    int B, H, S, S_pad, D, bq, bk, Cq, Ck;
+    int text_kblocks;       // key blocks holding text tokens
+    int f0_first, f0_last;  // frame-0 query-block range, f0_last < f0_first when empty
+};
+
+Geometry make_geometry(const bsa_layout &L);
+
+cudaError_t launch_pool(const Geometry &g, const void *q, const void *k, float *qc, float *kc,
+                        cudaStream_t st);
+cudaError_t launch_scores(const Geometry &g, const float *qc, const float *kc, float *probs,
+                          cudaStream_t st);
+
+struct TopP {
+    float p[kMaxHeads];
+};
+
+cudaError_t launch_mask(const Geometry &g, const float *probs, const TopP &tp, uint32_t flags,
+                        float eps, uint8_t *mask, int32_t *kv_index, int32_t *kv_count,
+                        float *row_entropy, cudaStream_t st);
+cudaError_t launch_entropy_reduce(const Geometry &g, const float *row_entropy, float *entropy,
+                                  float *entropy_norm, cudaStream_t st);
+
+// Returns BSA_* status.
+int launch_attention(const Geometry &g, const void *q, const void *k, const void *v,
+                     const int32_t *kv_index, const int32_t *kv_count, float softmax_scale,
+                     void *out, float *lse, int32_t *err_flag, cudaStream_t st);
+
+}  // namespace bsa

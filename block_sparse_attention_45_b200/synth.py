@@ -22,7 +22,9 @@ same shapes:
 Each (tensor, b, h) uses its own numpy PCG64 stream seeded with
 [seed, tensor, b, h], so any head can be generated on its own.
 """
-from dataclasses import dataclass, field, asdict
+import os
+from concurrent.futures import ThreadPoolExecutor
+from dataclasses import dataclass, asdict
 
 import numpy as np
 
@@ -153,15 +155,29 @@ def _draw_head(w, tensor, b, h):
     return x
 
 
-def generate(w, tensors=("q", "k", "v"), heads=None, batches=None):
-    """Raw bf16 bits, dict tensor -> uint16 [len(batches), len(heads), seq_pad, D]."""
+def generate(w, tensors=("q", "k", "v"), heads=None, batches=None, workers=None):
+    """Raw bf16 bits, dict tensor -> uint16 [len(batches), len(heads), seq_pad, D].
+
+    Every (tensor, b, h) has its own stream, so the result does not depend on
+    `workers` (threads that fill different heads at the same time).
+    """
     heads = list(range(w.heads)) if heads is None else list(heads)
     batches = list(range(w.batch)) if batches is None else list(batches)
-    out = {}
-    for t in tensors:
-        a = np.zeros((len(batches), len(heads), w.seq_pad, w.head_dim), np.uint16)
-        for bi, b in enumerate(batches):
-            for hi, h in enumerate(heads):
-                a[bi, hi, :w.seq_len] = f32_to_bf16_bits(_draw_head(w, t, b, h))
-        out[t] = a
+    out = {t: np.zeros((len(batches), len(heads), w.seq_pad, w.head_dim), np.uint16)
+           for t in tensors}
+    jobs = [(t, bi, b, hi, h) for t in tensors for bi, b in enumerate(batches)
+            for hi, h in enumerate(heads)]
+
+    def fill(job):
+        t, bi, b, hi, h = job
+        out[t][bi, hi, :w.seq_len] = f32_to_bf16_bits(_draw_head(w, t, b, h))
+
+    if workers is None:
+        workers = min(len(jobs), max(1, (os.cpu_count() or 1)))
+    if workers <= 1 or len(jobs) <= 1:
+        for j in jobs:
+            fill(j)
+    else:
+        with ThreadPoolExecutor(max_workers=workers) as ex:
+            list(ex.map(fill, jobs))
     return out

@@ -1,0 +1,192 @@
+/*
+ * bsa.h -- C ABI of the B200 (sm_100a) dynamic block-sparse attention library.
+ *
+ * The library implements the selection-then-attention path for video
+ * diffusion transformers:
+ *
+ *   bsa_block_scores   block centroids of Q and K, then the cluster-size-
+ *                      weighted softmax P' over key blocks
+ *   bsa_build_mask     per-row top-p over P', text-block keep, frame-0 dense
+ *                      override, per-head entropy, compacted key-block lists
+ *   bsa_attention_fwd  exact softmax attention over the listed key blocks only
+ *   bsa_dense_fwd      the same kernel with every key block listed
+ *
+ * Sources (pages by title and section):
+ *   "Attention matrix view: make only frame-0 query rows dense"
+ *       s1 token packing [text] + frame0 + frame1 + ...; s2 dense rows vs
+ *       sparse rows; s4 block-level override of the query blocks that overlap
+ *       frame 0; s7 keep text/global blocks.
+ *   "Competition Domains Matter: Selective Head Globalization for
+ *    Training-Free Sparse Attention in Video Diffusion Transformers"
+ *       s3: centroids with cluster sizes n_i, n_j; cluster-size-weighted
+ *       softmax P' (Eq. 1; rows sum to one); per-head entropy H_h (Eq. 3)
+ *       and H_h / log C_k; per-row local top-p (domain 1, Eq. 2).
+ *   "AB-Attention: accurate block-sparse attention for video diffusion"
+ *       TL;DR: exact attention computed only on the selected K/V blocks; key
+ *       blocks smaller than a tensor-core tile gathered into full tiles.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are dense, row-major, and live in device memory that the caller
+ *     allocated.  The library allocates nothing, frees nothing and keeps no
+ *     state between calls beyond a cached driver entry point.
+ *   - Q, K, V and O are bf16 [batch, heads, seq_pad, head_dim].  Token t of
+ *     (b, h) is row t; rows seq_len..seq_pad-1 are padding and are never read
+ *     as keys.  Every other array is described at its entry point.
+ *   - Query block i covers tokens [i*q_block, (i+1)*q_block); key block j
+ *     covers [j*k_block, (j+1)*k_block).  C_q = seq_pad / q_block,
+ *     C_k = seq_pad / k_block.  n_j = number of tokens of block j below
+ *     seq_len.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and never synchronises.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     failed check returns BSA_ERR_INVALID_ARG (or BSA_ERR_UNSUPPORTED for a
+ *     valid shape this build has no kernel for) and launches nothing.
+ *   - A launch failure returns BSA_ERR_LAUNCH; a failure of the driver's
+ *     tensor-map encoder returns BSA_ERR_DRIVER.
+ *   - Bad data found on the device (a list entry outside [0, C_k), a count
+ *     outside [0, C_k], a wait that timed out) never traps: the kernel skips
+ *     the offending item and ORs a BSA_DEVERR_* bit into *err_flag when the
+ *     caller passed one (a device int32 the caller zeroes beforehand).
+ */
+#ifndef BSA_H
+#define BSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Problem geometry ("Attention matrix view ..." s1 and s4). */
+typedef struct bsa_layout {
+    int32_t batch;            /* B >= 1 */
+    int32_t heads;            /* H, 1..256 */
+    int32_t seq_len;          /* S valid tokens, >= 1 */
+    int32_t seq_pad;          /* padded length: a multiple of max(q_block, k_block),
+                                 seq_pad - seq_len < min(q_block, k_block) so that
+                                 every block holds at least one valid token */
+    int32_t head_dim;         /* D: 64 or 128 */
+    int32_t q_block;          /* 64 or 128 */
+    int32_t k_block;          /* 64 or 128 */
+    int32_t text_len;         /* text tokens at the front of the sequence, >= 0 */
+    int32_t tokens_per_frame; /* latent_h * latent_w, >= 0 */
+    int32_t num_frames;       /* >= 0; text_len + num_frames*tokens_per_frame <= seq_len */
+} bsa_layout;
+
+enum bsa_status {
+    BSA_OK = 0,
+    BSA_ERR_INVALID_ARG = 1,
+    BSA_ERR_UNSUPPORTED = 2,
+    BSA_ERR_LAUNCH = 3,
+    BSA_ERR_DRIVER = 4
+};
+
+/* bsa_build_mask flags */
+enum bsa_flags {
+    BSA_TEXT_KEEP = 1u,     /* keep every key block that holds a text token ("... s7") */
+    BSA_FRAME0_DENSE = 2u   /* every key block for query blocks overlapping frame 0 ("... s4") */
+};
+
+/* Bits ORed into *err_flag by device code. */
+enum bsa_device_error {
+    BSA_DEVERR_BAD_INDEX = 1,  /* a kv_index entry outside [0, C_k): entry skipped */
+    BSA_DEVERR_BAD_COUNT = 2,  /* a kv_count outside [0, C_k]: clamped */
+    BSA_DEVERR_TIMEOUT = 4     /* an internal pipeline wait gave up: the tile's output is invalid */
+};
+
+/*
+ * Block centroids and block scores ("Competition Domains Matter" s3, Eq. 1).
+ *
+ *   q_centroids[b,h,i,:] = mean of Q rows of query block i below seq_len
+ *   k_centroids[b,h,j,:] = mean of K rows of key block j below seq_len
+ *   s_ij  = q_centroids_i . k_centroids_j / sqrt(head_dim)
+ *   probs[b,h,i,j] = P'_ij = n_j exp(s_ij) / sum_j' n_j' exp(s_ij')
+ *
+ * q, k          bf16 [B,H,seq_pad,D], 16-byte aligned (read only)
+ * q_centroids   fp32 [B,H,C_q,D], 16-byte aligned (written)
+ * k_centroids   fp32 [B,H,C_k,D], 16-byte aligned (written)
+ * probs         fp32 [B,H,C_q,C_k], 16-byte aligned (written; each row sums to 1)
+ * Accumulation is fp32.  Supports C_k up to 2048.
+ */
+int bsa_block_scores(const bsa_layout *layout, const void *q, const void *k,
+                     float *q_centroids, float *k_centroids, float *probs, void *stream);
+
+/* Bytes of device workspace bsa_build_mask needs (per-row entropies). */
+size_t bsa_build_mask_workspace_bytes(const bsa_layout *layout);
+
+/*
+ * Selection ("Competition Domains Matter" s3 domain 1 and Eq. 3;
+ * "Attention matrix view ..." s4, s6, s7).  For every row (b,h,i):
+ *   1. top-p: order the row by (P' descending, j ascending) and keep the
+ *      shortest prefix whose running sum reaches top_p[h] (the entry that
+ *      reaches it included); keep the whole row if it never does;
+ *   2. BSA_TEXT_KEEP: also keep key blocks j < ceil(text_len / k_block);
+ *   3. BSA_FRAME0_DENSE: keep every key block when
+ *      text_len / q_block <= i <= (text_len + tokens_per_frame - 1) / q_block;
+ *   4. write the kept key blocks in ascending order to kv_index[b,h,i,0..n-1]
+ *      and n to kv_count[b,h,i]; entries from n on are left unspecified.
+ * Per head: entropy[b,h] = (1/C_q) sum_i -sum_j P'_ij ln(P'_ij + eps) and
+ * entropy_norm[b,h] = entropy[b,h] / ln C_k.
+ *
+ * probs         fp32 [B,H,C_q,C_k] (read only)
+ * top_p         HOST fp32 [H], per-head p (read during the call only)
+ * flags         BSA_TEXT_KEEP | BSA_FRAME0_DENSE
+ * eps           entropy stabiliser (e.g. 1e-8)
+ * mask          u8 [B,H,C_q,C_k] 0/1 block mask, or NULL to skip it
+ * kv_index      int32 [B,H,C_q,C_k], 4-byte aligned (written)
+ * kv_count      int32 [B,H,C_q] (written)
+ * entropy       fp32 [B,H], or NULL to skip the entropy
+ * entropy_norm  fp32 [B,H], or NULL
+ * workspace     device scratch of bsa_build_mask_workspace_bytes(layout) bytes,
+ *               16-byte aligned; required when entropy or entropy_norm is set;
+ *               its contents on entry do not matter and are clobbered
+ * Supports C_k up to 2048.
+ */
+int bsa_build_mask(const bsa_layout *layout, const float *probs, const float *top_p,
+                   uint32_t flags, float eps, uint8_t *mask, int32_t *kv_index,
+                   int32_t *kv_count, float *entropy, float *entropy_norm,
+                   void *workspace, void *stream);
+
+/*
+ * Block-sparse exact attention ("Attention matrix view ..." s2;
+ * "AB-Attention ..." TL;DR).  For every valid query token t of query block i:
+ *   U = tokens u < seq_len of the key blocks kv_index[b,h,i,0..kv_count-1]
+ *   O_t = sum_{u in U} softmax_u(softmax_scale * Q_t . K_u) V_u
+ *   lse_t = ln sum_{u in U} exp(softmax_scale * Q_t . K_u)
+ * computed with bf16 tensor-core products and fp32 softmax/accumulation.
+ * Padded query rows (t >= seq_len) get O = 0 and lse = -inf; a row with no
+ * valid key gets the same.  With k_block = 64, consecutive list entries are
+ * paired into one 128-key tensor-core tile.
+ *
+ * q, k, v       bf16 [B,H,seq_pad,D], 16-byte aligned (read only)
+ * kv_index      int32 [B,H,C_q,C_k], ascending within a row (read only)
+ * kv_count      int32 [B,H,C_q] (read only)
+ * softmax_scale usually 1/sqrt(D)
+ * out           bf16 [B,H,seq_pad,D], 16-byte aligned (written)
+ * lse           fp32 [B,H,seq_pad], or NULL
+ * err_flag      device int32, or NULL (see BSA_DEVERR_*)
+ */
+int bsa_attention_fwd(const bsa_layout *layout, const void *q, const void *k, const void *v,
+                      const int32_t *kv_index, const int32_t *kv_count, float softmax_scale,
+                      void *out, float *lse, int32_t *err_flag, void *stream);
+
+/*
+ * Dense exact attention: bsa_attention_fwd with every key block selected for
+ * every query block ("Attention matrix view ..." s2, the dense rows).
+ * Arguments as for bsa_attention_fwd.
+ */
+int bsa_dense_fwd(const bsa_layout *layout, const void *q, const void *k, const void *v,
+                  float softmax_scale, void *out, float *lse, int32_t *err_flag, void *stream);
+
+/* Human-readable name of a bsa_status value (static storage). */
+const char *bsa_status_string(int status);
+
+/* ABI version: major * 100 + minor. */
+int bsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H */

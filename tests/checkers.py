@@ -1,0 +1,100 @@
+"""Comparison rules between the CUDA path and the oracle.
+
+Masks: a row whose oracle top-p decision has a margin above MARGIN must match
+bit for bit; a row closer to the cut than that may differ by rounding, and
+must then still be a valid top-p set (size within one of k*, mass >= p - MARGIN,
+and without its smallest member, mass < p + MARGIN).  The margin of row i is
+    min(p - c_{k*-1} (inf if k* = 1),  c_{k*} - p,  P'_(k*) - P'_(k*+1) (inf if k* = C_k))
+with c_k the fp64 running sum of the row sorted by (P' desc, j asc).
+
+Attention: given identical masks, the bf16 output must be within MAX_ABS of
+the fp64-computed fp32 oracle at every element and MEAN_ABS on average; the
+log-sum-exp within LSE_ABS.  Entropy within ENTROPY_REL relative.
+"""
+import numpy as np
+
+MARGIN = 1e-4
+MAX_ABS = 2e-2
+MEAN_ABS = 2e-3
+LSE_ABS = 1e-3
+ENTROPY_REL = 1e-3
+
+
+def row_margins(probs, top_p, heads_axis=1):
+    """k* and the margin of every row of probs [B,H,Cq,Ck] (oracle fp32 values)."""
+    B, H, Cq, Ck = probs.shape
+    tp = np.broadcast_to(np.asarray(top_p, np.float64), (H,))
+    kstar = np.empty((B, H, Cq), np.int64)
+    margin = np.empty((B, H, Cq), np.float64)
+    order_all = np.argsort(-probs.astype(np.float64), axis=-1, kind="stable")
+    for b in range(B):
+        for h in range(H):
+            p = np.float64(np.float32(tp[h]))
+            srt = np.take_along_axis(probs[b, h].astype(np.float64), order_all[b, h], axis=-1)
+            c = np.cumsum(srt, axis=-1)
+            reach = c >= p
+            k = np.where(reach.any(-1), reach.argmax(-1) + 1, Ck)
+            kstar[b, h] = k
+            idx = np.arange(Cq)
+            ck = c[idx, k - 1]
+            ckm1 = np.where(k > 1, c[idx, np.maximum(k - 2, 0)], -np.inf)
+            gap = np.where(k < Ck, srt[idx, k - 1] - srt[idx, np.minimum(k, Ck - 1)], np.inf)
+            m1 = np.where(k > 1, p - ckm1, np.inf)
+            m2 = np.where(reach.any(-1), ck - p, np.inf)
+            margin[b, h] = np.minimum(np.minimum(m1, m2), gap)
+    return kstar, margin
+
+
+def check_topp_masks(gpu_mask, ora_mask, probs, top_p, kstar=None, margin=None):
+    """Compare top-p masks (no overrides).  Returns the exempt fraction."""
+    if kstar is None:
+        kstar, margin = row_margins(probs, top_p)
+    gpu_mask = gpu_mask.astype(bool)
+    ora_mask = ora_mask.astype(bool)
+    strict = margin > MARGIN
+    diff = (gpu_mask != ora_mask).any(-1)
+    bad = np.argwhere(diff & strict)
+    assert bad.size == 0, "rows with margin > %g differ: %s (of %d)" % (MARGIN, bad[:5].tolist(), len(bad))
+    H = probs.shape[1]
+    tp = np.broadcast_to(np.asarray(top_p, np.float64), (H,))
+    for b, h, i in np.argwhere(diff & ~strict):
+        p = np.float64(np.float32(tp[h]))
+        row = probs[b, h, i].astype(np.float64)
+        sel = np.nonzero(gpu_mask[b, h, i])[0]
+        k = kstar[b, h, i]
+        assert abs(len(sel) - k) <= 1, (b, h, i, len(sel), k)
+        mass = row[sel].sum()
+        assert mass >= p - MARGIN, (b, h, i, mass, p)
+        assert mass - row[sel].min() < p + MARGIN, (b, h, i, mass, p)
+    return float((~strict).mean())
+
+
+def check_lists(kv_index, kv_count, mask):
+    """kv_index/kv_count must be the ascending compaction of mask."""
+    kv_index = np.asarray(kv_index)
+    kv_count = np.asarray(kv_count)
+    mask = np.asarray(mask).astype(bool)
+    assert np.array_equal(kv_count, mask.sum(-1))
+    Ck = mask.shape[-1]
+    pos = np.arange(Ck)
+    valid = pos < kv_count[..., None]
+    ref = np.sort(np.where(mask, pos, Ck), axis=-1)
+    assert np.array_equal(np.where(valid, kv_index, -1), np.where(valid, ref, -1))
+
+
+def check_attention(out_gpu, out_ora, lse_gpu=None, lse_ora=None, what=""):
+    out_gpu = np.asarray(out_gpu, np.float64)
+    out_ora = np.asarray(out_ora, np.float64)
+    assert np.isfinite(out_gpu).all(), what + ": non-finite output"
+    err = np.abs(out_gpu - out_ora)
+    assert err.max() <= MAX_ABS, "%s: max abs err %.3g > %g" % (what, err.max(), MAX_ABS)
+    assert err.mean() <= MEAN_ABS, "%s: mean abs err %.3g > %g" % (what, err.mean(), MEAN_ABS)
+    if lse_gpu is not None:
+        lg = np.asarray(lse_gpu, np.float64)
+        lo = np.asarray(lse_ora, np.float64)
+        fin = np.isfinite(lo)
+        assert np.array_equal(fin, np.isfinite(lg)), what + ": lse finiteness differs"
+        if fin.any():
+            e = np.abs(lg[fin] - lo[fin]).max()
+            assert e <= LSE_ABS, "%s: lse err %.3g" % (what, e)
+    return float(err.max()), float(err.mean())

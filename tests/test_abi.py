@@ -1,0 +1,88 @@
+"""The C ABI on a host without a GPU: the library loads, exports every symbol
+include/bsa.h declares, and rejects bad arguments before launching anything."""
+import ctypes
+
+import pytest
+
+from block_sparse_attention_45_b200 import binding as bsa
+from block_sparse_attention_45_b200 import synth
+
+
+def test_library_exports_every_declared_symbol():
+    lib = bsa.load()
+    names = bsa.declared_symbols()
+    assert {"bsa_block_scores", "bsa_build_mask", "bsa_attention_fwd", "bsa_dense_fwd"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert lib.bsa_version() >= 100
+    for s in range(5):
+        assert bsa.status_string(s).startswith("BSA_")
+
+
+def _layout(**kw):
+    d = synth.WORKLOADS["tiny"].layout()
+    d.update(kw)
+    return bsa.make_layout(d)
+
+
+FAKE = ctypes.c_void_p(0x10000)      # never dereferenced: validation fails first
+MISALIGNED = ctypes.c_void_p(0x10002)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(head_dim=96), bsa.BSA_ERR_UNSUPPORTED),
+    (dict(q_block=32), bsa.BSA_ERR_UNSUPPORTED),
+    (dict(heads=0), bsa.BSA_ERR_INVALID_ARG),
+    (dict(heads=257), bsa.BSA_ERR_UNSUPPORTED),
+    (dict(seq_pad=300), bsa.BSA_ERR_INVALID_ARG),          # not a multiple of the block
+    (dict(seq_len=200), bsa.BSA_ERR_INVALID_ARG),          # a whole empty block at the end
+    (dict(seq_len=400), bsa.BSA_ERR_INVALID_ARG),          # seq_pad < seq_len
+    (dict(text_len=300), bsa.BSA_ERR_INVALID_ARG),         # text + frames beyond seq_len
+    (dict(num_frames=-1), bsa.BSA_ERR_INVALID_ARG),
+])
+def test_bad_layouts_are_rejected(kw, expect):
+    L = _layout(**kw)
+    lib = bsa.load()
+    assert lib.bsa_dense_fwd(ctypes.byref(L), FAKE, FAKE, FAKE, 0.125, FAKE, None, None, None) == expect
+    assert lib.bsa_block_scores(ctypes.byref(L), FAKE, FAKE, FAKE, FAKE, FAKE, None) == expect
+    assert lib.bsa_build_mask_workspace_bytes(ctypes.byref(L)) == 0
+
+
+def test_bad_pointers_are_rejected():
+    L = _layout()
+    lib = bsa.load()
+    r = ctypes.byref(L)
+    assert lib.bsa_dense_fwd(r, MISALIGNED, FAKE, FAKE, 0.125, FAKE, None, None, None) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_dense_fwd(r, None, FAKE, FAKE, 0.125, FAKE, None, None, None) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_dense_fwd(r, FAKE, FAKE, FAKE, -1.0, FAKE, None, None, None) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_attention_fwd(r, FAKE, FAKE, FAKE, None, FAKE, 0.125, FAKE, None, None,
+                                 None) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_block_scores(r, FAKE, FAKE, FAKE, FAKE, MISALIGNED, None) == bsa.BSA_ERR_INVALID_ARG
+    tp = (ctypes.c_float * 2)(0.5, 0.5)
+    tpv = ctypes.cast(tp, ctypes.c_void_p)
+    # entropy requested without a workspace; unknown flag bit; no top_p
+    assert lib.bsa_build_mask(r, FAKE, tpv, 3, 1e-8, None, FAKE, FAKE, FAKE, None, None,
+                              None) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_build_mask(r, FAKE, tpv, 8, 1e-8, None, FAKE, FAKE, None, None, None,
+                              None) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_build_mask(r, FAKE, None, 3, 1e-8, None, FAKE, FAKE, None, None, None,
+                              None) == bsa.BSA_ERR_INVALID_ARG
+    nan_tp = (ctypes.c_float * 2)(float("nan"), 0.5)
+    assert lib.bsa_build_mask(r, FAKE, ctypes.cast(nan_tp, ctypes.c_void_p), 3, 1e-8, None, FAKE,
+                              FAKE, None, None, None, None) == bsa.BSA_ERR_INVALID_ARG
+
+
+def test_workspace_size():
+    L = _layout()
+    # one fp32 per (b, h, query block), rounded up to 256 bytes
+    assert bsa.load().bsa_build_mask_workspace_bytes(ctypes.byref(L)) == 256
+    w = synth.WORKLOADS["hunyuan"]
+    L = bsa.make_layout(w)
+    assert bsa.load().bsa_build_mask_workspace_bytes(ctypes.byref(L)) == -(-24 * 931 * 4 // 256) * 256
+
+
+def test_calls_fail_loudly_without_the_library(monkeypatch):
+    monkeypatch.setattr(bsa, "_LIB", None)
+    monkeypatch.setattr(bsa, "LIB_PATH", "/nonexistent/libbsa.so")
+    with pytest.raises(RuntimeError, match="not built"):
+        bsa.load()

@@ -1,0 +1,175 @@
+"""Edge cases of the CUDA path against the oracle (needs a B200).
+
+Ragged sequence ends, every (head_dim, q_block, k_block) combination, text and
+frame 0 that start or end inside a block, hand-built lists (one block, every
+block, none, odd counts in gather mode, invalid entries and counts) and
+garbage in the padded rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_45_b200 import binding as bsa
+from block_sparse_attention_45_b200 import synth
+from tests import checkers
+from tests.gpu_util import to_dev, to_host_f32
+
+pytestmark = pytest.mark.gpu
+
+EDGE = {
+    # D, bq, bk, text_len, frames, latent (h, w), pad_to  -> seq_len, seq_pad
+    "d128_q64_k128": synth.custom("d128_q64_k128", heads=3, head_dim=128, q_block=64, k_block=128,
+                                  text_len=40, num_frames=3, latent_h=10, latent_w=10, top_p=0.8,
+                                  seed=11),                                  # 340 -> 384
+    "d128_q128_k64": synth.custom("d128_q128_k64", heads=2, head_dim=128, q_block=128, k_block=64,
+                                  text_len=90, num_frames=4, latent_h=10, latent_w=16, top_p=0.75,
+                                  seed=12),                                  # 730 -> 768
+    "d64_q128_k128": synth.custom("d64_q128_k128", heads=2, head_dim=64, q_block=128, k_block=128,
+                                  text_len=20, num_frames=3, latent_h=10, latent_w=16, top_p=0.85,
+                                  seed=13),                                  # 500 -> 512
+    "d64_q64_k64": synth.custom("d64_q64_k64", heads=2, head_dim=64, q_block=64, k_block=64,
+                                text_len=10, num_frames=2, latent_h=6, latent_w=10, top_p=0.6,
+                                pad_to=64, seed=14),                         # 130 -> 192
+    "d64_q128_k64": synth.custom("d64_q128_k64", batch=2, heads=2, head_dim=64, q_block=128,
+                                 k_block=64, text_len=0, num_frames=5, latent_h=9, latent_w=22,
+                                 top_p=0.7, seed=15, kind="clustered"),      # 990 -> 1024
+}
+
+
+def _data(w):
+    x = synth.generate(w)
+    return x, {k: to_dev(v) for k, v in x.items()}
+
+
+def _attn_vs_oracle(w, x, xd, mask, idx, cnt, what):
+    L = w.layout()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = bsa.attention_fwd(w, xd["q"], xd["k"], xd["v"], torch.from_numpy(idx).cuda(),
+                                 torch.from_numpy(cnt).cuda(), err_flag=err)
+    torch.cuda.synchronize()
+    o_ora, l_ora = oracle.attention(L, x["q"], x["k"], x["v"], mask)
+    cq = w.seq_pad // w.q_block
+    og = to_host_f32(out).reshape(o_ora.shape)
+    lg = lse.cpu().numpy().reshape(l_ora.shape)
+    checkers.check_attention(og, o_ora, lg, l_ora, what=what)
+    return out, lse, int(err.item())
+
+
+@pytest.mark.parametrize("name", sorted(EDGE))
+def test_pipeline_edge_shapes(name):
+    w = EDGE[name]
+    x, xd = _data(w)
+    L = w.layout()
+    tp = [w.top_p] * w.heads
+    sel = oracle.select(L, x["q"], x["k"], tp, w.flags)
+    qc, kc, probs = bsa.block_scores(w, xd["q"], xd["k"])
+    np.testing.assert_allclose(to_host_f32(qc), sel["q_centroids"], rtol=1e-5, atol=2e-6)
+    np.testing.assert_allclose(to_host_f32(kc), sel["k_centroids"], rtol=1e-5, atol=2e-6)
+    assert np.abs(to_host_f32(probs) - sel["probs"]).max() <= 1e-4
+    g0 = bsa.build_mask(w, torch.from_numpy(sel["probs"]).cuda(), tp, 0)
+    checkers.check_topp_masks(g0["mask"].cpu().numpy(), sel["topp_mask"], sel["probs"], tp)
+    g = bsa.build_mask(w, torch.from_numpy(sel["probs"]).cuda(), tp, w.flags)
+    m = g["mask"].cpu().numpy()
+    assert np.array_equal(m, oracle.overrides(L, w.flags, g0["mask"].cpu().numpy()))
+    checkers.check_lists(g["kv_index"].cpu().numpy(), g["kv_count"].cpu().numpy(), m)
+    np.testing.assert_allclose(g["entropy"].cpu().numpy(), sel["entropy"], rtol=checkers.ENTROPY_REL)
+    _attn_vs_oracle(w, x, xd, sel["mask"], sel["kv_index"], sel["kv_count"], name)
+    out, lse = bsa.dense_fwd(w, xd["q"], xd["k"], xd["v"])
+    o_ora, l_ora = oracle.attention(L, x["q"], x["k"], x["v"], None)
+    checkers.check_attention(to_host_f32(out).reshape(o_ora.shape), o_ora,
+                             lse.cpu().numpy().reshape(l_ora.shape), l_ora, what=name + " dense")
+
+
+def _lists_from_mask(mask):
+    Ck = mask.shape[-1]
+    pos = np.arange(Ck)
+    idx = np.sort(np.where(mask.astype(bool), pos, Ck), axis=-1).astype(np.int32)
+    cnt = mask.astype(bool).sum(-1).astype(np.int32)
+    idx[idx == Ck] = -1
+    return idx, cnt
+
+
+@pytest.mark.parametrize("name", ["d128_q128_k64", "d64_q64_k64", "d128_q64_k128"])
+def test_hand_built_lists(name):
+    w = EDGE[name]
+    x, xd = _data(w)
+    cq, ck = w.seq_pad // w.q_block, w.seq_pad // w.k_block
+    rng = np.random.default_rng(7)
+    shape = (w.batch, w.heads, cq, ck)
+    # one block per row, including the ragged last key block
+    m = np.zeros(shape, np.uint8)
+    m[..., :] = 0
+    js = rng.integers(ck, size=shape[:-1])
+    js.reshape(-1)[0] = ck - 1
+    np.put_along_axis(m, js[..., None], 1, axis=-1)
+    _attn_vs_oracle(w, x, xd, m, *_lists_from_mask(m), what=name + " one block")
+    # every block (equals dense)
+    m = np.ones(shape, np.uint8)
+    out, _, _ = _attn_vs_oracle(w, x, xd, m, *_lists_from_mask(m), what=name + " all blocks")
+    dn, _ = bsa.dense_fwd(w, xd["q"], xd["k"], xd["v"])
+    assert torch.equal(out, dn)
+    # random counts: odd and even, 1..C_k
+    m = (rng.random(shape) < 0.4).astype(np.uint8)
+    m[..., 0, :] = 0
+    m[..., 0, ck // 2] = 1
+    _attn_vs_oracle(w, x, xd, m, *_lists_from_mask(m), what=name + " random")
+
+
+def test_empty_rows_and_bad_entries():
+    w = EDGE["d128_q128_k64"]
+    x, xd = _data(w)
+    cq, ck = w.seq_pad // w.q_block, w.seq_pad // w.k_block
+    shape = (w.batch, w.heads, cq, ck)
+    m = np.zeros(shape, np.uint8)
+    m[..., 1:, :3] = 1          # query block 0 of every head selects nothing
+    idx, cnt = _lists_from_mask(m)
+    out, lse, e = _attn_vs_oracle(w, x, xd, m, idx, cnt, what="empty rows")
+    assert e == 0
+    assert (out[:, :, :w.q_block] == 0).all()
+    assert torch.isneginf(lse[:, :, :w.q_block]).all()
+    # invalid entries are skipped and flagged; counts beyond C_k are clamped and flagged
+    idx2 = idx.copy()
+    cnt2 = cnt.copy()
+    idx2[0, 0, 1, 3] = ck + 5      # list of (0,0,1) = [0,1,2, bad]
+    cnt2[0, 0, 1] = 4
+    idx2[0, 1, 2, :4] = [0, -3, 1, 2]
+    cnt2[0, 1, 2] = 4
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out2, _ = bsa.attention_fwd(w, xd["q"], xd["k"], xd["v"], torch.from_numpy(idx2).cuda(),
+                                torch.from_numpy(cnt2).cuda(), err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & bsa.DEVERR_BAD_INDEX
+    assert torch.equal(out2[0, 0, w.q_block:2 * w.q_block], out[0, 0, w.q_block:2 * w.q_block])
+    # a bad entry inside a gathered pair changes the pairing, so compare within tolerance
+    a = out2[0, 1, 2 * w.q_block:3 * w.q_block].float()
+    b = out[0, 1, 2 * w.q_block:3 * w.q_block].float()
+    assert (a - b).abs().max().item() <= checkers.MAX_ABS
+    cnt3 = np.full_like(cnt, ck + 7)
+    err.zero_()
+    out3, _ = bsa.attention_fwd(w, xd["q"], xd["k"], xd["v"],
+                                torch.from_numpy(np.broadcast_to(np.arange(ck, dtype=np.int32),
+                                                                 shape).copy()).cuda(),
+                                torch.from_numpy(cnt3).cuda(), err_flag=err)
+    dn, _ = bsa.dense_fwd(w, xd["q"], xd["k"], xd["v"])
+    torch.cuda.synchronize()
+    assert int(err.item()) & bsa.DEVERR_BAD_COUNT
+    assert torch.equal(out3, dn)
+
+
+def test_padding_rows_are_ignored_and_zeroed():
+    w = EDGE["d64_q128_k128"]
+    x, xd = _data(w)
+    S = w.seq_len
+    ref, ref_lse = bsa.dense_fwd(w, xd["q"], xd["k"], xd["v"])
+    dirty = {k: v.clone() for k, v in xd.items()}
+    for t in dirty.values():
+        t[:, :, S:] = float("nan")
+    out = torch.full_like(ref, float("nan"))
+    lse = torch.full_like(ref_lse, 123.0)
+    bsa.dense_fwd(w, dirty["q"], dirty["k"], dirty["v"], out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    assert (out[:, :, S:] == 0).all()
+    assert torch.isneginf(lse[:, :, S:]).all()
+    assert torch.equal(lse[:, :, :S], ref_lse[:, :, :S])

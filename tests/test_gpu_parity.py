@@ -1,0 +1,159 @@
+"""CUDA path vs the CPU oracle on the five workload shapes (needs a B200).
+
+Every call goes through the C ABI (libbsa.so) via the ctypes binding.
+  * scores: centroids and P' element by element;
+  * mask: on the oracle's own P' (bit-exact outside the top-p margin rule),
+    then end to end on the GPU's P';
+  * attention: the oracle's lists fed to both sides; every output at the small
+    shapes, sampled query blocks (frame-0, text, ragged last, random) at full
+    size, in the launch configuration the bench times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_45_b200 import binding as bsa
+from block_sparse_attention_45_b200 import synth
+from tests import checkers
+from tests.gpu_util import (inputs, oracle_selection, sample_rows, to_dev, to_host_f32, top_p_of)
+
+pytestmark = pytest.mark.gpu
+
+ALL = ["tiny", "small", "wan1.3b", "wan14b", "hunyuan"]
+SMALL = ["tiny", "small"]
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_block_scores(name):
+    w, x = inputs(name)
+    sel = oracle_selection(name)
+    qc, kc, probs = bsa.block_scores(w, to_dev(x["q"]), to_dev(x["k"]))
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(to_host_f32(qc), sel["q_centroids"], rtol=1e-5, atol=2e-6)
+    np.testing.assert_allclose(to_host_f32(kc), sel["k_centroids"], rtol=1e-5, atol=2e-6)
+    P = to_host_f32(probs)
+    err = np.abs(P - sel["probs"]).max()
+    assert err <= 1e-4, "P' max abs err %.3g" % err
+    np.testing.assert_allclose(P.astype(np.float64).sum(-1), 1.0, atol=1e-5)
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_mask_on_oracle_probs(name):
+    """Same fp32 P' on both sides: top-p sets, overrides, lists and entropy."""
+    w, _ = inputs(name)
+    sel = oracle_selection(name)
+    L = w.layout()
+    tp = top_p_of(w)
+    probs = torch.from_numpy(sel["probs"]).cuda()
+    g0 = bsa.build_mask(w, probs, tp, 0)
+    torch.cuda.synchronize()
+    exempt = checkers.check_topp_masks(g0["mask"].cpu().numpy(), sel["topp_mask"], sel["probs"], tp)
+    assert exempt < 0.01
+    checkers.check_lists(g0["kv_index"].cpu().numpy(), g0["kv_count"].cpu().numpy(),
+                         g0["mask"].cpu().numpy())
+    g = bsa.build_mask(w, probs, tp, w.flags)
+    torch.cuda.synchronize()
+    m = g["mask"].cpu().numpy()
+    expect = oracle.overrides(L, w.flags, g0["mask"].cpu().numpy())
+    assert np.array_equal(m, expect)
+    checkers.check_lists(g["kv_index"].cpu().numpy(), g["kv_count"].cpu().numpy(), m)
+    H = g["entropy"].cpu().numpy()
+    Hn = g["entropy_norm"].cpu().numpy()
+    np.testing.assert_allclose(H, sel["entropy"], rtol=checkers.ENTROPY_REL)
+    np.testing.assert_allclose(Hn, sel["entropy_norm"], rtol=checkers.ENTROPY_REL)
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_selection_end_to_end(name):
+    """GPU P' -> GPU mask against the oracle's mask (margin rule on the oracle's P')."""
+    w, x = inputs(name)
+    sel = oracle_selection(name)
+    tp = top_p_of(w)
+    _, _, probs = bsa.block_scores(w, to_dev(x["q"]), to_dev(x["k"]))
+    g0 = bsa.build_mask(w, probs, tp, 0)
+    g = bsa.build_mask(w, probs, tp, w.flags)
+    torch.cuda.synchronize()
+    exempt = checkers.check_topp_masks(g0["mask"].cpu().numpy(), sel["topp_mask"], sel["probs"], tp)
+    assert exempt < 0.01
+    m = g["mask"].cpu().numpy()
+    assert np.array_equal(m, oracle.overrides(w.layout(), w.flags, g0["mask"].cpu().numpy()))
+    np.testing.assert_allclose(g["entropy"].cpu().numpy(), sel["entropy"], rtol=checkers.ENTROPY_REL)
+    density = g["kv_count"].cpu().numpy().mean() / m.shape[-1]
+    assert abs(density - m.mean()) < 1e-12
+
+
+def _attention_rows(name, rows):
+    w, x = inputs(name)
+    sel = oracle_selection(name)
+    L = w.layout()
+    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
+    kv_index = torch.from_numpy(sel["kv_index"]).cuda()
+    kv_count = torch.from_numpy(sel["kv_count"]).cuda()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = bsa.attention_fwd(w, q, k, v, kv_index, kv_count, err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    o_ora, l_ora = oracle.attention(L, x["q"], x["k"], x["v"], sel["mask"], rows=rows)
+    cq = w.seq_pad // w.q_block
+    og = to_host_f32(out).reshape(w.batch * w.heads, cq, w.q_block, w.head_dim)
+    lg = lse.cpu().numpy().reshape(w.batch * w.heads, cq, w.q_block)
+    og = og[rows // cq, rows % cq]
+    lg = lg[rows // cq, rows % cq]
+    return checkers.check_attention(og, o_ora, lg, l_ora, what=name)
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_sparse_attention_all_rows(name):
+    w, _ = inputs(name)
+    cq = w.seq_pad // w.q_block
+    rows = np.arange(w.batch * w.heads * cq, dtype=np.int64)
+    if name == "small":
+        rows = rows[::3]   # every third query block keeps the oracle to seconds
+    _attention_rows(name, rows)
+
+
+@pytest.mark.parametrize("name", ["wan1.3b", "wan14b", "hunyuan"])
+def test_sparse_attention_sampled(name):
+    w, _ = inputs(name)
+    _attention_rows(name, sample_rows(w))
+
+
+@pytest.mark.parametrize("name", ["tiny", "small", "wan1.3b"])
+def test_dense_attention(name):
+    w, x = inputs(name)
+    L = w.layout()
+    out, lse = bsa.dense_fwd(w, to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"]))
+    torch.cuda.synchronize()
+    rows = sample_rows(w, n_random=2)
+    o_ora, l_ora = oracle.attention(L, x["q"], x["k"], x["v"], None, rows=rows)
+    cq = w.seq_pad // w.q_block
+    og = to_host_f32(out).reshape(w.batch * w.heads, cq, w.q_block, w.head_dim)[rows // cq, rows % cq]
+    lg = lse.cpu().numpy().reshape(w.batch * w.heads, cq, w.q_block)[rows // cq, rows % cq]
+    checkers.check_attention(og, o_ora, lg, l_ora, what=name + " dense")
+
+
+def test_dense_matches_torch_sdpa():
+    """An independent library check of the dense path at the small shape."""
+    w, x = inputs("small")
+    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
+    out, _ = bsa.dense_fwd(w, q, k, v)
+    S = w.seq_len
+    ref = torch.nn.functional.scaled_dot_product_attention(q[:, :, :S].float(), k[:, :, :S].float(),
+                                                           v[:, :, :S].float())
+    err = (out[:, :, :S].float() - ref).abs()
+    assert err.max().item() <= checkers.MAX_ABS and err.mean().item() <= checkers.MEAN_ABS
+    assert (out[:, :, S:] == 0).all()
+
+
+@pytest.mark.parametrize("name", ["small", "hunyuan"])
+def test_frame0_rows_equal_dense(name):
+    """Frame-0 query rows are dense ("Attention matrix view ..." s2): identical to bsa_dense_fwd."""
+    w, x = inputs(name)
+    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
+    res = bsa.sparse_attention(w, q, k, v, top_p_of(w), w.flags)
+    dn, _ = bsa.dense_fwd(w, q, k, v)
+    torch.cuda.synchronize()
+    f0, f1 = oracle.frame0_qblocks(w.layout())
+    a, b = f0 * w.q_block, (f1 + 1) * w.q_block
+    assert torch.equal(res["out"][:, :, a:b], dn[:, :, a:b])
