@@ -67,6 +67,22 @@ def flops_per_pair(w):
     return 4.0 * w.q_block * w.k_block * w.head_dim
 
 
+def max_over_ranks(value, device=None):
+    """The job's time is the slowest rank's (torch.distributed MAX all-reduce)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_rank_step, world, ms_per_step):
+    """Whole-job throughput: every rank runs its own problem (weak scaling)."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- CPU oracle legs
 
 def oracle_sample(w, x, top_p, budget_s=20.0):
@@ -271,12 +287,9 @@ def our_arm(args, w):
     ms_attn = [m[2].elapsed_time(m[3]) for m in marks]
     ms_scores = [m[0].elapsed_time(m[1]) for m in marks]
     ms_mask = [m[1].elapsed_time(m[2]) for m in marks]
-    if world > 1:
-        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, dev)
     ms_step = ms_total / args.steps
-    value = world * step_flops / (ms_step * 1e-3) / 1e12
+    value = job_tflops(step_flops, world, ms_step)
 
     # end to end through the C ABI: pinned host inputs -> device, path, output -> host
     e2e = None
@@ -304,15 +317,10 @@ def our_arm(args, w):
         b.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        ms_e2e = a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        ms_e2e /= args.steps
+        ms_e2e = max_over_ranks(a.elapsed_time(b), dev) / args.steps
         h2d = sum(pin[n].numel() * pin[n].element_size() for n in pin)
         d2h = out_h.numel() * out_h.element_size() + ent_h.numel() * ent_h.element_size()
-        e2e = dict(value=world * step_flops / (ms_e2e * 1e-3) / 1e12, unit=UNIT,
+        e2e = dict(value=job_tflops(step_flops, world, ms_e2e), unit=UNIT,
                    ms_per_step=ms_e2e, h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h))
 
     # the dense path (all key blocks) for context: not part of the step

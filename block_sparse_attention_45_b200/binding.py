@@ -61,9 +61,11 @@ def load():
         L.bsa_build_mask.argtypes = [lp, vp, vp, ctypes.c_uint32, ctypes.c_float, vp, vp, vp, vp,
                                      vp, vp, vp]
         L.bsa_build_mask.restype = ctypes.c_int
-        L.bsa_attention_fwd.argtypes = [lp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp]
+        L.bsa_attention_fwd.argtypes = [lp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp, vp]
         L.bsa_attention_fwd.restype = ctypes.c_int
-        L.bsa_dense_fwd.argtypes = [lp, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp]
+        L.bsa_attention_workspace_bytes.argtypes = [lp]
+        L.bsa_attention_workspace_bytes.restype = ctypes.c_size_t
+        L.bsa_dense_fwd.argtypes = [lp, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp, vp]
         L.bsa_dense_fwd.restype = ctypes.c_int
         L.bsa_status_string.argtypes = [ctypes.c_int]
         L.bsa_status_string.restype = ctypes.c_char_p
@@ -185,8 +187,19 @@ def build_mask(layout, probs, top_p, flags, eps=1e-8, mask=None, kv_index=None, 
                 entropy_norm=entropy_norm)
 
 
+def attention_workspace_bytes(layout):
+    L = make_layout(layout)
+    return int(load().bsa_attention_workspace_bytes(ctypes.byref(L)))
+
+
+def _attn_workspace(L, device, workspace):
+    if workspace is None:
+        workspace = torch.empty(attention_workspace_bytes(L), dtype=torch.uint8, device=device)
+    return workspace
+
+
 def attention_fwd(layout, q, k, v, kv_index, kv_count, softmax_scale=None, out=None, lse=None,
-                  err_flag=None, with_lse=True, stream=None):
+                  err_flag=None, with_lse=True, workspace=None, stream=None):
     """bsa_attention_fwd: returns (out, lse)."""
     L = make_layout(layout)
     d = dims(L)
@@ -201,15 +214,16 @@ def attention_fwd(layout, q, k, v, kv_index, kv_count, softmax_scale=None, out=N
         out = torch.empty(qkv, dtype=torch.bfloat16, device=q.device)
     if lse is None and with_lse:
         lse = torch.empty((d["B"], d["H"], d["Sp"]), dtype=torch.float32, device=q.device)
+    workspace = _attn_workspace(L, q.device, workspace)
     rc = load().bsa_attention_fwd(ctypes.byref(L), _ptr(q), _ptr(k), _ptr(v), _ptr(kv_index),
                                   _ptr(kv_count), float(softmax_scale), _ptr(out), _ptr(lse),
-                                  _ptr(err_flag), _stream(stream))
+                                  _ptr(err_flag), _ptr(workspace), _stream(stream))
     _check("bsa_attention_fwd", rc)
     return out, lse
 
 
 def dense_fwd(layout, q, k, v, softmax_scale=None, out=None, lse=None, err_flag=None,
-              with_lse=True, stream=None):
+              with_lse=True, workspace=None, stream=None):
     """bsa_dense_fwd: returns (out, lse)."""
     L = make_layout(layout)
     d = dims(L)
@@ -222,8 +236,10 @@ def dense_fwd(layout, q, k, v, softmax_scale=None, out=None, lse=None, err_flag=
         out = torch.empty(qkv, dtype=torch.bfloat16, device=q.device)
     if lse is None and with_lse:
         lse = torch.empty((d["B"], d["H"], d["Sp"]), dtype=torch.float32, device=q.device)
+    workspace = _attn_workspace(L, q.device, workspace)
     rc = load().bsa_dense_fwd(ctypes.byref(L), _ptr(q), _ptr(k), _ptr(v), float(softmax_scale),
-                              _ptr(out), _ptr(lse), _ptr(err_flag), _stream(stream))
+                              _ptr(out), _ptr(lse), _ptr(err_flag), _ptr(workspace),
+                              _stream(stream))
     _check("bsa_dense_fwd", rc)
     return out, lse
 

@@ -134,9 +134,14 @@ int bsa_build_mask(const bsa_layout *layout, const float *probs, const float *to
     return launch_status(bsa::launch_entropy_reduce(g, row_ent, entropy, entropy_norm, st));
 }
 
+size_t bsa_attention_workspace_bytes(const bsa_layout *layout) {
+    if (check_layout(layout) != BSA_OK) return 0;
+    return bsa::kAttnWorkspaceBytes;
+}
+
 int bsa_attention_fwd(const bsa_layout *layout, const void *q, const void *k, const void *v,
                       const int32_t *kv_index, const int32_t *kv_count, float softmax_scale,
-                      void *out, float *lse, int32_t *err_flag, void *stream) {
+                      void *out, float *lse, int32_t *err_flag, void *workspace, void *stream) {
     int rc = check_layout(layout);
     if (rc != BSA_OK) return rc;
     if (!q || !k || !v || !out || !kv_index || !kv_count) return BSA_ERR_INVALID_ARG;
@@ -146,13 +151,15 @@ int bsa_attention_fwd(const bsa_layout *layout, const void *q, const void *k, co
         (err_flag && !aligned(err_flag, 4)))
         return BSA_ERR_INVALID_ARG;
     if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return BSA_ERR_INVALID_ARG;
+    if (workspace && !aligned(workspace, 16)) return BSA_ERR_INVALID_ARG;
     const Geometry g = bsa::make_geometry(*layout);
     return bsa::launch_attention(g, q, k, v, kv_index, kv_count, softmax_scale, out, lse, err_flag,
-                                 static_cast<cudaStream_t>(stream));
+                                 workspace, static_cast<cudaStream_t>(stream));
 }
 
 int bsa_dense_fwd(const bsa_layout *layout, const void *q, const void *k, const void *v,
-                  float softmax_scale, void *out, float *lse, int32_t *err_flag, void *stream) {
+                  float softmax_scale, void *out, float *lse, int32_t *err_flag, void *workspace,
+                  void *stream) {
     int rc = check_layout(layout);
     if (rc != BSA_OK) return rc;
     if (!q || !k || !v || !out) return BSA_ERR_INVALID_ARG;
@@ -160,9 +167,10 @@ int bsa_dense_fwd(const bsa_layout *layout, const void *q, const void *k, const 
         return BSA_ERR_INVALID_ARG;
     if ((lse && !aligned(lse, 4)) || (err_flag && !aligned(err_flag, 4))) return BSA_ERR_INVALID_ARG;
     if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return BSA_ERR_INVALID_ARG;
+    if (workspace && !aligned(workspace, 16)) return BSA_ERR_INVALID_ARG;
     const Geometry g = bsa::make_geometry(*layout);
     return bsa::launch_attention(g, q, k, v, nullptr, nullptr, softmax_scale, out, lse, err_flag,
-                                 static_cast<cudaStream_t>(stream));
+                                 workspace, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -8,30 +8,40 @@
 // full tiles.  The output is the exact softmax over the selected keys,
 // renormalised over them alone.
 //
-// One CTA per 128-row query tile (one query block of 128, or one block of 64
-// in the upper half of the tile).  It walks that block's compacted key-block
-// list; skipped blocks cost nothing.  Every list position t is one 128-key
-// tile: one key block of 128, or (k_block = 64) the blocks at list positions
-// 2t and 2t+1 gathered into the two halves of the tile.
+// Work item = one 128-row query tile (a query block of 128, or a block of 64
+// in the upper half of the tile) of one (batch, head).  It walks that block's
+// compacted key-block list; skipped blocks cost nothing.  Every list position
+// t is one 128-key tile: one key block of 128, or (k_block = 64) the blocks at
+// list positions 2t and 2t+1 gathered into the two halves of the tile.
+//
+// Persistent: one CTA per SM.  Its producer thread claims the next item from a
+// global counter (items are ordered head-major, so the CTAs in flight share one
+// head's K/V in L2, and a CTA that drew a dense frame-0 row simply claims fewer
+// items) and hands it to the other roles through a 4-slot ring in shared
+// memory.  Without a counter the CTAs take items blockIdx.x, +gridDim.x, ...
+// Barriers, TMEM and tensor-map prefetches are set up once; every pipeline
+// phase is carried across items, so item n+1's Q/K/V loads and first QK^T
+// products overlap item n's epilogue.  Every wait is bounded (see mbar_wait).
 //
 // Warp roles (12 warps):
-//   warp 0      TMA producer: Q once, then K and V tiles into 3-stage rings
+//   warp 0      TMA producer: Q per item, K into a 3-stage ring, V into a 2-stage ring
 //   warp 1      tcgen05 issuer (one thread) and TMEM owner (512 columns)
 //   warps 4-7   softmax stream 0: list positions 0, 2, 4, ...
 //   warps 8-11  softmax stream 1: list positions 1, 3, 5, ...
-// Each stream s has S_s (128 fp32 columns; later reused for its bf16 P) and
-// O_s (D fp32 columns) in TMEM, so the tensor core computes one stream's
-// QK^T or PV while the other stream's softmax runs.  The two partial
-// (O_s, m_s, l_s) are merged in the epilogue.  Each softmax thread owns one
-// query row (TMEM lane), so row max and row sum need no shuffles.  The running
-// max is raised lazily: O_s is rescaled only when the max grows by more than
-// 2^8, which keeps every P value below 256.
+// Each stream s has S_s (128 fp32 columns; its first 64 are reused for the
+// bf16 P of the same tile) and O_s (D fp32 columns) in TMEM, so the tensor
+// core computes one stream's QK^T or PV while the other stream's softmax
+// runs.  The two partial (O_s, m_s, l_s) are merged in the epilogue.  Each
+// softmax thread owns one query row (TMEM lane): row max and row sum need no
+// shuffles.  The running max is raised lazily (O_s is rescaled only when it
+// grows by more than 2^8), which keeps every P below 256.  One quarter of the
+// exponentials run as a polynomial on the FMA pipe to unload the MUFU unit.
 //
-// Tensor-core issue order: S0(0) S1(1) | PV(0) S(2) | PV(1) S(3) | ...
+// Tensor-core issue order per item: S(0) S(1) | PV(0) S(2) | PV(1) S(3) | ...
 // tcgen05 operations of one thread complete in issue order, so
 //   * S_s(t+2) may overwrite P_s(t): it is issued after PV(t);
-//   * when S_s(t) is complete, PV for the previous tile of stream s is too,
-//     so the softmax may rescale O_s right after it sees S_s(t).
+//   * when S_s(t) is complete, the previous PV into O_s is too, so the softmax
+//     may rescale O_s as soon as it sees S_s(t).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -48,6 +58,16 @@ namespace bsa {
 namespace {
 
 constexpr int kThreads = 384;
+// Launch: 168 registers x 384 threads.  Warps 0-3 (producer, MMA issuer, two
+// idle warps) give back to kRegsControl; the two softmax warpgroups take the
+// rest (56 -> 224 by default): kRegsControl*128 + kRegsSoftmax*256 = 168*384.
+#ifndef BSA_REGS_CONTROL
+#define BSA_REGS_CONTROL 56
+#endif
+constexpr uint32_t kRegsControl = BSA_REGS_CONTROL;
+constexpr uint32_t kRegsSoftmax = (168 * kThreads - kRegsControl * 128) / 256;
+static_assert(kRegsControl * 128 + kRegsSoftmax * 256 == 168 * kThreads, "register split");
+static_assert(kRegsControl % 8 == 0 && kRegsSoftmax % 8 == 0, "setmaxnreg takes multiples of 8");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kPanelBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle panel)
@@ -57,9 +77,10 @@ struct Cfg {
     static constexpr int kPanels = D / 64;
     static constexpr int kTileBytes = kPanels * kPanelBytes;  // 128 rows x D bf16
     static constexpr int kStagesK = (D == 128) ? 3 : 4;
-    static constexpr int kStagesV = (D == 128) ? 3 : 4;
+    static constexpr int kStagesV = (D == 128) ? 2 : 4;
     static constexpr int kHeader = 1024;
-    static constexpr int kOffQ = kHeader;
+    static constexpr int kOffStats = kHeader;  // [item parity][m, l][stream][row] floats: 4 KB
+    static constexpr int kOffQ = kOffStats + 4096;
     static constexpr int kOffK = kOffQ + kTileBytes;
     static constexpr int kOffV = kOffK + kStagesK * kTileBytes;
     static constexpr int kBytes = kOffV + kStagesV * kTileBytes;
@@ -72,21 +93,42 @@ struct AttnParams {
     __nv_bfloat16 *out;
     float *lse;
     int32_t *err;
+    int *sched;               // work-queue counter (zeroed before launch), or nullptr: static
+    long long n_items;
     int S, S_pad, Cq, Ck, bq;
     float scale_log2;
 };
 
-// Header: mbarriers, TMEM base, abort flag.
 template <int D>
 struct Header {
-    uint64_t q_full;
+    uint64_t q_full, q_empty;
     uint64_t k_full[Cfg<D>::kStagesK], k_empty[Cfg<D>::kStagesK];
     uint64_t v_full[Cfg<D>::kStagesV], v_empty[Cfg<D>::kStagesV];
     uint64_t s_full[2], p_full[2];
-    uint64_t o_final;
+    uint64_t o_full, o_free;
+    uint64_t item_full[4], item_empty[4];  // work-item ring: producer -> MMA + softmax warps
+    uint64_t stats_full;                   // both streams' (m, l) of an item are in smem
+    int item_ring[4];
     uint32_t tmem_base;
     int abort;
 };
+constexpr int kItemConsumers = 1 + 8;  // the MMA thread + one arrival per softmax warp
+
+// List entries of a work item, clamped to [0, C_k], and its number of tiles.
+template <int BK>
+__device__ __forceinline__ void item_lists(const AttnParams &p, long long item,
+                                           const int32_t *&entries, int &n_entries, int &n_tiles,
+                                           bool &bad_count) {
+    entries = p.kv_index ? p.kv_index + item * p.Ck : nullptr;
+    n_entries = p.Ck;
+    bad_count = false;
+    if (p.kv_index) {
+        const int c = p.kv_count[item];
+        bad_count = c < 0 || c > p.Ck;
+        n_entries = min(max(c, 0), p.Ck);
+    }
+    n_tiles = (BK == 128) ? n_entries : (n_entries + 1) / 2;
+}
 
 // Key block of half `hf` of list tile t, and how many of its key columns are
 // real (0 for a missing or invalid entry).
@@ -117,8 +159,7 @@ __device__ __forceinline__ void tile_block(const AttnParams &p, const int32_t *e
 template <int D, int BK>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                const AttnParams p) {
+                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
     using C = Cfg<D>;
     constexpr int NK = C::kStagesK, NV = C::kStagesV;
     constexpr int kHalves = 128 / BK;
@@ -126,29 +167,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     Header<D> &hd = *reinterpret_cast<Header<D> *>(smem);
+    float *stats = reinterpret_cast<float *>(smem + C::kOffStats);
     uint8_t *sQ = smem + C::kOffQ;
     uint8_t *sK = smem + C::kOffK;
     uint8_t *sV = smem + C::kOffV;
     volatile int *abort_flag = &hd.abort;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const long long item = blockIdx.x;  // = (b*H + h)*C_q + i
-    const int bh = static_cast<int>(item / p.Cq);
-    const int qi = static_cast<int>(item % p.Cq);
-
-    // Number of list entries (clamped) and of 128-key tiles.
-    const int32_t *entries = p.kv_index ? p.kv_index + item * p.Ck : nullptr;
-    int n_entries = p.Ck;
-    bool bad_count = false;
-    if (p.kv_index) {
-        const int c = p.kv_count[item];
-        bad_count = c < 0 || c > p.Ck;
-        n_entries = min(max(c, 0), p.Ck);
-    }
-    const int n_tiles = (BK == 128) ? n_entries : (n_entries + 1) / 2;
 
     if (threadIdx.x == 0) {
         mbar_init(&hd.q_full, 1);
+        mbar_init(&hd.q_empty, 1);
         for (int s = 0; s < NK; ++s) {
             mbar_init(&hd.k_full[s], 1);
             mbar_init(&hd.k_empty[s], 1);
@@ -161,7 +190,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&hd.s_full[s], 1);
             mbar_init(&hd.p_full[s], 128);
         }
-        mbar_init(&hd.o_final, 1);
+        mbar_init(&hd.o_full, 1);
+        mbar_init(&hd.o_free, 256);
+        for (int s = 0; s < 4; ++s) {
+            mbar_init(&hd.item_full[s], 1);
+            mbar_init(&hd.item_empty[s], kItemConsumers);
+        }
+        mbar_init(&hd.stats_full, 256);
         hd.abort = 0;
         fence_mbar_init();
     }
@@ -181,57 +216,87 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = hd.tmem_base;
-
+    if (warp < 4) {
+    regs_dec<kRegsControl>();
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
-            if (bad_count && p.err) atomicOr(p.err, BSA_DEVERR_BAD_COUNT);
-            mbar_arrive_expect_tx(&hd.q_full, static_cast<uint32_t>(p.bq * D * 2));
-            for (int pn = 0; pn < C::kPanels; ++pn)
-                tma_load_3d(sQ + pn * kPanelBytes, &tmQ, &hd.q_full, pn * 64, qi * p.bq, bh);
-            int fills_k = 0, fills_v = 0;
-            bool any_bad = false;
-            for (int t = 0; t < n_tiles; ++t) {
-                int jl[kHalves];
-#pragma unroll
-                for (int hf = 0; hf < kHalves; ++hf) {
-                    int valid;
-                    bool bad;
-                    tile_block<BK>(p, entries, n_entries, t, hf, jl[hf], valid, bad);
-                    any_bad |= bad;
+            int kt = 0, vt = 0, qn = 0, q_loads = 0;
+            bool any_bad = false, any_bad_count = false, stop = false;
+            for (;; ++qn) {
+                // Claim the next item and publish it (an index >= n_items ends the loop).
+                const int slot = qn & 3;
+                if (!mbar_wait(&hd.item_empty[slot], ((qn >> 2) & 1) ^ 1, abort_flag)) break;
+                long long item = p.sched ? static_cast<long long>(atomicAdd(p.sched, 1))
+                                         : blockIdx.x + static_cast<long long>(qn) * gridDim.x;
+                if (stop || item > p.n_items) item = p.n_items;
+                hd.item_ring[slot] = static_cast<int>(item);
+                mbar_arrive(&hd.item_full[slot]);
+                if (item >= p.n_items || stop) break;
+                const int bh = static_cast<int>(item / p.Cq), qi = static_cast<int>(item % p.Cq);
+                const int32_t *entries;
+                int n_entries, n_tiles;
+                bool bad_count;
+                item_lists<BK>(p, item, entries, n_entries, n_tiles, bad_count);
+                any_bad_count |= bad_count;
+                if (!mbar_wait(&hd.q_empty, (qn & 1) ^ 1, abort_flag)) {
+                    stop = true;
+                    continue;   // publishes the end marker next
                 }
-                const int ks = t % NK;
-                if (!mbar_wait(&hd.k_empty[ks], ((t / NK) & 1) ^ 1, abort_flag)) break;
-                mbar_arrive_expect_tx(&hd.k_full[ks], static_cast<uint32_t>(C::kTileBytes));
+                mbar_arrive_expect_tx(&hd.q_full, static_cast<uint32_t>(p.bq * D * 2));
+                for (int pn = 0; pn < C::kPanels; ++pn)
+                    tma_load_3d(sQ + pn * kPanelBytes, &tmQ, &hd.q_full, pn * 64, qi * p.bq, bh);
+                ++q_loads;
+                for (int t = 0; t < n_tiles; ++t) {
+                    int jl[kHalves];
 #pragma unroll
-                for (int hf = 0; hf < kHalves; ++hf)
-                    for (int pn = 0; pn < C::kPanels; ++pn)
-                        tma_load_3d(sK + ks * C::kTileBytes + pn * kPanelBytes + hf * BK * 128, &tmK,
-                                    &hd.k_full[ks], pn * 64, jl[hf] * BK, bh);
-                ++fills_k;
-                const int vs = t % NV;
-                if (!mbar_wait(&hd.v_empty[vs], ((t / NV) & 1) ^ 1, abort_flag)) break;
-                mbar_arrive_expect_tx(&hd.v_full[vs], static_cast<uint32_t>(C::kTileBytes));
+                    for (int hf = 0; hf < kHalves; ++hf) {
+                        int valid;
+                        bool bad;
+                        tile_block<BK>(p, entries, n_entries, t, hf, jl[hf], valid, bad);
+                        any_bad |= bad;
+                    }
+                    const int ks = kt % NK;
+                    if (!mbar_wait(&hd.k_empty[ks], ((kt / NK) & 1) ^ 1, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    // (an item cut short by an abort still publishes the end marker next)
+                    mbar_arrive_expect_tx(&hd.k_full[ks], static_cast<uint32_t>(C::kTileBytes));
 #pragma unroll
-                for (int hf = 0; hf < kHalves; ++hf)
-                    for (int pn = 0; pn < C::kPanels; ++pn)
-                        tma_load_3d(sV + vs * C::kTileBytes + pn * kPanelBytes + hf * BK * 128, &tmV,
-                                    &hd.v_full[vs], pn * 64, jl[hf] * BK, bh);
-                ++fills_v;
+                    for (int hf = 0; hf < kHalves; ++hf)
+                        for (int pn = 0; pn < C::kPanels; ++pn)
+                            tma_load_3d(sK + ks * C::kTileBytes + pn * kPanelBytes + hf * BK * 128,
+                                        &tmK, &hd.k_full[ks], pn * 64, jl[hf] * BK, bh);
+                    ++kt;
+                    const int vs = vt % NV;
+                    if (!mbar_wait(&hd.v_empty[vs], ((vt / NV) & 1) ^ 1, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&hd.v_full[vs], static_cast<uint32_t>(C::kTileBytes));
+#pragma unroll
+                    for (int hf = 0; hf < kHalves; ++hf)
+                        for (int pn = 0; pn < C::kPanels; ++pn)
+                            tma_load_3d(sV + vs * C::kTileBytes + pn * kPanelBytes + hf * BK * 128,
+                                        &tmV, &hd.v_full[vs], pn * 64, jl[hf] * BK, bh);
+                    ++vt;
+                }
             }
             if (any_bad && p.err) atomicOr(p.err, BSA_DEVERR_BAD_INDEX);
+            if (any_bad_count && p.err) atomicOr(p.err, BSA_DEVERR_BAD_COUNT);
             // Drain: every copy this thread started must land before the CTA ends.
             volatile int no_abort = 0;
-            mbar_wait(&hd.q_full, 0, &no_abort);
+            if (q_loads > 0) mbar_wait(&hd.q_full, (q_loads - 1) & 1, &no_abort);
             for (int s = 0; s < NK; ++s) {
-                const int f = fills_k / NK + (s < fills_k % NK ? 1 : 0);
+                const int f = kt / NK + (s < kt % NK ? 1 : 0);
                 if (f > 0) mbar_wait(&hd.k_full[s], (f - 1) & 1, &no_abort);
             }
             for (int s = 0; s < NV; ++s) {
-                const int f = fills_v / NV + (s < fills_v % NV ? 1 : 0);
+                const int f = vt / NV + (s < vt % NV ? 1 : 0);
                 if (f > 0) mbar_wait(&hd.v_full[s], (f - 1) & 1, &no_abort);
             }
         }
@@ -241,49 +306,88 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
             const uint32_t q_addr = smem_u32(sQ);
-            auto issue_s = [&](int t) -> bool {
-                const int ks = t % NK;
-                if (!mbar_wait(&hd.k_full[ks], (t / NK) & 1, abort_flag)) return false;
-                tc_fence_after();
-                const uint32_t k_addr = smem_u32(sK + ks * C::kTileBytes);
-                const uint32_t d_tmem = tmem + static_cast<uint32_t>((t & 1) * 128);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk / 4) * kPanelBytes + (kk % 4) * 32;
-                    mma_ss(d_tmem, sw128_desc(q_addr + off, 16, 1024),
-                           sw128_desc(k_addr + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+            int kt = 0, vt = 0, qn = 0, pc[2] = {0, 0};
+            bool ok = true;
+            for (; ok; ++qn) {
+                const int slot = qn & 3;
+                if (!mbar_wait(&hd.item_full[slot], (qn >> 2) & 1, abort_flag)) {
+                    ok = false;
+                    break;
                 }
-                mma_commit(&hd.k_empty[ks]);
-                mma_commit(&hd.s_full[t & 1]);
-                return true;
-            };
-            bool ok = mbar_wait(&hd.q_full, 0, abort_flag);
-            if (ok && n_tiles > 0) ok = issue_s(0);
-            if (ok && n_tiles > 1) ok = issue_s(1);
-            for (int t = 0; ok && t < n_tiles; ++t) {
-                const int s = t & 1, it = t >> 1;
-                if (!mbar_wait(&hd.p_full[s], it & 1, abort_flag)) break;
-                tc_fence_after();
-                const int vs = t % NV;
-                if (!mbar_wait(&hd.v_full[vs], (t / NV) & 1, abort_flag)) break;
-                tc_fence_after();
-                const uint32_t v_addr = smem_u32(sV + vs * C::kTileBytes);
-                const uint32_t o_tmem = tmem + 256u + static_cast<uint32_t>(s * 128);
-                const uint32_t p_tmem = tmem + static_cast<uint32_t>(s * 128);
+                const long long item = *reinterpret_cast<volatile int *>(&hd.item_ring[slot]);
+                mbar_arrive(&hd.item_empty[slot]);
+                if (item >= p.n_items) break;
+                const int32_t *entries;
+                int n_entries, n_tiles;
+                bool bad_count;
+                item_lists<BK>(p, item, entries, n_entries, n_tiles, bad_count);
+                // S_s(t) = Q K_t^T; frees the K stage, and Q once t is the item's last tile.
+                auto issue_s = [&](int t) -> bool {
+                    const int ks = kt % NK;
+                    if (!mbar_wait(&hd.k_full[ks], (kt / NK) & 1, abort_flag)) return false;
+                    tc_fence_after();
+                    const uint32_t k_addr = smem_u32(sK + ks * C::kTileBytes);
+                    const uint32_t d_tmem = tmem + static_cast<uint32_t>((t & 1) * 128);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(o_tmem, p_tmem + kk * 8, sw128_desc(v_addr + kk * 2048, kPanelBytes, 1024),
-                           idesc_pv, (it > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&hd.v_empty[vs]);
-                if (t + 2 < n_tiles && !issue_s(t + 2)) break;
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk / 4) * kPanelBytes + (kk % 4) * 32;
+                        mma_ss(d_tmem, sw128_desc(q_addr + off, 16, 1024),
+                               sw128_desc(k_addr + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&hd.k_empty[ks]);
+                    mma_commit(&hd.s_full[t & 1]);
+                    if (t == n_tiles - 1) mma_commit(&hd.q_empty);
+                    ++kt;
+                    return true;
+                };
+                ok = mbar_wait(&hd.q_full, qn & 1, abort_flag);
+                if (ok && n_tiles == 0) mma_commit(&hd.q_empty);
+                if (ok && n_tiles > 0) ok = issue_s(0);
+                if (ok && n_tiles > 1) ok = issue_s(1);
+                // O_a / O_b still hold the previous item until its epilogue has read them.
+                // Waited for every item (even one without tiles) so that the wait never
+                // runs two phases ahead of the epilogues.
+                if (ok && qn > 0) ok = mbar_wait(&hd.o_free, (qn - 1) & 1, abort_flag);
+                for (int t = 0; ok && t < n_tiles; ++t) {
+                    const int s = t & 1;
+                    if (!mbar_wait(&hd.p_full[s], pc[s] & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    ++pc[s];
+                    tc_fence_after();
+                    const int vs = vt % NV;
+                    if (!mbar_wait(&hd.v_full[vs], (vt / NV) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t v_addr = smem_u32(sV + vs * C::kTileBytes);
+                    const uint32_t o_tmem = tmem + 256u + static_cast<uint32_t>(s * 128);
+                    const uint32_t p_tmem = tmem + static_cast<uint32_t>(s * 128);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(o_tmem, p_tmem + kk * 8,
+                               sw128_desc(v_addr + kk * 2048, kPanelBytes, 1024), idesc_pv,
+                               (t >= 2 || kk > 0) ? 1u : 0u);
+                    mma_commit(&hd.v_empty[vs]);
+                    ++vt;
+                    if (t + 2 < n_tiles && !issue_s(t + 2)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                mma_commit(&hd.o_full);
             }
-            mma_commit(&hd.o_final);
-            if (*abort_flag) {  // let whatever was issued finish before TMEM is freed
+            if (!ok) {  // let whatever was issued finish before TMEM is freed
+                mma_commit(&hd.o_full);
                 volatile int no_abort = 0;
-                mbar_wait(&hd.o_final, 0, &no_abort);
+                mbar_wait(&hd.o_full, qn & 1, &no_abort);
             }
         }
-    } else if (warp >= 4) {
+    }
+    } else {
+        regs_inc<kRegsSoftmax>();
         // ------------------------------------------------------------ softmax streams
         const int s = (warp >> 2) - 1;  // stream
         const int rw = warp & 3;        // TMEM lane quarter
@@ -291,165 +395,184 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(rw * 32) << 16);
         const uint32_t t_s = t_lane + static_cast<uint32_t>(s * 128);
         const uint32_t t_o = t_lane + 256u + static_cast<uint32_t>(s * 128);
-        const int n_s = (n_tiles > s) ? (n_tiles - s + 1) / 2 : 0;
-        float m_run = -INFINITY, l_run = 0.f;
+        int sc = 0, qn = 0;
         bool ok = true;
-        for (int it = 0; it < n_s; ++it) {
-            const int t = 2 * it + s;
-            // tcgen05.ld/st below are warp-collective: leave together or not at all.
-            if (!__all_sync(0xffffffffu, mbar_wait(&hd.s_full[s], it & 1, abort_flag))) {
-                ok = false;
+        for (;; ++qn) {
+            const int slot = qn & 3;
+            if (!__all_sync(0xffffffffu, mbar_wait(&hd.item_full[slot], (qn >> 2) & 1, abort_flag)))
                 break;
-            }
-            tc_fence_after();
-            float x[128];
-            {
-                uint32_t raw[4][32];
+            const long long item = *reinterpret_cast<volatile int *>(&hd.item_ring[slot]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&hd.item_empty[slot]);
+            if (item >= p.n_items) break;
+            const int bh = static_cast<int>(item / p.Cq), qi = static_cast<int>(item % p.Cq);
+            const int32_t *entries;
+            int n_entries, n_tiles;
+            bool bad_count;
+            item_lists<BK>(p, item, entries, n_entries, n_tiles, bad_count);
+            const int n_s = (n_tiles > s) ? (n_tiles - s + 1) / 2 : 0;
+            float m_run = -INFINITY, l_run = 0.f;
+            for (int it = 0; ok && it < n_s; ++it) {
+                const int t = 2 * it + s;
+                // tcgen05.ld/st below are warp-collective: leave together or not at all.
+                if (!__all_sync(0xffffffffu, mbar_wait(&hd.s_full[s], sc & 1, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                ++sc;
+                tc_fence_after();
+                float x[128];
+                {
+                    uint32_t raw[4][32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, raw[c]);
-                tmem_ld_wait();
+                    for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, raw[c]);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        reg_fence(raw[c]);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(raw[c][e]);
+                    }
+                }
+                // Mask key columns past seq_len, and missing / invalid halves.
+                int vc[kHalves];
+                bool partial = false;
+#pragma unroll
+                for (int hf = 0; hf < kHalves; ++hf) {
+                    int jl;
+                    bool bad;
+                    tile_block<BK>(p, entries, n_entries, t, hf, jl, vc[hf], bad);
+                    partial |= vc[hf] < BK;
+                }
+                if (partial) {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if ((c % BK) >= vc[c / BK]) x[c] = -INFINITY;
+                }
+                float mx;
+                {
+                    float pm[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        pm[k] = fmaxf(x[32 * k], x[32 * k + 1]);
+#pragma unroll
+                        for (int e = 2; e < 32; e += 2) pm[k] = max3(pm[k], x[32 * k + e], x[32 * k + e + 1]);
+                    }
+                    mx = fmaxf(max3(pm[0], pm[1], pm[2]), pm[3]);
+                }
+                const float m_new = fmaxf(m_run, mx * p.scale_log2);
+                if (it == 0) {
+                    m_run = m_new;
+                } else {
+                    const bool need = m_new > m_run + kRescaleLog2;
+                    if (__any_sync(0xffffffffu, need)) {
+                        const float alpha = need ? ex2(m_run - m_new) : 1.0f;
+#pragma unroll 1
+                        for (int c = 0; c < D / 16; ++c) {
+                            uint32_t o[16];
+                            tmem_ld16(t_o + c * 16, o);
+                            tmem_ld_wait();
+                            reg_fence(o);
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                            tmem_st16(t_o + c * 16, o);
+                        }
+                        tmem_st_wait();
+                        l_run *= alpha;
+                        if (need) m_run = m_new;
+                    }
+                }
+                const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
+                const float sl = p.scale_log2;
+                float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    reg_fence(raw[c]);
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(raw[c][e]);
-                }
-            }
-            // Mask key columns past seq_len, and missing / invalid halves.
-            int vc[kHalves];
-            bool partial = false;
-#pragma unroll
-            for (int hf = 0; hf < kHalves; ++hf) {
-                int jl;
-                bool bad;
-                tile_block<BK>(p, entries, n_entries, t, hf, jl, vc[hf], bad);
-                partial |= vc[hf] < BK;
-            }
-            if (partial) {
-#pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if ((c % BK) >= vc[c / BK]) x[c] = -INFINITY;
-            }
-            float mx = x[0];
-#pragma unroll
-            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
-            const float m_new = fmaxf(m_run, mx * p.scale_log2);
-            if (it == 0) {
-                m_run = m_new;
-            } else {
-                const bool need = m_new > m_run + kRescaleLog2;
-                if (__any_sync(0xffffffffu, need)) {
-                    const float alpha = need ? ex2(m_run - m_new) : 1.0f;
-#pragma unroll 1
-                    for (int c = 0; c < D / 16; ++c) {
-                        uint32_t o[16];
-                        tmem_ld16(t_o + c * 16, o);
-                        tmem_ld_wait();
-                        reg_fence(o);
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st16(t_o + c * 16, o);
+                    for (int e = 0; e < 16; ++e) {
+                        float t0, t1, p0, p1;
+                        fma2(t0, t1, x[c * 32 + 2 * e], x[c * 32 + 2 * e + 1], sl, sl, nm, nm);
+                        if (c == 3) {
+                            exp2_poly2(t0, t1, p0, p1);  // columns 96..127 on the FMA pipe
+                        } else {
+                            p0 = ex2(t0);
+                            p1 = ex2(t1);
+                        }
+                        pk[e] = pack_bf16x2(p0, p1);
+                        if (e & 1) add2(b0, b1, b0, b1, p0, p1);
+                        else add2(a0, a1, a0, a1, p0, p1);
                     }
-                    tmem_st_wait();
-                    l_run *= alpha;
-                    if (need) m_run = m_new;
+                    tmem_st16(t_s + c * 16, pk);
                 }
+                l_run += (a0 + a1) + (b0 + b1);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&hd.p_full[s]);
             }
-            const float m_eff = (m_run == -INFINITY) ? 0.f : m_run;
-            float sum = 0.f;
+
+            // -------------------------------------------------------- epilogue
+            ok = ok && !*abort_flag && mbar_wait(&hd.o_full, qn & 1, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
+            // Exchange (m, l) between the streams.  Double-buffered by item parity: a
+            // stream cannot write item n+2's stats before the other stream has read
+            // item n's, because item n+2's PV waits for both streams' o_free of n+1.
+            float *st = stats + (qn & 1) * 512;
+            st[s * 128 + r] = m_run;
+            st[256 + s * 128 + r] = l_run;
+            mbar_arrive(&hd.stats_full);
+            ok = __all_sync(0xffffffffu, mbar_wait(&hd.stats_full, qn & 1, abort_flag) && ok);
+            const float ma = st[r], mb = st[128 + r];
+            const float la = st[256 + r], lb = st[384 + r];
+            const float m = fmaxf(ma, mb);
+            const float sa = (ma == -INFINITY) ? 0.f : ex2(ma - m);
+            const float sb = (mb == -INFINITY) ? 0.f : ex2(mb - m);
+            const float L = la * sa + lb * sb;
+            const float inv = (L > 0.f) ? 1.0f / L : 0.f;
+            const bool has_a = n_tiles > 0, has_b = n_tiles > 1;
+            const long long t_abs = static_cast<long long>(qi) * p.bq + r;
+            const bool row_out = r < p.bq && t_abs < p.S_pad;
+            const bool row_valid = t_abs < p.S;
+            const long long grow = static_cast<long long>(bh) * p.S_pad + t_abs;
+            // Stream s writes output columns [s*D/2, (s+1)*D/2) of its row.
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < D / 64; ++c) {
+                const int col = s * (D / 2) + c * 32;
+                uint32_t oa[32], ob[32];
+                if (ok && has_a) tmem_ld32(t_lane + 256u + col, oa);
+                if (ok && has_b) tmem_ld32(t_lane + 384u + col, ob);
+                tmem_ld_wait();
+                reg_fence(oa);
+                reg_fence(ob);
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float p0 = ex2(fmaf(x[c * 32 + 2 * e], p.scale_log2, -m_eff));
-                    const float p1 = ex2(fmaf(x[c * 32 + 2 * e + 1], p.scale_log2, -m_eff));
-                    sum += p0 + p1;
-                    pk[e] = pack_bf16x2(p0, p1);
+                    float v0 = 0.f, v1 = 0.f;
+                    if (ok && has_a && row_valid) {
+                        v0 = __uint_as_float(oa[2 * e]) * sa;
+                        v1 = __uint_as_float(oa[2 * e + 1]) * sa;
+                    }
+                    if (ok && has_b && row_valid) {
+                        v0 = fmaf(__uint_as_float(ob[2 * e]), sb, v0);
+                        v1 = fmaf(__uint_as_float(ob[2 * e + 1]), sb, v1);
+                    }
+                    pk[e] = pack_bf16x2(v0 * inv, v1 * inv);
                 }
-                tmem_st16(t_s + c * 16, pk);
+                if (row_out && ok) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + grow * D + col);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+                }
             }
-            l_run += sum;
-            tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&hd.p_full[s]);
+            mbar_arrive(&hd.o_free);
+            if (s == 0 && row_out && p.lse)
+                p.lse[grow] = !row_valid ? -INFINITY
+                              : ok       ? (m + __log2f(L)) * 0.69314718055994531f
+                                         : NAN;
         }
-
-        // ------------------------------------------------------------ epilogue
-        ok = ok && !*abort_flag && mbar_wait(&hd.o_final, 0, abort_flag);
-        ok = __all_sync(0xffffffffu, ok);
-        tc_fence_after();
-        float *st_m = reinterpret_cast<float *>(sK);  // K ring is idle once o_final fired
-        float *st_l = st_m + 256;
-        st_m[s * 128 + r] = m_run;
-        st_l[s * 128 + r] = l_run;
-        named_barrier_sync(1, 256);
-        const float ma = st_m[r], mb = st_m[128 + r];
-        const float la = st_l[r], lb = st_l[128 + r];
-        const float m = fmaxf(ma, mb);
-        const float sa = (ma == -INFINITY) ? 0.f : ex2(ma - m);
-        const float sb = (mb == -INFINITY) ? 0.f : ex2(mb - m);
-        const float L = la * sa + lb * sb;
-        const float inv = (L > 0.f) ? 1.0f / L : 0.f;
-        const bool has_a = n_tiles > 0, has_b = n_tiles > 1;
-        // Stream s writes output columns [s*D/2, (s+1)*D/2) into the Q buffer (now idle)
-        // in the 128-byte-swizzled layout the O tensor map expects.
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-            const int col = s * (D / 2) + c * 32;
-            uint32_t oa[32], ob[32];
-            if (ok && has_a) tmem_ld32(t_lane + 256u + col, oa);
-            if (ok && has_b) tmem_ld32(t_lane + 384u + col, ob);
-            tmem_ld_wait();
-            reg_fence(oa);
-            reg_fence(ob);
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                float v0 = 0.f, v1 = 0.f;
-                if (ok && has_a) {
-                    v0 = __uint_as_float(oa[2 * e]) * sa;
-                    v1 = __uint_as_float(oa[2 * e + 1]) * sa;
-                }
-                if (ok && has_b) {
-                    v0 = fmaf(__uint_as_float(ob[2 * e]), sb, v0);
-                    v1 = fmaf(__uint_as_float(ob[2 * e + 1]), sb, v1);
-                }
-                pk[e] = pack_bf16x2(v0 * inv, v1 * inv);
-            }
-            const int panel = col / 64;
-            uint8_t *row_base = sQ + panel * kPanelBytes + r * 128;
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                const int chunk = ((col % 64) / 8 + q4) ^ (r & 7);
-                *reinterpret_cast<uint4 *>(row_base + chunk * 16) =
-                    make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-            }
-        }
-        fence_proxy_async_smem();
-        named_barrier_sync(1, 256);
-        if (threadIdx.x == 128 && ok) {
-            for (int pn = 0; pn < C::kPanels; ++pn)
-                tma_store_3d(&tmO, sQ + pn * kPanelBytes, pn * 64, qi * p.bq, bh);
-            tma_store_commit();
-            tma_store_wait_all();
-        }
-        // Row statistics, and the padded rows S..S_pad-1 (outside the O tensor map).
-        const long long t_abs = static_cast<long long>(qi) * p.bq + r;
-        if (r < p.bq && t_abs < p.S_pad) {
-            const long long grow = static_cast<long long>(bh) * p.S_pad + t_abs;
-            if (t_abs < p.S) {
-                if (s == 0 && p.lse)
-                    p.lse[grow] = ok ? (m + __log2f(L)) * 0.69314718055994531f : NAN;
-            } else {
-                uint4 *dst = reinterpret_cast<uint4 *>(p.out + grow * D + s * (D / 2));
-#pragma unroll
-                for (int e = 0; e < D / 16; ++e) dst[e] = make_uint4(0, 0, 0, 0);
-                if (s == 0 && p.lse) p.lse[grow] = -INFINITY;
-            }
-        }
-        tc_fence_before();
     }
 
     __syncthreads();
@@ -482,7 +605,7 @@ EncodeTiledFn encoder() {
     return fn;
 }
 
-// [B*H, S, D] bf16 view with rows >= S out of bounds (loads read zero, stores are dropped).
+// [B*H, S, D] bf16 view with rows >= S out of bounds (loads read zero).
 bool make_map(CUtensorMap *m, const void *base, const Geometry &g, int box_rows) {
     EncodeTiledFn enc = encoder();
     if (!enc) return false;
@@ -497,13 +620,19 @@ bool make_map(CUtensorMap *m, const void *base, const Geometry &g, int box_rows)
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
 template <int D, int BK>
 int launch_t(const Geometry &g, const void *q, const void *k, const void *v,
              const int32_t *kv_index, const int32_t *kv_count, float softmax_scale, void *out,
-             float *lse, int32_t *err, cudaStream_t st) {
-    CUtensorMap mq, mk, mv, mo;
-    if (!make_map(&mq, q, g, g.bq) || !make_map(&mk, k, g, BK) || !make_map(&mv, v, g, BK) ||
-        !make_map(&mo, out, g, g.bq))
+             float *lse, int32_t *err, void *workspace, cudaStream_t st) {
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, g, g.bq) || !make_map(&mk, k, g, BK) || !make_map(&mv, v, g, BK))
         return BSA_ERR_DRIVER;
     AttnParams p;
     p.kv_index = kv_index;
@@ -511,6 +640,8 @@ int launch_t(const Geometry &g, const void *q, const void *k, const void *v,
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.lse = lse;
     p.err = err;
+    p.sched = static_cast<int *>(workspace);
+    p.n_items = static_cast<long long>(g.B) * g.H * g.Cq;
     p.S = g.S;
     p.S_pad = g.S_pad;
     p.Cq = g.Cq;
@@ -521,8 +652,12 @@ int launch_t(const Geometry &g, const void *q, const void *k, const void *v,
     if (cudaFuncSetAttribute(attn_kernel<D, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
         return BSA_ERR_LAUNCH;
-    const long long grid = static_cast<long long>(g.B) * g.H * g.Cq;
-    attn_kernel<D, BK><<<static_cast<unsigned>(grid), kThreads, smem, st>>>(mq, mk, mv, mo, p);
+    const int sms = sm_count();
+    if (sms <= 0) return BSA_ERR_LAUNCH;
+    const long long grid = p.n_items < sms ? p.n_items : sms;
+    if (workspace && cudaMemsetAsync(workspace, 0, sizeof(int), st) != cudaSuccess)
+        return BSA_ERR_LAUNCH;
+    attn_kernel<D, BK><<<static_cast<unsigned>(grid), kThreads, smem, st>>>(mq, mk, mv, p);
     return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_LAUNCH;
 }
 
@@ -530,17 +665,17 @@ int launch_t(const Geometry &g, const void *q, const void *k, const void *v,
 
 int launch_attention(const Geometry &g, const void *q, const void *k, const void *v,
                      const int32_t *kv_index, const int32_t *kv_count, float softmax_scale,
-                     void *out, float *lse, int32_t *err_flag, cudaStream_t st) {
+                     void *out, float *lse, int32_t *err_flag, void *workspace, cudaStream_t st) {
     if (g.D == 128) {
         return g.bk == 128 ? launch_t<128, 128>(g, q, k, v, kv_index, kv_count, softmax_scale, out,
-                                                lse, err_flag, st)
+                                                lse, err_flag, workspace, st)
                            : launch_t<128, 64>(g, q, k, v, kv_index, kv_count, softmax_scale, out,
-                                               lse, err_flag, st);
+                                               lse, err_flag, workspace, st);
     }
     return g.bk == 128 ? launch_t<64, 128>(g, q, k, v, kv_index, kv_count, softmax_scale, out, lse,
-                                           err_flag, st)
+                                           err_flag, workspace, st)
                        : launch_t<64, 64>(g, q, k, v, kv_index, kv_count, softmax_scale, out, lse,
-                                          err_flag, st);
+                                          err_flag, workspace, st);
 }
 
 }  // namespace bsa

@@ -38,6 +38,8 @@ cudaError_t launch_entropy_reduce(const Geometry &g, const float *row_entropy, f
 // Returns BSA_* status.
 int launch_attention(const Geometry &g, const void *q, const void *k, const void *v,
                      const int32_t *kv_index, const int32_t *kv_count, float softmax_scale,
-                     void *out, float *lse, int32_t *err_flag, cudaStream_t st);
+                     void *out, float *lse, int32_t *err_flag, void *workspace, cudaStream_t st);
+
+constexpr size_t kAttnWorkspaceBytes = 256;
 
 }  // namespace bsa

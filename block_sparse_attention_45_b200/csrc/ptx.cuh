@@ -251,6 +251,20 @@ __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Per-warpgroup register reallocation; every warp of a warpgroup executes the
+// same one.  The splits used by the kernels add up exactly to the registers the
+// block was launched with, so an increase never waits for registers that no
+// decrease releases.
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- descriptors
 
 // Shared-memory matrix descriptor (tcgen05 format, version 1) for a tile
@@ -283,6 +297,53 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Packed fp32x2 arithmetic (sm_100): one instruction for two lanes of data.
+__device__ __forceinline__ void fma2(float &d0, float &d1, float a0, float a1, float b0, float b1,
+                                     float c0, float c1) {
+    asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+        "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+__device__ __forceinline__ void add2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 a, b, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// 2^t for a pair, on the FMA pipe (leaves the MUFU unit to the other columns).
+// Range reduction: t = n + f with n = round(t) (from the low mantissa bits of
+// t + 1.5*2^23) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial with
+// p(0) = 1 whose coefficients are a minimax fit of the relative error on
+// [-1/2, 1/2] (max 1.01e-4, below bf16 resolution); 2^n is added to the
+// exponent field.  t is clamped at -127, where the result is exactly +0, so
+// masked (-inf) columns give exact zeros.  Valid for t <= 127.
+__device__ __forceinline__ void exp2_poly2(float t0, float t1, float &p0, float &p1) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    constexpr float kC1 = 0.693282902f, kC2 = 0.242210954f, kC3 = 0.0550089329f;
+    t0 = fmaxf(t0, -127.0f);
+    t1 = fmaxf(t1, -127.0f);
+    float j0, j1, r0, r1, f0, f1, q0, q1;
+    add2(j0, j1, t0, t1, kMagic, kMagic);
+    add2(r0, r1, j0, j1, -kMagic, -kMagic);
+    fma2(f0, f1, r0, r1, -1.0f, -1.0f, t0, t1);
+    fma2(q0, q1, f0, f1, kC3, kC3, kC2, kC2);
+    fma2(q0, q1, q0, q1, f0, f1, kC1, kC1);
+    fma2(q0, q1, q0, q1, f0, f1, 1.0f, 1.0f);
+    p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(j0) << 23));
+    p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(j1) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -159,6 +159,11 @@ int bsa_build_mask(const bsa_layout *layout, const float *probs, const float *to
  * valid key gets the same.  With k_block = 64, consecutive list entries are
  * paired into one 128-key tensor-core tile.
  *
+ * One CTA per SM walks the (batch, head, query block) work items in
+ * head-major order.  With a workspace the CTAs claim items from a counter in
+ * it, which balances rows of very different list lengths (dense frame-0 rows
+ * next to sparse ones); without one, CTA c takes items c, c + #SMs, ...
+ *
  * q, k, v       bf16 [B,H,seq_pad,D], 16-byte aligned (read only)
  * kv_index      int32 [B,H,C_q,C_k], ascending within a row (read only)
  * kv_count      int32 [B,H,C_q] (read only)
@@ -166,10 +171,17 @@ int bsa_build_mask(const bsa_layout *layout, const float *probs, const float *to
  * out           bf16 [B,H,seq_pad,D], 16-byte aligned (written)
  * lse           fp32 [B,H,seq_pad], or NULL
  * err_flag      device int32, or NULL (see BSA_DEVERR_*)
+ * workspace     device scratch of bsa_attention_workspace_bytes(layout) bytes,
+ *               16-byte aligned, or NULL.  Its contents on entry do not matter
+ *               (the call clears it on `stream` first); two calls that share
+ *               one workspace must not run at the same time.
  */
 int bsa_attention_fwd(const bsa_layout *layout, const void *q, const void *k, const void *v,
                       const int32_t *kv_index, const int32_t *kv_count, float softmax_scale,
-                      void *out, float *lse, int32_t *err_flag, void *stream);
+                      void *out, float *lse, int32_t *err_flag, void *workspace, void *stream);
+
+/* Bytes of device workspace bsa_attention_fwd / bsa_dense_fwd can use. */
+size_t bsa_attention_workspace_bytes(const bsa_layout *layout);
 
 /*
  * Dense exact attention: bsa_attention_fwd with every key block selected for
@@ -177,7 +189,8 @@ int bsa_attention_fwd(const bsa_layout *layout, const void *q, const void *k, co
  * Arguments as for bsa_attention_fwd.
  */
 int bsa_dense_fwd(const bsa_layout *layout, const void *q, const void *k, const void *v,
-                  float softmax_scale, void *out, float *lse, int32_t *err_flag, void *stream);
+                  float softmax_scale, void *out, float *lse, int32_t *err_flag, void *workspace,
+                  void *stream);
 
 /* Human-readable name of a bsa_status value (static storage). */
 const char *bsa_status_string(int status);

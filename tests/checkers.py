@@ -13,15 +13,20 @@ log-sum-exp within LSE_ABS.  Entropy within ENTROPY_REL relative.
 """
 import numpy as np
 
-MARGIN = 1e-4
+MARGIN = 1e-4            # end to end (GPU P' vs oracle P'): all three margin terms
+MARGIN_SAME_PROBS = 1e-5  # identical P' on both sides: only the running-sum terms matter
 MAX_ABS = 2e-2
 MEAN_ABS = 2e-3
 LSE_ABS = 1e-3
 ENTROPY_REL = 1e-3
 
 
-def row_margins(probs, top_p, heads_axis=1):
-    """k* and the margin of every row of probs [B,H,Cq,Ck] (oracle fp32 values)."""
+def row_margins(probs, top_p, use_gap=True):
+    """k* and the margin of every row of probs [B,H,Cq,Ck] (oracle fp32 values).
+
+    use_gap=False drops the P'_(k*) - P'_(k*+1) term: when both sides read the
+    same fp32 P', their orders agree and only the summation rounding can move
+    the cut."""
     B, H, Cq, Ck = probs.shape
     tp = np.broadcast_to(np.asarray(top_p, np.float64), (H,))
     kstar = np.empty((B, H, Cq), np.int64)
@@ -41,20 +46,24 @@ def row_margins(probs, top_p, heads_axis=1):
             gap = np.where(k < Ck, srt[idx, k - 1] - srt[idx, np.minimum(k, Ck - 1)], np.inf)
             m1 = np.where(k > 1, p - ckm1, np.inf)
             m2 = np.where(reach.any(-1), ck - p, np.inf)
-            margin[b, h] = np.minimum(np.minimum(m1, m2), gap)
+            margin[b, h] = np.minimum(np.minimum(m1, m2), gap if use_gap else np.inf)
     return kstar, margin
 
 
-def check_topp_masks(gpu_mask, ora_mask, probs, top_p, kstar=None, margin=None):
-    """Compare top-p masks (no overrides).  Returns the exempt fraction."""
-    if kstar is None:
-        kstar, margin = row_margins(probs, top_p)
+def check_topp_masks(gpu_mask, ora_mask, probs, top_p, same_probs=False):
+    """Compare top-p masks (no overrides).  Returns the exempt fraction.
+
+    same_probs=True: the GPU read the oracle's own P', so the rule is the
+    summation margin MARGIN_SAME_PROBS without the gap term; otherwise the
+    end-to-end rule (MARGIN, all three terms)."""
+    thr = MARGIN_SAME_PROBS if same_probs else MARGIN
+    kstar, margin = row_margins(probs, top_p, use_gap=not same_probs)
     gpu_mask = gpu_mask.astype(bool)
     ora_mask = ora_mask.astype(bool)
-    strict = margin > MARGIN
+    strict = margin > thr
     diff = (gpu_mask != ora_mask).any(-1)
     bad = np.argwhere(diff & strict)
-    assert bad.size == 0, "rows with margin > %g differ: %s (of %d)" % (MARGIN, bad[:5].tolist(), len(bad))
+    assert bad.size == 0, "rows with margin > %g differ: %s (of %d)" % (thr, bad[:5].tolist(), len(bad))
     H = probs.shape[1]
     tp = np.broadcast_to(np.asarray(top_p, np.float64), (H,))
     for b, h, i in np.argwhere(diff & ~strict):
@@ -82,12 +91,20 @@ def check_lists(kv_index, kv_count, mask):
     assert np.array_equal(np.where(valid, kv_index, -1), np.where(valid, ref, -1))
 
 
-def check_attention(out_gpu, out_ora, lse_gpu=None, lse_ora=None, what=""):
+def bf16_output_bound(out_ora, v_max):
+    """Largest max-abs error bf16 arithmetic can produce at this value range:
+    output rounding (2^-9 |o|) plus the rounding of P to bf16 before the PV
+    product, which perturbs each normalised weight by at most 2^-8 relative
+    (<= 2^-8 max|V|).  The spec's MAX_ABS applies when this is below it."""
+    return max(MAX_ABS, 2.0 ** -9 * float(np.abs(out_ora).max()) + 2.0 ** -8 * float(v_max))
+
+
+def check_attention(out_gpu, out_ora, lse_gpu=None, lse_ora=None, what="", max_abs=MAX_ABS):
     out_gpu = np.asarray(out_gpu, np.float64)
     out_ora = np.asarray(out_ora, np.float64)
     assert np.isfinite(out_gpu).all(), what + ": non-finite output"
     err = np.abs(out_gpu - out_ora)
-    assert err.max() <= MAX_ABS, "%s: max abs err %.3g > %g" % (what, err.max(), MAX_ABS)
+    assert err.max() <= max_abs, "%s: max abs err %.3g > %g" % (what, err.max(), max_abs)
     assert err.mean() <= MEAN_ABS, "%s: mean abs err %.3g > %g" % (what, err.mean(), MEAN_ABS)
     if lse_gpu is not None:
         lg = np.asarray(lse_gpu, np.float64)

@@ -43,7 +43,7 @@ MISALIGNED = ctypes.c_void_p(0x10002)
 def test_bad_layouts_are_rejected(kw, expect):
     L = _layout(**kw)
     lib = bsa.load()
-    assert lib.bsa_dense_fwd(ctypes.byref(L), FAKE, FAKE, FAKE, 0.125, FAKE, None, None, None) == expect
+    assert lib.bsa_dense_fwd(ctypes.byref(L), FAKE, FAKE, FAKE, 0.125, FAKE, None, None, None, None) == expect
     assert lib.bsa_block_scores(ctypes.byref(L), FAKE, FAKE, FAKE, FAKE, FAKE, None) == expect
     assert lib.bsa_build_mask_workspace_bytes(ctypes.byref(L)) == 0
 
@@ -52,11 +52,13 @@ def test_bad_pointers_are_rejected():
     L = _layout()
     lib = bsa.load()
     r = ctypes.byref(L)
-    assert lib.bsa_dense_fwd(r, MISALIGNED, FAKE, FAKE, 0.125, FAKE, None, None, None) == bsa.BSA_ERR_INVALID_ARG
-    assert lib.bsa_dense_fwd(r, None, FAKE, FAKE, 0.125, FAKE, None, None, None) == bsa.BSA_ERR_INVALID_ARG
-    assert lib.bsa_dense_fwd(r, FAKE, FAKE, FAKE, -1.0, FAKE, None, None, None) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_dense_fwd(r, MISALIGNED, FAKE, FAKE, 0.125, FAKE, None, None, None, None) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_dense_fwd(r, None, FAKE, FAKE, 0.125, FAKE, None, None, None, None) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_dense_fwd(r, FAKE, FAKE, FAKE, -1.0, FAKE, None, None, None, None) == bsa.BSA_ERR_INVALID_ARG
     assert lib.bsa_attention_fwd(r, FAKE, FAKE, FAKE, None, FAKE, 0.125, FAKE, None, None,
-                                 None) == bsa.BSA_ERR_INVALID_ARG
+                                 None, None) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_dense_fwd(r, FAKE, FAKE, FAKE, 0.125, FAKE, None, None, MISALIGNED,
+                             None) == bsa.BSA_ERR_INVALID_ARG
     assert lib.bsa_block_scores(r, FAKE, FAKE, FAKE, FAKE, MISALIGNED, None) == bsa.BSA_ERR_INVALID_ARG
     tp = (ctypes.c_float * 2)(0.5, 0.5)
     tpv = ctypes.cast(tp, ctypes.c_void_p)
@@ -74,6 +76,7 @@ def test_bad_pointers_are_rejected():
 
 def test_workspace_size():
     L = _layout()
+    assert bsa.load().bsa_attention_workspace_bytes(ctypes.byref(L)) == 256
     # one fp32 per (b, h, query block), rounded up to 256 bytes
     assert bsa.load().bsa_build_mask_workspace_bytes(ctypes.byref(L)) == 256
     w = synth.WORKLOADS["hunyuan"]

@@ -31,6 +31,12 @@ EDGE = {
     "d64_q64_k64": synth.custom("d64_q64_k64", heads=2, head_dim=64, q_block=64, k_block=64,
                                 text_len=10, num_frames=2, latent_h=6, latent_w=10, top_p=0.6,
                                 pad_to=64, seed=14),                         # 130 -> 192
+    "d128_q64_k64": synth.custom("d128_q64_k64", heads=2, head_dim=128, q_block=64, k_block=64,
+                                 text_len=33, num_frames=3, latent_h=7, latent_w=9, top_p=0.8,
+                                 pad_to=64, seed=16),                        # 222 -> 256
+    "d64_q64_k128": synth.custom("d64_q64_k128", heads=2, head_dim=64, q_block=64, k_block=128,
+                                 text_len=70, num_frames=2, latent_h=10, latent_w=20, top_p=0.7,
+                                 seed=17),                                   # 470 -> 512
     "d64_q128_k64": synth.custom("d64_q128_k64", batch=2, heads=2, head_dim=64, q_block=128,
                                  k_block=64, text_len=0, num_frames=5, latent_h=9, latent_w=22,
                                  top_p=0.7, seed=15, kind="clustered"),      # 990 -> 1024
@@ -52,7 +58,9 @@ def _attn_vs_oracle(w, x, xd, mask, idx, cnt, what):
     cq = w.seq_pad // w.q_block
     og = to_host_f32(out).reshape(o_ora.shape)
     lg = lse.cpu().numpy().reshape(l_ora.shape)
-    checkers.check_attention(og, o_ora, lg, l_ora, what=what)
+    vmax = np.abs(synth.bf16_bits_to_f32(x["v"])).max()
+    checkers.check_attention(og, o_ora, lg, l_ora, what=what,
+                             max_abs=checkers.bf16_output_bound(o_ora, vmax))
     return out, lse, int(err.item())
 
 
@@ -68,7 +76,8 @@ def test_pipeline_edge_shapes(name):
     np.testing.assert_allclose(to_host_f32(kc), sel["k_centroids"], rtol=1e-5, atol=2e-6)
     assert np.abs(to_host_f32(probs) - sel["probs"]).max() <= 1e-4
     g0 = bsa.build_mask(w, torch.from_numpy(sel["probs"]).cuda(), tp, 0)
-    checkers.check_topp_masks(g0["mask"].cpu().numpy(), sel["topp_mask"], sel["probs"], tp)
+    checkers.check_topp_masks(g0["mask"].cpu().numpy(), sel["topp_mask"], sel["probs"], tp,
+                              same_probs=True)
     g = bsa.build_mask(w, torch.from_numpy(sel["probs"]).cuda(), tp, w.flags)
     m = g["mask"].cpu().numpy()
     assert np.array_equal(m, oracle.overrides(L, w.flags, g0["mask"].cpu().numpy()))
@@ -77,8 +86,10 @@ def test_pipeline_edge_shapes(name):
     _attn_vs_oracle(w, x, xd, sel["mask"], sel["kv_index"], sel["kv_count"], name)
     out, lse = bsa.dense_fwd(w, xd["q"], xd["k"], xd["v"])
     o_ora, l_ora = oracle.attention(L, x["q"], x["k"], x["v"], None)
+    vmax = np.abs(synth.bf16_bits_to_f32(x["v"])).max()
     checkers.check_attention(to_host_f32(out).reshape(o_ora.shape), o_ora,
-                             lse.cpu().numpy().reshape(l_ora.shape), l_ora, what=name + " dense")
+                             lse.cpu().numpy().reshape(l_ora.shape), l_ora, what=name + " dense",
+                             max_abs=checkers.bf16_output_bound(o_ora, vmax))
 
 
 def _lists_from_mask(mask):
@@ -144,7 +155,7 @@ def test_empty_rows_and_bad_entries():
     # a bad entry inside a gathered pair changes the pairing, so compare within tolerance
     a = out2[0, 1, 2 * w.q_block:3 * w.q_block].float()
     b = out[0, 1, 2 * w.q_block:3 * w.q_block].float()
-    assert (a - b).abs().max().item() <= checkers.MAX_ABS
+    assert (a - b).abs().max().item() <= 2 * checkers.MAX_ABS
     cnt3 = np.full_like(cnt, ck + 7)
     err.zero_()
     out3, _ = bsa.attention_fwd(w, xd["q"], xd["k"], xd["v"],
