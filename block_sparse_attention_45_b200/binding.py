@@ -61,6 +61,9 @@ def load():
         L.bsa_build_mask.argtypes = [lp, vp, vp, ctypes.c_uint32, ctypes.c_float, vp, vp, vp, vp,
                                      vp, vp, vp]
         L.bsa_build_mask.restype = ctypes.c_int
+        L.bsa_build_mask_noalloc.argtypes = [lp, vp, vp, ctypes.c_uint32, ctypes.c_float, vp, vp,
+                                             vp, vp, vp, vp]
+        L.bsa_build_mask_noalloc.restype = ctypes.c_int
         L.bsa_attention_fwd.argtypes = [lp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp, vp]
         L.bsa_attention_fwd.restype = ctypes.c_int
         L.bsa_attention_workspace_bytes.argtypes = [lp]

@@ -149,6 +149,30 @@ int bsa_build_mask(const bsa_layout *layout, const float *probs, const float *to
                    void *workspace, void *stream);
 
 /*
+ * bsa_build_mask without a workspace, for callers that cannot allocate device
+ * memory (a framework allocator or memory-planning pass, a process whose device
+ * memory is reserved up front, a plugin whose host owns every allocation).
+ * The pages have no counterpart: this is a deployment variant of
+ * bsa_build_mask, not a step of the method.
+ *
+ * Same arguments and results as bsa_build_mask minus `workspace`: the
+ * per-row entropies go to a fixed array inside the library (4 bytes per row,
+ * BSA_NOALLOC_MAX_MASK_ROWS rows, resident on every GPU that loads the
+ * library until the process exits).  Returns BSA_ERR_UNSUPPORTED when
+ * batch * heads * (seq_pad / q_block) exceeds BSA_NOALLOC_MAX_MASK_ROWS and
+ * BSA_ERR_LAUNCH if the array's device address cannot be obtained.  The call
+ * allocates and frees nothing.  All calls on a device share the array (it
+ * keeps the last call's contents; nothing in it needs clearing), so calls that
+ * overlap on the GPU race.  The first call on each device looks the array up
+ * (cudaGetSymbolAddress) with that device current; make it before any stream
+ * capture.
+ */
+#define BSA_NOALLOC_MAX_MASK_ROWS 262144
+int bsa_build_mask_noalloc(const bsa_layout *layout, const float *probs, const float *top_p,
+                           uint32_t flags, float eps, uint8_t *mask, int32_t *kv_index,
+                           int32_t *kv_count, float *entropy, float *entropy_norm, void *stream);
+
+/*
  * Block-sparse exact attention ("Attention matrix view ..." s2;
  * "AB-Attention ..." TL;DR).  For every valid query token t of query block i:
  *   U = tokens u < seq_len of the key blocks kv_index[b,h,i,0..kv_count-1]

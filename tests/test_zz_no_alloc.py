@@ -1,0 +1,85 @@
+"""bsa_build_mask_noalloc against bsa_build_mask (needs a B200).
+
+bsa_build_mask_noalloc exists for callers that cannot allocate device memory
+(a framework allocator or memory-planning pass, a process whose device memory
+is reserved up front, a plugin whose host owns every allocation) and so have no
+workspace to pass: it keeps the per-row entropies in an array inside the
+library.  These tests call it through the C ABI twice in a row, on two
+different geometries, and require the same masks, lists and entropies as the
+ordinary entry point given a workspace; and they check that a problem larger
+than the array is refused.
+
+This file is collected last on purpose; it works alone in a fresh process too.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_45_b200 import binding as bsa
+from block_sparse_attention_45_b200 import synth
+from tests import checkers
+
+pytestmark = pytest.mark.gpu
+
+
+def _probs(name):
+    w = synth.WORKLOADS[name]
+    x = synth.generate(w, ("q", "k"))
+    to = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)  # noqa: E731
+    _, _, probs = bsa.block_scores(w, to(x["q"]), to(x["k"]))
+    return w, probs
+
+
+def _noalloc(w, probs, top_p, flags):
+    L = bsa.make_layout(w)
+    B, H = w.batch, w.heads
+    cq, ck = w.seq_pad // w.q_block, w.seq_pad // w.k_block
+    dev = probs.device
+    mask = torch.full((B, H, cq, ck), 7, dtype=torch.uint8, device=dev)
+    idx = torch.full((B, H, cq, ck), -5, dtype=torch.int32, device=dev)
+    cnt = torch.full((B, H, cq), -5, dtype=torch.int32, device=dev)
+    ent = torch.full((B, H), float("nan"), dtype=torch.float32, device=dev)
+    entn = torch.full((B, H), float("nan"), dtype=torch.float32, device=dev)
+    tp = (ctypes.c_float * H)(*top_p)
+    rc = bsa.load().bsa_build_mask_noalloc(
+        ctypes.byref(L), ctypes.c_void_p(probs.data_ptr()), ctypes.cast(tp, ctypes.c_void_p),
+        flags, 1e-8, ctypes.c_void_p(mask.data_ptr()), ctypes.c_void_p(idx.data_ptr()),
+        ctypes.c_void_p(cnt.data_ptr()), ctypes.c_void_p(ent.data_ptr()),
+        ctypes.c_void_p(entn.data_ptr()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == bsa.BSA_OK, bsa.status_string(rc)
+    return dict(mask=mask, kv_index=idx, kv_count=cnt, entropy=ent, entropy_norm=entn)
+
+
+def _same(a, b):
+    torch.cuda.synchronize()
+    assert torch.equal(a["mask"], b["mask"])
+    assert torch.equal(a["kv_count"], b["kv_count"])
+    m = b["mask"].cpu().numpy()
+    checkers.check_lists(a["kv_index"].cpu().numpy(), a["kv_count"].cpu().numpy(), m)
+    for k in ("entropy", "entropy_norm"):
+        np.testing.assert_allclose(a[k].cpu().numpy(), b[k].cpu().numpy(),
+                                   rtol=checkers.ENTROPY_REL)
+
+
+def test_noalloc_matches_workspace_entry_point_twice():
+    # two calls in a row with different geometries: the second must not see the first's scratch
+    for name in ("small", "tiny"):
+        w, probs = _probs(name)
+        tp = [float(w.top_p)] * w.heads
+        ref = bsa.build_mask(w, probs, tp, w.flags)
+        got = _noalloc(w, probs, tp, w.flags)
+        _same(got, ref)
+
+
+def test_noalloc_rejects_problems_larger_than_its_array():
+    w = synth.WORKLOADS["hunyuan"]
+    d = w.layout()
+    d["batch"] = 12            # 12 * 24 * 931 rows > 262144
+    L = bsa.make_layout(d)
+    fake = ctypes.c_void_p(0x10000)
+    tp = (ctypes.c_float * w.heads)(*([0.9] * w.heads))
+    rc = bsa.load().bsa_build_mask_noalloc(ctypes.byref(L), fake, ctypes.cast(tp, ctypes.c_void_p),
+                                           3, 1e-8, None, fake, fake, fake, None, None)
+    assert rc == bsa.BSA_ERR_UNSUPPORTED
