@@ -24,7 +24,7 @@
 // products overlap item n's epilogue.  Every wait is bounded (see mbar_wait).
 //
 // Warp roles (12 warps):
-//   warp 0      TMA producer: Q per item, K into a 3-stage ring, V into a 2-stage ring
+//   warp 0      TMA producer: Q per item, K into a 2-stage ring, V into a 3-stage ring
 //   warp 1      tcgen05 issuer (one thread) and TMEM owner (512 columns)
 //   warps 4-7   softmax stream 0: list positions 0, 2, 4, ...
 //   warps 8-11  softmax stream 1: list positions 1, 3, 5, ...
@@ -69,6 +69,7 @@ constexpr uint32_t kRegsSoftmax = (168 * kThreads - kRegsControl * 128) / 256;
 static_assert(kRegsControl * 128 + kRegsSoftmax * 256 == 168 * kThreads, "register split");
 static_assert(kRegsControl % 8 == 0 && kRegsSoftmax % 8 == 0, "setmaxnreg takes multiples of 8");
 constexpr uint32_t kTmemCols = 512;
+// O is rescaled only when a row's max grows by more than 2^8 (P stays below 256).
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kPanelBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle panel)
 
@@ -76,8 +77,10 @@ template <int D>
 struct Cfg {
     static constexpr int kPanels = D / 64;
     static constexpr int kTileBytes = kPanels * kPanelBytes;  // 128 rows x D bf16
-    static constexpr int kStagesK = (D == 128) ? 3 : 4;
-    static constexpr int kStagesV = (D == 128) ? 2 : 4;
+    // K is released as soon as its QK^T product is done; V only after the PV product
+    // that follows the softmax, so V gets the deeper ring.
+    static constexpr int kStagesK = (D == 128) ? 2 : 4;
+    static constexpr int kStagesV = (D == 128) ? 3 : 4;
     static constexpr int kHeader = 1024;
     static constexpr int kOffStats = kHeader;  // [item parity][m, l][stream][row] floats: 4 KB
     static constexpr int kOffQ = kOffStats + 4096;
@@ -305,7 +308,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-            const uint32_t q_addr = smem_u32(sQ);
+            // Descriptor halves: the start address (>> 4) is in the low word, so every
+            // K-step below is a compile-time offset added to it.
+            const uint64_t q_desc = sw128_desc(smem_u32(sQ), 16, 1024);
+            const uint64_t k_desc0 = sw128_desc(smem_u32(sK), 16, 1024);
+            const uint64_t v_desc0 = sw128_desc(smem_u32(sV), kPanelBytes, 1024);
+            const uint32_t q_lo = static_cast<uint32_t>(q_desc);
+            const uint32_t kv_hi_k = static_cast<uint32_t>(k_desc0 >> 32);
+            const uint32_t kv_hi_v = static_cast<uint32_t>(v_desc0 >> 32);
+            const uint32_t q_hi = static_cast<uint32_t>(q_desc >> 32);
             int kt = 0, vt = 0, qn = 0, pc[2] = {0, 0};
             bool ok = true;
             for (; ok; ++qn) {
@@ -322,17 +333,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bool bad_count;
                 item_lists<BK>(p, item, entries, n_entries, n_tiles, bad_count);
                 // S_s(t) = Q K_t^T; frees the K stage, and Q once t is the item's last tile.
-                auto issue_s = [&](int t) -> bool {
+                auto issue_s = [&](int t, bool k_ready) -> bool {
                     const int ks = kt % NK;
-                    if (!mbar_wait(&hd.k_full[ks], (kt / NK) & 1, abort_flag)) return false;
+                    if (!k_ready && !mbar_wait(&hd.k_full[ks], (kt / NK) & 1, abort_flag))
+                        return false;
                     tc_fence_after();
-                    const uint32_t k_addr = smem_u32(sK + ks * C::kTileBytes);
+                    const uint32_t k_lo = static_cast<uint32_t>(k_desc0) +
+                                          static_cast<uint32_t>(ks * (C::kTileBytes >> 4));
                     const uint32_t d_tmem = tmem + static_cast<uint32_t>((t & 1) * 128);
+                    mma_ss_c<0>(d_tmem, q_lo, q_hi, k_lo, kv_hi_k, idesc_qk);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk / 4) * kPanelBytes + (kk % 4) * 32;
-                        mma_ss(d_tmem, sw128_desc(q_addr + off, 16, 1024),
-                               sw128_desc(k_addr + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                    for (int kk = 1; kk < D / 16; ++kk) {
+                        const uint32_t off = ((kk / 4) * kPanelBytes + (kk % 4) * 32) >> 4;
+                        mma_ss_c<1>(d_tmem, q_lo + off, q_hi, k_lo + off, kv_hi_k, idesc_qk);
                     }
                     mma_commit(&hd.k_empty[ks]);
                     mma_commit(&hd.s_full[t & 1]);
@@ -342,37 +355,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                 };
                 ok = mbar_wait(&hd.q_full, qn & 1, abort_flag);
                 if (ok && n_tiles == 0) mma_commit(&hd.q_empty);
-                if (ok && n_tiles > 0) ok = issue_s(0);
-                if (ok && n_tiles > 1) ok = issue_s(1);
+                if (ok && n_tiles > 0) ok = issue_s(0, false);
+                if (ok && n_tiles > 1) ok = issue_s(1, false);
                 // O_a / O_b still hold the previous item until its epilogue has read them.
                 // Waited for every item (even one without tiles) so that the wait never
                 // runs two phases ahead of the epilogues.
                 if (ok && qn > 0) ok = mbar_wait(&hd.o_free, (qn - 1) & 1, abort_flag);
                 for (int t = 0; ok && t < n_tiles; ++t) {
                     const int s = t & 1;
+                    // V(t) and K(t+2) normally landed long ago; checking them before P(t)
+                    // keeps those barrier round trips off the softmax -> PV path.
+                    const int vs = vt % NV;
+                    if (!mbar_wait(&hd.v_full[vs], (vt / NV) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (t + 2 < n_tiles &&
+                        !mbar_wait(&hd.k_full[kt % NK], (kt / NK) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     if (!mbar_wait(&hd.p_full[s], pc[s] & 1, abort_flag)) {
                         ok = false;
                         break;
                     }
                     ++pc[s];
                     tc_fence_after();
-                    const int vs = vt % NV;
-                    if (!mbar_wait(&hd.v_full[vs], (vt / NV) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t v_addr = smem_u32(sV + vs * C::kTileBytes);
+                    const uint32_t v_lo = static_cast<uint32_t>(v_desc0) +
+                                          static_cast<uint32_t>(vs * (C::kTileBytes >> 4));
                     const uint32_t o_tmem = tmem + 256u + static_cast<uint32_t>(s * 128);
                     const uint32_t p_tmem = tmem + static_cast<uint32_t>(s * 128);
+                    mma_ts_r(o_tmem, p_tmem, v_lo, kv_hi_v, idesc_pv, t >= 2 ? 1u : 0u);
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(o_tmem, p_tmem + kk * 8,
-                               sw128_desc(v_addr + kk * 2048, kPanelBytes, 1024), idesc_pv,
-                               (t >= 2 || kk > 0) ? 1u : 0u);
+                    for (int kk = 1; kk < 8; ++kk)
+                        mma_ts_r(o_tmem, p_tmem + kk * 8, v_lo + ((kk * 2048) >> 4), kv_hi_v,
+                                 idesc_pv, 1u);
                     mma_commit(&hd.v_empty[vs]);
                     ++vt;
-                    if (t + 2 < n_tiles && !issue_s(t + 2)) {
+                    if (t + 2 < n_tiles && !issue_s(t + 2, true)) {
                         ok = false;
                         break;
                     }
@@ -412,8 +432,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             item_lists<BK>(p, item, entries, n_entries, n_tiles, bad_count);
             const int n_s = (n_tiles > s) ? (n_tiles - s + 1) / 2 : 0;
             float m_run = -INFINITY, l_run = 0.f;
+            // The list entries of this stream's next tile are read one tile ahead
+            // (raw block indices; -1 = no block) so their latency is hidden.
+            int j_next0 = -1, j_next1 = -1;
+            if (n_s > 0) {
+                const int e0 = (BK == 128) ? s : 2 * s;
+                j_next0 = entries ? __ldg(entries + e0) : e0;
+                if (BK != 128 && e0 + 1 < n_entries) j_next1 = entries ? __ldg(entries + e0 + 1) : e0 + 1;
+            }
             for (int it = 0; ok && it < n_s; ++it) {
                 const int t = 2 * it + s;
+                const int j0 = j_next0, j1 = j_next1;
+                if (t + 2 < n_tiles) {
+                    const int e0 = (BK == 128) ? t + 2 : 2 * (t + 2);
+                    j_next0 = entries ? __ldg(entries + e0) : e0;
+                    j_next1 = -1;
+                    if (BK != 128 && e0 + 1 < n_entries)
+                        j_next1 = entries ? __ldg(entries + e0 + 1) : e0 + 1;
+                }
                 // tcgen05.ld/st below are warp-collective: leave together or not at all.
                 if (!__all_sync(0xffffffffu, mbar_wait(&hd.s_full[s], sc & 1, abort_flag))) {
                     ok = false;
@@ -421,66 +457,49 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ++sc;
                 tc_fence_after();
-                float x[128];
-                {
-                    uint32_t raw[4][32];
+                uint32_t raw[4][32];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, raw[c]);
-                    tmem_ld_wait();
+                for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, raw[c]);
+                tmem_ld_wait();
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        reg_fence(raw[c]);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(raw[c][e]);
-                    }
-                }
+                for (int c = 0; c < 4; ++c) reg_fence(raw[c]);
+#define X(i) (*reinterpret_cast<float *>(&raw[(i) >> 5][(i) & 31]))
                 // Mask key columns past seq_len, and missing / invalid halves.
                 int vc[kHalves];
+                vc[0] = (j0 >= 0 && j0 < p.Ck) ? min(BK, p.S - j0 * BK) : 0;
+                if (kHalves > 1) vc[kHalves - 1] = (j1 >= 0 && j1 < p.Ck) ? min(BK, p.S - j1 * BK) : 0;
                 bool partial = false;
 #pragma unroll
-                for (int hf = 0; hf < kHalves; ++hf) {
-                    int jl;
-                    bool bad;
-                    tile_block<BK>(p, entries, n_entries, t, hf, jl, vc[hf], bad);
-                    partial |= vc[hf] < BK;
-                }
+                for (int hf = 0; hf < kHalves; ++hf) partial |= vc[hf] < BK;
                 if (partial) {
 #pragma unroll
                     for (int c = 0; c < 128; ++c)
-                        if ((c % BK) >= vc[c / BK]) x[c] = -INFINITY;
+                        if ((c % BK) >= vc[c / BK]) X(c) = -INFINITY;
                 }
                 float mx;
                 {
                     float pm[4];
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        pm[k] = fmaxf(x[32 * k], x[32 * k + 1]);
+                        pm[k] = fmaxf(X(32 * k), X(32 * k + 1));
 #pragma unroll
-                        for (int e = 2; e < 32; e += 2) pm[k] = max3(pm[k], x[32 * k + e], x[32 * k + e + 1]);
+                        for (int e = 2; e < 32; e += 2) pm[k] = max3(pm[k], X(32 * k + e), X(32 * k + e + 1));
                     }
                     mx = fmaxf(max3(pm[0], pm[1], pm[2]), pm[3]);
                 }
                 const float m_new = fmaxf(m_run, mx * p.scale_log2);
+                // Raise the row's max lazily; O_s is rescaled below, after P is written
+                // (the S values are dead by then, so the O round trip has registers).
+                float alpha = 1.0f;
+                bool rescale = false;
                 if (it == 0) {
                     m_run = m_new;
                 } else {
                     const bool need = m_new > m_run + kRescaleLog2;
-                    if (__any_sync(0xffffffffu, need)) {
-                        const float alpha = need ? ex2(m_run - m_new) : 1.0f;
-#pragma unroll 1
-                        for (int c = 0; c < D / 16; ++c) {
-                            uint32_t o[16];
-                            tmem_ld16(t_o + c * 16, o);
-                            tmem_ld_wait();
-                            reg_fence(o);
-#pragma unroll
-                            for (int e = 0; e < 16; ++e)
-                                o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                            tmem_st16(t_o + c * 16, o);
-                        }
-                        tmem_st_wait();
-                        l_run *= alpha;
-                        if (need) m_run = m_new;
+                    rescale = __any_sync(0xffffffffu, need);
+                    if (need) {
+                        alpha = ex2(m_run - m_new);
+                        m_run = m_new;
                     }
                 }
                 const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
@@ -492,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         float t0, t1, p0, p1;
-                        fma2(t0, t1, x[c * 32 + 2 * e], x[c * 32 + 2 * e + 1], sl, sl, nm, nm);
+                        fma2(t0, t1, X(c * 32 + 2 * e), X(c * 32 + 2 * e + 1), sl, sl, nm, nm);
                         if (c == 3) {
                             exp2_poly2(t0, t1, p0, p1);  // columns 96..127 on the FMA pipe
                         } else {
@@ -505,7 +524,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tmem_st16(t_s + c * 16, pk);
                 }
-                l_run += (a0 + a1) + (b0 + b1);
+                l_run = l_run * alpha + ((a0 + a1) + (b0 + b1));
+#undef X
+                if (rescale) {  // O_s *= alpha; PV(t) waits for p_full below, so no race
+                    uint32_t o[D / 32][32];
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) tmem_ld32(t_o + c * 32, o[c]);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        reg_fence(o[c]);
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            float y0, y1;
+                            fma2(y0, y1, __uint_as_float(o[c][e]), __uint_as_float(o[c][e + 1]), alpha,
+                                 alpha, 0.f, 0.f);
+                            o[c][e] = __float_as_uint(y0);
+                            o[c][e + 1] = __float_as_uint(y1);
+                        }
+                        tmem_st32(t_o + c * 32, o[c]);
+                    }
+                }
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&hd.p_full[s]);
