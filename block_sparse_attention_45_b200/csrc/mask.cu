@@ -8,14 +8,16 @@
 // s7: text/global key blocks are always kept.
 //
 // One warp per row; element j of the row lives in lane j % 32, slot j / 32.
-// Top-p without sorting: P' >= 0, so the fp32 bit patterns order like the
-// values.  With f(u) = sum of the values whose pattern is >= u (a step
-// function, non-increasing in u), the cut value v* is the largest pattern u*
-// with f(u*) >= p, found by bisection on u; the row keeps every value above
-// v* plus, among the entries equal to v*, the lowest-index ones needed for the
-// running sum to reach p -- the same set as sorting by (P' desc, j asc) and
-// taking the shortest prefix whose sum reaches p.  Row entropies go to a
-// workspace; a second kernel sums them per head in a fixed order.
+// Top-p without sorting: P' >= 0, so fp32 bit patterns order like the values.
+// Stage A bisects on the exponent field, with fp64 sums, for the binade that
+// holds the cut (the largest e with mass(exponent >= e) >= p); Stage B gathers
+// that binade's entries into shared memory and keeps entry m iff it is the
+// first of the (P' desc, j asc) order or the fp64 mass strictly before it is
+// below p -- the shortest prefix of the sorted row whose running sum reaches p
+// (at least one entry, also for p <= 0).  Rows whose binade holds more than
+// kCandMax entries fall back to an fp64 bisection on the full bit pattern
+// inside that binade.  Row entropies go to a workspace; a second kernel sums them
+// per head in a fixed order.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -51,10 +53,152 @@ __device__ __forceinline__ int warp_sum_i(int v) {
     return v;
 }
 
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ uint64_t warp_min_u64(uint64_t v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t w = __shfl_xor_sync(0xffffffffu, v, o);
+        v = w < v ? w : v;
+    }
+    return v;
+}
+
+// Candidates of the cut binade kept in shared memory per warp.
+constexpr int kCandMax = 128;
+
+// Row (b,h,i) keeps every entry whose key (P' bits, -j) is at least (ucut, -jcut):
+// u > ucut, or u == ucut and j <= jcut -- the shortest prefix of the (P' desc,
+// j asc) order whose running sum reaches p.
+template <int VPL>
+__device__ __forceinline__ void find_cut(const float (&v)[VPL], int Ck,
+                                         float p, uint32_t umax, int lane, float *cv, int *cj,
+                                         uint32_t &ucut, int &jcut) {
+    // Stage A: the binade (fp32 exponent field) that holds the cut: the largest e
+    // with mass(exponent >= e) >= p, by bisection on e with fp64 sums (fp32 sums
+    // cannot tell 1 - 2^-30 from 1 when p is close to the row total).
+#define U(s) __float_as_uint(v[s])
+    const double pd = static_cast<double>(p);
+    uint32_t lo = 0, hi = umax >> 23;
+    while (lo < hi) {
+        const uint32_t mid = lo + ((hi - lo + 1) >> 1);
+        const uint32_t thr = mid << 23;
+        double f = 0.0;
+#pragma unroll
+        for (int s = 0; s < VPL; ++s) f += (U(s) >= thr) ? static_cast<double>(v[s]) : 0.0;
+        if (warp_sum_d(f) >= pd) lo = mid;
+        else hi = mid - 1;
+    }
+    const uint32_t e = lo;
+    double above = 0.0;
+    {
+        double a_l = 0.0;
+#pragma unroll
+        for (int s = 0; s < VPL; ++s) a_l += ((U(s) >> 23) > e) ? static_cast<double>(v[s]) : 0.0;
+        above = warp_sum_d(a_l);
+    }
+    // Stage B: the binade's entries, compacted in ascending j.
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    int c = 0;
+#pragma unroll
+    for (int s = 0; s < VPL; ++s) {
+        const int j = lane + 32 * s;
+        const bool is_c = j < Ck && (U(s) >> 23) == e;
+        const uint32_t bal = __ballot_sync(0xffffffffu, is_c);
+        const int pos = c + __popc(bal & lt_mask);
+        if (is_c && pos < kCandMax) {
+            cv[pos] = v[s];
+            cj[pos] = j;
+        }
+        c += __popc(bal);
+    }
+    __syncwarp();
+    if (c <= kCandMax) {
+        // Candidate m is kept iff the fp64 mass strictly before it in
+        // (P' desc, j asc) order is below p; the cut is the last kept one.
+        // The first entry of the order is always kept (k* >= 1, also for p <= 0).
+        uint64_t best = ~0ull;
+        for (int m = lane; m < c; m += 32) {
+            const float vm = cv[m];
+            const int jm = cj[m];
+            double before = above;
+            bool first = above == 0.0;
+            for (int n = 0; n < c; ++n) {
+                const float vn = cv[n];
+                if (vn > vm || (vn == vm && cj[n] < jm)) {
+                    before += static_cast<double>(vn);
+                    first = false;
+                }
+            }
+            if (before < pd || first) {
+                const uint64_t key = (static_cast<uint64_t>(__float_as_uint(vm)) << 32) |
+                                     (0xFFFFFFFFu - static_cast<uint32_t>(jm));
+                best = key < best ? key : best;
+            }
+        }
+        best = warp_min_u64(best);
+        ucut = static_cast<uint32_t>(best >> 32);
+        jcut = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(best));
+        return;
+    }
+    // A binade with more than kCandMax entries (nearly flat rows): bisection on
+    // the full bit pattern, then ties at the cut value in ascending j.
+    uint32_t lo2 = e << 23, hi2 = min(umax, (e << 23) | 0x7FFFFFu);
+    while (lo2 < hi2) {
+        const uint32_t mid = lo2 + ((hi2 - lo2 + 1) >> 1);
+        double f = 0.0;
+#pragma unroll
+        for (int s = 0; s < VPL; ++s) f += (U(s) >= mid) ? static_cast<double>(v[s]) : 0.0;
+        if (warp_sum_d(f) >= pd) lo2 = mid;
+        else hi2 = mid - 1;
+    }
+    ucut = lo2;
+    double abv = 0.0;
+    int ties = 0;
+#pragma unroll
+    for (int s = 0; s < VPL; ++s) {
+        abv += (U(s) > ucut) ? static_cast<double>(v[s]) : 0.0;
+        ties += (U(s) == ucut && lane + 32 * s < Ck) ? 1 : 0;
+    }
+    abv = warp_sum_d(abv);
+    ties = warp_sum_i(ties);
+    const double vcut = static_cast<double>(__uint_as_float(ucut));
+    int need = 1;
+    double run = abv + vcut;
+    while (run < pd && need < ties) {
+        run += vcut;
+        ++need;
+    }
+    // jcut = index of the need-th tie in ascending j
+    int seen = 0;
+    jcut = -1;
+#pragma unroll
+    for (int s = 0; s < VPL; ++s) {
+        const int j = lane + 32 * s;
+        const bool is_t = j < Ck && U(s) == ucut;
+        const uint32_t bal = __ballot_sync(0xffffffffu, is_t);
+        const int cnt = __popc(bal);
+        if (jcut < 0 && seen + cnt >= need) {
+            // the (need - seen)-th set bit of bal
+            uint32_t b = bal;
+            for (int k = 1; k < need - seen; ++k) b &= b - 1;
+            jcut = 32 * s + __ffs(b) - 1;
+        }
+        seen += cnt;
+    }
+#undef U
+}
+
 template <int VPL>
 __global__ void __launch_bounds__(256) mask_kernel(MaskArgs a, TopP tp) {
-    const int lane = threadIdx.x % 32;
-    const long long row = static_cast<long long>(blockIdx.x) * 8 + threadIdx.x / 32;
+    __shared__ float s_cv[8][kCandMax];
+    __shared__ int s_cj[8][kCandMax];
+    const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
+    const long long row = static_cast<long long>(blockIdx.x) * 8 + wid;
     if (row >= a.rows) return;  // whole warp leaves together
     const int Ck = a.Ck;
     const int i = static_cast<int>(row % a.Cq);
@@ -63,8 +207,8 @@ __global__ void __launch_bounds__(256) mask_kernel(MaskArgs a, TopP tp) {
     const float *src = a.probs + row * Ck;
 
     float v[VPL];
-    uint32_t u[VPL];
-    float ent = 0.f, total = 0.f;
+    float ent = 0.f;
+    double total = 0.0;
     uint32_t umax = 0;
 #pragma unroll
     for (int s = 0; s < VPL; ++s) {
@@ -72,12 +216,11 @@ __global__ void __launch_bounds__(256) mask_kernel(MaskArgs a, TopP tp) {
         float x = (j < Ck) ? __ldg(src + j) : 0.f;
         x = fmaxf(x, 0.f);
         v[s] = x;
-        u[s] = __float_as_uint(x);
-        umax = max(umax, u[s]);
-        total += x;
-        if (j < Ck) ent -= x * logf(x + a.eps);
+        umax = max(umax, __float_as_uint(x));
+        total += static_cast<double>(x);
+        if (j < Ck) ent -= x * __logf(x + a.eps);
     }
-    total = warp_sum(total);
+    total = warp_sum_d(total);
     if (a.row_entropy) {
         ent = warp_sum(ent);
         if (lane == 0) a.row_entropy[row] = ent;
@@ -85,54 +228,24 @@ __global__ void __launch_bounds__(256) mask_kernel(MaskArgs a, TopP tp) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) umax = max(umax, __shfl_xor_sync(0xffffffffu, umax, o));
 
-    bool keep_all = !(total >= p);  // the row never reaches p: keep everything
+    // fp64 totals, like the running sum of the rule: the row never reaches p -> keep it all
+    const bool keep_all = !(total >= static_cast<double>(p));
     uint32_t ucut = 0;
-    int ties_needed = 0;
-    if (!keep_all) {
-        uint32_t lo = 0, hi = umax;  // invariant: f(lo) >= p
-        while (lo < hi) {
-            const uint32_t mid = lo + ((hi - lo + 1) >> 1);
-            float f = 0.f;
-#pragma unroll
-            for (int s = 0; s < VPL; ++s) f += (u[s] >= mid) ? v[s] : 0.f;
-            f = warp_sum(f);
-            if (f >= p) lo = mid;
-            else hi = mid - 1;
-        }
-        ucut = lo;
-        float above = 0.f;
-        int ties = 0;
-#pragma unroll
-        for (int s = 0; s < VPL; ++s) {
-            above += (u[s] > ucut) ? v[s] : 0.f;
-            ties += (u[s] == ucut && lane + 32 * s < Ck) ? 1 : 0;
-        }
-        above = warp_sum(above);
-        ties = warp_sum_i(ties);
-        const float vcut = __uint_as_float(ucut);
-        float run = above + vcut;
-        ties_needed = 1;
-        while (run < p && ties_needed < ties) {
-            run += vcut;
-            ++ties_needed;
-        }
-    }
+    int jcut = 0x7FFFFFFF;
+    if (!keep_all) find_cut<VPL>(v, Ck, p, umax, lane, s_cv[wid], s_cj[wid], ucut, jcut);
 
     const bool dense_row = (a.flags & BSA_FRAME0_DENSE) && i >= a.f0_first && i <= a.f0_last;
     const bool text = (a.flags & BSA_TEXT_KEEP) != 0;
     uint8_t *mrow = a.mask ? a.mask + row * Ck : nullptr;
     int32_t *irow = a.kv_index + row * Ck;
     const uint32_t lt_mask = (1u << lane) - 1u;
-    int base = 0, tie_base = 0;
+    int base = 0;
 #pragma unroll
     for (int s = 0; s < VPL; ++s) {
         const int j = lane + 32 * s;
         const bool valid = j < Ck;
-        const bool is_tie = valid && !keep_all && u[s] == ucut;
-        const uint32_t tie_bal = __ballot_sync(0xffffffffu, is_tie);
-        const int tie_rank = tie_base + __popc(tie_bal & lt_mask);
-        tie_base += __popc(tie_bal);
-        bool sel = keep_all || u[s] > ucut || (is_tie && tie_rank < ties_needed);
+        const uint32_t us = __float_as_uint(v[s]);
+        bool sel = keep_all || us > ucut || (us == ucut && j <= jcut);
         sel = valid && (sel || dense_row || (text && j < a.text_kblocks));
         if (mrow && valid) mrow[j] = sel ? 1 : 0;
         const uint32_t bal = __ballot_sync(0xffffffffu, sel);

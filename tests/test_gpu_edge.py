@@ -184,3 +184,52 @@ def test_padding_rows_are_ignored_and_zeroed():
     assert (out[:, :, S:] == 0).all()
     assert torch.isneginf(lse[:, :, S:]).all()
     assert torch.equal(lse[:, :, :S], ref_lse[:, :, :S])
+
+
+def _crafted_probs(rng, rows, ck):
+    """P' rows that exercise every branch of the GPU cut search."""
+    out = []
+    for r in range(rows):
+        kind = r % 8
+        if kind == 0:                                    # generic
+            x = rng.dirichlet(np.full(ck, 0.3))
+        elif kind == 1:                                  # flat: one binade holds every entry
+            x = np.full(ck, 1.0 / ck)
+        elif kind == 2:                                  # flat with noise inside one binade
+            x = (1.0 + 0.5 * rng.random(ck)) / ck
+        elif kind == 3:                                  # many exact ties at the cut
+            x = np.full(ck, 0.25 / ck)
+            x[rng.choice(ck, 5, replace=False)] = 0.15
+        elif kind == 4:                                  # very peaked with tiny tail values
+            x = rng.random(ck) ** 12
+            x[rng.integers(ck)] = 50.0
+        elif kind == 5:                                  # two-level
+            x = np.where(rng.random(ck) < 0.1, 1.0, 1e-3)
+        elif kind == 6:                                  # some exact zeros
+            x = rng.dirichlet(np.full(ck, 0.5))
+            x[rng.random(ck) < 0.3] = 0.0
+        else:                                            # a few equal maxima
+            x = rng.random(ck) * 0.1
+            x[:3] = 1.0
+        x = np.asarray(x, np.float64)
+        out.append((x / x.sum()).astype(np.float32))
+    return np.stack(out)
+
+
+@pytest.mark.parametrize("ck_blocks", [5, 64, 300, 931])
+def test_topp_crafted_rows_exact(ck_blocks):
+    """On identical fp32 P' the GPU top-p must equal the oracle's row for row:
+    both sum in fp64 in the same order-independent way at the cut."""
+    rng = np.random.default_rng(ck_blocks)
+    L = dict(batch=1, heads=4, seq_len=ck_blocks * 128, seq_pad=ck_blocks * 128, head_dim=128,
+             q_block=128, k_block=128, text_len=0, tokens_per_frame=0, num_frames=0)
+    cq = L["seq_pad"] // L["q_block"]
+    probs = _crafted_probs(rng, 4 * cq, ck_blocks).reshape(1, 4, cq, ck_blocks)
+    for tp in ([0.5, 0.9, 0.99, 0.999999], [1e-9, 0.3, 1.0, 2.0], [-1.0, 0.7, 0.75, 0.8]):
+        m_ora, _ = oracle.topp(L, probs, tp)
+        g = bsa.build_mask(L, torch.from_numpy(probs).cuda(), tp, 0)
+        torch.cuda.synchronize()
+        got = g["mask"].cpu().numpy()
+        bad = np.argwhere((got != m_ora).any(-1))
+        assert bad.size == 0, (tp, bad[:5].tolist())
+        checkers.check_lists(g["kv_index"].cpu().numpy(), g["kv_count"].cpu().numpy(), got)
