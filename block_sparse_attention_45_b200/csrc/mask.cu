@@ -8,16 +8,16 @@
 // s7: text/global key blocks are always kept.
 //
 // One warp per row; element j of the row lives in lane j % 32, slot j / 32.
-// Top-p without sorting: P' >= 0, so fp32 bit patterns order like the values.
-// Stage A bisects on the exponent field, with fp64 sums, for the binade that
-// holds the cut (the largest e with mass(exponent >= e) >= p); Stage B gathers
-// that binade's entries into shared memory and keeps entry m iff it is the
-// first of the (P' desc, j asc) order or the fp64 mass strictly before it is
-// below p -- the shortest prefix of the sorted row whose running sum reaches p
-// (at least one entry, also for p <= 0).  Rows whose binade holds more than
-// kCandMax entries fall back to an fp64 bisection on the full bit pattern
-// inside that binade.  Row entropies go to a workspace; a second kernel sums them
-// per head in a fixed order.
+// Top-p without sorting: P' >= 0, so fp32 bit patterns order like the values,
+// and the kept set is every entry whose key (bits, -j) is at least the cut's.
+// The cut is found by an exact radix selection (below): histograms of integer
+// significand sums pick the binade, then 5 mantissa bits at a time, until at
+// most 32 candidates remain; candidate m is kept iff it is the first of the
+// (P' desc, j asc) order or the mass strictly before it is below p -- the
+// shortest prefix of the sorted row whose running sum reaches p (at least one
+// entry, also for p <= 0).  Masses inside one binade are exact integers; the
+// binades above it are summed in fp64.  Row entropies go to a workspace; a
+// second kernel sums them per head in a fixed order.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -68,137 +68,336 @@ __device__ __forceinline__ uint64_t warp_min_u64(uint64_t v) {
     return v;
 }
 
-// Candidates of the cut binade kept in shared memory per warp.
-constexpr int kCandMax = 128;
+// ---------------------------------------------------------------------------
+// Exact radix selection of the cut.
+//
+// Keys order like (P' desc, j asc).  Level 1 histograms the fp32 exponent
+// field over the 31 binades below the row's largest one (binade r holds the
+// entries whose exponent is emax - r; everything further down lands in row 31,
+// the underflow bin); the later levels histogram 5 mantissa bits at a time
+// inside the chosen range, until at most 32 entries remain.  Each lane owns one
+// column of a 32 x 32 table in shared memory and adds (1 << 40 | mantissa) of
+// its own entries to it; the implicit leading bits are added per bin from the
+// count, so a bin holds the exact integer sum of its entries' significands.
+// Within one binade masses are integers times one power of two, so every
+// prefix below the level-1 split is exact.  Row r of the table is the r-th bin
+// in descending order; lane r sums row r and the warp scans the rows.
+//
+// Padding slots (j >= Ck) hold +0.0, which has exponent field 0 and mantissa 0:
+// they add no mass, and their count is taken off the one bin they fall in.
+constexpr int kLanes = 32;
+constexpr uint64_t kCountOne = 1ull << 40;
+constexpr uint64_t kSigMask = kCountOne - 1;
+constexpr uint64_t kImplicit = 1ull << 23;
 
-// Row (b,h,i) keeps every entry whose key (P' bits, -j) is at least (ucut, -jcut):
-// u > ucut, or u == ucut and j <= jcut -- the shortest prefix of the (P' desc,
-// j asc) order whose running sum reaches p.
+struct WarpScratch {
+    unsigned long long bins[32][kLanes];  // [row][lane]
+    uint32_t cand_u[32];
+    int cand_j[32];
+};
+
+__device__ __forceinline__ uint32_t significand(uint32_t u) {
+    return (u & 0x7FFFFFu) | ((u >> 23) ? 0x800000u : 0u);
+}
+
+// 2^(max(e, 1) - 150): the weight of one significand unit in binade e.
+__device__ __forceinline__ double unit_of_binade(uint32_t e) {
+    const int k = static_cast<int>(e > 1u ? e : 1u) - 150;
+    return __longlong_as_double(static_cast<long long>(k + 1023) << 52);
+}
+
+// Lane r returns the sum of row r and clears it.  Quarter-warps read 8
+// distinct bank groups thanks to the rotation.
+__device__ __forceinline__ unsigned long long bin_row_sum(unsigned long long (*bins)[kLanes],
+                                                         int lane) {
+    ulonglong2 *row = reinterpret_cast<ulonglong2 *>(bins[lane]);
+    unsigned long long acc = 0;
+#pragma unroll
+    for (int k = 0; k < kLanes / 2; ++k) {
+        const int kk = (k + lane) & (kLanes / 2 - 1);
+        const ulonglong2 x = row[kk];
+        acc += x.x + x.y;
+        row[kk] = make_ulonglong2(0ull, 0ull);
+    }
+    return acc;
+}
+
+__device__ __forceinline__ unsigned long long scan_incl_u64(unsigned long long x, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long t = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += t;
+    }
+    return x;
+}
+
+__device__ __forceinline__ double scan_incl_d(double x, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double t = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += t;
+    }
+    return x;
+}
+
+// The row of the cut: the first non-empty row whose inclusive mass reaches p,
+// else (rounding left the whole range short of p) the last non-empty row.
+__device__ __forceinline__ int pick_row(bool nonempty, bool reaches) {
+    const uint32_t hit = __ballot_sync(0xffffffffu, nonempty && reaches);
+    if (hit) return __ffs(hit) - 1;
+    const uint32_t ne = __ballot_sync(0xffffffffu, nonempty);
+    return ne ? 31 - __clz(ne) : 0;
+}
+
+// j of the n-th (1-based) entry with bit pattern uc, in ascending j.
 template <int VPL>
-__device__ __forceinline__ void find_cut(const float (&v)[VPL], int Ck,
-                                         float p, uint32_t umax, int lane, float *cv, int *cj,
-                                         uint32_t &ucut, int &jcut) {
-    // Stage A: the binade (fp32 exponent field) that holds the cut: the largest e
-    // with mass(exponent >= e) >= p, by bisection on e with fp64 sums (fp32 sums
-    // cannot tell 1 - 2^-30 from 1 when p is close to the row total).
-#define U(s) __float_as_uint(v[s])
-    const double pd = static_cast<double>(p);
-    uint32_t lo = 0, hi = umax >> 23;
-    while (lo < hi) {
-        const uint32_t mid = lo + ((hi - lo + 1) >> 1);
-        const uint32_t thr = mid << 23;
-        double f = 0.0;
-#pragma unroll
-        for (int s = 0; s < VPL; ++s) f += (U(s) >= thr) ? static_cast<double>(v[s]) : 0.0;
-        if (warp_sum_d(f) >= pd) lo = mid;
-        else hi = mid - 1;
-    }
-    const uint32_t e = lo;
-    double above = 0.0;
-    {
-        double a_l = 0.0;
-#pragma unroll
-        for (int s = 0; s < VPL; ++s) a_l += ((U(s) >> 23) > e) ? static_cast<double>(v[s]) : 0.0;
-        above = warp_sum_d(a_l);
-    }
-    // Stage B: the binade's entries, compacted in ascending j.
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    int c = 0;
+__device__ __forceinline__ int nth_tie(const float (&v)[VPL], int Ck, uint32_t uc, int n, int lane) {
+    int seen = 0, jc = -1;
 #pragma unroll
     for (int s = 0; s < VPL; ++s) {
-        const int j = lane + 32 * s;
-        const bool is_c = j < Ck && (U(s) >> 23) == e;
-        const uint32_t bal = __ballot_sync(0xffffffffu, is_c);
-        const int pos = c + __popc(bal & lt_mask);
-        if (is_c && pos < kCandMax) {
-            cv[pos] = v[s];
-            cj[pos] = j;
-        }
-        c += __popc(bal);
-    }
-    __syncwarp();
-    if (c <= kCandMax) {
-        // Candidate m is kept iff the fp64 mass strictly before it in
-        // (P' desc, j asc) order is below p; the cut is the last kept one.
-        // The first entry of the order is always kept (k* >= 1, also for p <= 0).
-        uint64_t best = ~0ull;
-        for (int m = lane; m < c; m += 32) {
-            const float vm = cv[m];
-            const int jm = cj[m];
-            double before = above;
-            bool first = above == 0.0;
-            for (int n = 0; n < c; ++n) {
-                const float vn = cv[n];
-                if (vn > vm || (vn == vm && cj[n] < jm)) {
-                    before += static_cast<double>(vn);
-                    first = false;
-                }
-            }
-            if (before < pd || first) {
-                const uint64_t key = (static_cast<uint64_t>(__float_as_uint(vm)) << 32) |
-                                     (0xFFFFFFFFu - static_cast<uint32_t>(jm));
-                best = key < best ? key : best;
-            }
-        }
-        best = warp_min_u64(best);
-        ucut = static_cast<uint32_t>(best >> 32);
-        jcut = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(best));
-        return;
-    }
-    // A binade with more than kCandMax entries (nearly flat rows): bisection on
-    // the full bit pattern, then ties at the cut value in ascending j.
-    uint32_t lo2 = e << 23, hi2 = min(umax, (e << 23) | 0x7FFFFFu);
-    while (lo2 < hi2) {
-        const uint32_t mid = lo2 + ((hi2 - lo2 + 1) >> 1);
-        double f = 0.0;
-#pragma unroll
-        for (int s = 0; s < VPL; ++s) f += (U(s) >= mid) ? static_cast<double>(v[s]) : 0.0;
-        if (warp_sum_d(f) >= pd) lo2 = mid;
-        else hi2 = mid - 1;
-    }
-    ucut = lo2;
-    double abv = 0.0;
-    int ties = 0;
-#pragma unroll
-    for (int s = 0; s < VPL; ++s) {
-        abv += (U(s) > ucut) ? static_cast<double>(v[s]) : 0.0;
-        ties += (U(s) == ucut && lane + 32 * s < Ck) ? 1 : 0;
-    }
-    abv = warp_sum_d(abv);
-    ties = warp_sum_i(ties);
-    const double vcut = static_cast<double>(__uint_as_float(ucut));
-    int need = 1;
-    double run = abv + vcut;
-    while (run < pd && need < ties) {
-        run += vcut;
-        ++need;
-    }
-    // jcut = index of the need-th tie in ascending j
-    int seen = 0;
-    jcut = -1;
-#pragma unroll
-    for (int s = 0; s < VPL; ++s) {
-        const int j = lane + 32 * s;
-        const bool is_t = j < Ck && U(s) == ucut;
+        const bool is_t = lane + 32 * s < Ck && __float_as_uint(v[s]) == uc;
         const uint32_t bal = __ballot_sync(0xffffffffu, is_t);
         const int cnt = __popc(bal);
-        if (jcut < 0 && seen + cnt >= need) {
-            // the (need - seen)-th set bit of bal
+        if (jc < 0 && seen + cnt >= n) {
             uint32_t b = bal;
-            for (int k = 1; k < need - seen; ++k) b &= b - 1;
-            jcut = 32 * s + __ffs(b) - 1;
+            for (int k = 1; k < n - seen; ++k) b &= b - 1;
+            jc = 32 * s + __ffs(b) - 1;
         }
         seen += cnt;
     }
-#undef U
+    return jc;
+}
+
+// Bit pattern of max(y, +0.0), NaN -> +0.0: the value every pass works on.
+__device__ __forceinline__ uint32_t pos_bits(float y) { return __float_as_uint(y > 0.f ? y : 0.f); }
+
+// fp64 mass of the row's entries with bit pattern in [lo_u, hi_u].
+__device__ __noinline__ double mass_between(const float *__restrict__ src, int Ck, uint32_t lo_u,
+                                            uint32_t hi_u, int lane) {
+    double f = 0.0;
+    for (int j = lane; j < Ck; j += 32) {
+        const float y = __ldg(src + j);
+        const float x = y > 0.f ? y : 0.f;
+        const uint32_t u = __float_as_uint(x);
+        if (u >= lo_u && u <= hi_u) f += static_cast<double>(x);
+    }
+    return warp_sum_d(f);
+}
+
+// Cut inside the underflow range u <= hi (entries 31 or more binades below the
+// row maximum), given that the row reaches p only there: fp64 bisection on the
+// bit pattern, then ties in ascending j.  Reached only when p lies within about
+// 2^-30 of the row total, so it re-reads the row from global memory instead of
+// holding fp64 copies in registers.
+__device__ __noinline__ void cut_in_underflow(const float *__restrict__ src, int Ck, double pd,
+                                              double above, uint32_t hi, int lane,
+                                              uint32_t *ucut_out, int *jcut_out) {
+    uint32_t lo = 0, top = hi;
+    while (lo < top) {
+        const uint32_t mid = lo + ((top - lo + 1) >> 1);
+        if (above + mass_between(src, Ck, mid, hi, lane) >= pd) lo = mid;
+        else top = mid - 1;
+    }
+    const uint32_t uc = lo;
+    const double abv = uc < hi ? above + mass_between(src, Ck, uc + 1, hi, lane) : above;
+    int ties = 0;
+    for (int j = lane; j < Ck; j += 32) ties += pos_bits(__ldg(src + j)) == uc;
+    ties = warp_sum_i(ties);
+    const double vc = static_cast<double>(__uint_as_float(uc));
+    int need = 1;
+    double run = abv + vc;
+    while (run < pd && need < ties) {
+        run += vc;
+        ++need;
+    }
+    int seen = 0, jc = -1;
+    for (int j0 = 0; j0 < Ck; j0 += 32) {
+        const int j = j0 + lane;
+        const bool is_t = j < Ck && pos_bits(__ldg(src + j)) == uc;
+        const uint32_t bal = __ballot_sync(0xffffffffu, is_t);
+        const int cnt = __popc(bal);
+        if (jc < 0 && seen + cnt >= need) {
+            uint32_t b = bal;
+            for (int k = 1; k < need - seen; ++k) b &= b - 1;
+            jc = j0 + __ffs(b) - 1;
+        }
+        seen += cnt;
+    }
+    *ucut_out = uc;
+    *jcut_out = jc;
+}
+
+// Sets (ucut, jcut) so that the row keeps exactly the entries with u > ucut,
+// or u == ucut and j <= jcut; (0, INT_MAX) keeps the whole row (it never
+// reaches p).
+template <int VPL>
+__device__ __forceinline__ void find_cut(const float (&v)[VPL], const float *__restrict__ src,
+                                         int Ck, float p, uint32_t umax, int lane,
+                                         WarpScratch &ws, uint32_t &ucut, int &jcut) {
+    const double pd = static_cast<double>(p);
+    const uint32_t emax = umax >> 23;
+    const int npad = 32 * VPL - Ck;
+    // ---- level 1: binades emax .. emax-30 in rows 0..30, the rest in row 31
+#pragma unroll
+    for (int s = 0; s < VPL; ++s) {
+        const uint32_t u = __float_as_uint(v[s]);
+        const uint32_t r = min(emax - (u >> 23), 31u);
+        ws.bins[r][lane] += kCountOne | (u & 0x7FFFFFu);
+    }
+    __syncwarp();
+    const unsigned long long acc1 = bin_row_sum(ws.bins, lane);
+    __syncwarp();
+    const uint32_t pad_row = min(emax, 31u);
+    const int cnt_r = static_cast<int>(acc1 >> 40) - (lane == static_cast<int>(pad_row) ? npad : 0);
+    const uint32_t ex_r = emax - static_cast<uint32_t>(lane);  // exponent field of row `lane`
+    double mass_r = 0.0;
+    if (lane < 31 && lane <= static_cast<int>(emax)) {
+        const unsigned long long sig = (acc1 & kSigMask) +
+            (ex_r > 0u ? kImplicit * static_cast<unsigned long long>(cnt_r) : 0ull);
+        mass_r = static_cast<double>(sig) * unit_of_binade(ex_r);
+    }
+    const double incl = scan_incl_d(mass_r, lane);  // row 31 adds nothing here
+    const int cincl = static_cast<int>(scan_incl_u64(static_cast<unsigned long long>(cnt_r), lane));
+    double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) excl = 0.0;
+    const uint32_t hit = __ballot_sync(0xffffffffu, lane < 31 && cnt_r > 0 && incl >= pd);
+    if (!hit) {
+        // Binades emax..emax-30 do not reach p: the row total decides.
+        const double head = __shfl_sync(0xffffffffu, incl, 31);
+        const int n_under = __shfl_sync(0xffffffffu, cnt_r, 31);
+        const double tail = n_under > 0 ? mass_between(src, Ck, 0u, ((emax - 30u) << 23) - 1u, lane)
+                                        : 0.0;
+        if (!(head + tail >= pd)) {
+            ucut = 0u;
+            jcut = 0x7FFFFFFF;
+            return;
+        }
+        // Reaching p needs the underflow entries (tail > 0 here).
+        cut_in_underflow(src, Ck, pd, head, ((emax - 30u) << 23) - 1u, lane, &ucut, &jcut);
+        return;
+    }
+    const int b = __ffs(hit) - 1;
+    const double above = __shfl_sync(0xffffffffu, excl, b);
+    int cnt_above = __shfl_sync(0xffffffffu, cincl - cnt_r, b);
+    int cnt = __shfl_sync(0xffffffffu, cnt_r, b);
+    // ---- mantissa levels inside binade e: candidates share (u >> sh) == pre
+    const uint32_t e = emax - static_cast<uint32_t>(b);
+    const double unit = unit_of_binade(e);
+    const unsigned long long implicit = e > 0u ? kImplicit : 0ull;
+    bool pad_in = e == 0u;           // padding (+0.0) still inside the range
+    unsigned long long s_above = 0;  // significands of the binade's entries above the range
+    uint32_t pre = e;
+    int sh = 23;
+    while (cnt > 32 && sh > 0) {
+        const int w = sh >= 5 ? 5 : sh;
+        sh -= w;
+        const uint32_t top = (1u << w) - 1u;
+#pragma unroll
+        for (int s = 0; s < VPL; ++s) {
+            const uint32_t u = __float_as_uint(v[s]);
+            if ((u >> (sh + w)) == pre)
+                ws.bins[top - ((u >> sh) & top)][lane] += kCountOne | (u & 0x7FFFFFu);
+        }
+        __syncwarp();
+        const unsigned long long acc = bin_row_sum(ws.bins, lane);
+        __syncwarp();
+        const int c_r = static_cast<int>(acc >> 40) -
+                        (pad_in && lane == static_cast<int>(top) ? npad : 0);
+        const unsigned long long sg_r = (acc & kSigMask) +
+                                        implicit * static_cast<unsigned long long>(c_r);
+        const unsigned long long sg_incl = scan_incl_u64(sg_r, lane);
+        const int c_incl = static_cast<int>(scan_incl_u64(static_cast<unsigned long long>(c_r), lane));
+        const bool reaches = above + static_cast<double>(s_above + sg_incl) * unit >= pd;
+        const int r = pick_row(c_r > 0, reaches);
+        s_above += __shfl_sync(0xffffffffu, sg_incl - sg_r, r);
+        cnt_above += __shfl_sync(0xffffffffu, c_incl - c_r, r);
+        cnt = __shfl_sync(0xffffffffu, c_r, r);
+        pad_in = pad_in && r == static_cast<int>(top);
+        pre = (pre << w) | (top - static_cast<uint32_t>(r));
+    }
+    if (cnt <= 32) {
+        // ---- at most 32 candidates: each one knows the exact mass before it
+        const uint32_t lt_mask = (1u << lane) - 1u;
+        int c = 0;
+#pragma unroll
+        for (int s = 0; s < VPL; ++s) {
+            const uint32_t u = __float_as_uint(v[s]);
+            const int j = lane + 32 * s;
+            const bool is_c = (u >> sh) == pre && j < Ck;
+            const uint32_t bal = __ballot_sync(0xffffffffu, is_c);
+            if (is_c) {
+                const int pos = c + __popc(bal & lt_mask);
+                ws.cand_u[pos] = u;
+                ws.cand_j[pos] = j;
+            }
+            c += __popc(bal);
+        }
+        __syncwarp();
+        const bool mine = lane < cnt;
+        const uint32_t um = mine ? ws.cand_u[lane] : 0u;
+        const int jm = mine ? ws.cand_j[lane] : 0;
+        unsigned long long s_before = 0;
+        int n_before = 0;
+#pragma unroll 4
+        for (int n = 0; n < cnt; ++n) {
+            const uint32_t un = ws.cand_u[n];
+            if (un > um || (un == um && n < lane)) {
+                s_before += significand(un);
+                ++n_before;
+            }
+        }
+        __syncwarp();
+        const double before = above + static_cast<double>(s_above + s_before) * unit;
+        const bool kept = mine && (before < pd || (cnt_above == 0 && n_before == 0));
+        const uint64_t key = kept ? ((static_cast<uint64_t>(um) << 32) |
+                                     (0xFFFFFFFFu - static_cast<uint32_t>(jm)))
+                                  : ~0ull;
+        const uint64_t best = warp_min_u64(key);
+        if (best == ~0ull) {  // the range starts past p (rounding): keep only what is above it
+            uint32_t mx = mine ? um : 0u;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            ucut = mx;
+            jcut = -1;
+        } else {
+            ucut = static_cast<uint32_t>(best >> 32);
+            jcut = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(best));
+        }
+        return;
+    }
+    // ---- more than 32 entries with one bit pattern: ties in ascending j
+    const uint32_t uc = pre;
+    const unsigned long long sg = significand(uc);
+    int n_keep = 0;
+    for (int k = lane; k < cnt; k += 32)
+        n_keep += (above + static_cast<double>(s_above + sg * static_cast<unsigned long long>(k)) *
+                               unit < pd) ? 1 : 0;
+    n_keep = warp_sum_i(n_keep);
+    if (n_keep == 0 && cnt_above == 0) n_keep = 1;
+    ucut = uc;
+    jcut = n_keep == 0 ? -1 : nth_tie<VPL>(v, Ck, uc, n_keep, lane);
+}
+
+// Hardware base-2 logarithm (MUFU approximation, relative error ~2^-22).
+__device__ __forceinline__ float lg2_approx(float y) {
+    float r;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(y));
+    return r;
 }
 
 template <int VPL>
-__global__ void __launch_bounds__(256) mask_kernel(MaskArgs a, TopP tp) {
-    __shared__ float s_cv[8][kCandMax];
-    __shared__ int s_cj[8][kCandMax];
+__global__ void __launch_bounds__(128, VPL <= 16 ? 6 : VPL <= 32 ? 5 : 3)
+mask_kernel(MaskArgs a, TopP tp) {
+    __shared__ __align__(16) WarpScratch s_ws[4];
     const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
-    const long long row = static_cast<long long>(blockIdx.x) * 8 + wid;
+    WarpScratch &ws = s_ws[wid];
+    {   // clear this warp's table once; every level leaves it cleared
+        ulonglong2 *t = reinterpret_cast<ulonglong2 *>(&ws.bins[0][0]);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) t[lane + 32 * k] = make_ulonglong2(0ull, 0ull);
+        __syncwarp();
+    }
+    const long long row = static_cast<long long>(blockIdx.x) * 4 + wid;
     if (row >= a.rows) return;  // whole warp leaves together
     const int Ck = a.Ck;
     const int i = static_cast<int>(row % a.Cq);
@@ -206,36 +405,35 @@ __global__ void __launch_bounds__(256) mask_kernel(MaskArgs a, TopP tp) {
     const float p = tp.p[h];
     const float *src = a.probs + row * Ck;
 
+    // Issue every load before any arithmetic on them.
     float v[VPL];
-    float ent = 0.f;
-    double total = 0.0;
-    uint32_t umax = 0;
 #pragma unroll
     for (int s = 0; s < VPL; ++s) {
         const int j = lane + 32 * s;
-        float x = (j < Ck) ? __ldg(src + j) : 0.f;
-        x = fmaxf(x, 0.f);
+        v[s] = (j < Ck) ? __ldg(src + j) : 0.f;
+    }
+    float ent = 0.f;
+    uint32_t umax = 0;
+#pragma unroll
+    for (int s = 0; s < VPL; ++s) {
+        const float x = v[s] > 0.f ? v[s] : 0.f;  // -0.0 and NaN become +0.0
         v[s] = x;
         umax = max(umax, __float_as_uint(x));
-        total += static_cast<double>(x);
-        if (j < Ck) ent -= x * __logf(x + a.eps);
+        if (lane + 32 * s < Ck) ent = fmaf(x, lg2_approx(x + a.eps), ent);
     }
-    total = warp_sum_d(total);
     if (a.row_entropy) {
-        ent = warp_sum(ent);
+        ent = -warp_sum(ent) * 0.6931471805599453f;  // ln 2
         if (lane == 0) a.row_entropy[row] = ent;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) umax = max(umax, __shfl_xor_sync(0xffffffffu, umax, o));
 
-    // fp64 totals, like the running sum of the rule: the row never reaches p -> keep it all
-    const bool keep_all = !(total >= static_cast<double>(p));
-    uint32_t ucut = 0;
-    int jcut = 0x7FFFFFFF;
-    if (!keep_all) find_cut<VPL>(v, Ck, p, umax, lane, s_cv[wid], s_cj[wid], ucut, jcut);
-
     const bool dense_row = (a.flags & BSA_FRAME0_DENSE) && i >= a.f0_first && i <= a.f0_last;
-    const bool text = (a.flags & BSA_TEXT_KEEP) != 0;
+    uint32_t ucut = 0;
+    int jcut = 0x7FFFFFFF;  // keep every entry
+    if (!dense_row) find_cut<VPL>(v, src, Ck, p, umax, lane, ws, ucut, jcut);
+
+    const int text_k = (a.flags & BSA_TEXT_KEEP) ? a.text_kblocks : 0;
     uint8_t *mrow = a.mask ? a.mask + row * Ck : nullptr;
     int32_t *irow = a.kv_index + row * Ck;
     const uint32_t lt_mask = (1u << lane) - 1u;
@@ -243,11 +441,9 @@ __global__ void __launch_bounds__(256) mask_kernel(MaskArgs a, TopP tp) {
 #pragma unroll
     for (int s = 0; s < VPL; ++s) {
         const int j = lane + 32 * s;
-        const bool valid = j < Ck;
         const uint32_t us = __float_as_uint(v[s]);
-        bool sel = keep_all || us > ucut || (us == ucut && j <= jcut);
-        sel = valid && (sel || dense_row || (text && j < a.text_kblocks));
-        if (mrow && valid) mrow[j] = sel ? 1 : 0;
+        const bool sel = j < Ck && (us > ucut || (us == ucut && j <= jcut) || j < text_k);
+        if (mrow && j < Ck) mrow[j] = sel ? 1 : 0;
         const uint32_t bal = __ballot_sync(0xffffffffu, sel);
         if (sel) irow[base + __popc(bal & lt_mask)] = j;
         base += __popc(bal);
@@ -276,8 +472,8 @@ __global__ void __launch_bounds__(256) entropy_reduce_kernel(const float *__rest
 
 template <int VPL>
 cudaError_t launch_mask_t(const MaskArgs &a, const TopP &tp, cudaStream_t st) {
-    const unsigned grid = static_cast<unsigned>((a.rows + 7) / 8);
-    mask_kernel<VPL><<<grid, 256, 0, st>>>(a, tp);
+    const unsigned grid = static_cast<unsigned>((a.rows + 3) / 4);
+    mask_kernel<VPL><<<grid, 128, 0, st>>>(a, tp);
     return cudaGetLastError();
 }
 
