@@ -18,7 +18,9 @@ by head with no collective; weak scaling).  `--impl reference` times the CPU
 oracle on a bounded sample of the same workload (rank 0 only).
 """
 import argparse
+import glob
 import json
+import re
 import math
 import os
 import signal
@@ -353,15 +355,7 @@ def our_arm(args, w):
         hbm = peaks["hbm_gbs"]
     else:
         peak, peak_note, burst, hbm = 1400.0, "fallback sustained", 1590.0, 6650.0
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(prof):
-        try:
-            t = json.load(open(prof)).get(w.name)
-            if t and t.get("kernel_sha") == kernel_sha():
-                traffic = t["bytes_per_launch"]
-        except (OSError, ValueError, KeyError):
-            traffic = None
+    traffic = profiled_traffic(w.name)
     # scoring and mask: algorithmic bytes (read Q, K once; write centroids, P'; read P',
     # write mask, lists, counts) over their measured durations
     bytes_scores = 2 * B * H * w.seq_len * D * 2 + 4 * B * H * (Cq + Ck) * D + 4 * B * H * Cq * Ck
@@ -403,6 +397,21 @@ def our_arm(args, w):
                    "query blocks (%d selected block pairs), %.1f s" % (r["blocks"], r["pairs"],
                                                                        r["seconds"]))
     print(json.dumps(line), flush=True)
+
+
+TRAFFIC_LINE = re.compile(r"traffic: kernel=attn_kernel workload=(\S+) kernel_sha=([0-9a-f]+) "
+                          r"bytes_per_launch=(\d+)")
+
+
+def profiled_traffic(workload):
+    """DRAM bytes (read + write) per attention launch from the ncu summaries
+    under profiles/, valid only while the kernel source still hashes the same."""
+    sha = kernel_sha()
+    for f in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for m in TRAFFIC_LINE.finditer(open(f).read()):
+            if m.group(1) == workload and m.group(2) == sha:
+                return int(m.group(3))
+    return None
 
 
 def kernel_sha():
