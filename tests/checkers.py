@@ -14,19 +14,15 @@ log-sum-exp within LSE_ABS.  Entropy within ENTROPY_REL relative.
 import numpy as np
 
 MARGIN = 1e-4            # end to end (GPU P' vs oracle P'): all three margin terms
-MARGIN_SAME_PROBS = 1e-5  # identical P' on both sides: only the running-sum terms matter
 MAX_ABS = 2e-2
 MEAN_ABS = 2e-3
 LSE_ABS = 1e-3
 ENTROPY_REL = 1e-3
 
 
-def row_margins(probs, top_p, use_gap=True):
-    """k* and the margin of every row of probs [B,H,Cq,Ck] (oracle fp32 values).
-
-    use_gap=False drops the P'_(k*) - P'_(k*+1) term: when both sides read the
-    same fp32 P', their orders agree and only the summation rounding can move
-    the cut."""
+def row_margins(probs, top_p):
+    """k* and the margin of every row of probs [B,H,Cq,Ck] (oracle fp32 values):
+    min(p - c_{k*-1}, c_{k*} - p, P'_(k*) - P'_(k*+1))."""
     B, H, Cq, Ck = probs.shape
     tp = np.broadcast_to(np.asarray(top_p, np.float64), (H,))
     kstar = np.empty((B, H, Cq), np.int64)
@@ -46,18 +42,26 @@ def row_margins(probs, top_p, use_gap=True):
             gap = np.where(k < Ck, srt[idx, k - 1] - srt[idx, np.minimum(k, Ck - 1)], np.inf)
             m1 = np.where(k > 1, p - ckm1, np.inf)
             m2 = np.where(reach.any(-1), ck - p, np.inf)
-            margin[b, h] = np.minimum(np.minimum(m1, m2), gap if use_gap else np.inf)
+            margin[b, h] = np.minimum(np.minimum(m1, m2), gap)
     return kstar, margin
 
 
 def check_topp_masks(gpu_mask, ora_mask, probs, top_p, same_probs=False):
     """Compare top-p masks (no overrides).  Returns the exempt fraction.
 
-    same_probs=True: the GPU read the oracle's own P', so the rule is the
-    summation margin MARGIN_SAME_PROBS without the gap term; otherwise the
-    end-to-end rule (MARGIN, all three terms)."""
-    thr = MARGIN_SAME_PROBS if same_probs else MARGIN
-    kstar, margin = row_margins(probs, top_p, use_gap=not same_probs)
+    same_probs=True: the GPU read the oracle's own P'.  Both sides then sum
+    exactly (the oracle's fp64 running sum of fp32 values spans fewer than 53
+    bits down to any cut above 2^-29; the GPU sums integer significands per
+    binade), so every row must match bit for bit.  Otherwise the end-to-end
+    rule: bit-exact where the margin exceeds MARGIN (all three terms), a valid
+    top-p set elsewhere."""
+    if same_probs:
+        gpu_b, ora_b = gpu_mask.astype(bool), ora_mask.astype(bool)
+        bad = np.argwhere((gpu_b != ora_b).any(-1))
+        assert bad.size == 0, "rows differ on identical P': %s (of %d)" % (bad[:5].tolist(), len(bad))
+        return 0.0
+    thr = MARGIN
+    kstar, margin = row_margins(probs, top_p)
     gpu_mask = gpu_mask.astype(bool)
     ora_mask = ora_mask.astype(bool)
     strict = margin > thr
