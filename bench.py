@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="hunyuan")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-group", type=int, default=1,
+                    help="heads per group of the pipelined host-buffer call timed as e2e")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     return ap.parse_args()
@@ -293,21 +295,23 @@ def our_arm(args, w):
     ms_step = ms_total / args.steps
     value = job_tflops(step_flops, world, ms_step)
 
-    # end to end through the C ABI: pinned host inputs -> device, path, output -> host
+    # end to end through the C ABI with HOST buffers: bsa_sparse_attention_host copies
+    # Q, K, V in and O (+ entropy) out per head group on two copy streams, overlapped
+    # with the kernels of the neighbouring groups
     e2e = None
     if not args.no_e2e:
         pin = {n: host[n].pin_memory() for n in ("q", "k", "v")}
         out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        ent_h = torch.empty(ent.shape, dtype=ent.dtype).pin_memory()
-        qd, kd, vd = (torch.empty_like(q) for _ in range(3))
+        ent_h = torch.empty((B, H), dtype=torch.float32).pin_memory()
+        h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        nws = bsa.pipeline_workspace_bytes(w, args.e2e_group)
+        pws = torch.empty(nws, dtype=torch.uint8, device=dev)
 
         def e2e_step():
-            qd.copy_(pin["q"], non_blocking=True)
-            kd.copy_(pin["k"], non_blocking=True)
-            vd.copy_(pin["v"], non_blocking=True)
-            step(qd, kd, vd)
-            out_h.copy_(out, non_blocking=True)
-            ent_h.copy_(ent, non_blocking=True)
+            bsa.sparse_attention_host(w, pin["q"], pin["k"], pin["v"], top_p, w.flags,
+                                      heads_per_group=args.e2e_group, out=out_h, entropy=ent_h,
+                                      workspace=pws, stream=stream, h2d_stream=h2d_s,
+                                      d2h_stream=d2h_s, device=dev)
 
         e2e_step()
         torch.cuda.synchronize(dev)
@@ -323,7 +327,10 @@ def our_arm(args, w):
         h2d = sum(pin[n].numel() * pin[n].element_size() for n in pin)
         d2h = out_h.numel() * out_h.element_size() + ent_h.numel() * ent_h.element_size()
         e2e = dict(value=job_tflops(step_flops, world, ms_e2e), unit=UNIT,
-                   ms_per_step=ms_e2e, h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h))
+                   ms_per_step=ms_e2e, h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h),
+                   call="bsa_sparse_attention_host (page-locked host buffers, heads_per_group=%d)"
+                        % args.e2e_group)
+        del pws
 
     # the dense path (all key blocks) for context: not part of the step
     dense = None

@@ -70,6 +70,12 @@ def load():
         L.bsa_attention_workspace_bytes.restype = ctypes.c_size_t
         L.bsa_dense_fwd.argtypes = [lp, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp, vp]
         L.bsa_dense_fwd.restype = ctypes.c_int
+        L.bsa_sparse_attention_host.argtypes = [lp, ctypes.c_int, vp, vp, vp, vp, ctypes.c_uint32,
+                                                ctypes.c_float, ctypes.c_float, vp, vp, vp, vp, vp,
+                                                vp, ctypes.c_size_t, vp, vp, vp]
+        L.bsa_sparse_attention_host.restype = ctypes.c_int
+        L.bsa_pipeline_workspace_bytes.argtypes = [lp, ctypes.c_int]
+        L.bsa_pipeline_workspace_bytes.restype = ctypes.c_size_t
         L.bsa_status_string.argtypes = [ctypes.c_int]
         L.bsa_status_string.restype = ctypes.c_char_p
         L.bsa_version.restype = ctypes.c_int
@@ -255,3 +261,69 @@ def sparse_attention(layout, q, k, v, top_p, flags, eps=1e-8, softmax_scale=None
                              stream=stream)
     sel.update(q_centroids=qc, k_centroids=kc, probs=probs, out=out, lse=lse)
     return sel
+
+
+def pipeline_workspace_bytes(layout, heads_per_group):
+    return int(load().bsa_pipeline_workspace_bytes(ctypes.byref(make_layout(layout)),
+                                                   int(heads_per_group)))
+
+
+def _need_host(t, name, dtype, shape):
+    if t.dtype != dtype:
+        raise TypeError("%s: expected %s, got %s" % (name, dtype, t.dtype))
+    if t.is_cuda:
+        raise ValueError("%s must be a host tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s: expected shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+
+
+def sparse_attention_host(layout, q, k, v, top_p, flags, eps=1e-8, softmax_scale=None,
+                          heads_per_group=2, out=None, entropy=None, entropy_norm=None,
+                          kv_count=None, err_flag=None, workspace=None, stream=None,
+                          h2d_stream=None, d2h_stream=None, device=None):
+    """bsa_sparse_attention_host: the whole path on HOST q, k, v (page-locked
+    for overlap), writing HOST out (and optional entropy / kv_count).  Queued
+    on `stream` (default: the current stream of `device`); returns a dict of
+    the host outputs, valid once that stream is synchronised."""
+    L = make_layout(layout)
+    B, H, Sp, D = L.batch, L.heads, L.seq_pad, L.head_dim
+    Cq = Sp // L.q_block
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need_host(t, n, torch.bfloat16, (B, H, Sp, D))
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if out is None:
+        out = torch.empty((B, H, Sp, D), dtype=torch.bfloat16, pin_memory=True)
+    _need_host(out, "out", torch.bfloat16, (B, H, Sp, D))
+    if entropy is not None:
+        _need_host(entropy, "entropy", torch.float32, (B, H))
+    if entropy_norm is not None:
+        _need_host(entropy_norm, "entropy_norm", torch.float32, (B, H))
+    if kv_count is not None:
+        _need_host(kv_count, "kv_count", torch.int32, (B, H, Cq))
+    if err_flag is not None:
+        _need_host(err_flag, "err_flag", torch.int32, (1,))
+    nbytes = pipeline_workspace_bytes(L, heads_per_group)
+    if nbytes == 0:
+        raise BsaError("bsa_pipeline_workspace_bytes", BSA_ERR_INVALID_ARG)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    elif workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError("workspace: %d bytes needed" % nbytes)
+    scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
+    if len(top_p) != H:
+        raise ValueError("top_p: expected %d values" % H)
+    tp = (ctypes.c_float * H)(*[float(x) for x in top_p])
+    cs = torch.cuda.current_stream(dev) if stream is None else stream
+    hs = cs if h2d_stream is None else h2d_stream
+    ds = cs if d2h_stream is None else d2h_stream
+    rc = load().bsa_sparse_attention_host(
+        ctypes.byref(L), int(heads_per_group), _ptr(q), _ptr(k), _ptr(v),
+        ctypes.cast(tp, ctypes.c_void_p), int(flags), float(eps), scale, _ptr(out), _ptr(entropy),
+        _ptr(entropy_norm), _ptr(kv_count), _ptr(err_flag), _ptr(workspace), nbytes,
+        ctypes.c_void_p(cs.cuda_stream), ctypes.c_void_p(hs.cuda_stream),
+        ctypes.c_void_p(ds.cuda_stream))
+    _check("bsa_sparse_attention_host", rc)
+    return dict(out=out, entropy=entropy, entropy_norm=entropy_norm, kv_count=kv_count,
+                err_flag=err_flag, workspace=workspace)

@@ -35,14 +35,6 @@ Geometry make_geometry(const bsa_layout &L) {
     return g;
 }
 
-}  // namespace bsa
-
-namespace {
-
-using bsa::Geometry;
-
-bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-
 int check_layout(const bsa_layout *L) {
     if (!L) return BSA_ERR_INVALID_ARG;
     if (L->batch < 1 || L->heads < 1 || L->seq_len < 1 || L->seq_pad < L->seq_len)
@@ -65,6 +57,15 @@ int check_layout(const bsa_layout *L) {
         return BSA_ERR_UNSUPPORTED;
     return BSA_OK;
 }
+
+}  // namespace bsa
+
+namespace {
+
+using bsa::check_layout;
+using bsa::Geometry;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 int launch_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_LAUNCH; }
 

@@ -20,6 +20,10 @@ struct Geometry {
 
 Geometry make_geometry(const bsa_layout &L);
 
+// Host-side validation of a layout shared by every entry point: BSA_OK,
+// BSA_ERR_INVALID_ARG or BSA_ERR_UNSUPPORTED.
+int check_layout(const bsa_layout *L);
+
 cudaError_t launch_pool(const Geometry &g, const void *q, const void *k, float *qc, float *kc,
                         cudaStream_t st);
 cudaError_t launch_scores(const Geometry &g, const float *qc, const float *kc, float *probs,

@@ -348,29 +348,6 @@ __device__ __forceinline__ void add2(float &d0, float &d1, float a0, float a1, f
         : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-// 2^t for a pair, on the FMA pipe (leaves the MUFU unit to the other columns).
-// Range reduction: t = n + f with n = round(t) (from the low mantissa bits of
-// t + 1.5*2^23) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial with
-// p(0) = 1 whose coefficients are a minimax fit of the relative error on
-// [-1/2, 1/2] (max 1.01e-4, below bf16 resolution); 2^n is added to the
-// exponent field.  t is clamped at -127, where the result is exactly +0, so
-// masked (-inf) columns give exact zeros.  Valid for t <= 127.
-__device__ __forceinline__ void exp2_poly2(float t0, float t1, float &p0, float &p1) {
-    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-    constexpr float kC1 = 0.693282902f, kC2 = 0.242210954f, kC3 = 0.0550089329f;
-    t0 = fmaxf(t0, -127.0f);
-    t1 = fmaxf(t1, -127.0f);
-    float j0, j1, r0, r1, f0, f1, q0, q1;
-    add2(j0, j1, t0, t1, kMagic, kMagic);
-    add2(r0, r1, j0, j1, -kMagic, -kMagic);
-    fma2(f0, f1, r0, r1, -1.0f, -1.0f, t0, t1);
-    fma2(q0, q1, f0, f1, kC3, kC3, kC2, kC2);
-    fma2(q0, q1, q0, q1, f0, f1, kC1, kC1);
-    fma2(q0, q1, q0, q1, f0, f1, 1.0f, 1.0f);
-    p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(j0) << 23));
-    p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(j1) << 23));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);

@@ -216,6 +216,51 @@ int bsa_dense_fwd(const bsa_layout *layout, const void *q, const void *k, const 
                   float softmax_scale, void *out, float *lse, int32_t *err_flag, void *workspace,
                   void *stream);
 
+/*
+ * The whole path for host-resident tensors: bsa_block_scores, bsa_build_mask
+ * (mask bytes not kept) and bsa_attention_fwd, with the host<->device copies
+ * overlapped with the kernels.  The path is independent per (b, h) ("Competition
+ * Domains Matter ..." s3 domain 1 selects per head and query row; attention is
+ * per head), so the heads of each batch entry are cut into groups of
+ * heads_per_group: while group c computes on compute_stream, Q, K, V of group
+ * c+1 travel in on h2d_stream and O of group c-1 travels out on d2h_stream,
+ * through two device slots inside `workspace`.  Results equal those of the
+ * three device entry points called on the same data.
+ *
+ * heads_per_group  heads per group (>= 1; larger than H means all heads)
+ * q, k, v          HOST bf16 [B,H,seq_pad,D] (read).  Page-locked memory
+ *                  (cudaHostAlloc / cudaHostRegister) is needed for the copies
+ *                  to overlap anything; pageable memory works but serialises.
+ * top_p            host fp32 [H]; flags, eps, softmax_scale as above
+ * out              HOST bf16 [B,H,seq_pad,D] (written)
+ * entropy          HOST fp32 [B,H], or NULL; entropy_norm likewise
+ * kv_count         HOST int32 [B,H,C_q] (the list lengths), or NULL
+ * err_flag         HOST int32, or NULL: receives the OR of the BSA_DEVERR_*
+ *                  bits of every attention launch of the call
+ * workspace        device memory, 256-byte aligned, of at least
+ *                  bsa_pipeline_workspace_bytes(layout, heads_per_group)
+ *                  bytes; owned by the call until it completes
+ * compute_stream, h2d_stream, d2h_stream
+ *                  cudaStream_t values; they may coincide (no overlap then).
+ *
+ * Asynchronous: everything is ordered after the work already queued on
+ * compute_stream, and compute_stream is made to wait for the last copy, so
+ * synchronising compute_stream (or an event recorded on it after the call)
+ * means every output is on the host.  The host buffers must stay valid until
+ * then.  The call creates and releases a few CUDA events; it allocates no
+ * memory.  On an error return some copies may already be queued: synchronise
+ * all three streams before reusing the buffers.
+ */
+int bsa_sparse_attention_host(const bsa_layout *layout, int heads_per_group, const void *q,
+                              const void *k, const void *v, const float *top_p, uint32_t flags,
+                              float eps, float softmax_scale, void *out, float *entropy,
+                              float *entropy_norm, int32_t *kv_count, int32_t *err_flag,
+                              void *workspace, size_t workspace_bytes, void *compute_stream,
+                              void *h2d_stream, void *d2h_stream);
+
+/* Device workspace bytes bsa_sparse_attention_host needs (0: invalid layout). */
+size_t bsa_pipeline_workspace_bytes(const bsa_layout *layout, int heads_per_group);
+
 /* Human-readable name of a bsa_status value (static storage). */
 const char *bsa_status_string(int status);
 

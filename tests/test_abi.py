@@ -84,6 +84,51 @@ def test_workspace_size():
     assert bsa.load().bsa_build_mask_workspace_bytes(ctypes.byref(L)) == -(-24 * 931 * 4 // 256) * 256
 
 
+def _host_call(lib, L, hpg=1, q=FAKE, out=FAKE, top_p=None, flags=3, eps=1e-8, scale=0.125,
+               ws=ctypes.c_void_p(0x100000), ws_bytes=1 << 40):
+    tp = (ctypes.c_float * L.heads)(*([0.5] * L.heads)) if top_p is None else top_p
+    return lib.bsa_sparse_attention_host(
+        ctypes.byref(L), hpg, q, FAKE, FAKE, ctypes.cast(tp, ctypes.c_void_p), flags, eps, scale,
+        out, None, None, None, None, ws, ws_bytes, None, None, None)
+
+
+def test_pipeline_entry_point_validates_before_any_cuda_call():
+    lib = bsa.load()
+    L = _layout()
+    # every rejection below happens on the host, before a stream or event is touched
+    assert _host_call(lib, _layout(head_dim=96)) == bsa.BSA_ERR_UNSUPPORTED
+    assert _host_call(lib, _layout(seq_len=200)) == bsa.BSA_ERR_INVALID_ARG
+    assert _host_call(lib, L, hpg=0) == bsa.BSA_ERR_INVALID_ARG
+    assert _host_call(lib, L, q=None) == bsa.BSA_ERR_INVALID_ARG
+    assert _host_call(lib, L, out=None) == bsa.BSA_ERR_INVALID_ARG
+    assert _host_call(lib, L, ws=None) == bsa.BSA_ERR_INVALID_ARG
+    assert _host_call(lib, L, ws=ctypes.c_void_p(0x100010)) == bsa.BSA_ERR_INVALID_ARG  # not 256-aligned
+    need = lib.bsa_pipeline_workspace_bytes(ctypes.byref(L), 1)
+    assert _host_call(lib, L, ws_bytes=need - 1) == bsa.BSA_ERR_INVALID_ARG
+    assert _host_call(lib, L, flags=8) == bsa.BSA_ERR_INVALID_ARG
+    assert _host_call(lib, L, eps=-1.0) == bsa.BSA_ERR_INVALID_ARG
+    assert _host_call(lib, L, scale=0.0) == bsa.BSA_ERR_INVALID_ARG
+    nan_tp = (ctypes.c_float * 2)(0.5, float("nan"))
+    assert _host_call(lib, L, top_p=nan_tp) == bsa.BSA_ERR_INVALID_ARG
+
+
+def test_pipeline_workspace_size():
+    lib = bsa.load()
+    w = synth.WORKLOADS["hunyuan"]
+    L = bsa.make_layout(w)
+    assert lib.bsa_pipeline_workspace_bytes(ctypes.byref(L), 0) == 0
+    assert lib.bsa_pipeline_workspace_bytes(ctypes.byref(_layout(head_dim=96)), 1) == 0
+    one = lib.bsa_pipeline_workspace_bytes(ctypes.byref(L), 1)
+    two = lib.bsa_pipeline_workspace_bytes(ctypes.byref(L), 2)
+    # two slots, each holding q, k, v, out of the group plus its selection buffers
+    per_head = 4 * w.seq_pad * w.head_dim * 2
+    assert one > 2 * per_head and two > 2 * (2 * per_head)
+    assert two - one >= 2 * per_head
+    # a group larger than H is clamped to H
+    assert lib.bsa_pipeline_workspace_bytes(ctypes.byref(L), 1000) == \
+        lib.bsa_pipeline_workspace_bytes(ctypes.byref(L), w.heads)
+
+
 def test_calls_fail_loudly_without_the_library(monkeypatch):
     monkeypatch.setattr(bsa, "_LIB", None)
     monkeypatch.setattr(bsa, "LIB_PATH", "/nonexistent/libbsa.so")
