@@ -1,6 +1,7 @@
 // internal.h -- launchers shared between the C ABI (api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -19,6 +20,15 @@ struct Geometry {
 };
 
 Geometry make_geometry(const bsa_layout &L);
+
+// cuTensorMapEncodeTiled, looked up once through the runtime (nullptr if the
+// driver lacks it), and the current device's SM count (0 on error).
+typedef CUresult (*TensorMapEncoder)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                     const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                     const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                     CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+TensorMapEncoder tensor_map_encoder();
+int sm_count();
 
 // Host-side validation of a layout shared by every entry point: BSA_OK,
 // BSA_ERR_INVALID_ARG or BSA_ERR_UNSUPPORTED.

@@ -10,9 +10,9 @@
 //
 // pool_kernel   HBM-bound: streams Q and K exactly once with 16-byte loads and
 //               writes fp32 centroids.
-// score_kernel  fp32 register-tiled centroid GEMM (C_q x C_k x D per head)
-//               with the row softmax fused: a CTA owns TM full rows, keeps
-//               their logits in shared memory and writes P' once.
+// score_kernel  the centroid GEMM (C_q x C_k x D per head) on the tensor
+//               cores in split-tf32 (three kind::tf32 MMAs per K step), with
+//               the n_j-weighted row softmax fused into the TMEM epilogue.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -89,116 +89,394 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint4 *__restrict__ q,
     }
 }
 
-// CTA = (head, TM query rows) x all C_k key blocks.  Thread (ty, tx) owns
-// rows ty*RPT .. +RPT-1 and columns tx + 32c (c < 4) of each 128-column tile.
-template <int TM, int D>
-__global__ void __launch_bounds__(256) score_kernel(const float *__restrict__ qc,
-                                                    const float *__restrict__ kc,
-                                                    float *__restrict__ probs, int S, int bk,
-                                                    int Cq, int Ck, float inv_sqrt_d) {
-    constexpr int TN = 128;
-    constexpr int RPT = TM / 8;
-    constexpr int KS = D + 4;  // padded k row stride (floats): conflict-free float4 reads
-    extern __shared__ __align__(16) float smem[];
-    float *ks = smem;              // [TN][KS]
-    float *qs = ks + TN * KS;      // [TM][D]
-    float *logit = qs + TM * D;    // [TM][Ck]
+// ---------------------------------------------------------------------------
+// score_kernel: the centroid GEMM on the tensor cores, row softmax fused.
+//
+// Work item = (b*h, 128 query-block rows).  For each chunk of 256 key-block
+// columns the item's logits accumulate in TMEM (two chunk buffers of 256
+// columns), fed by 2 shared-memory stages that each hold one 32-wide slice of
+// D ("panel") of q-bar (128 x 32 fp32) and k-bar (256 x 32 fp32).
+//
+// Precision: plain tf32 keeps ~11 significant bits, far too coarse for logits
+// of magnitude ~50 (P' must stay within 1e-4).  Each operand x is split
+// exactly into hi = x with the low 13 mantissa bits cleared (a tf32 value)
+// and lo = x - hi, and the product is hi_a hi_b + hi_a lo_b + lo_a hi_b
+// (three tf32 MMAs), which leaves an error near 2^-21 relative.
+//
+// Warp roles (384 threads):
+//   warp 0      TMA producer: q-bar and k-bar panels into the stage's hi halves
+//   warp 1      TMEM owner; lane 0 issues the tcgen05.mma (kind::tf32)
+//   warps 4-7   split workers: hi/lo in place for each landed stage
+//   warps 8-11  epilogue: thread = query-block row (TMEM lane); per 32-column
+//               slice s2 = acc * log2(e)/sqrt(D) + log2 n_j, a running row
+//               max m2 and sum z of 2^(s2 - m2); the slice goes through shared
+//               memory so a warp writes one row's 32 values contiguously.  After
+//               the last chunk a warp per row rewrites s2 -> 2^(s2 - m2) / z.
+namespace sc {
 
-    const int tid = threadIdx.x, ty = tid / 32, tx = tid % 32;
-    const int tiles_per_head = (Cq + TM - 1) / TM;
-    const long long bh = blockIdx.x / tiles_per_head;
-    const int i0 = (blockIdx.x % tiles_per_head) * TM;
-    const int rows = min(TM, Cq - i0);
+constexpr int kThreads = 384;
+constexpr int kRows = 128;                           // MMA M
+constexpr int kCols = 256;                           // MMA N: key-block columns per chunk
+constexpr int kAPanelBytes = kRows * 128;            // 128 rows x 32 fp32
+constexpr int kBPanelBytes = kCols * 128;            // 256 rows x 32 fp32
+constexpr int kStageBytes = 2 * (kAPanelBytes + kBPanelBytes);  // A, A_lo, B, B_lo
+constexpr int kStages = 2;
+constexpr int kTmemCols = 2 * kCols;
+constexpr int kPitch = 33;                           // staging row pitch (floats)
 
-    const float4 *qsrc = reinterpret_cast<const float4 *>(qc + (bh * Cq + i0) * D);
-    for (int e = tid; e < TM * D / 4; e += 256) {
-        const int r = e / (D / 4);
-        reinterpret_cast<float4 *>(qs)[e] = (r < rows) ? __ldg(qsrc + e) : make_float4(0, 0, 0, 0);
+struct Header {
+    uint64_t full[kStages];    // TMA landed (expect_tx)
+    uint64_t split[kStages];   // hi / lo written (128 arrivals)
+    uint64_t empty[kStages];   // MMAs done with the stage (commit)
+    uint64_t acc_full[2];      // chunk accumulated (commit)
+    uint64_t acc_empty[2];     // epilogue read the chunk (128 arrivals)
+    uint64_t mma_done;         // every issued MMA finished (commit)
+    uint32_t tmem_base;
+    int abort;
+    float m2[kRows], inv_z[kRows];
+};
+constexpr int kHeaderBytes = 2048;
+static_assert(sizeof(Header) <= kHeaderBytes, "header");
+constexpr int kOffLog2n = kHeaderBytes;
+constexpr int kOffStaging = kOffLog2n + kMaxScoreCk * 4;
+constexpr int kOffStages = ((kOffStaging + kRows * kPitch * 4) + 1023) / 1024 * 1024;
+constexpr int kSmemBytes = kOffStages + kStages * kStageBytes;
+constexpr int kSmemAlloc = kSmemBytes + 1024;
+static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
+
+struct Params {
+    float *probs;
+    int Cq, Ck, S, bk, n_rt, n_items;
+    float scale2;  // log2(e) / sqrt(D)
+};
+
+// Clear the low 13 mantissa bits: an exact tf32 value, and x - hi is exact.
+__device__ __forceinline__ void split4(uint4 &x, uint4 &lo) {
+    const uint32_t m = 0xFFFFE000u;
+    const uint4 hi = make_uint4(x.x & m, x.y & m, x.z & m, x.w & m);
+    lo = make_uint4(__float_as_uint(__uint_as_float(x.x) - __uint_as_float(hi.x)),
+                    __float_as_uint(__uint_as_float(x.y) - __uint_as_float(hi.y)),
+                    __float_as_uint(__uint_as_float(x.z) - __uint_as_float(hi.z)),
+                    __float_as_uint(__uint_as_float(x.w) - __uint_as_float(hi.w)));
+    x = hi;
+}
+
+}  // namespace sc
+
+template <int D>
+__global__ void __launch_bounds__(sc::kThreads, 1)
+    score_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                 sc::Params p) {
+    using namespace sc;
+    constexpr int NP = D / 32;  // panels per chunk
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    Header &hd = *reinterpret_cast<Header *>(smem);
+    float *log2n = reinterpret_cast<float *>(smem + kOffLog2n);
+    float *stg = reinterpret_cast<float *>(smem + kOffStaging);
+    uint8_t *stages = smem + kOffStages;
+    volatile int *abort_flag = &hd.abort;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int nch = (p.Ck + kCols - 1) / kCols;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&hd.full[s], 1);
+            mbar_init(&hd.split[s], 128);
+            mbar_init(&hd.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&hd.acc_full[b], 1);
+            mbar_init(&hd.acc_empty[b], 128);
+        }
+        mbar_init(&hd.mma_done, 1);
+        hd.abort = 0;
+        fence_mbar_init();
     }
-    const float4 *kbase = reinterpret_cast<const float4 *>(kc + bh * Ck * D);
-
-    for (int j0 = 0; j0 < Ck; j0 += TN) {
-        __syncthreads();  // previous tile fully consumed (and qs visible on the first pass)
-        const int ncols = min(TN, Ck - j0);
-        for (int e = tid; e < TN * D / 4; e += 256) {
-            const int col = e / (D / 4), d4 = e % (D / 4);
-            const float4 val = (col < ncols) ? __ldg(kbase + (j0 + col) * (D / 4) + d4)
-                                             : make_float4(0, 0, 0, 0);
-            *reinterpret_cast<float4 *>(ks + col * KS + d4 * 4) = val;
-        }
-        __syncthreads();
-        float acc[RPT][4];
-#pragma unroll
-        for (int r = 0; r < RPT; ++r)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
-#pragma unroll 4
-        for (int d = 0; d < D; d += 4) {
-            float4 a[RPT], b[4];
-#pragma unroll
-            for (int r = 0; r < RPT; ++r)
-                a[r] = *reinterpret_cast<const float4 *>(qs + (ty * RPT + r) * D + d);
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                b[c] = *reinterpret_cast<const float4 *>(ks + (tx + 32 * c) * KS + d);
-#pragma unroll
-            for (int r = 0; r < RPT; ++r)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    acc[r][c] = fmaf(a[r].x, b[c].x, acc[r][c]);
-                    acc[r][c] = fmaf(a[r].y, b[c].y, acc[r][c]);
-                    acc[r][c] = fmaf(a[r].z, b[c].z, acc[r][c]);
-                    acc[r][c] = fmaf(a[r].w, b[c].w, acc[r][c]);
-                }
-        }
-#pragma unroll
-        for (int r = 0; r < RPT; ++r)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int col = tx + 32 * c;
-                if (col < ncols) logit[(ty * RPT + r) * Ck + j0 + col] = acc[r][c] * inv_sqrt_d;
-            }
+    // log2 of the key-block sizes n_j (every block holds at least one token)
+    for (int j = threadIdx.x; j < p.Ck; j += kThreads)
+        log2n[j] = log2f(static_cast<float>(min(p.bk, p.S - j * p.bk)));
+    if (warp == 1) {
+        tmem_alloc(&hd.tmem_base, kTmemCols);
+        tmem_relinquish();
     }
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = hd.tmem_base;
 
-    // Row softmax weighted by the key-block sizes n_j: P'_j = n_j e^{s_j - m} / Z.
-    const int warp = tid / 32, lane = tid % 32;
-    for (int r = warp; r < rows; r += 8) {
-        float *lr = logit + r * Ck;
-        float m = -INFINITY;
-        for (int j = lane; j < Ck; j += 32) m = fmaxf(m, lr[j]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float z = 0.f;
-        for (int j = lane; j < Ck; j += 32) {
-            const int nj = min(bk, S - j * bk);
-            const float w = static_cast<float>(nj) * expf(lr[j] - m);
-            lr[j] = w;
-            z += w;
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&mq);
+            prefetch_tmap(&mk);
+            int it = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+                const int bh = item / p.n_rt, r0 = (item % p.n_rt) * kRows;
+                for (int c = 0; ok && c < nch; ++c) {
+                    for (int pn = 0; pn < NP; ++pn, ++it) {
+                        const int st = it % kStages;
+                        if (it >= kStages &&
+                            !mbar_wait(&hd.empty[st], ((it / kStages) - 1) & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        uint8_t *sb = stages + st * kStageBytes;
+                        mbar_arrive_expect_tx(&hd.full[st], kAPanelBytes + kBPanelBytes);
+                        tma_load_3d(sb, &mq, &hd.full[st], pn * 32, r0, bh);
+                        tma_load_3d(sb + 2 * kAPanelBytes, &mk, &hd.full[st], pn * 32, c * kCols,
+                                    bh);
+                    }
+                }
+            }
+            // the last loads must land before the CTA may exit
+            volatile int no_abort = 0;
+            for (int k = it > kStages ? it - kStages : 0; k < it; ++k)
+                mbar_wait(&hd.full[k % kStages], (k / kStages) & 1, &no_abort);
         }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_tf32_f32(kRows, kCols);
+            int it = 0, ch = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+                for (int c = 0; ok && c < nch; ++c, ++ch) {
+                    const int buf = ch & 1;
+                    if (ch >= 2 && !mbar_wait(&hd.acc_empty[buf], ((ch >> 1) - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d = tmem + static_cast<uint32_t>(buf * kCols);
+                    for (int pn = 0; pn < NP; ++pn, ++it) {
+                        const int st = it % kStages;
+                        if (!mbar_wait(&hd.split[st], (it / kStages) & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t sb = smem_u32(stages + st * kStageBytes);
+                        const uint64_t a_hi = sw128_desc(sb, 16, 1024);
+                        const uint64_t a_lo = sw128_desc(sb + kAPanelBytes, 16, 1024);
+                        const uint64_t b_hi = sw128_desc(sb + 2 * kAPanelBytes, 16, 1024);
+                        const uint64_t b_lo =
+                            sw128_desc(sb + 2 * kAPanelBytes + kBPanelBytes, 16, 1024);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-        float *dst = probs + (bh * Cq + i0 + r) * static_cast<long long>(Ck);
-        for (int j = lane; j < Ck; j += 32) dst[j] = lr[j] / z;
+                        for (int k = 0; k < 4; ++k) {  // K = 8 tf32 = 32 bytes per MMA
+                            const uint64_t o = static_cast<uint64_t>(k * 2);
+                            mma_tf32_ss(d, a_hi + o, b_hi + o, idesc, (pn | k) ? 1u : 0u);
+                            mma_tf32_ss(d, a_hi + o, b_lo + o, idesc, 1u);
+                            mma_tf32_ss(d, a_lo + o, b_hi + o, idesc, 1u);
+                        }
+                        mma_commit(&hd.empty[st]);
+                    }
+                    if (!ok) break;
+                    mma_commit(&hd.acc_full[buf]);
+                }
+            }
+            // every issued MMA completes before TMEM is released
+            mma_commit(&hd.mma_done);
+            volatile int no_abort = 0;
+            mbar_wait(&hd.mma_done, 0, &no_abort);
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ split workers
+        const int tid = threadIdx.x - 128;
+        int it = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+            for (int c = 0; ok && c < nch; ++c) {
+                for (int pn = 0; pn < NP; ++pn, ++it) {
+                    const int st = it % kStages;
+                    if (!mbar_wait(&hd.full[st], (it / kStages) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    uint4 *a = reinterpret_cast<uint4 *>(stages + st * kStageBytes);
+                    uint4 *a_lo = a + kAPanelBytes / 16;
+                    uint4 *b = a_lo + kAPanelBytes / 16;
+                    uint4 *b_lo = b + kBPanelBytes / 16;
+                    // same byte offset in the lo half: the 128-byte swizzle depends only
+                    // on the address bits inside the 1024-byte-aligned atom
+#pragma unroll 4
+                    for (int i = tid; i < kAPanelBytes / 16; i += 128) {
+                        uint4 x = a[i], lo;
+                        split4(x, lo);
+                        a[i] = x;
+                        a_lo[i] = lo;
+                    }
+#pragma unroll 4
+                    for (int i = tid; i < kBPanelBytes / 16; i += 128) {
+                        uint4 x = b[i], lo;
+                        split4(x, lo);
+                        b[i] = x;
+                        b_lo[i] = lo;
+                    }
+                    fence_proxy_async_smem();
+                    mbar_arrive(&hd.split[st]);
+                }
+            }
+        }
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------ epilogue
+        // Named barrier 1 over the 128 epilogue threads.  Every bounded wait is
+        // followed by a vote (bar.red.and), so the four warps leave together and
+        // no bar.sync can wait for a warp that is gone.
+        const int ew = warp - 8;
+        const int rl = ew * 32 + lane;  // row within the tile = TMEM lane
+        const uint32_t t_lane = tmem + (static_cast<uint32_t>(ew * 32) << 16);
+        int ch = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+            const int bh = item / p.n_rt, r0 = (item % p.n_rt) * kRows;
+            const int nrows = min(kRows, p.Cq - r0);
+            float *tile = p.probs + (static_cast<long long>(bh) * p.Cq + r0) * p.Ck;
+            float m2 = -INFINITY, z = 0.f;
+            for (int c = 0; c < nch; ++c, ++ch) {
+                const int buf = ch & 1;
+                const bool got = mbar_wait(&hd.acc_full[buf], (ch >> 1) & 1, abort_flag);
+                if (!bar_red_and(1, 128, got)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int n_sl = min(kCols / 32, (p.Ck - c * kCols + 31) / 32);
+                uint32_t nxt[32];
+                tmem_ld32(t_lane + static_cast<uint32_t>(buf * kCols), nxt);
+                tmem_ld_wait();
+                reg_fence(nxt);  // no read of nxt may move above the wait
+                for (int s = 0; s < n_sl; ++s) {
+                    const int col0 = c * kCols + s * 32;
+                    uint32_t r[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) r[j] = nxt[j];
+                    reg_fence(r);
+                    // the next slice's TMEM load runs while this one is processed
+                    if (s + 1 < n_sl)
+                        tmem_ld32(t_lane + static_cast<uint32_t>(buf * kCols + (s + 1) * 32), nxt);
+                    float mx = -INFINITY;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int col = col0 + j;
+                        const float t = col < p.Ck
+                                            ? fmaf(__uint_as_float(r[j]), p.scale2, log2n[col])
+                                            : -INFINITY;
+                        r[j] = __float_as_uint(t);
+                        mx = fmaxf(mx, t);
+                    }
+                    const float mn = fmaxf(m2, mx);
+                    float sum = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) sum += ex2(__uint_as_float(r[j]) - mn);
+                    z = z * ex2(m2 - mn) + sum;
+                    m2 = mn;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) stg[rl * kPitch + j] = __uint_as_float(r[j]);
+                    named_barrier_sync(1, 128);
+                    // warp ew writes rows ew, ew+4, ...: all 32 staging reads first
+                    const int col = col0 + lane;
+                    if (col < p.Ck) {
+                        float v[kRows / 4];
+#pragma unroll
+                        for (int i = 0; i < kRows / 4; ++i) v[i] = stg[(ew + 4 * i) * kPitch + lane];
+                        float *dst = tile + static_cast<long long>(ew) * p.Ck + col;
+                        const long long step = 4ll * p.Ck;
+#pragma unroll
+                        for (int i = 0; i < kRows / 4; ++i)
+                            if (ew + 4 * i < nrows) dst[i * step] = v[i];
+                    }
+                    named_barrier_sync(1, 128);
+                    tmem_ld_wait();  // the prefetched slice has landed
+                    reg_fence(nxt);
+                }
+                tc_fence_before();
+                mbar_arrive(&hd.acc_empty[buf]);
+            }
+            if (!ok) break;
+            // P' = 2^(s2 - m2) / z, one warp per row, every load of a 1024-column
+            // segment issued before the arithmetic on it
+            hd.m2[rl] = m2;
+            hd.inv_z[rl] = 1.0f / z;
+            named_barrier_sync(1, 128);
+            // two rows at a time: 64 loads in flight per lane
+            for (int rr = ew; rr < nrows; rr += 8) {
+                const bool two = rr + 4 < nrows;
+                const float ma = hd.m2[rr], iza = hd.inv_z[rr];
+                const float mb = two ? hd.m2[rr + 4] : 0.f, izb = two ? hd.inv_z[rr + 4] : 0.f;
+                float *ra = tile + static_cast<long long>(rr) * p.Ck;
+                float *rb = ra + 4ll * p.Ck;
+                for (int c0 = 0; c0 < p.Ck; c0 += 1024) {
+                    float va[32], vb[32];
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        const int col = c0 + lane + 32 * k;
+                        va[k] = col < p.Ck ? ra[col] : 0.f;
+                        vb[k] = (two && col < p.Ck) ? rb[col] : 0.f;
+                    }
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        const int col = c0 + lane + 32 * k;
+                        if (col < p.Ck) {
+                            ra[col] = ex2(va[k] - ma) * iza;
+                            if (two) rb[col] = ex2(vb[k] - mb) * izb;
+                        }
+                    }
+                }
+            }
+            named_barrier_sync(1, 128);  // m2 / inv_z are reused by the next item
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
     }
 }
 
-template <int TM, int D>
-size_t score_smem_bytes(int Ck) {
-    return sizeof(float) * (static_cast<size_t>(128) * (D + 4) + TM * D + static_cast<size_t>(TM) * Ck);
+// [B*H, rows, D] fp32 view, box = 32 x box_rows x 1 with the 128-byte swizzle;
+// rows past `rows` read as zeros.
+bool make_f32_map(CUtensorMap *m, const float *base, long long BH, int rows, int D, int box_rows) {
+    TensorMapEncoder enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
+                                static_cast<cuuint64_t>(BH)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 4,
+                                   static_cast<cuuint64_t>(rows) * D * 4};
+    const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(box_rows), 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(base), dims, strides, box,
+               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int TM, int D>
+template <int D>
 cudaError_t launch_scores_t(const Geometry &g, const float *qc, const float *kc, float *probs,
                             cudaStream_t st) {
-    const size_t smem = score_smem_bytes<TM, D>(g.Ck);
-    cudaError_t e = cudaFuncSetAttribute(score_kernel<TM, D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    const long long BH = static_cast<long long>(g.B) * g.H;
+    CUtensorMap mq, mk;
+    if (!make_f32_map(&mq, qc, BH, g.Cq, D, sc::kRows) || !make_f32_map(&mk, kc, BH, g.Ck, D, sc::kCols))
+        return cudaErrorInvalidValue;
+    sc::Params p;
+    p.probs = probs;
+    p.Cq = g.Cq;
+    p.Ck = g.Ck;
+    p.S = g.S;
+    p.bk = g.bk;
+    p.n_rt = (g.Cq + sc::kRows - 1) / sc::kRows;
+    const long long items = BH * p.n_rt;
+    if (items > 0x7FFFFFFFll) return cudaErrorInvalidValue;
+    p.n_items = static_cast<int>(items);
+    p.scale2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+    cudaError_t e = cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         sc::kSmemAlloc);
     if (e != cudaSuccess) return e;
-    const long long grid = static_cast<long long>(g.B) * g.H * ((g.Cq + TM - 1) / TM);
-    score_kernel<TM, D><<<static_cast<unsigned>(grid), 256, smem, st>>>(
-        qc, kc, probs, g.S, g.bk, g.Cq, g.Ck, 1.0f / sqrtf(static_cast<float>(g.D)));
+    const int sms = sm_count();
+    if (sms <= 0) return cudaErrorInvalidValue;
+    const int grid = p.n_items < sms ? p.n_items : sms;
+    score_kernel<D><<<grid, sc::kThreads, sc::kSmemAlloc, st>>>(mq, mk, p);
     return cudaGetLastError();
 }
 
@@ -221,12 +499,8 @@ cudaError_t launch_pool(const Geometry &g, const void *q, const void *k, float *
 
 cudaError_t launch_scores(const Geometry &g, const float *qc, const float *kc, float *probs,
                           cudaStream_t st) {
-    if (g.Ck <= 1024) {
-        return g.D == 128 ? launch_scores_t<32, 128>(g, qc, kc, probs, st)
-                          : launch_scores_t<32, 64>(g, qc, kc, probs, st);
-    }
-    return g.D == 128 ? launch_scores_t<16, 128>(g, qc, kc, probs, st)
-                      : launch_scores_t<16, 64>(g, qc, kc, probs, st);
+    return g.D == 128 ? launch_scores_t<128>(g, qc, kc, probs, st)
+                      : launch_scores_t<64>(g, qc, kc, probs, st);
 }
 
 }  // namespace bsa
