@@ -11,7 +11,7 @@
 // Top-p without sorting: P' >= 0, so fp32 bit patterns order like the values,
 // and the kept set is every entry whose key (bits, -j) is at least the cut's.
 // The cut is found by an exact radix selection (below): histograms of integer
-// significand sums pick the binade, then 5 mantissa bits at a time, until at
+// significand sums pick the binade, then 4 mantissa bits at a time, until at
 // most 32 candidates remain; candidate m is kept iff it is the first of the
 // (P' desc, j asc) order or the mass strictly before it is below p -- the
 // shortest prefix of the sorted row whose running sum reaches p (at least one
@@ -72,11 +72,12 @@ __device__ __forceinline__ uint64_t warp_min_u64(uint64_t v) {
 // Exact radix selection of the cut.
 //
 // Keys order like (P' desc, j asc).  Level 1 histograms the fp32 exponent
-// field over the 31 binades below the row's largest one (binade r holds the
-// entries whose exponent is emax - r; everything further down lands in row 31,
-// the underflow bin); the later levels histogram 5 mantissa bits at a time
-// inside the chosen range, until at most 32 entries remain.  Each lane owns one
-// column of a 32 x 32 table in shared memory and adds (1 << 40 | mantissa) of
+// field over the 27 binades from the row's largest one down (binade r holds the
+// entries whose exponent is emax - r; everything further down lands in row
+// kUnder, the underflow bin); the later levels histogram 4 mantissa bits at a
+// time inside the chosen range, until at most 32 entries remain.  Each lane
+// owns one column of a kRowsTab x 32 table in shared memory (28 rows keep a
+// 4-warp CTA at 30 KB, so 7 CTAs fit an SM) and adds (1 << 40 | mantissa) of
 // its own entries to it; the implicit leading bits are added per bin from the
 // count, so a bin holds the exact integer sum of its entries' significands.
 // Within one binade masses are integers times one power of two, so every
@@ -86,12 +87,15 @@ __device__ __forceinline__ uint64_t warp_min_u64(uint64_t v) {
 // Padding slots (j >= Ck) hold +0.0, which has exponent field 0 and mantissa 0:
 // they add no mass, and their count is taken off the one bin they fall in.
 constexpr int kLanes = 32;
+constexpr int kRowsTab = 28;          // table rows
+constexpr int kUnder = kRowsTab - 1;  // level-1 row of everything below the binade window
+constexpr int kDigitBits = 4;         // mantissa bits per later level (16 rows)
 constexpr uint64_t kCountOne = 1ull << 40;
 constexpr uint64_t kSigMask = kCountOne - 1;
 constexpr uint64_t kImplicit = 1ull << 23;
 
 struct WarpScratch {
-    unsigned long long bins[32][kLanes];  // [row][lane]
+    unsigned long long bins[kRowsTab][kLanes];  // [row][lane]
     uint32_t cand_u[32];
     int cand_j[32];
 };
@@ -106,18 +110,20 @@ __device__ __forceinline__ double unit_of_binade(uint32_t e) {
     return __longlong_as_double(static_cast<long long>(k + 1023) << 52);
 }
 
-// Lane r returns the sum of row r and clears it.  Quarter-warps read 8
-// distinct bank groups thanks to the rotation.
+// Lane r < kRowsTab returns the sum of row r and clears it (other lanes 0).
+// Quarter-warps read 8 distinct bank groups thanks to the rotation.
 __device__ __forceinline__ unsigned long long bin_row_sum(unsigned long long (*bins)[kLanes],
                                                          int lane) {
-    ulonglong2 *row = reinterpret_cast<ulonglong2 *>(bins[lane]);
     unsigned long long acc = 0;
+    if (lane < kRowsTab) {
+        ulonglong2 *row = reinterpret_cast<ulonglong2 *>(bins[lane]);
 #pragma unroll
-    for (int k = 0; k < kLanes / 2; ++k) {
-        const int kk = (k + lane) & (kLanes / 2 - 1);
-        const ulonglong2 x = row[kk];
-        acc += x.x + x.y;
-        row[kk] = make_ulonglong2(0ull, 0ull);
+        for (int k = 0; k < kLanes / 2; ++k) {
+            const int kk = (k + lane) & (kLanes / 2 - 1);
+            const ulonglong2 x = row[kk];
+            acc += x.x + x.y;
+            row[kk] = make_ulonglong2(0ull, 0ull);
+        }
     }
     return acc;
 }
@@ -184,7 +190,7 @@ __device__ __noinline__ double mass_between(const float *__restrict__ src, int C
     return warp_sum_d(f);
 }
 
-// Cut inside the underflow range u <= hi (entries 31 or more binades below the
+// Cut inside the underflow range u <= hi (entries kUnder or more binades below the
 // row maximum), given that the row reaches p only there: fp64 bisection on the
 // bit pattern, then ties in ascending j.  Reached only when p lies within about
 // 2^-30 of the row total, so it re-reads the row from global memory instead of
@@ -237,35 +243,35 @@ __device__ __forceinline__ void find_cut(const float (&v)[VPL], const float *__r
     const double pd = static_cast<double>(p);
     const uint32_t emax = umax >> 23;
     const int npad = 32 * VPL - Ck;
-    // ---- level 1: binades emax .. emax-30 in rows 0..30, the rest in row 31
+    // ---- level 1: binades emax .. emax-(kUnder-1) in rows 0..kUnder-1, the rest in kUnder
 #pragma unroll
     for (int s = 0; s < VPL; ++s) {
         const uint32_t u = __float_as_uint(v[s]);
-        const uint32_t r = min(emax - (u >> 23), 31u);
+        const uint32_t r = min(emax - (u >> 23), static_cast<uint32_t>(kUnder));
         ws.bins[r][lane] += kCountOne | (u & 0x7FFFFFu);
     }
     __syncwarp();
     const unsigned long long acc1 = bin_row_sum(ws.bins, lane);
     __syncwarp();
-    const uint32_t pad_row = min(emax, 31u);
+    const uint32_t pad_row = min(emax, static_cast<uint32_t>(kUnder));
     const int cnt_r = static_cast<int>(acc1 >> 40) - (lane == static_cast<int>(pad_row) ? npad : 0);
     const uint32_t ex_r = emax - static_cast<uint32_t>(lane);  // exponent field of row `lane`
     double mass_r = 0.0;
-    if (lane < 31 && lane <= static_cast<int>(emax)) {
+    if (lane < kUnder && lane <= static_cast<int>(emax)) {
         const unsigned long long sig = (acc1 & kSigMask) +
             (ex_r > 0u ? kImplicit * static_cast<unsigned long long>(cnt_r) : 0ull);
         mass_r = static_cast<double>(sig) * unit_of_binade(ex_r);
     }
-    const double incl = scan_incl_d(mass_r, lane);  // row 31 adds nothing here
+    const double incl = scan_incl_d(mass_r, lane);  // rows kUnder.. add nothing here
     const int cincl = static_cast<int>(scan_incl_u64(static_cast<unsigned long long>(cnt_r), lane));
     double excl = __shfl_up_sync(0xffffffffu, incl, 1);
     if (lane == 0) excl = 0.0;
-    const uint32_t hit = __ballot_sync(0xffffffffu, lane < 31 && cnt_r > 0 && incl >= pd);
+    const uint32_t hit = __ballot_sync(0xffffffffu, lane < kUnder && cnt_r > 0 && incl >= pd);
     if (!hit) {
         // Binades emax..emax-30 do not reach p: the row total decides.
-        const double head = __shfl_sync(0xffffffffu, incl, 31);
-        const int n_under = __shfl_sync(0xffffffffu, cnt_r, 31);
-        const double tail = n_under > 0 ? mass_between(src, Ck, 0u, ((emax - 30u) << 23) - 1u, lane)
+        const double head = __shfl_sync(0xffffffffu, incl, kUnder);
+        const int n_under = __shfl_sync(0xffffffffu, cnt_r, kUnder);
+        const double tail = n_under > 0 ? mass_between(src, Ck, 0u, ((emax - static_cast<uint32_t>(kUnder - 1)) << 23) - 1u, lane)
                                         : 0.0;
         if (!(head + tail >= pd)) {
             ucut = 0u;
@@ -273,7 +279,7 @@ __device__ __forceinline__ void find_cut(const float (&v)[VPL], const float *__r
             return;
         }
         // Reaching p needs the underflow entries (tail > 0 here).
-        cut_in_underflow(src, Ck, pd, head, ((emax - 30u) << 23) - 1u, lane, &ucut, &jcut);
+        cut_in_underflow(src, Ck, pd, head, ((emax - static_cast<uint32_t>(kUnder - 1)) << 23) - 1u, lane, &ucut, &jcut);
         return;
     }
     const int b = __ffs(hit) - 1;
@@ -289,7 +295,7 @@ __device__ __forceinline__ void find_cut(const float (&v)[VPL], const float *__r
     uint32_t pre = e;
     int sh = 23;
     while (cnt > 32 && sh > 0) {
-        const int w = sh >= 5 ? 5 : sh;
+        const int w = sh >= kDigitBits ? kDigitBits : sh;
         sh -= w;
         const uint32_t top = (1u << w) - 1u;
 #pragma unroll
@@ -386,7 +392,7 @@ __device__ __forceinline__ float lg2_approx(float y) {
 }
 
 template <int VPL>
-__global__ void __launch_bounds__(128, VPL <= 16 ? 6 : VPL <= 32 ? 5 : 3)
+__global__ void __launch_bounds__(128, VPL <= 32 ? 7 : 3)
 mask_kernel(MaskArgs a, TopP tp) {
     __shared__ __align__(16) WarpScratch s_ws[4];
     const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
@@ -394,7 +400,7 @@ mask_kernel(MaskArgs a, TopP tp) {
     {   // clear this warp's table once; every level leaves it cleared
         ulonglong2 *t = reinterpret_cast<ulonglong2 *>(&ws.bins[0][0]);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) t[lane + 32 * k] = make_ulonglong2(0ull, 0ull);
+        for (int k = lane; k < kRowsTab * kLanes / 2; k += 32) t[k] = make_ulonglong2(0ull, 0ull);
         __syncwarp();
     }
     const long long row = static_cast<long long>(blockIdx.x) * 4 + wid;

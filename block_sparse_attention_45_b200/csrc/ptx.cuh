@@ -116,18 +116,6 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthread
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Barrier `id` over n threads that also ANDs a predicate across them.
-__device__ __forceinline__ bool bar_red_and(uint32_t id, uint32_t nthreads, bool x) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %2, 0;\n\t"
-        "bar.red.and.pred po, %1, %3, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
-        : "=r"(r)
-        : "r"(id), "r"(x ? 1u : 0u), "r"(nthreads)
-        : "memory");
-    return r != 0;
-}
-
 // ---------------------------------------------------------------- tcgen05 / TMEM
 
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {

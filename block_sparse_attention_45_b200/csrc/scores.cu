@@ -109,9 +109,10 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint4 *__restrict__ q,
 //   warps 4-7   split workers: hi/lo in place for each landed stage
 //   warps 8-11  epilogue: thread = query-block row (TMEM lane); per 32-column
 //               slice s2 = acc * log2(e)/sqrt(D) + log2 n_j, a running row
-//               max m2 and sum z of 2^(s2 - m2); the slice goes through shared
-//               memory so a warp writes one row's 32 values contiguously.  After
-//               the last chunk a warp per row rewrites s2 -> 2^(s2 - m2) / z.
+//               max m2 and sum z of 2^(s2 - m2); each warp transposes its own
+//               32 x 32 slice through shared memory so it writes one row's 32
+//               values contiguously.  After the last chunk the warp rewrites its
+//               rows s2 -> 2^(s2 - m2) / z, a row at a time across the warp.
 namespace sc {
 
 constexpr int kThreads = 384;
@@ -321,23 +322,26 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
         }
     } else if (warp >= 8) {
         // ------------------------------------------------------------ epilogue
-        // Named barrier 1 over the 128 epilogue threads.  Every bounded wait is
-        // followed by a vote (bar.red.and), so the four warps leave together and
-        // no bar.sync can wait for a warp that is gone.
+        // Warp ew owns rows 32*ew .. 32*ew+31 of the tile (its TMEM lanes) for the
+        // whole item: it transposes its own 32 x 32 slices in a private staging
+        // block and normalises its own rows, so the four warps never wait for one
+        // another.
         const int ew = warp - 8;
         const int rl = ew * 32 + lane;  // row within the tile = TMEM lane
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(ew * 32) << 16);
+        float *wst = stg + ew * 32 * kPitch;  // this warp's 32 x kPitch staging block
         int ch = 0;
         bool ok = true;
         for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
             const int bh = item / p.n_rt, r0 = (item % p.n_rt) * kRows;
             const int nrows = min(kRows, p.Cq - r0);
-            float *tile = p.probs + (static_cast<long long>(bh) * p.Cq + r0) * p.Ck;
+            const int my_rows = max(0, min(32, nrows - ew * 32));  // rows of this warp
+            float *wtile = p.probs + (static_cast<long long>(bh) * p.Cq + r0 + ew * 32) * p.Ck;
             float m2 = -INFINITY, z = 0.f;
             for (int c = 0; c < nch; ++c, ++ch) {
                 const int buf = ch & 1;
-                const bool got = mbar_wait(&hd.acc_full[buf], (ch >> 1) & 1, abort_flag);
-                if (!bar_red_and(1, 128, got)) {
+                if (!__all_sync(0xffffffffu,
+                                mbar_wait(&hd.acc_full[buf], (ch >> 1) & 1, abort_flag))) {
                     ok = false;
                     break;
                 }
@@ -373,21 +377,19 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
                     z = z * ex2(m2 - mn) + sum;
                     m2 = mn;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) stg[rl * kPitch + j] = __uint_as_float(r[j]);
-                    named_barrier_sync(1, 128);
-                    // warp ew writes rows ew, ew+4, ...: all 32 staging reads first
+                    for (int j = 0; j < 32; ++j) wst[lane * kPitch + j] = __uint_as_float(r[j]);
+                    __syncwarp();
+                    // row i of this warp: 32 consecutive columns, one 128-byte store
                     const int col = col0 + lane;
                     if (col < p.Ck) {
-                        float v[kRows / 4];
+                        float v[32];
 #pragma unroll
-                        for (int i = 0; i < kRows / 4; ++i) v[i] = stg[(ew + 4 * i) * kPitch + lane];
-                        float *dst = tile + static_cast<long long>(ew) * p.Ck + col;
-                        const long long step = 4ll * p.Ck;
+                        for (int i = 0; i < 32; ++i) v[i] = wst[i * kPitch + lane];
 #pragma unroll
-                        for (int i = 0; i < kRows / 4; ++i)
-                            if (ew + 4 * i < nrows) dst[i * step] = v[i];
+                        for (int i = 0; i < 32; ++i)
+                            if (i < my_rows) wtile[static_cast<long long>(i) * p.Ck + col] = v[i];
                     }
-                    named_barrier_sync(1, 128);
+                    __syncwarp();
                     tmem_ld_wait();  // the prefetched slice has landed
                     reg_fence(nxt);
                 }
@@ -395,18 +397,18 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
                 mbar_arrive(&hd.acc_empty[buf]);
             }
             if (!ok) break;
-            // P' = 2^(s2 - m2) / z, one warp per row, every load of a 1024-column
-            // segment issued before the arithmetic on it
+            // P' = 2^(s2 - m2) / z for this warp's rows, one row at a time across the
+            // warp (coalesced), two rows in flight
             hd.m2[rl] = m2;
             hd.inv_z[rl] = 1.0f / z;
-            named_barrier_sync(1, 128);
-            // two rows at a time: 64 loads in flight per lane
-            for (int rr = ew; rr < nrows; rr += 8) {
-                const bool two = rr + 4 < nrows;
-                const float ma = hd.m2[rr], iza = hd.inv_z[rr];
-                const float mb = two ? hd.m2[rr + 4] : 0.f, izb = two ? hd.inv_z[rr + 4] : 0.f;
-                float *ra = tile + static_cast<long long>(rr) * p.Ck;
-                float *rb = ra + 4ll * p.Ck;
+            __syncwarp();
+            for (int i = 0; i < my_rows; i += 2) {
+                const bool two = i + 1 < my_rows;
+                const float ma = hd.m2[ew * 32 + i], iza = hd.inv_z[ew * 32 + i];
+                const float mb = two ? hd.m2[ew * 32 + i + 1] : 0.f;
+                const float izb = two ? hd.inv_z[ew * 32 + i + 1] : 0.f;
+                float *ra = wtile + static_cast<long long>(i) * p.Ck;
+                float *rb = ra + p.Ck;
                 for (int c0 = 0; c0 < p.Ck; c0 += 1024) {
                     float va[32], vb[32];
 #pragma unroll
@@ -425,7 +427,7 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
                     }
                 }
             }
-            named_barrier_sync(1, 128);  // m2 / inv_z are reused by the next item
+            __syncwarp();  // m2 / inv_z of this warp's rows are reused by the next item
         }
     }
     __syncthreads();
