@@ -123,7 +123,10 @@ constexpr int kBPanelBytes = kCols * 128;            // 256 rows x 32 fp32
 constexpr int kStageBytes = 2 * (kAPanelBytes + kBPanelBytes);  // A, A_lo, B, B_lo
 constexpr int kStages = 2;
 constexpr int kTmemCols = 2 * kCols;
-constexpr int kPitch = 33;                           // staging row pitch (floats)
+// Staging row pitch (floats): a multiple of 4, so a lane writes its row with
+// 16-byte stores (conflict-free per quarter-warp), and 4i + lane keeps the
+// column reads of one row conflict-free.
+constexpr int kPitch = 36;
 
 struct Header {
     uint64_t full[kStages];    // TMA landed (expect_tx)
@@ -377,7 +380,9 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
                     z = z * ex2(m2 - mn) + sum;
                     m2 = mn;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) wst[lane * kPitch + j] = __uint_as_float(r[j]);
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<uint4 *>(wst + lane * kPitch + j) =
+                            make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]);
                     __syncwarp();
                     // row i of this warp: 32 consecutive columns, one 128-byte store
                     const int col = col0 + lane;
