@@ -64,6 +64,9 @@ class Oracle:
         L.ora_lists.argtypes = [lp, vp, vp, vp]
         L.ora_attention.argtypes = [lp, vp, vp, vp, vp, ctypes.c_double, ctypes.c_long,
                                     vp, vp, vp]
+        L.ora_value_norms.argtypes = [lp, vp, vp]
+        L.ora_eg_route.argtypes = [lp, vp, vp]
+        L.ora_eg_select.argtypes = [lp, vp, vp, vp, ctypes.c_float, vp, vp]
         L.ora_num_threads.restype = ctypes.c_int
         self.lib = L
 
@@ -158,6 +161,52 @@ class Oracle:
         self.lib.ora_attention(ctypes.byref(L), _ptr(q), _ptr(k), _ptr(v), _ptr(m),
                                float(scale), n, _ptr(r), _ptr(out), _ptr(lse))
         return out, lse
+
+    def value_norms(self, L, v):
+        """||c^V_{h,j}||_2 of the value centroids, fp32 [B,H,C_k]."""
+        L = _layout(L)
+        v = _u16(v)
+        out = np.empty((L.batch, L.heads, L.ck), np.float32)
+        self.lib.ora_value_norms(ctypes.byref(L), _ptr(v), _ptr(out))
+        return out
+
+    def eg_route(self, L, H):
+        """Median split per batch entry: u8 [B,H], 1 for the floor(H/2) lowest-entropy heads."""
+        L = _layout(L)
+        H = np.ascontiguousarray(H, np.float64)
+        low = np.empty((L.batch, L.heads), np.uint8)
+        self.lib.ora_eg_route(ctypes.byref(L), _ptr(H), _ptr(low))
+        return low
+
+    def eg_select(self, L, probs, vnorm, top_p, pool_p, low):
+        """Entropy-guided selection mask u8 [B,H,C_q,C_k] (no overrides): per-row top-p for
+        the heads with low == 0, one cross-head pool per batch entry for the others.
+        vnorm None ranks the pool by P' alone."""
+        L = _layout(L)
+        probs = np.ascontiguousarray(probs, np.float32)
+        vn = None if vnorm is None else np.ascontiguousarray(vnorm, np.float32)
+        tp = np.ascontiguousarray(np.broadcast_to(np.asarray(top_p, np.float32), (L.heads,)))
+        low = np.ascontiguousarray(low, np.uint8)
+        mask = np.empty((L.batch, L.heads, L.cq, L.ck), np.uint8)
+        self.lib.ora_eg_select(ctypes.byref(L), _ptr(probs), _ptr(vn), _ptr(tp), float(pool_p),
+                               _ptr(low), _ptr(mask))
+        return mask
+
+    def eg_selection(self, L, q, k, v, top_p, pool_p, flags, eps=1e-8, value_aware=True):
+        """The entropy-guided selection stage: centroids, P', entropy, median split,
+        per-row / pooled top-p with the safeguard, overrides, lists."""
+        L = _layout(L)
+        qc = self.pool(L, q, L.q_block)
+        kc = self.pool(L, k, L.k_block)
+        probs = self.scores(L, qc, kc)
+        H, Hn = self.entropy(L, probs, eps)
+        low = self.eg_route(L, H)
+        vn = self.value_norms(L, v) if value_aware else None
+        smask = self.eg_select(L, probs, vn, top_p, pool_p, low)
+        m = self.overrides(L, flags, smask)
+        idx, cnt = self.lists(L, m)
+        return dict(probs=probs, entropy=H, entropy_norm=Hn, low=low, vnorm=vn, sel_mask=smask,
+                    mask=m, kv_index=idx, kv_count=cnt)
 
     def select(self, L, q, k, top_p, flags, eps=1e-8):
         """The whole selection stage: centroids, P', entropy, top-p, overrides, lists."""

@@ -20,7 +20,9 @@
  *       s3 setup: centroids with cluster sizes n_i, n_j and the
  *       cluster-size-weighted softmax P' (Eq. 1, rows sum to one);
  *       per-head entropy H_h (Eq. 3) and its normalisation by log C_k;
- *       domain 1 "per-row local" top-p (Eq. 2).
+ *       domain 1 "per-row local" top-p (Eq. 2); domain 3 "grouped
+ *       cross-head" with the median split on H_h and the safeguard; s4 the
+ *       value-aware score of the cross-head pool (EG-Sparse).
  *  [p5] "AB-Attention: accurate block-sparse attention for video diffusion"
  *       TL;DR: exact attention computed only on the selected K/V blocks.
  *
@@ -324,6 +326,175 @@ void ora_attention(const ora_layout *L, const uint16_t *q, const uint16_t *k, co
         free(s);
         free(u_of);
         free(acc);
+    }
+}
+
+/*
+ * ---------------------------------------------------------------------------
+ * Entropy-guided competition domains ([p3] s3.3 domain 3 "Grouped
+ * cross-head", the minimum one-key-per-row safeguard; s4 the value-aware
+ * importance score in the cross-head pool).  Readings where the page is
+ * silent (its equations are lost in the extracted text):
+ *  - the value centroid c^V_{h,j} is the mean of V over key block j's valid
+ *    tokens (like the key centroid), and the score of a pool pair is
+ *    I_{h,i,j} = P'_{h,i,j} * ||c^V_{h,j}||_2, the product of the two fp32
+ *    values rounded to fp32;
+ *  - "split by the median of H_h": per batch entry, heads ordered by
+ *    (H_h ascending, h ascending); the first floor(H/2) are the low-entropy
+ *    heads (an odd middle head stays with the high-entropy, per-row heads);
+ *  - a pool's top-p keeps the shortest prefix of its (I desc, h, i, j asc)
+ *    order whose fp64 running sum reaches pool_p times the pool's total
+ *    (rows of a pool are not normalised to one as a single row is);
+ *  - the safeguard gives an empty pool row its highest-scoring key block
+ *    (lowest j on ties), by the pool's score.
+ * ---------------------------------------------------------------------------
+ */
+
+/* ||c^V_{h,j}||_2 with the centroid a fp64 mean over the block's valid tokens
+ * in ascending token order; fp32 [B,H,C_k]. */
+void ora_value_norms(const ora_layout *L, const uint16_t *v, float *out)
+{
+    const int D = L->head_dim, Ck = L->seq_pad / L->k_block;
+    const long BH = (long)L->batch * L->heads;
+    #pragma omp parallel for schedule(static)
+    for (long r = 0; r < BH * Ck; ++r) {
+        long bh = r / Ck;
+        int j = (int)(r % Ck);
+        int n = ora_block_count(L->seq_len, L->k_block, j);
+        const uint16_t *base = v + (bh * L->seq_pad + (long)j * L->k_block) * D;
+        double ss = 0.0;
+        for (int d = 0; d < D; ++d) {
+            double s = 0.0;
+            for (int t = 0; t < n; ++t) s += bf16_val(base[(long)t * D + d]);
+            double c = n > 0 ? s / n : 0.0;
+            ss += c * c;
+        }
+        out[r] = (float)sqrt(ss);
+    }
+}
+
+typedef struct { double H; int h; } ora_head;
+
+static int ora_head_cmp(const void *a, const void *b)
+{
+    const ora_head *x = (const ora_head *)a, *y = (const ora_head *)b;
+    if (x->H < y->H) return -1;
+    if (x->H > y->H) return 1;
+    return (x->h > y->h) - (x->h < y->h);
+}
+
+/* Median split of the heads of every batch entry: low[b,h] = 1 for the
+ * floor(H/2) heads first in (H_h asc, h asc) order, else 0.  H is [B,H]. */
+void ora_eg_route(const ora_layout *L, const double *H, uint8_t *low)
+{
+    const int nh = L->heads;
+    ora_head *o = (ora_head *)malloc(sizeof(ora_head) * nh);
+    for (int b = 0; b < L->batch; ++b) {
+        for (int h = 0; h < nh; ++h) {
+            o[h].H = H[(long)b * nh + h];
+            o[h].h = h;
+        }
+        qsort(o, (size_t)nh, sizeof(ora_head), ora_head_cmp);
+        for (int h = 0; h < nh; ++h) low[(long)b * nh + h] = 0;
+        for (int k = 0; k < nh / 2; ++k) low[(long)b * nh + o[k].h] = 1;
+    }
+    free(o);
+}
+
+typedef struct { float I; int h, i, j; } ora_pair;
+
+static int ora_pair_cmp(const void *a, const void *b)
+{
+    const ora_pair *x = (const ora_pair *)a, *y = (const ora_pair *)b;
+    if (x->I > y->I) return -1;
+    if (x->I < y->I) return 1;
+    if (x->h != y->h) return (x->h > y->h) - (x->h < y->h);
+    if (x->i != y->i) return (x->i > y->i) - (x->i < y->i);
+    if (x->j != y->j) return x->j < y->j ? -1 : 1;
+    return 0;
+}
+
+/* Score of pair (bh, i, j) in the cross-head pool: P' * ||c^V||, rounded to
+ * fp32, or P' itself when there are no value norms. */
+static float ora_pool_score(const float *probs, const float *vnorm, long bh, int Cq, int Ck,
+                            int i, int j)
+{
+    float p = probs[(bh * Cq + i) * (long)Ck + j];
+    if (!vnorm) return p;
+    float v = vnorm[bh * Ck + j];
+    return p * v;
+}
+
+/*
+ * Entropy-guided selection.  Heads with low[b,h] == 0 keep the per-row local
+ * top-p of ora_topp with p = top_p[h].  For every batch entry, all pairs
+ * (h,i,j) of its low heads form one pool ranked by I in (I desc, h, i, j asc)
+ * order; the pool keeps its first k* pairs, k* = min{k >= 1 : c_k >= pool_p * T}
+ * with c_k the fp64 running sum of the first k fp32 scores and T = c_N, or
+ * every pair when no k qualifies.  Then every pool row (h,i) left without a
+ * kept pair keeps its highest-scoring key block.  mask is u8 [B,H,C_q,C_k].
+ */
+void ora_eg_select(const ora_layout *L, const float *probs, const float *vnorm,
+                   const float *top_p, float pool_p, const uint8_t *low, uint8_t *mask)
+{
+    const int Cq = L->seq_pad / L->q_block, Ck = L->seq_pad / L->k_block;
+    const int nh = L->heads;
+    /* per-row heads: the domain-1 rule, whole layout at once */
+    ora_topp(L, probs, top_p, mask, NULL);
+    for (int b = 0; b < L->batch; ++b) {
+        long n = 0;
+        for (int h = 0; h < nh; ++h)
+            if (low[(long)b * nh + h]) n += (long)Cq * Ck;
+        if (n == 0) continue;
+        ora_pair *e = (ora_pair *)malloc(sizeof(ora_pair) * (size_t)n);
+        long k = 0;
+        for (int h = 0; h < nh; ++h) {
+            if (!low[(long)b * nh + h]) continue;
+            long bh = (long)b * nh + h;
+            for (int i = 0; i < Cq; ++i) {
+                memset(mask + (bh * Cq + i) * (long)Ck, 0, (size_t)Ck);
+                for (int j = 0; j < Ck; ++j) {
+                    e[k].I = ora_pool_score(probs, vnorm, bh, Cq, Ck, i, j);
+                    e[k].h = h;
+                    e[k].i = i;
+                    e[k].j = j;
+                    ++k;
+                }
+            }
+        }
+        qsort(e, (size_t)n, sizeof(ora_pair), ora_pair_cmp);
+        double T = 0.0;
+        for (long t = 0; t < n; ++t) T += (double)e[t].I;
+        const double target = (double)pool_p * T;
+        long kstar = n;
+        double c = 0.0;
+        for (long t = 0; t < n; ++t) {
+            c += (double)e[t].I;
+            if (c >= target) { kstar = t + 1; break; }
+        }
+        for (long t = 0; t < kstar; ++t) {
+            long bh = (long)b * nh + e[t].h;
+            mask[(bh * Cq + e[t].i) * (long)Ck + e[t].j] = 1;
+        }
+        free(e);
+        /* safeguard: an empty pool row keeps its best key block */
+        for (int h = 0; h < nh; ++h) {
+            if (!low[(long)b * nh + h]) continue;
+            long bh = (long)b * nh + h;
+            for (int i = 0; i < Cq; ++i) {
+                uint8_t *m = mask + (bh * Cq + i) * (long)Ck;
+                int any = 0;
+                for (int j = 0; j < Ck; ++j) any |= m[j];
+                if (any) continue;
+                int best = 0;
+                float bv = ora_pool_score(probs, vnorm, bh, Cq, Ck, i, 0);
+                for (int j = 1; j < Ck; ++j) {
+                    float x = ora_pool_score(probs, vnorm, bh, Cq, Ck, i, j);
+                    if (x > bv) { bv = x; best = j; }
+                }
+                m[best] = 1;
+            }
+        }
     }
 }
 

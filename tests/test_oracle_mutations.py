@@ -27,13 +27,25 @@ MUTATIONS = [
     ("ties to the higher index", "return (x->j > y->j) - (x->j < y->j);",
      "return (x->j < y->j) - (x->j > y->j);"),
     ("ascending order", "if (x->p > y->p) return -1;", "if (x->p > y->p) return 1;"),
-    ("pool divides by block size", "s / n : 0.0", "s / block : 0.0"),
+    ("pool divides by block size", "out[r * D + d] = (float)(n > 0 ? s / n : 0.0);",
+     "out[r * D + d] = (float)(n > 0 ? s / block : 0.0);"),
     ("text blocks floored", "(L->text_len + L->k_block - 1) / L->k_block", "L->text_len / L->k_block"),
     ("padded keys attended", "int cnt = ora_block_count(L->seq_len, bk, j);", "int cnt = bk;"),
     ("attention scale dropped", "s[a] = dot * scale;", "s[a] = dot;"),
     ("lse without log", "(float)(m + log(z))", "(float)(m + z)"),
     ("text keep on query rows", "for (int j = 0; j < tk; ++j) m[j] = 1;",
      "for (int j = 0; j < tk && i < tk; ++j) m[j] = 1;"),
+    ("value norm of the block sum", "double c = n > 0 ? s / n : 0.0;", "double c = s;"),
+    ("high-entropy heads pooled", "low[(long)b * nh + o[k].h] = 1;", "low[(long)b * nh + o[nh - 1 - k].h] = 1;"),
+    ("pool ranked by P' alone", "return p * v;", "return p;"),
+    ("pool target not scaled by the total", "const double target = (double)pool_p * T;",
+     "const double target = (double)pool_p;"),
+    ("pool cut entry excluded", "if (c >= target)", "if (c > target)"),
+    ("pool ties by descending row", "if (x->i != y->i) return (x->i > y->i) - (x->i < y->i);",
+     "if (x->i != y->i) return (x->i < y->i) - (x->i > y->i);"),
+    ("no safeguard", "m[best] = 1;", "(void)best;"),
+    ("safeguard takes the last maximum", "if (x > bv) { bv = x; best = j; }",
+     "if (x >= bv) { bv = x; best = j; }"),
 ]
 
 

@@ -391,5 +391,141 @@ def test_pipeline_invariants(ora):
     check_pipeline(ora)
 
 
+# --------------------------------------------------------------------------- entropy-guided domains
+
+def check_value_norms(ora):
+    # constant vector per block: the norm is that vector's; padded tokens (garbage) do not count
+    D = 4
+    L = lay(seq_len=14, seq_pad=16, D=D, bq=4, bk=4, heads=2)
+    rng = np.random.default_rng(11)
+    c = np.round(rng.normal(size=(1, 2, 4, D)) * 8) / 8           # exact in bf16
+    v = np.repeat(c, 4, axis=2).astype(np.float32)                 # [1, 2, 16, D]
+    v[:, :, 14:, :] = 1000.0                                       # padding
+    got = ora.value_norms(L, bits(v))
+    exp = np.sqrt((c.astype(np.float64) ** 2).sum(-1)).astype(np.float32)
+    assert np.array_equal(got, exp), (got, exp)
+    # a block whose tokens differ: the norm of the mean, not the mean of the norms
+    v = np.zeros((1, 1, 4, 2), np.float32)
+    v[0, 0, :, 0] = [1.0, -1.0, 3.0, -3.0]
+    v[0, 0, :, 1] = [2.0, 2.0, 2.0, 2.0]
+    L1 = lay(seq_len=4, seq_pad=4, D=2, bq=4, bk=4)
+    assert ora.value_norms(L1, bits(v))[0, 0, 0] == np.float32(2.0)
+
+
+def check_eg_route(ora):
+    def low(H):
+        H = np.asarray(H, np.float64)
+        L = lay(seq_len=4, seq_pad=4, heads=H.shape[1], batch=H.shape[0])
+        return ora.eg_route(L, H).tolist()
+    assert low([[0.3, 0.1, 0.5, 0.2]]) == [[0, 1, 0, 1]]
+    assert low([[0.2, 0.4, 0.1]]) == [[0, 0, 1]]                   # odd H: floor(H/2) low heads
+    assert low([[0.2, 0.2, 0.3, 0.4]]) == [[1, 1, 0, 0]]
+    assert low([[0.5, 0.5, 0.5, 0.5]]) == [[1, 1, 0, 0]]           # ties: lower head index first
+    assert low([[0.1, 0.9], [0.9, 0.1]]) == [[1, 0], [0, 1]]       # per batch entry
+    assert low([[0.7]]) == [[0]]                                   # one head: nothing pooled
+
+
+def _brute_pool(I, target):
+    """Smallest subset of the flat scores with mass >= target; the heaviest among those."""
+    n = len(I)
+    v = I.astype(np.float64)
+    for k in range(1, n + 1):
+        best = None
+        for sub in itertools.combinations(range(n), k):
+            m = float(v[list(sub)].sum())
+            if m >= target:
+                key = (-m, sub)
+                if best is None or key < best:
+                    best = key
+        if best is not None:
+            return set(best[1])
+    return set(range(n))
+
+
+def check_eg_select(ora):
+    # a one-row pool with vnorm = 1 is the per-row rule (dyadic row: the pool total is exactly 1)
+    L = lay(seq_len=16, seq_pad=16, D=4, bq=16, bk=4, heads=2)
+    row = np.array([0.125, 0.5, 0.125, 0.25], np.float32)
+    P = np.broadcast_to(row, (1, 2, 1, 4)).copy()
+    low = np.array([[1, 0]], np.uint8)
+    for p in (0.75, 0.7, 0.76, 0.5, 1e-6, 1.0):
+        m = ora.eg_select(L, P, np.ones((1, 2, 4), np.float32), [p, p], p, low)
+        ref, _ = ora.topp(L, P, p)
+        assert np.array_equal(m, ref), p
+    # brute force on small pools: heads 0 and 2 pooled, head 1 per-row
+    rng = np.random.default_rng(5)
+    H, Cq, Ck = 3, 2, 3
+    L = lay(seq_len=12, seq_pad=12, D=4, bq=6, bk=4, heads=H)
+    low = np.array([[1, 0, 1]], np.uint8)
+    for trial in range(25):
+        P = rng.dirichlet(np.full(Ck, 0.8), size=(1, H, Cq)).astype(np.float32)
+        vn = rng.uniform(0.2, 3.0, size=(1, H, Ck)).astype(np.float32)
+        pp = float(np.float32(rng.uniform(0.1, 0.95)))
+        tp = [0.6, 0.6, 0.6]
+        m = ora.eg_select(L, P, vn, tp, pp, low)
+        # pooled pairs in (h, i, j) order, scores rounded to fp32
+        pairs = [(h, i, j) for h in (0, 2) for i in range(Cq) for j in range(Ck)]
+        I = np.array([P[0, h, i, j] * vn[0, h, j] for (h, i, j) in pairs], np.float32)
+        keep = _brute_pool(I, np.float64(np.float32(pp)) * I.astype(np.float64).sum())
+        exp = np.zeros_like(m)
+        for t in keep:
+            h, i, j = pairs[t]
+            exp[0, h, i, j] = 1
+        for h in (0, 2):
+            for i in range(Cq):
+                if not exp[0, h, i].any():                         # safeguard
+                    exp[0, h, i, int(np.argmax(P[0, h, i] * vn[0, h]))] = 1
+        exp[0, 1] = ora.topp(lay(seq_len=12, seq_pad=12, D=4, bq=6, bk=4), P[:, 1:2], 0.6)[0][0, 0]
+        if not np.array_equal(m, exp):
+            raise AssertionError((trial, m, exp))
+    # p <= 0: the pool keeps its best pair only; every other pool row gets its own argmax
+    P = rng.dirichlet(np.full(Ck, 0.8), size=(1, H, Cq)).astype(np.float32)
+    vn = rng.uniform(0.2, 3.0, size=(1, H, Ck)).astype(np.float32)
+    m = ora.eg_select(L, P, vn, [0.6] * 3, -1.0, low)
+    for h in (0, 2):
+        for i in range(Cq):
+            exp = np.zeros(Ck, np.uint8)
+            exp[int(np.argmax(P[0, h, i] * vn[0, h]))] = 1
+            assert np.array_equal(m[0, h, i], exp), (h, i)
+    # p above one: every pooled pair
+    m = ora.eg_select(L, P, vn, [0.6] * 3, 1.5, low)
+    assert m[0, 0].all() and m[0, 2].all()
+    # ranking by P' alone when there are no value norms, and ties to the lower j in the safeguard
+    P = np.zeros((1, H, Cq, Ck), np.float32)
+    P[0, 0, 0] = [0.9, 0.05, 0.05]
+    P[0, 0, 1] = [1 / 3, 1 / 3, 1 / 3]                             # tied row, left empty by the pool
+    P[0, 2] = [[0.8, 0.1, 0.1], [0.7, 0.2, 0.1]]
+    P[0, 1] = 1 / 3
+    m = ora.eg_select(L, P, None, [0.6] * 3, 0.5, low)
+    assert m[0, 0, 0].tolist() == [1, 0, 0] and m[0, 0, 1].tolist() == [1, 0, 0]
+    assert m[0, 2, 0].tolist() == [1, 0, 0] and m[0, 2, 1].tolist() == [1, 0, 0]
+    # tied scores in two rows at the cut: the lower (h, i) is kept (neither row empties)
+    P = np.zeros((1, H, Cq, Ck), np.float32)
+    P[0, 0, 0] = [0.4, 0.6, 0.0]
+    P[0, 0, 1] = [0.6, 0.4, 0.0]
+    P[0, 2, :, 0] = 1.0
+    P[0, 1] = 1 / 3
+    m = ora.eg_select(L, P, None, [0.6] * 3, 0.875, low)           # target 3.5 of 4: one 0.4 kept
+    assert m[0, 0, 0].tolist() == [1, 1, 0] and m[0, 0, 1].tolist() == [1, 0, 0], m[0, 0]
+    # with value norms the small-P' column with a large value centroid wins its place
+    vn = np.ones((1, H, Ck), np.float32)
+    vn[0, 0, 1] = 40.0
+    m = ora.eg_select(L, P, vn, [0.6] * 3, 0.5, low)
+    assert m[0, 0, 0, 1] == 1
+
+
+def test_eg_value_norms(ora):
+    check_value_norms(ora)
+
+
+def test_eg_route(ora):
+    check_eg_route(ora)
+
+
+def test_eg_select(ora):
+    check_eg_select(ora)
+
+
 ALL_CHECKS = [check_geometry, check_pooling, check_scores, check_entropy, check_topp,
-              check_overrides_lists, check_attention, check_pipeline]
+              check_overrides_lists, check_attention, check_pipeline, check_value_norms,
+              check_eg_route, check_eg_select]
