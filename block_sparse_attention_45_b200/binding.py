@@ -76,6 +76,13 @@ def load():
         L.bsa_sparse_attention_host.restype = ctypes.c_int
         L.bsa_pipeline_workspace_bytes.argtypes = [lp, ctypes.c_int]
         L.bsa_pipeline_workspace_bytes.restype = ctypes.c_size_t
+        L.bsa_value_norms.argtypes = [lp, vp, vp, vp]
+        L.bsa_value_norms.restype = ctypes.c_int
+        L.bsa_build_mask_eg.argtypes = [lp, vp, vp, vp, ctypes.c_float, ctypes.c_uint32,
+                                        ctypes.c_float, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.bsa_build_mask_eg.restype = ctypes.c_int
+        L.bsa_build_mask_eg_workspace_bytes.argtypes = [lp]
+        L.bsa_build_mask_eg_workspace_bytes.restype = ctypes.c_size_t
         L.bsa_status_string.argtypes = [ctypes.c_int]
         L.bsa_status_string.restype = ctypes.c_char_p
         L.bsa_version.restype = ctypes.c_int
@@ -194,6 +201,59 @@ def build_mask(layout, probs, top_p, flags, eps=1e-8, mask=None, kv_index=None, 
     _check("bsa_build_mask", rc)
     return dict(mask=mask, kv_index=kv_index, kv_count=kv_count, entropy=entropy,
                 entropy_norm=entropy_norm)
+
+
+def value_norms(layout, v, vnorm=None, stream=None):
+    """bsa_value_norms: ||c^V_{h,j}||_2 of the value centroids, fp32 [B,H,C_k]."""
+    L = make_layout(layout)
+    d = dims(L)
+    _need(v, "v", torch.bfloat16, (d["B"], d["H"], L.seq_pad, L.head_dim))
+    if vnorm is None:
+        vnorm = torch.empty((d["B"], d["H"], d["Ck"]), dtype=torch.float32, device=v.device)
+    _check("bsa_value_norms", load().bsa_value_norms(ctypes.byref(L), _ptr(v), _ptr(vnorm),
+                                                     _stream(stream)))
+    return vnorm
+
+
+def eg_workspace_bytes(layout):
+    L = make_layout(layout)
+    return int(load().bsa_build_mask_eg_workspace_bytes(ctypes.byref(L)))
+
+
+def build_mask_eg(layout, probs, vnorm, top_p, pool_p, flags, eps=1e-8, mask=None,
+                  kv_index=None, kv_count=None, workspace=None, with_mask=True, stream=None):
+    """bsa_build_mask_eg (entropy-guided grouped cross-head selection): returns
+    dict(mask, kv_index, kv_count, entropy, entropy_norm, low_heads).  vnorm None
+    ranks the pools by P' alone."""
+    L = make_layout(layout)
+    d = dims(L)
+    _need(probs, "probs", torch.float32, (d["B"], d["H"], d["Cq"], d["Ck"]))
+    if vnorm is not None:
+        _need(vnorm, "vnorm", torch.float32, (d["B"], d["H"], d["Ck"]))
+    dev = probs.device
+    vals = list(top_p) if hasattr(top_p, "__len__") else [top_p] * d["H"]
+    if len(vals) != d["H"]:
+        raise ValueError("top_p needs one value per head")
+    tp = (ctypes.c_float * d["H"])(*[float(x) for x in vals])
+    if mask is None and with_mask:
+        mask = torch.empty((d["B"], d["H"], d["Cq"], d["Ck"]), dtype=torch.uint8, device=dev)
+    if kv_index is None:
+        kv_index = torch.empty((d["B"], d["H"], d["Cq"], d["Ck"]), dtype=torch.int32, device=dev)
+    if kv_count is None:
+        kv_count = torch.empty((d["B"], d["H"], d["Cq"]), dtype=torch.int32, device=dev)
+    entropy = torch.empty((d["B"], d["H"]), dtype=torch.float32, device=dev)
+    entropy_norm = torch.empty((d["B"], d["H"]), dtype=torch.float32, device=dev)
+    low = torch.empty((d["B"], d["H"]), dtype=torch.uint8, device=dev)
+    if workspace is None:
+        workspace = torch.empty(eg_workspace_bytes(L), dtype=torch.uint8, device=dev)
+    rc = load().bsa_build_mask_eg(ctypes.byref(L), _ptr(probs), _ptr(vnorm),
+                                  ctypes.cast(tp, ctypes.c_void_p), float(pool_p), int(flags),
+                                  float(eps), _ptr(mask), _ptr(kv_index), _ptr(kv_count),
+                                  _ptr(entropy), _ptr(entropy_norm), _ptr(low), _ptr(workspace),
+                                  _stream(stream))
+    _check("bsa_build_mask_eg", rc)
+    return dict(mask=mask, kv_index=kv_index, kv_count=kv_count, entropy=entropy,
+                entropy_norm=entropy_norm, low_heads=low)
 
 
 def attention_workspace_bytes(layout):

@@ -158,6 +158,50 @@ int bsa_build_mask(const bsa_layout *layout, const float *probs, const float *to
     return launch_status(bsa::launch_entropy_reduce(g, row_ent, entropy, entropy_norm, st));
 }
 
+int bsa_value_norms(const bsa_layout *layout, const void *v, float *vnorm, void *stream) {
+    int rc = check_layout(layout);
+    if (rc != BSA_OK) return rc;
+    if (!v || !vnorm || !aligned(v, 16) || !aligned(vnorm, 4)) return BSA_ERR_INVALID_ARG;
+    const Geometry g = bsa::make_geometry(*layout);
+    return launch_status(bsa::launch_value_norms(g, v, vnorm, static_cast<cudaStream_t>(stream)));
+}
+
+size_t bsa_build_mask_eg_workspace_bytes(const bsa_layout *layout) {
+    if (check_layout(layout) != BSA_OK) return 0;
+    return bsa::eg_workspace(bsa::make_geometry(*layout)).bytes;
+}
+
+int bsa_build_mask_eg(const bsa_layout *layout, const float *probs, const float *vnorm,
+                      const float *top_p, float pool_p, uint32_t flags, float eps, uint8_t *mask,
+                      int32_t *kv_index, int32_t *kv_count, float *entropy, float *entropy_norm,
+                      uint8_t *low_heads, void *workspace, void *stream) {
+    int rc = check_layout(layout);
+    if (rc != BSA_OK) return rc;
+    if (!probs || !top_p || !kv_index || !kv_count || !workspace) return BSA_ERR_INVALID_ARG;
+    if (flags & ~static_cast<uint32_t>(BSA_TEXT_KEEP | BSA_FRAME0_DENSE)) return BSA_ERR_INVALID_ARG;
+    if (!aligned(probs, 4) || !aligned(kv_index, 4) || !aligned(kv_count, 4) ||
+        (vnorm && !aligned(vnorm, 4)) || !aligned(workspace, 256))
+        return BSA_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || !isfinite(eps) || isnan(pool_p)) return BSA_ERR_INVALID_ARG;
+    const Geometry g = bsa::make_geometry(*layout);
+    if (g.Ck > bsa::kMaxMaskCk) return BSA_ERR_UNSUPPORTED;
+    bsa::TopP tp;
+    memset(&tp, 0, sizeof tp);
+    for (int h = 0; h < g.H; ++h) {
+        if (isnan(top_p[h])) return BSA_ERR_INVALID_ARG;
+        tp.p[h] = top_p[h];
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    rc = launch_status(bsa::launch_eg_prepare(g, probs, vnorm, pool_p, eps, entropy, entropy_norm,
+                                              low_heads, ws, st));
+    if (rc != BSA_OK) return rc;
+    const bsa::EgWorkspace w = bsa::eg_workspace(g);
+    return launch_status(bsa::launch_mask_eg(
+        g, probs, vnorm, tp, flags, mask, kv_index, kv_count, ws + w.low,
+        reinterpret_cast<const bsa::PoolState *>(ws + w.state), st));
+}
+
 size_t bsa_attention_workspace_bytes(const bsa_layout *layout) {
     if (check_layout(layout) != BSA_OK) return 0;
     return bsa::kAttnWorkspaceBytes;

@@ -39,6 +39,10 @@ struct MaskArgs {
     uint32_t flags;
     float eps;
     int text_kblocks, f0_first, f0_last;
+    // entropy-guided mode: pooled heads take the batch entry's pool cut
+    const float *vnorm;           // value-centroid norms [B,H,C_k], or nullptr
+    const uint8_t *low;           // [B,H]: 1 = pooled head
+    const PoolState *state;       // [B]
 };
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -391,7 +395,13 @@ __device__ __forceinline__ float lg2_approx(float y) {
     return r;
 }
 
-template <int VPL>
+// EG = false: every row takes its per-row top-p.  EG = true ("Competition
+// Domains Matter ..." s3.3 domain 3): rows of pooled heads keep the pairs of the
+// batch entry's pool cut (scores P' * ||c^V|| above the cut pattern, ties at
+// it up to the cut row's rank) and, if that leaves them empty, their single
+// best key block (the one-key-per-row safeguard); the other rows keep their
+// per-row top-p.  Entropies are not computed in that mode.
+template <int VPL, bool EG>
 __global__ void __launch_bounds__(128, VPL <= 32 ? 7 : 3)
 mask_kernel(MaskArgs a, TopP tp) {
     __shared__ __align__(16) WarpScratch s_ws[4];
@@ -418,16 +428,24 @@ mask_kernel(MaskArgs a, TopP tp) {
         const int j = lane + 32 * s;
         v[s] = (j < Ck) ? __ldg(src + j) : 0.f;
     }
+    const long long bh = row / a.Cq;
+    const bool pooled = EG && a.low[bh];
     float ent = 0.f;
     uint32_t umax = 0;
 #pragma unroll
     for (int s = 0; s < VPL; ++s) {
         const float x = v[s] > 0.f ? v[s] : 0.f;  // -0.0 and NaN become +0.0
-        v[s] = x;
-        umax = max(umax, __float_as_uint(x));
-        if (lane + 32 * s < Ck) ent = fmaf(x, lg2_approx(x + a.eps), ent);
+        if (!EG && lane + 32 * s < Ck) ent = fmaf(x, lg2_approx(x + a.eps), ent);
+        float y = x;
+        if (pooled && a.vnorm) {  // the pool's value-aware score, rounded to fp32
+            const int j = lane + 32 * s;
+            y = (j < Ck) ? __fmul_rn(x, __ldg(a.vnorm + bh * Ck + j)) : 0.f;
+            y = y > 0.f ? y : 0.f;
+        }
+        v[s] = y;
+        umax = max(umax, __float_as_uint(y));
     }
-    if (a.row_entropy) {
+    if (!EG && a.row_entropy) {
         ent = -warp_sum(ent) * 0.6931471805599453f;  // ln 2
         if (lane == 0) a.row_entropy[row] = ent;
     }
@@ -437,7 +455,31 @@ mask_kernel(MaskArgs a, TopP tp) {
     const bool dense_row = (a.flags & BSA_FRAME0_DENSE) && i >= a.f0_first && i <= a.f0_last;
     uint32_t ucut = 0;
     int jcut = 0x7FFFFFFF;  // keep every entry
-    if (!dense_row) find_cut<VPL>(v, src, Ck, p, umax, lane, ws, ucut, jcut);
+    if (!dense_row) {
+        if (!pooled) {
+            find_cut<VPL>(v, src, Ck, p, umax, lane, ws, ucut, jcut);
+        } else {
+            const PoolState st = a.state[bh / a.H];
+            if (!st.keep_all) {
+                ucut = st.ucut;
+                jcut = row < st.cut_row ? 0x7FFFFFFF
+                       : row == st.cut_row ? nth_tie<VPL>(v, Ck, ucut, st.cut_rank, lane)
+                                           : -1;
+                // safeguard: an empty row keeps its best key block (lowest j on ties)
+                bool any = false;
+#pragma unroll
+                for (int s = 0; s < VPL; ++s) {
+                    const int j = lane + 32 * s;
+                    const uint32_t us = __float_as_uint(v[s]);
+                    any |= j < Ck && (us > ucut || (us == ucut && j <= jcut));
+                }
+                if (!__any_sync(0xffffffffu, any)) {
+                    ucut = umax;
+                    jcut = nth_tie<VPL>(v, Ck, umax, 1, lane);
+                }
+            }
+        }
+    }
 
     const int text_k = (a.flags & BSA_TEXT_KEEP) ? a.text_kblocks : 0;
     uint8_t *mrow = a.mask ? a.mask + row * Ck : nullptr;
@@ -476,11 +518,21 @@ __global__ void __launch_bounds__(256) entropy_reduce_kernel(const float *__rest
     }
 }
 
-template <int VPL>
+template <int VPL, bool EG>
 cudaError_t launch_mask_t(const MaskArgs &a, const TopP &tp, cudaStream_t st) {
     const unsigned grid = static_cast<unsigned>((a.rows + 3) / 4);
-    mask_kernel<VPL><<<grid, 128, 0, st>>>(a, tp);
+    mask_kernel<VPL, EG><<<grid, 128, 0, st>>>(a, tp);
     return cudaGetLastError();
+}
+
+template <bool EG>
+cudaError_t launch_mask_vpl(const MaskArgs &a, const TopP &tp, int Ck, cudaStream_t st) {
+    const int vpl = (Ck + 31) / 32;
+    if (vpl <= 4) return launch_mask_t<4, EG>(a, tp, st);
+    if (vpl <= 8) return launch_mask_t<8, EG>(a, tp, st);
+    if (vpl <= 16) return launch_mask_t<16, EG>(a, tp, st);
+    if (vpl <= 32) return launch_mask_t<32, EG>(a, tp, st);
+    return launch_mask_t<64, EG>(a, tp, st);
 }
 
 }  // namespace
@@ -503,12 +555,35 @@ cudaError_t launch_mask(const Geometry &g, const float *probs, const TopP &tp, u
     a.text_kblocks = g.text_kblocks;
     a.f0_first = g.f0_first;
     a.f0_last = g.f0_last;
-    const int vpl = (g.Ck + 31) / 32;
-    if (vpl <= 4) return launch_mask_t<4>(a, tp, st);
-    if (vpl <= 8) return launch_mask_t<8>(a, tp, st);
-    if (vpl <= 16) return launch_mask_t<16>(a, tp, st);
-    if (vpl <= 32) return launch_mask_t<32>(a, tp, st);
-    return launch_mask_t<64>(a, tp, st);
+    a.vnorm = nullptr;
+    a.low = nullptr;
+    a.state = nullptr;
+    return launch_mask_vpl<false>(a, tp, g.Ck, st);
+}
+
+cudaError_t launch_mask_eg(const Geometry &g, const float *probs, const float *vnorm,
+                           const TopP &tp, uint32_t flags, uint8_t *mask, int32_t *kv_index,
+                           int32_t *kv_count, const uint8_t *low, const PoolState *state,
+                           cudaStream_t st) {
+    MaskArgs a;
+    a.probs = probs;
+    a.mask = mask;
+    a.kv_index = kv_index;
+    a.kv_count = kv_count;
+    a.row_entropy = nullptr;
+    a.rows = static_cast<long long>(g.B) * g.H * g.Cq;
+    a.H = g.H;
+    a.Cq = g.Cq;
+    a.Ck = g.Ck;
+    a.flags = flags;
+    a.eps = 0.f;
+    a.text_kblocks = g.text_kblocks;
+    a.f0_first = g.f0_first;
+    a.f0_last = g.f0_last;
+    a.vnorm = vnorm;
+    a.low = low;
+    a.state = state;
+    return launch_mask_vpl<true>(a, tp, g.Ck, st);
 }
 
 cudaError_t launch_entropy_reduce(const Geometry &g, const float *row_entropy, float *entropy,

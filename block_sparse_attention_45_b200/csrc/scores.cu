@@ -89,6 +89,56 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint4 *__restrict__ q,
     }
 }
 
+// One CTA per key block: the value centroid (mean of V over the block's valid
+// tokens, as for the key centroid) and its L2 norm ||c^V_{h,j}||, the weight of
+// the value-aware score ("Competition Domains Matter ..." s4).
+template <int D>
+__global__ void __launch_bounds__(256) vnorm_kernel(const uint4 *__restrict__ v,
+                                                    float *__restrict__ vnorm, int S, int S_pad,
+                                                    int bk, int Ck) {
+    constexpr int CH = D / 8;      // 16-byte chunks per token row
+    constexpr int RPI = 256 / CH;  // rows covered per pass of the CTA
+    constexpr int PASSES = 128 / RPI;
+    __shared__ float red[RPI][D];
+    __shared__ float sq[8];
+    const long long item = blockIdx.x;
+    const long long bh = item / Ck;
+    const int j = static_cast<int>(item % Ck);
+    const int n = min(bk, S - j * bk);
+    const uint4 *base = v + ((bh * S_pad + static_cast<long long>(j) * bk) * D) / 8;
+    const int c = threadIdx.x % CH, r0 = threadIdx.x / CH;
+    uint4 x[PASSES];
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p) {
+        const int r = r0 + p * RPI;
+        x[p] = (r < n) ? __ldg(base + r * CH + c) : make_uint4(0, 0, 0, 0);
+    }
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p) bf16x8_add(x[p], acc);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[r0][c * 8 + e] = acc[e];
+    __syncthreads();
+    float part = 0.f;
+    for (int d = threadIdx.x; d < D; d += 256) {
+        float sum = 0.f;
+#pragma unroll
+        for (int r = 0; r < RPI; ++r) sum += red[r][d];
+        const float m = sum / static_cast<float>(n);
+        part = fmaf(m, m, part);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (threadIdx.x % 32 == 0) sq[threadIdx.x / 32] = part;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) t += sq[w];
+        vnorm[item] = sqrtf(t);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // score_kernel: the centroid GEMM on the tensor cores, row softmax fused.
 //
@@ -501,6 +551,16 @@ cudaError_t launch_pool(const Geometry &g, const void *q, const void *k, float *
     else
         pool_kernel<64><<<static_cast<unsigned>(nq + nk), 256, 0, st>>>(
             q4, k4, qc, kc, g.S, g.S_pad, g.bq, g.bk, g.Cq, g.Ck, nq);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_value_norms(const Geometry &g, const void *v, float *vnorm, cudaStream_t st) {
+    const long long nk = static_cast<long long>(g.B) * g.H * g.Ck;
+    const auto *v4 = static_cast<const uint4 *>(v);
+    if (g.D == 128)
+        vnorm_kernel<128><<<static_cast<unsigned>(nk), 256, 0, st>>>(v4, vnorm, g.S, g.S_pad, g.bk, g.Ck);
+    else
+        vnorm_kernel<64><<<static_cast<unsigned>(nk), 256, 0, st>>>(v4, vnorm, g.S, g.S_pad, g.bk, g.Ck);
     return cudaGetLastError();
 }
 

@@ -173,6 +173,53 @@ int bsa_build_mask_noalloc(const bsa_layout *layout, const float *probs, const f
                            int32_t *kv_count, float *entropy, float *entropy_norm, void *stream);
 
 /*
+ * Value-centroid norms for the value-aware score of the entropy-guided
+ * selection ("Competition Domains Matter ..." s4): for every key block j of
+ * every (b, h), the centroid c^V = mean of V over the block's valid tokens
+ * (as for the key centroid) and vnorm[b,h,j] = ||c^V||_2.
+ *
+ * v      bf16 [B,H,seq_pad,D], 16-byte aligned (read)
+ * vnorm  fp32 [B,H,C_k] (written)
+ */
+int bsa_value_norms(const bsa_layout *layout, const void *v, float *vnorm, void *stream);
+
+/*
+ * Entropy-guided selection (EG-Sparse; "Competition Domains Matter ..."
+ * s3.3 domain 3 "grouped cross-head", the one-key-per-row safeguard, s4 the
+ * value-aware score).  Per batch entry the heads are split at the median of
+ * their entropy H_h: ordered by (H_h ascending, h ascending), the first
+ * floor(H/2) are pooled, the others keep the per-row local top-p of
+ * bsa_build_mask with their top_p[h].  All pairs (h, i, j) of the pooled heads
+ * of one batch entry compete in one pool, ranked by the score
+ * I = P'[b,h,i,j] * vnorm[b,h,j] (the fp32 product; P' alone when vnorm is
+ * NULL) in (I descending, h, i, j ascending) order; the pool keeps the
+ * shortest prefix whose running sum reaches pool_p times the pool's total
+ * score (everything if it never does; its first pair if pool_p <= 0).  A
+ * pooled row left empty then keeps its single highest-scoring key block
+ * (lowest j on ties).  The text-keep and frame-0 overrides and the lists
+ * follow as in bsa_build_mask.  The cut is found without sorting by an exact
+ * radix select over the scores' bit patterns with integer significand sums.
+ *
+ * probs         fp32 [B,H,C_q,C_k] (read)
+ * vnorm         fp32 [B,H,C_k] from bsa_value_norms, or NULL (rank by P')
+ * top_p         HOST fp32 [H]: p of the per-row heads
+ * pool_p        p of the cross-head pools
+ * flags, eps    as for bsa_build_mask
+ * mask, kv_index, kv_count   as for bsa_build_mask (mask may be NULL)
+ * entropy, entropy_norm      fp32 [B,H], or NULL (always computed)
+ * low_heads     u8 [B,H]: 1 for the pooled heads, or NULL
+ * workspace     device scratch of bsa_build_mask_eg_workspace_bytes(layout)
+ *               bytes, 256-byte aligned; contents on entry do not matter
+ */
+int bsa_build_mask_eg(const bsa_layout *layout, const float *probs, const float *vnorm,
+                      const float *top_p, float pool_p, uint32_t flags, float eps, uint8_t *mask,
+                      int32_t *kv_index, int32_t *kv_count, float *entropy, float *entropy_norm,
+                      uint8_t *low_heads, void *workspace, void *stream);
+
+/* Bytes of device workspace bsa_build_mask_eg needs (0: invalid layout). */
+size_t bsa_build_mask_eg_workspace_bytes(const bsa_layout *layout);
+
+/*
  * Block-sparse exact attention ("Attention matrix view ..." s2;
  * "AB-Attention ..." TL;DR).  For every valid query token t of query block i:
  *   U = tokens u < seq_len of the key blocks kv_index[b,h,i,0..kv_count-1]

@@ -129,6 +129,42 @@ def test_pipeline_workspace_size():
         lib.bsa_pipeline_workspace_bytes(ctypes.byref(L), w.heads)
 
 
+def test_eg_entry_points_validate_before_any_cuda_call():
+    lib = bsa.load()
+    L = _layout()
+    r = ctypes.byref(L)
+    tp = (ctypes.c_float * 2)(0.5, 0.5)
+    tpv = ctypes.cast(tp, ctypes.c_void_p)
+    ws = ctypes.c_void_p(0x100000)
+
+    def eg(probs=FAKE, vnorm=None, top=tpv, pool_p=0.9, flags=3, idx=FAKE, cnt=FAKE, w=ws):
+        return lib.bsa_build_mask_eg(r, probs, vnorm, top, pool_p, flags, 1e-8, None, idx, cnt,
+                                     None, None, None, w, None)
+    assert eg(probs=None) == bsa.BSA_ERR_INVALID_ARG
+    assert eg(top=None) == bsa.BSA_ERR_INVALID_ARG
+    assert eg(idx=None) == bsa.BSA_ERR_INVALID_ARG
+    assert eg(w=None) == bsa.BSA_ERR_INVALID_ARG
+    assert eg(w=ctypes.c_void_p(0x100010)) == bsa.BSA_ERR_INVALID_ARG     # not 256-aligned
+    assert eg(vnorm=MISALIGNED) == bsa.BSA_ERR_INVALID_ARG
+    assert eg(flags=8) == bsa.BSA_ERR_INVALID_ARG
+    assert eg(pool_p=float("nan")) == bsa.BSA_ERR_INVALID_ARG
+    nan_tp = (ctypes.c_float * 2)(float("nan"), 0.5)
+    assert eg(top=ctypes.cast(nan_tp, ctypes.c_void_p)) == bsa.BSA_ERR_INVALID_ARG
+    bad = _layout(head_dim=96)
+    assert lib.bsa_build_mask_eg(ctypes.byref(bad), FAKE, None, tpv, 0.9, 3, 1e-8, None, FAKE, FAKE,
+                                 None, None, None, ws, None) == bsa.BSA_ERR_UNSUPPORTED
+    assert lib.bsa_value_norms(r, None, FAKE, None) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_value_norms(r, MISALIGNED, FAKE, None) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_value_norms(ctypes.byref(bad), FAKE, FAKE, None) == bsa.BSA_ERR_UNSUPPORTED
+    # workspace: row entropies + per-row tie counts + per-head values + one pool state and
+    # 4096-bin histogram per batch entry
+    assert lib.bsa_build_mask_eg_workspace_bytes(ctypes.byref(bad)) == 0
+    w = synth.WORKLOADS["hunyuan"]
+    n = lib.bsa_build_mask_eg_workspace_bytes(ctypes.byref(bsa.make_layout(w)))
+    rows = w.heads * (w.seq_pad // w.q_block)
+    assert n >= rows * 8 + 4096 * 16 and n % 256 == 0
+
+
 def test_calls_fail_loudly_without_the_library(monkeypatch):
     monkeypatch.setattr(bsa, "_LIB", None)
     monkeypatch.setattr(bsa, "LIB_PATH", "/nonexistent/libbsa.so")
