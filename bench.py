@@ -50,6 +50,11 @@ def parse():
                     help="heads per group of the pipelined host-buffer call timed as e2e")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--selection", default="top_p", choices=["top_p", "eg"],
+                    help="per-row top-p (bsa_build_mask) or entropy-guided grouped selection "
+                         "(bsa_value_norms + bsa_build_mask_eg) inside the step")
+    ap.add_argument("--pool-p", type=float, default=None,
+                    help="threshold of the low-entropy pool (default: the mean per-head top-p)")
     return ap.parse_args()
 
 
@@ -240,6 +245,16 @@ def our_arm(args, w):
     ent = torch.empty((B, H), **f32)
     ent_n = torch.empty((B, H), **f32)
     ws = torch.empty(bsa.workspace_bytes(w), dtype=torch.uint8, device=dev)
+    eg = args.selection == "eg"
+    pool_p = float(np.mean(top_p)) if args.pool_p is None else args.pool_p
+    vnorm = torch.empty((B, H, Ck), **f32)
+    low = torch.empty((B, H), dtype=torch.uint8, device=dev)
+    ws_eg = torch.empty(bsa.eg_workspace_bytes(w), dtype=torch.uint8, device=dev)
+
+    def select_eg():
+        bsa.value_norms(w, v, vnorm, stream=stream)
+        bsa.build_mask_eg(w, probs, vnorm, top_p, pool_p, w.flags, 1e-8, mask, kv_index, kv_count,
+                          ws_eg, stream=stream, entropy=ent, entropy_norm=ent_n, low_heads=low)
     out = torch.empty((B, H, Sp, D), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((B, H, Sp), **f32)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -252,15 +267,21 @@ def our_arm(args, w):
         bsa.block_scores(w, qq, kk, qc, kc, probs, stream=stream)
         if marks is not None:
             marks[1].record(stream)
-        bsa.build_mask(w, probs, top_p, w.flags, 1e-8, mask, kv_index, kv_count, ent, ent_n, ws,
-                       stream=stream)
+        if eg:
+            select_eg()
+        else:
+            bsa.build_mask(w, probs, top_p, w.flags, 1e-8, mask, kv_index, kv_count, ent, ent_n,
+                           ws, stream=stream)
         if marks is not None:
             marks[2].record(stream)
         bsa.attention_fwd(w, qq, kk, vv, kv_index, kv_count, None, out, lse, err, stream=stream)
         if marks is not None:
             marks[3].record(stream)
 
-    launches_per_step = 5   # pool, score, mask, entropy reduce, attention
+    # pool, score, mask, entropy reduce, attention; the entropy-guided selection runs
+    # value norms, row entropy, entropy reduce, route, 3 x (pool histogram, pick), tie count,
+    # tie scan and the mask kernel in place of mask + entropy reduce
+    launches_per_step = 15 if eg else 5
     for _ in range(max(3, args.warmup)):
         step(q, k, v)
     torch.cuda.synchronize(dev)
@@ -348,6 +369,25 @@ def our_arm(args, w):
         dflops = B * H * Cq * Ck * flops_per_pair(w)
         dense = dict(ms=dms, tflops=dflops / (dms * 1e-3) / 1e12)
 
+    # the entropy-guided selection for context when it is not the step's selection:
+    # value norms + bsa_build_mask_eg on the step's P' (not part of the step)
+    eg_ctx = None
+    if not eg:
+        for _ in range(2):
+            select_eg()
+        a, b = ev(), ev()
+        a.record(stream)
+        ne = max(3, args.steps)
+        for _ in range(ne):
+            select_eg()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        eg_pairs = int(kv_count.sum().item())
+        eg_ctx = dict(ms=a.elapsed_time(b) / ne, pool_p=pool_p,
+                      density=eg_pairs / float(B * H * Cq * Ck),
+                      pooled_heads=int(low.sum().item()),
+                      call="bsa_value_norms + bsa_build_mask_eg on the step's P'")
+
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -367,6 +407,8 @@ def our_arm(args, w):
     # write mask, lists, counts) over their measured durations
     bytes_scores = 2 * B * H * w.seq_len * D * 2 + 4 * B * H * (Cq + Ck) * D + 4 * B * H * Cq * Ck
     bytes_mask = 4 * B * H * Cq * Ck + B * H * Cq * Ck + 4 * pairs + 4 * B * H * Cq
+    if eg:   # value norms read V and write ||c^V||; the pools read them too
+        bytes_mask += B * H * w.seq_len * D * 2 + 2 * 4 * B * H * Ck
     line = dict(
         metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
         ms_per_step=ms_step, higher_is_better=True, scaling="weak", vs_baseline=None,
@@ -375,6 +417,8 @@ def our_arm(args, w):
         config=dict(workload=w.name, batch=B, heads=H, seq_len=w.seq_len, seq_pad=Sp, head_dim=D,
                     q_block=w.q_block, k_block=w.k_block, text_len=w.text_len,
                     frames=w.num_frames, latent=[w.latent_h, w.latent_w],
+                    selection="entropy-guided grouped (pool_p %.4g)" % pool_p if eg
+                              else "per-row top-p",
                     density=density, skipped=1 - density, selected_pairs=pairs,
                     computed_tflop_per_step=step_flops / 1e12,
                     dense_equiv_tflop=4.0 * B * H * w.seq_len ** 2 * D / 1e12,
@@ -388,6 +432,7 @@ def our_arm(args, w):
         mask=dict(ms=float(np.mean(ms_mask)), gbs=bytes_mask / (np.mean(ms_mask) * 1e-3) / 1e9,
                   frac_hbm=bytes_mask / (np.mean(ms_mask) * 1e-3) / 1e9 / hbm),
         dense=dense,
+        eg_selection=eg_ctx,
         roofline=dict(bound="tensor", kernel="attn_kernel", achieved=achieved, peak=peak,
                       unit="TFLOP/s", frac=achieved / peak, peak_source=peak_note,
                       traffic=traffic, flop_per_launch=step_flops,

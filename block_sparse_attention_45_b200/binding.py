@@ -221,7 +221,8 @@ def eg_workspace_bytes(layout):
 
 
 def build_mask_eg(layout, probs, vnorm, top_p, pool_p, flags, eps=1e-8, mask=None,
-                  kv_index=None, kv_count=None, workspace=None, with_mask=True, stream=None):
+                  kv_index=None, kv_count=None, workspace=None, with_mask=True, stream=None,
+                  entropy=None, entropy_norm=None, low_heads=None):
     """bsa_build_mask_eg (entropy-guided grouped cross-head selection): returns
     dict(mask, kv_index, kv_count, entropy, entropy_norm, low_heads).  vnorm None
     ranks the pools by P' alone."""
@@ -241,9 +242,16 @@ def build_mask_eg(layout, probs, vnorm, top_p, pool_p, flags, eps=1e-8, mask=Non
         kv_index = torch.empty((d["B"], d["H"], d["Cq"], d["Ck"]), dtype=torch.int32, device=dev)
     if kv_count is None:
         kv_count = torch.empty((d["B"], d["H"], d["Cq"]), dtype=torch.int32, device=dev)
-    entropy = torch.empty((d["B"], d["H"]), dtype=torch.float32, device=dev)
-    entropy_norm = torch.empty((d["B"], d["H"]), dtype=torch.float32, device=dev)
-    low = torch.empty((d["B"], d["H"]), dtype=torch.uint8, device=dev)
+    if entropy is None:
+        entropy = torch.empty((d["B"], d["H"]), dtype=torch.float32, device=dev)
+    if entropy_norm is None:
+        entropy_norm = torch.empty((d["B"], d["H"]), dtype=torch.float32, device=dev)
+    low = low_heads
+    if low is None:
+        low = torch.empty((d["B"], d["H"]), dtype=torch.uint8, device=dev)
+    _need(entropy, "entropy", torch.float32, (d["B"], d["H"]))
+    _need(entropy_norm, "entropy_norm", torch.float32, (d["B"], d["H"]))
+    _need(low, "low_heads", torch.uint8, (d["B"], d["H"]))
     if workspace is None:
         workspace = torch.empty(eg_workspace_bytes(L), dtype=torch.uint8, device=dev)
     rc = load().bsa_build_mask_eg(ctypes.byref(L), _ptr(probs), _ptr(vnorm),

@@ -18,16 +18,18 @@
 // the target then lies in one bit pattern u*: every pair above u* is kept, and
 // of the pairs equal to u* the first `need` in (h, i, j) order.
 //
-// Kernels (all on the caller's stream):
-//   row_entropy_kernel   -sum_j P' ln(P' + eps) per row (warp per row)
-//   (entropy_reduce of mask.cu: per-head mean)
-//   route_kernel         median split per batch entry, pool state reset
-//   pool_hist_kernel     one radix level: shared-memory histogram, flushed
-//                        with 64-bit atomics (persistent CTAs per batch entry)
-//   pool_pick_kernel     one warp per batch entry: the bin that reaches target
-//   tie_count_kernel     pairs equal to u* per pool row
-//   tie_scan_kernel      the row and rank of the last kept tie
+// Launches (all on the caller's stream; the last CTA of each launch to finish
+// does that launch's serial step, so no launch waits on another's CTAs):
+//   entropy_level1_kernel  -sum_j P' ln(P' + eps) per row and a per-head
+//                          histogram of the scores' exponent fields; its last
+//                          CTA takes the per-head means, the median split and
+//                          the level-1 pick of every batch entry
+//   pool_level_kernel x2   mantissa bits 22..11, then 10..0, over the pooled
+//                          heads only; the last CTA picks the bin
+//   tie_kernel             pairs equal to the cut pattern per pooled row; the
+//                          last CTA finds the row and rank of the last kept tie
 #include <cuda_runtime.h>
+#include <limits.h>
 #include <math.h>
 #include <stdint.h>
 
@@ -37,8 +39,15 @@ namespace bsa {
 
 namespace {
 
-constexpr int kMaxBins = 4096;
-constexpr int kLevelBits[3] = {8, 12, 11};  // exponent, mantissa 22..11, mantissa 10..0
+constexpr int kThreads = 256;                 // every launch of this file
+constexpr int kWarps = kThreads / 32;
+constexpr int kL1Bins = 256;                  // exponent field
+constexpr int kL1Copies = 4;                  // level-1 histograms per warp
+constexpr int kL1Stride = 2 * kL1Bins + 1;    // words between copies (lo, hi; bank offset 1)
+constexpr size_t kL1Smem = static_cast<size_t>(kThreads / 32) * kL1Copies * kL1Stride * sizeof(uint32_t);
+constexpr int kMaxBins = 4096;                // widest later level
+constexpr int kLevelBits[2] = {12, 11};       // mantissa 22..11, 10..0
+constexpr uint32_t kBinCap = (1u << 20) - 1;  // pairs one 32-bit shared bin may take (12-bit halves)
 
 __device__ __forceinline__ float lg2_fast(float y) {
     float r;
@@ -58,13 +67,47 @@ __device__ __forceinline__ double unit_of_binade(uint32_t e) {
     return __longlong_as_double(static_cast<long long>(k + 1023) << 52);
 }
 
-// Score of pair (row, j) of a pooled head, as a bit pattern: P' * ||c^V|| rounded
-// to fp32 (P' alone without value norms); -0 and NaN count as +0.
-__device__ __forceinline__ uint32_t pool_score(const float *__restrict__ prow,
-                                               const float *__restrict__ vrow, int j) {
-    const float p = __ldg(prow + j);
-    const float s = vrow ? __fmul_rn(p, __ldg(vrow + j)) : p;
-    return pos_bits(s);
+// Score of a pooled pair as a bit pattern: P' (negatives and NaN as +0) times
+// ||c^V|| (vn), rounded to fp32; P' alone without value norms.
+__device__ __forceinline__ uint32_t score_bits(float p, bool value_aware, float vn) {
+    const float x = p > 0.f ? p : 0.f;
+    return pos_bits(value_aware ? __fmul_rn(x, vn) : x);
+}
+
+// The value norms of head bh, lane + 32 s in slot s (0 past C_k).
+template <int VPL>
+__device__ __forceinline__ void load_vnorm(const float *vnorm, long long bh, int Ck, int lane, float (&vn)[VPL]) {
+#pragma unroll
+    for (int s = 0; s < VPL; ++s) {
+        const int j = lane + 32 * s;
+        vn[s] = (vnorm && j < Ck) ? __ldg(vnorm + bh * Ck + j) : 0.f;
+    }
+}
+
+// A shared-memory bin: count, and the significand split into 12-bit halves so
+// that 32-bit atomics stay exact for up to kBinCap pairs.
+__device__ __forceinline__ void bin_add(uint32_t *c, uint32_t *lo, uint32_t *hi, uint32_t bin,
+                                        uint32_t u) {
+    const uint32_t s = significand(u);
+    atomicAdd(c + bin, 1u);
+    atomicAdd(lo + bin, s & 0xFFFu);
+    atomicAdd(hi + bin, s >> 12);
+}
+
+// Unsigned key ordering floats like <, with -0 == +0 and NaN above everything.
+__device__ __forceinline__ uint32_t order_key(float f) {
+    if (f != f) return 0xFFFFFFFFu;
+    const uint32_t u = __float_as_uint(f + 0.0f);  // -0 -> +0
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The same without the count, for levels whose pick only needs to know which
+// bins are empty: a bin of scores >= 2^-149 is non-empty iff its sum is
+// positive; zero scores are flagged separately.
+__device__ __forceinline__ void bin_add_sum(uint32_t *lo, uint32_t *hi, uint32_t bin, uint32_t u) {
+    const uint32_t s = significand(u);
+    atomicAdd(lo + bin, s & 0xFFFu);
+    atomicAdd(hi + bin, s >> 12);
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -73,297 +116,614 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// -sum_j P' ln(P' + eps) of every row, one warp per row.
-__global__ void __launch_bounds__(256) row_entropy_kernel(const float *__restrict__ probs,
-                                                          float *__restrict__ row_ent,
-                                                          long long rows, int Ck, float eps) {
-    const int lane = threadIdx.x % 32;
-    const long long row = static_cast<long long>(blockIdx.x) * 8 + threadIdx.x / 32;
-    if (row >= rows) return;
-    const float *src = probs + row * Ck;
-    float ent = 0.f;
-#pragma unroll 4
-    for (int j = lane; j < Ck; j += 32) {
-        const float y = __ldg(src + j);
-        const float x = y > 0.f ? y : 0.f;
-        ent = fmaf(x, lg2_fast(x + eps), ent);
-    }
-    ent = warp_sum(ent);
-    if (lane == 0) row_ent[row] = -ent * 0.6931471805599453f;  // ln 2
-}
-
-// Median split: heads of batch entry b ordered by (H_h asc, h asc); the first
-// floor(H/2) are pooled.  Also resets the pool state of b.
-__global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ heads_h, int H,
-                                                    uint8_t *low, uint8_t *low_out,
-                                                    PoolState *state) {
-    const int b = blockIdx.x, h = threadIdx.x;
-    const float *hb = heads_h + static_cast<long long>(b) * H;
-    if (h < H) {
-        const float x = hb[h];
-        int rank = 0;
-        for (int o = 0; o < H; ++o) {
-            const float y = hb[o];
-            rank += (y < x || (y == x && o < h)) ? 1 : 0;
-        }
-        const uint8_t l = rank < H / 2 ? 1 : 0;
-        low[static_cast<long long>(b) * H + h] = l;
-        if (low_out) low_out[static_cast<long long>(b) * H + h] = l;
-    }
-    if (h == 0) {
-        PoolState s;
-        s.target = 0.0;
-        s.above = 0.0;
-        s.cnt_above = 0;
-        s.pre = 0;
-        s.shift = 31;  // level 1 bins bits 30..23 of scores >= 0 (bit 31 is 0)
-        s.keep_all = 0;
-        s.empty = H / 2 == 0;
-        s.ucut = 0;
-        s.pad0 = 0;
-        s.need = 0;
-        s.cut_row = -1;
-        s.cut_rank = 0;
-        s.pad1 = 0;
-        state[b] = s;
-    }
-}
-
-// One radix level of batch entry blockIdx.y: every score in the current range
-// (bits above `shift` equal to `pre`) adds (1, significand) to bin
-// (u >> (shift - nbits)) & (2^nbits - 1) of a shared histogram, flushed at exit.
-__global__ void __launch_bounds__(256) pool_hist_kernel(const float *__restrict__ probs,
-                                                        const float *__restrict__ vnorm,
-                                                        const uint8_t *__restrict__ low,
-                                                        const PoolState *__restrict__ state,
-                                                        unsigned long long *__restrict__ hist,
-                                                        int H, int Cq, int Ck, int nbits) {
-    extern __shared__ unsigned long long sh[];  // [2^nbits][2]: count, significand sum
-    const int b = blockIdx.y;
-    const PoolState st = state[b];
-    if (st.empty || st.keep_all || st.shift < nbits) return;
-    const int nb = 1 << nbits;
-    for (int k = threadIdx.x; k < 2 * nb; k += blockDim.x) sh[k] = 0ull;
+// Called by every thread after its last global write: true in the one CTA of
+// the grid that finishes last, which then sees every other CTA's writes.
+__device__ bool last_cta(unsigned int *counter) {
+    __shared__ int s_last;
+    __threadfence();
     __syncthreads();
-    const int lo = st.shift - nbits;
-    const uint32_t pre = st.pre;
-    const uint32_t bmask = static_cast<uint32_t>(nb - 1);
-    const int lane = threadIdx.x % 32;
-    const long long rows_b = static_cast<long long>(H) * Cq;
-    const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
-    for (long long w = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
-         w < rows_b; w += warps) {
-        const int h = static_cast<int>(w / Cq);
-        if (!low[static_cast<long long>(b) * H + h]) continue;  // warp-uniform
-        const long long bh = static_cast<long long>(b) * H + h;
-        const float *prow = probs + (bh * Cq + (w % Cq)) * Ck;
-        const float *vrow = vnorm ? vnorm + bh * Ck : nullptr;
-        for (int j = lane; j < Ck; j += 32) {
-            const uint32_t u = pool_score(prow, vrow, j);
-            if ((u >> st.shift) == pre) {  // shift 31: every score (bit 31 clear)
-                const uint32_t bin = (u >> lo) & bmask;
-                atomicAdd(&sh[2 * bin], 1ull);
-                atomicAdd(&sh[2 * bin + 1], static_cast<unsigned long long>(significand(u)));
-            }
-        }
-    }
+    if (threadIdx.x == 0) s_last = atomicAdd(counter, 1u) == gridDim.x - 1 ? 1 : 0;
     __syncthreads();
-    unsigned long long *g = hist + static_cast<long long>(b) * 2 * kMaxBins;
-    for (int k = threadIdx.x; k < nb; k += blockDim.x) {
-        if (sh[2 * k]) {
-            atomicAdd(&g[2 * k], sh[2 * k]);
-            atomicAdd(&g[2 * k + 1], sh[2 * k + 1]);
-        }
-    }
+    const bool last = s_last != 0;
+    if (last) __threadfence();
+    return last;
 }
 
-// The bin of the current level that holds the cut: scanning bins from the
-// largest value down, the first non-empty bin whose inclusive mass (plus the
-// mass above the range) reaches the target; if rounding leaves the whole range
-// short of it, the last non-empty bin.  Level 1 also fixes the target
-// pool_p * total, and keep_all when the pool never reaches it.  One warp per
-// batch entry; lane l owns a contiguous run of bins from the top.
-__global__ void __launch_bounds__(32) pool_pick_kernel(const unsigned long long *__restrict__ hist,
-                                                       PoolState *state, float pool_p, int nbits,
-                                                       int first_level) {
-    const int b = blockIdx.x, lane = threadIdx.x;
-    PoolState st = state[b];
-    if (st.empty || st.keep_all || st.shift < nbits) return;
-    const int nb = 1 << nbits;
-    const int per = nb / 32;
-    const unsigned long long *g = hist + static_cast<long long>(b) * 2 * kMaxBins;
-    const int lo = st.shift - nbits;
-    // bin k (value order) -> its mass unit: level 1 bins are binades, later
-    // levels lie inside the binade fixed by level 1 (the top 8 bits of pre)
-    auto unit_of = [&](int k) -> double {
-        if (first_level) return unit_of_binade(static_cast<uint32_t>(k));
-        const uint32_t e = (st.pre << st.shift) >> 23;  // exponent of the range
-        return unit_of_binade(e);
-    };
-    // lane l: bins top - l*per - t, t = 0..per-1 (descending value)
-    double m_run = 0.0;
-    unsigned long long c_run = 0;
-    const int top = nb - 1 - lane * per;
-    for (int t = 0; t < per; ++t) {
-        const int k = top - t;
-        const unsigned long long c = g[2 * k];
-        if (c) {
-            m_run += static_cast<double>(g[2 * k + 1]) * unit_of(k);
-            c_run += c;
-        }
-    }
-    // exclusive prefix over lanes (value order)
-    double m_ex = m_run;
-    unsigned long long c_ex = c_run;
+struct ScanScratch {
+    double m[kThreads];
+    unsigned long long c[kThreads];
+    double wm[kWarps];
+    unsigned long long wc[kWarps];
+    int owner, last_ne;
+};
+
+// Inclusive scan of (m, c) over the threads of the CTA in thread order; every
+// thread's result also lands in sc.m / sc.c.
+__device__ void cta_scan(double &m, unsigned long long &c, ScanScratch &sc) {
+    const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const double mo = __shfl_up_sync(0xffffffffu, m_ex, o);
-        const unsigned long long co = __shfl_up_sync(0xffffffffu, c_ex, o);
+        const double mo = __shfl_up_sync(0xffffffffu, m, o);
+        const unsigned long long co = __shfl_up_sync(0xffffffffu, c, o);
         if (lane >= o) {
-            m_ex += mo;
-            c_ex += co;
+            m += mo;
+            c += co;
         }
     }
-    const double m_before = m_ex - m_run;   // mass of the lanes above this one
-    const unsigned long long c_before = c_ex - c_run;
+    if (lane == 31) {
+        sc.wm[wid] = m;
+        sc.wc[wid] = c;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < kWarps; ++w) {
+            sc.wm[w] += sc.wm[w - 1];
+            sc.wc[w] += sc.wc[w - 1];
+        }
+    }
+    __syncthreads();
+    if (wid > 0) {
+        m += sc.wm[wid - 1];
+        c += sc.wc[wid - 1];
+    }
+    sc.m[threadIdx.x] = m;
+    sc.c[threadIdx.x] = c;
+    __syncthreads();
+}
+
+// One radix level of one batch entry, by the whole CTA, on its histogram in
+// shared memory (sum[k] = significand sum of bin k; cnt[k] = its count at the
+// last level, before it only zero or not as the bin is empty or not).  The
+// level's bin holding the cut: scanning bins from the largest value down, the
+// first non-empty bin whose inclusive mass (plus the mass above the range)
+// reaches the target; if rounding leaves the range short of it, its last
+// non-empty bin.  Level 1 also fixes the target pool_p * total, and keep_all
+// when the pool never reaches it.  The last level fixes the cut pattern and
+// how many pairs equal to it are kept.  Thread t owns a run of bins from the
+// top; the thread whose run holds the cut walks it.
+__device__ void cta_pick(const uint32_t *cnt, const unsigned long long *sum, int nbits,
+                         bool first_level, float pool_p, PoolState &st, ScanScratch &sc) {
+    const int t = threadIdx.x;
+    const int nb = 1 << nbits;
+    const int per = nb / kThreads;
+    const int lo = st.shift - nbits;
+    const uint32_t range_e = first_level ? 0u : (st.pre << st.shift) >> 23;  // later levels: one binade
+    auto unit_of = [&](int k) -> double {
+        return unit_of_binade(first_level ? static_cast<uint32_t>(k) : range_e);
+    };
+    const int top = nb - 1 - t * per;
+    double m_run = 0.0;
+    unsigned long long c_run = 0;
+    for (int s = 0; s < per; ++s) {
+        const int k = top - s;
+        if (cnt[k]) {
+            m_run += static_cast<double>(sum[k]) * unit_of(k);
+            c_run += cnt[k];
+        }
+    }
+    double m_in = m_run;
+    unsigned long long c_in = c_run;
+    if (t == 0) {
+        sc.owner = INT_MAX;
+        sc.last_ne = -1;
+    }
+    cta_scan(m_in, c_in, sc);
+    const double m_before = t ? sc.m[t - 1] : 0.0;
+    double target = st.target;
     if (first_level) {
-        const double total = __shfl_sync(0xffffffffu, m_ex, 31);
-        st.target = static_cast<double>(pool_p) * total;
-        if (!(total >= st.target)) {
-            if (lane == 0) {
-                st.keep_all = 1;
-                state[b] = st;
-            }
+        const double total = sc.m[kThreads - 1];
+        target = static_cast<double>(pool_p) * total;
+        if (!(total >= target)) {  // every thread takes this branch
+            __syncthreads();
+            if (t == 0) st.keep_all = 1;
+            __syncthreads();
             return;
         }
     }
-    const double target = st.target;
     const bool reaches = c_run > 0 && st.above + m_before + m_run >= target;
-    const uint32_t hit = __ballot_sync(0xffffffffu, reaches);
-    int owner;
-    if (hit) {
-        owner = __ffs(hit) - 1;
-    } else {
-        const uint32_t ne = __ballot_sync(0xffffffffu, c_run > 0);
-        owner = ne ? 31 - __clz(ne) : 0;
-    }
-    if (lane == owner) {
+    if (reaches) atomicMin(&sc.owner, t);
+    if (c_run > 0) atomicMax(&sc.last_ne, t);
+    __syncthreads();
+    const bool hit = sc.owner != INT_MAX;
+    const int owner = hit ? sc.owner : max(sc.last_ne, 0);
+    if (t == owner) {
         double m = st.above + m_before;
-        unsigned long long c = st.cnt_above + c_before;
         int pick = -1, last_ne = -1;
-        for (int t = 0; t < per; ++t) {
-            const int k = top - t;
-            const unsigned long long ck = g[2 * k];
-            if (!ck) continue;
-            const double mk = static_cast<double>(g[2 * k + 1]) * unit_of(k);
+        for (int s = 0; s < per; ++s) {
+            const int k = top - s;
+            if (!cnt[k]) continue;
+            const double mk = static_cast<double>(sum[k]) * unit_of(k);
             if (hit && m + mk >= target) {
                 pick = k;
                 break;
             }
             last_ne = k;
             m += mk;
-            c += ck;
         }
-        if (pick < 0) {  // the range ends short of the target: its last bin
+        if (pick < 0 && last_ne >= 0) {  // the range ends short of the target: its last bin
             pick = last_ne;
-            // undo the last bin's mass: it is the cut bin itself
-            const double mk = static_cast<double>(g[2 * pick + 1]) * unit_of(pick);
-            m -= mk;
-            c -= g[2 * pick];
+            m -= static_cast<double>(sum[pick]) * unit_of(pick);
         }
-        st.above = m;
-        st.cnt_above = c;
-        st.pre = (st.pre << nbits) | static_cast<uint32_t>(pick);
-        st.shift = lo;
-        if (lo == 0) {
-            // the cut bit pattern; keep its first `need` pairs in (h, i, j) order
-            st.ucut = st.pre;
-            const double v = static_cast<double>(__uint_as_float(st.ucut));
-            const unsigned long long ties = g[2 * pick];
-            unsigned long long need = 1;
-            if (v > 0.0 && st.above < target) {
-                const double n = ceil((target - st.above) / v);
-                need = n < 1.0 ? 1ull : static_cast<unsigned long long>(n);
-                // the closed form against the running sum of the rule
-                while (need > 1 && st.above + static_cast<double>(need - 1) * v >= target) --need;
-                while (need < ties && st.above + static_cast<double>(need) * v < target) ++need;
-            }
-            st.need = need < ties ? need : ties;
-        }
-        state[b] = st;
-    }
-}
-
-// Pairs equal to the cut pattern in each pooled row.
-__global__ void __launch_bounds__(256) tie_count_kernel(const float *__restrict__ probs,
-                                                        const float *__restrict__ vnorm,
-                                                        const uint8_t *__restrict__ low,
-                                                        const PoolState *__restrict__ state,
-                                                        int *__restrict__ tiecnt, long long rows,
-                                                        int H, int Cq, int Ck) {
-    const int lane = threadIdx.x % 32;
-    const long long row = static_cast<long long>(blockIdx.x) * 8 + threadIdx.x / 32;
-    if (row >= rows) return;
-    const long long bh = row / Cq;
-    const int b = static_cast<int>(bh / H);
-    const PoolState st = state[b];
-    int n = 0;
-    if (!st.empty && !st.keep_all && low[bh]) {
-        const float *prow = probs + row * Ck;
-        const float *vrow = vnorm ? vnorm + bh * Ck : nullptr;
-        for (int j = lane; j < Ck; j += 32) n += pool_score(prow, vrow, j) == st.ucut ? 1 : 0;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
-    }
-    if (lane == 0) tiecnt[row] = n;
-}
-
-// The row (in (h, i) order) where the running count of ties reaches `need`,
-// and how many ties of that row are kept.  One block per batch entry.
-__global__ void __launch_bounds__(1024) tie_scan_kernel(const int *__restrict__ tiecnt,
-                                                        PoolState *state, int H, int Cq) {
-    __shared__ unsigned long long part[1024];
-    const int b = blockIdx.x;
-    const PoolState st = state[b];
-    if (st.empty || st.keep_all) return;
-    const long long rows_b = static_cast<long long>(H) * Cq;
-    const long long base = static_cast<long long>(b) * rows_b;
-    const long long per = (rows_b + blockDim.x - 1) / blockDim.x;
-    const long long r0 = threadIdx.x * per, r1 = min(rows_b, r0 + per);
-    unsigned long long s = 0;
-    for (long long r = r0; r < r1; ++r) s += static_cast<unsigned long long>(tiecnt[base + r]);
-    part[threadIdx.x] = s;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        unsigned long long run = 0;
-        int owner = -1;
-        for (int t = 0; t < static_cast<int>(blockDim.x); ++t) {
-            if (run + part[t] >= st.need) {
-                owner = t;
-                break;
-            }
-            run += part[t];
-        }
-        PoolState s2 = st;
-        s2.cut_row = -1;
-        s2.cut_rank = 0;
-        if (owner >= 0) {
-            const long long a = owner * per, e = min(rows_b, a + per);
-            for (long long r = a; r < e; ++r) {
-                const unsigned long long c = static_cast<unsigned long long>(tiecnt[base + r]);
-                if (run + c >= st.need) {
-                    s2.cut_row = base + r;
-                    s2.cut_rank = static_cast<int>(st.need - run);
-                    break;
+        if (first_level) st.target = target;
+        if (pick < 0) {
+            st.keep_all = 1;  // an empty range (not reachable from a non-empty pool)
+        } else {
+            st.above = m;
+            st.pre = (st.pre << nbits) | static_cast<uint32_t>(pick);
+            st.shift = lo;
+            if (lo == 0) {
+                // the cut bit pattern; keep its first `need` pairs in (h, i, j) order
+                st.ucut = st.pre;
+                const double v = static_cast<double>(__uint_as_float(st.ucut));
+                const unsigned long long ties = cnt[pick];
+                unsigned long long need = 1;
+                if (v > 0.0 && st.above < target) {
+                    const double n = ceil((target - st.above) / v);
+                    need = n < 1.0 ? 1ull : static_cast<unsigned long long>(n);
+                    // the closed form against the running sum of the rule
+                    while (need > 1 && st.above + static_cast<double>(need - 1) * v >= target) --need;
+                    while (need < ties && st.above + static_cast<double>(need) * v < target) ++need;
                 }
-                run += c;
+                st.need = need < ties ? need : ties;
+                // every tie kept: no row search needed
+                st.cut_row = st.need == ties ? LLONG_MAX : -1;
+                st.cut_rank = 0;
             }
         }
-        state[b] = s2;
     }
+    __syncthreads();
+}
+
+struct EgArgs {
+    const float *probs;     // [B,H,C_q,C_k]
+    const float *vnorm;     // [B,H,C_k] or nullptr
+    double *ent_part;       // [B,H,ctas]: row-entropy sums of one CTA of level 1
+    float *heads_h;         // [B,H]
+    float *entropy;         // [B,H] or nullptr (caller's)
+    float *entropy_norm;    // [B,H] or nullptr (caller's)
+    uint8_t *low;           // [B,H]
+    uint8_t *low_out;       // [B,H] or nullptr (caller's)
+    int *pool_heads;        // [B,H]: the pooled heads of b in ascending order
+    unsigned long long *hist1;  // [B,H,256,2]
+    unsigned long long *hist;   // [B,4096,2]
+    int *tiecnt;            // [B,H,C_q]
+    PoolState *state;       // [B]
+    unsigned int *counter;  // this launch's finish counter
+    int B, H, Cq, Ck;
+    int ctas;               // CTAs per head (level 1) or per batch entry (later passes)
+    float eps, inv_log_ck, pool_p;
+};
+
+__device__ __forceinline__ bool pool_active(const PoolState &st) { return !st.empty && !st.keep_all; }
+
+// Rows [r0, r1) of n rows split into contiguous runs, one per warp of the grid slice.
+__device__ __forceinline__ void warp_rows(long long n, long long warp, long long warps, long long &r0,
+                                          long long &r1) {
+    const long long per = (n + warps - 1) / warps;
+    r0 = min(n, warp * per);
+    r1 = min(n, r0 + per);
+}
+
+// Row entropies of every head and the level-1 histogram (exponent field of the
+// score) per head.  CTA blockIdx.x % ctas of head blockIdx.x / ctas takes a
+// contiguous run of rows, each warp a run of that; a warp holds a whole row in
+// registers (VPL values per lane) and bins into its own shared histogram.
+template <int VPL>
+__global__ void __launch_bounds__(kThreads) entropy_level1_kernel(EgArgs a) {
+    // per warp kL1Copies histograms (count, lo, hi), lane l bins into copy l % kL1Copies;
+    // copies kL1Stride words apart so that one bin's copies sit in different banks
+    extern __shared__ __align__(16) uint32_t sh[];
+    __shared__ ScanScratch sc;
+    __shared__ PoolState s_st;
+    __shared__ double s_wsum[kWarps];
+    __shared__ float s_h[kMaxHeads];
+    __shared__ int s_heads[kMaxHeads];
+    const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
+    __shared__ int s_zero;
+    {
+        uint32_t *wbase = sh + wid * kL1Copies * kL1Stride;
+        for (int k = lane; k < kL1Copies * kL1Stride; k += 32) wbase[k] = 0u;
+        if (threadIdx.x == 0) s_zero = 0;
+        __syncthreads();
+        uint32_t *wl = wbase + (lane % kL1Copies) * kL1Stride, *wh = wl + kL1Bins;
+        bool zero = false;
+        const long long bh = blockIdx.x / a.ctas;
+        const int part = blockIdx.x % a.ctas;
+        const int Ck = a.Ck;
+        const bool va = a.vnorm != nullptr;
+        float vn[VPL];
+        load_vnorm<VPL>(a.vnorm, bh, Ck, lane, vn);
+        long long i0, i1;
+        warp_rows(a.Cq, static_cast<long long>(part) * kWarps + wid, static_cast<long long>(a.ctas) * kWarps,
+                  i0, i1);
+        double wsum = 0.0;  // lane 0: this warp's rows, in row order
+        for (long long i = i0; i < i1; ++i) {
+            const float *prow = a.probs + (bh * a.Cq + i) * Ck;
+            float y[VPL];
+#pragma unroll
+            for (int s = 0; s < VPL; ++s) {
+                const int j = lane + 32 * s;
+                y[s] = j < Ck ? __ldg(prow + j) : 0.f;
+            }
+            float ent = 0.f;
+#pragma unroll
+            for (int s = 0; s < VPL; ++s) {
+                const int j = lane + 32 * s;
+                if (j < Ck) {
+                    const float x = y[s] > 0.f ? y[s] : 0.f;
+                    ent = fmaf(x, lg2_fast(x + a.eps), ent);
+                    const uint32_t u = score_bits(x, va, vn[s]);
+                    bin_add_sum(wl, wh, u >> 23, u);
+                    zero |= u == 0u;
+                }
+            }
+            ent = warp_sum(ent);
+            wsum += static_cast<double>(-ent * 0.6931471805599453f);  // ln 2
+        }
+        if (lane == 0) s_wsum[wid] = wsum;
+        if (__any_sync(0xffffffffu, zero) && lane == 0) atomicOr(&s_zero, 1);
+        __syncthreads();
+        const int t = threadIdx.x;  // bin t
+        unsigned long long s = 0;
+        for (int w = 0; w < kWarps * kL1Copies; ++w) {
+            const uint32_t *h = sh + w * kL1Stride;
+            s += h[t] + (static_cast<unsigned long long>(h[kL1Bins + t]) << 12);
+        }
+        if (s || (t == 0 && s_zero)) {  // the count slot only marks non-empty bins
+            atomicAdd(&a.hist1[(bh * kL1Bins + t) * 2], 1ull);
+            atomicAdd(&a.hist1[(bh * kL1Bins + t) * 2 + 1], s);
+        }
+        if (t == 0) {
+            double cs = 0.0;
+            for (int w = 0; w < kWarps; ++w) cs += s_wsum[w];
+            a.ent_part[bh * a.ctas + part] = cs;
+        }
+    }
+    if (!last_cta(a.counter)) return;
+
+    // ---- the last CTA: per-head means, median split, level-1 pick per batch entry
+    const long long BH = static_cast<long long>(a.B) * a.H;
+    for (long long bh = wid; bh < BH; bh += kWarps) {
+        double s = 0.0;  // fixed order: part-strided per lane, then a butterfly; lane 0's sum
+        for (int q = lane; q < a.ctas; q += 32) s += __ldcg(a.ent_part + bh * a.ctas + q);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) {
+            const float Hh = static_cast<float>(s / a.Cq);
+            a.heads_h[bh] = Hh;
+            if (a.entropy) a.entropy[bh] = Hh;
+            if (a.entropy_norm) a.entropy_norm[bh] = Hh * a.inv_log_ck;
+        }
+    }
+    __syncthreads();
+    uint32_t *cnt = sh;  // reuse: [256] counts, then [256] u64 sums
+    unsigned long long *sum = reinterpret_cast<unsigned long long *>(sh + 2 * kL1Bins);
+    const int H = a.H, np = H / 2;
+    for (int b = 0; b < a.B; ++b) {
+        for (int h = threadIdx.x; h < H; h += kThreads) s_h[h] = a.heads_h[static_cast<long long>(b) * H + h];
+        __syncthreads();
+        // heads ordered by (H_h asc, h asc); the first floor(H/2) are pooled.  The
+        // ranks form a permutation even for NaN entropies (ordered last).
+        for (int h = threadIdx.x; h < H; h += kThreads) {
+            const uint32_t x = order_key(s_h[h]);
+            int rank = 0;
+            for (int o = 0; o < H; ++o) {
+                const uint32_t y = order_key(s_h[o]);
+                rank += (y < x || (y == x && o < h)) ? 1 : 0;
+            }
+            const uint8_t l = rank < np ? 1 : 0;
+            a.low[static_cast<long long>(b) * H + h] = l;
+            if (a.low_out) a.low_out[static_cast<long long>(b) * H + h] = l;
+            s_heads[h] = l;  // flag for now, list below
+        }
+        if (threadIdx.x == 0) {
+            PoolState z;
+            z.target = 0.0;
+            z.above = 0.0;
+            z.pad2 = 0;
+            z.pre = 0;
+            z.shift = 31;  // level 1 bins bits 30..23 of scores >= 0 (bit 31 is 0)
+            z.keep_all = 0;
+            z.empty = np == 0;
+            z.ucut = 0;
+            z.pad0 = 0;
+            z.need = 0;
+            z.cut_row = -1;
+            z.cut_rank = 0;
+            z.pad1 = 0;
+            s_st = z;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {  // flags -> ascending list of pooled heads
+            int k = 0;
+            for (int h = 0; h < H; ++h)
+                if (s_heads[h]) s_heads[k++] = h;
+        }
+        __syncthreads();
+        for (int k = threadIdx.x; k < np; k += kThreads) a.pool_heads[static_cast<long long>(b) * H + k] = s_heads[k];
+        if (!s_st.empty) {
+            const int t = threadIdx.x;  // bin t over the pooled heads, loads 8 heads at a time
+            unsigned long long c = 0, s = 0;
+            for (int k0 = 0; k0 < np; k0 += 8) {
+                unsigned long long cc[8], ss[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    cc[q] = ss[q] = 0ull;
+                    if (k0 + q < np) {
+                        const unsigned long long *g =
+                            a.hist1 + ((static_cast<long long>(b) * H + s_heads[k0 + q]) * kL1Bins + t) * 2;
+                        cc[q] = __ldcg(g);
+                        ss[q] = __ldcg(g + 1);
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    c += cc[q];
+                    s += ss[q];
+                }
+            }
+            cnt[t] = static_cast<uint32_t>(c);
+            sum[t] = s;
+            __syncthreads();
+            cta_pick(cnt, sum, 8, true, a.pool_p, s_st, sc);
+        }
+        if (threadIdx.x == 0) a.state[b] = s_st;
+        __syncthreads();
+    }
+}
+
+// Pooled rows of batch entry b in (h, i) order: row r is row r % C_q of the
+// (r / C_q)-th pooled head.
+__device__ __forceinline__ long long pooled_row(const EgArgs &a, const int *heads, int b, long long r) {
+    const long long kk = r / a.Cq;
+    return (static_cast<long long>(b) * a.H + heads[kk]) * a.Cq + (r - kk * a.Cq);
+}
+
+// One later radix level over the pooled rows of batch entry blockIdx.x / ctas:
+// every score in the current range (bits above `shift` equal to `pre`) adds
+// (1, significand) to bin (u >> (shift - NBITS)) & (2^NBITS - 1).
+template <int VPL, int NBITS, bool COUNTS>
+__global__ void __launch_bounds__(kThreads) pool_level_kernel(EgArgs a) {
+    constexpr int nb = 1 << NBITS;
+    constexpr int per = nb / kThreads;
+    __shared__ int s_zero;
+    extern __shared__ __align__(16) uint32_t sh[];  // [3 * nb]: count, lo, hi; then count + u64 sum
+    __shared__ ScanScratch sc;
+    __shared__ PoolState s_st;
+    __shared__ int s_heads[kMaxHeads];
+    const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
+    {
+        const int b = blockIdx.x / a.ctas, part = blockIdx.x % a.ctas;
+        const PoolState st = a.state[b];
+        if (pool_active(st) && st.shift >= NBITS) {
+            uint32_t *c = sh, *lo = sh + nb, *hi = sh + 2 * nb;
+            for (int k = threadIdx.x; k < 3 * nb; k += kThreads) sh[k] = 0u;
+            if (threadIdx.x == 0) s_zero = 0;
+            bool zero = false;
+            for (int k = threadIdx.x; k < a.H / 2; k += kThreads)
+                s_heads[k] = a.pool_heads[static_cast<long long>(b) * a.H + k];
+            __syncthreads();
+            const int shift = st.shift, low_bits = st.shift - NBITS;
+            const uint32_t pre = st.pre;
+            const int Ck = a.Ck;
+            long long r0, r1;
+            warp_rows(static_cast<long long>(a.H / 2) * a.Cq, static_cast<long long>(part) * kWarps + wid,
+                      static_cast<long long>(a.ctas) * kWarps, r0, r1);
+            const bool va = a.vnorm != nullptr;
+            float vn[VPL];
+            long long cur_bh = -1;
+            for (long long r = r0; r < r1; ++r) {
+                const long long row = pooled_row(a, s_heads, b, r);
+                const long long bh = row / a.Cq;
+                if (va && bh != cur_bh) {
+                    load_vnorm<VPL>(a.vnorm, bh, Ck, lane, vn);
+                    cur_bh = bh;
+                }
+                const float *prow = a.probs + row * Ck;
+                float y[VPL];
+#pragma unroll
+                for (int s = 0; s < VPL; ++s) {
+                    const int j = lane + 32 * s;
+                    y[s] = j < Ck ? __ldg(prow + j) : 0.f;
+                }
+#pragma unroll
+                for (int s = 0; s < VPL; ++s) {
+                    const int j = lane + 32 * s;
+                    if (j < Ck) {
+                        const uint32_t u = score_bits(y[s], va, vn[s]);
+                        if ((u >> shift) == pre) {
+                            if (COUNTS) {
+                                bin_add(c, lo, hi, (u >> low_bits) & (nb - 1), u);
+                            } else {
+                                bin_add_sum(lo, hi, (u >> low_bits) & (nb - 1), u);
+                                zero |= u == 0u;
+                            }
+                        }
+                    }
+                }
+            }
+            if (!COUNTS && __any_sync(0xffffffffu, zero) && lane == 0) atomicOr(&s_zero, 1);
+            __syncthreads();
+            unsigned long long *g = a.hist + static_cast<long long>(b) * 2 * kMaxBins;
+            for (int k = threadIdx.x; k < nb; k += kThreads) {
+                const unsigned long long sk = lo[k] + (static_cast<unsigned long long>(hi[k]) << 12);
+                const unsigned long long ck = COUNTS ? c[k] : ((sk || (k == 0 && s_zero)) ? 1ull : 0ull);
+                if (ck) {
+                    atomicAdd(&g[2 * k], ck);
+                    atomicAdd(&g[2 * k + 1], sk);
+                }
+            }
+        }
+    }
+    if (!last_cta(a.counter)) return;
+
+    // ---- the last CTA: the pick of every active batch entry
+    uint32_t *cnt = sh;
+    unsigned long long *sum = reinterpret_cast<unsigned long long *>(sh + nb);
+    for (int b = 0; b < a.B; ++b) {
+        if (threadIdx.x == 0) s_st = a.state[b];
+        __syncthreads();
+        if (pool_active(s_st) && s_st.shift >= NBITS) {
+            unsigned long long *g = a.hist + static_cast<long long>(b) * 2 * kMaxBins;
+            unsigned long long cc[per], ss[per];
+#pragma unroll
+            for (int q = 0; q < per; ++q) {
+                const int k = threadIdx.x + q * kThreads;
+                cc[q] = __ldcg(&g[2 * k]);
+                ss[q] = __ldcg(&g[2 * k + 1]);
+            }
+#pragma unroll
+            for (int q = 0; q < per; ++q) {
+                const int k = threadIdx.x + q * kThreads;
+                cnt[k] = static_cast<uint32_t>(cc[q]);
+                sum[k] = ss[q];
+                g[2 * k] = 0ull;  // ready for the next level
+                g[2 * k + 1] = 0ull;
+            }
+            __syncthreads();
+            cta_pick(cnt, sum, NBITS, false, a.pool_p, s_st, sc);
+            if (threadIdx.x == 0) a.state[b] = s_st;
+        }
+        __syncthreads();
+    }
+}
+
+// Needed only when some but not all pairs equal to the cut pattern are kept:
+// ties per pooled row, then (last CTA) the row, in (h, i) order, where their
+// running count reaches `need` and how many of that row's ties are kept.
+template <int VPL>
+__global__ void __launch_bounds__(kThreads) tie_kernel(EgArgs a) {
+    __shared__ ScanScratch sc;
+    __shared__ int s_heads[kMaxHeads];
+    const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
+    const long long rows = static_cast<long long>(a.H / 2) * a.Cq;
+    {
+        const int b = blockIdx.x / a.ctas, part = blockIdx.x % a.ctas;
+        const PoolState st = a.state[b];
+        if (pool_active(st) && st.cut_row == -1) {
+            for (int k = threadIdx.x; k < a.H / 2; k += kThreads)
+                s_heads[k] = a.pool_heads[static_cast<long long>(b) * a.H + k];
+            __syncthreads();
+            const int Ck = a.Ck;
+            long long r0, r1;
+            warp_rows(rows, static_cast<long long>(part) * kWarps + wid, static_cast<long long>(a.ctas) * kWarps,
+                      r0, r1);
+            const bool va = a.vnorm != nullptr;
+            float vn[VPL];
+            long long cur_bh = -1;
+            for (long long r = r0; r < r1; ++r) {
+                const long long row = pooled_row(a, s_heads, b, r);
+                const long long bh = row / a.Cq;
+                if (va && bh != cur_bh) {
+                    load_vnorm<VPL>(a.vnorm, bh, Ck, lane, vn);
+                    cur_bh = bh;
+                }
+                const float *prow = a.probs + row * Ck;
+                float y[VPL];
+#pragma unroll
+                for (int s = 0; s < VPL; ++s) {
+                    const int j = lane + 32 * s;
+                    y[s] = j < Ck ? __ldg(prow + j) : 0.f;
+                }
+                int n = 0;
+#pragma unroll
+                for (int s = 0; s < VPL; ++s) {
+                    const int j = lane + 32 * s;
+                    n += __popc(__ballot_sync(0xffffffffu, j < Ck && score_bits(y[s], va, vn[s]) == st.ucut));
+                }
+                if (lane == 0) a.tiecnt[row] = n;
+            }
+        }
+    }
+    if (!last_cta(a.counter)) return;
+
+    // ---- the last CTA: a scan over the pooled rows of each batch entry that needs one
+    const int t = threadIdx.x;
+    for (int b = 0; b < a.B; ++b) {
+        const PoolState st = a.state[b];
+        if (!pool_active(st) || st.cut_row != -1) continue;  // uniform over the CTA
+        for (int k = t; k < a.H / 2; k += kThreads) s_heads[k] = a.pool_heads[static_cast<long long>(b) * a.H + k];
+        if (t == 0) sc.owner = INT_MAX;
+        __syncthreads();
+        const long long per = (rows + kThreads - 1) / kThreads;
+        const long long r0 = min(rows, t * per), r1 = min(rows, r0 + per);
+        unsigned long long n = 0;
+        for (long long r = r0; r < r1; r += 8) {  // 8 loads in flight
+            int v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) v[q] = r + q < r1 ? __ldcg(a.tiecnt + pooled_row(a, s_heads, b, r + q)) : 0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) n += static_cast<unsigned long long>(v[q]);
+        }
+        double dm = 0.0;
+        unsigned long long run = n;
+        cta_scan(dm, run, sc);  // inclusive tie counts in thread order
+        if (n > 0 && run >= st.need) atomicMin(&sc.owner, t);
+        __syncthreads();
+        if (t == sc.owner) {
+            unsigned long long acc = run - n;
+            long long cut_row = -1;
+            int cut_rank = 0;
+            for (long long r = r0; r < r1 && cut_row < 0; r += 8) {
+                int v[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) v[q] = r + q < r1 ? __ldcg(a.tiecnt + pooled_row(a, s_heads, b, r + q)) : 0;
+                for (int q = 0; q < 8 && r + q < r1; ++q) {
+                    const unsigned long long c = static_cast<unsigned long long>(v[q]);
+                    if (acc + c >= st.need) {
+                        cut_row = pooled_row(a, s_heads, b, r + q);
+                        cut_rank = static_cast<int>(st.need - acc);
+                        break;
+                    }
+                    acc += c;
+                }
+            }
+            a.state[b].cut_row = cut_row;
+            a.state[b].cut_rank = cut_rank;
+        }
+        __syncthreads();
+    }
+}
+
+template <int VPL>
+cudaError_t launch_eg_passes(const EgArgs &base, long long c1, long long c2, int B, long long BH,
+                             cudaStream_t st) {
+    unsigned int *counters = base.counter;
+    EgArgs a = base;
+    a.ctas = static_cast<int>(c1);
+    a.counter = counters + 0;
+    cudaError_t e = cudaFuncSetAttribute(entropy_level1_kernel<VPL>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kL1Smem));
+    if (e != cudaSuccess) return e;
+    entropy_level1_kernel<VPL><<<static_cast<unsigned>(BH * c1), kThreads, kL1Smem, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    a.ctas = static_cast<int>(c2);
+    const unsigned grid2 = static_cast<unsigned>(B * c2);
+    const size_t smem12 = 3 * (1 << kLevelBits[0]) * sizeof(uint32_t);
+    const size_t smem11 = 3 * (1 << kLevelBits[1]) * sizeof(uint32_t);
+    if ((e = cudaFuncSetAttribute(pool_level_kernel<VPL, kLevelBits[0], false>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(smem12))) != cudaSuccess)
+        return e;
+    a.counter = counters + 1;
+    pool_level_kernel<VPL, kLevelBits[0], false><<<grid2, kThreads, smem12, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    a.counter = counters + 2;
+    pool_level_kernel<VPL, kLevelBits[1], true><<<grid2, kThreads, smem11, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    a.counter = counters + 3;
+    tie_kernel<VPL><<<grid2, kThreads, 0, st>>>(a);
+    return cudaGetLastError();
 }
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Level-1 CTAs per head: at most one per kWarps rows.
+long long eg_level1_ctas_max(int Cq) { return max(1ll, (static_cast<long long>(Cq) + kWarps - 1) / kWarps); }
+
+static_assert(kL1Bins == kThreads, "the level-1 fold and pick take one bin per thread");
+static_assert(kMaxBins % kThreads == 0 && (1 << kLevelBits[1]) % kThreads == 0, "bins per thread");
 
 }  // namespace
 
@@ -372,18 +732,27 @@ EgWorkspace eg_workspace(const Geometry &g) {
     const size_t bh = static_cast<size_t>(g.B) * g.H;
     EgWorkspace w;
     size_t off = 0;
-    w.row_entropy = off;
-    off += round256(rows * sizeof(float));
+    w.ent_part = off;
+    off += round256(bh * static_cast<size_t>(eg_level1_ctas_max(g.Cq)) * sizeof(double));
     w.heads_h = off;
     off += round256(bh * sizeof(float));
     w.low = off;
     off += round256(bh);
-    w.hist = off;
-    off += round256(static_cast<size_t>(g.B) * 2 * kMaxBins * sizeof(unsigned long long));
+    w.pool_heads = off;
+    off += round256(bh * sizeof(int));
     w.state = off;
     off += round256(static_cast<size_t>(g.B) * sizeof(PoolState));
+    // zeroed once per call: histograms, tie counts, finish counters
+    w.zero_begin = off;
+    w.hist1 = off;
+    off += round256(bh * kL1Bins * 2 * sizeof(unsigned long long));
+    w.hist = off;
+    off += round256(static_cast<size_t>(g.B) * 2 * kMaxBins * sizeof(unsigned long long));
     w.tiecnt = off;
     off += round256(rows * sizeof(int));
+    w.counters = off;
+    off += round256(4 * sizeof(unsigned int));
+    w.zero_bytes = off - w.zero_begin;
     w.bytes = off;
     return w;
 }
@@ -392,54 +761,55 @@ cudaError_t launch_eg_prepare(const Geometry &g, const float *probs, const float
                               float pool_p, float eps, float *entropy, float *entropy_norm,
                               uint8_t *low_heads, uint8_t *workspace, cudaStream_t st) {
     const EgWorkspace w = eg_workspace(g);
-    float *row_ent = reinterpret_cast<float *>(workspace + w.row_entropy);
-    float *heads_h = reinterpret_cast<float *>(workspace + w.heads_h);
-    uint8_t *low = workspace + w.low;
-    unsigned long long *hist = reinterpret_cast<unsigned long long *>(workspace + w.hist);
-    PoolState *state = reinterpret_cast<PoolState *>(workspace + w.state);
-    int *tiecnt = reinterpret_cast<int *>(workspace + w.tiecnt);
-    const long long rows = static_cast<long long>(g.B) * g.H * g.Cq;
-    const unsigned rgrid = static_cast<unsigned>((rows + 7) / 8);
-
-    row_entropy_kernel<<<rgrid, 256, 0, st>>>(probs, row_ent, rows, g.Ck, eps);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = cudaMemsetAsync(workspace + w.zero_begin, 0, w.zero_bytes, st);
     if (e != cudaSuccess) return e;
-    e = launch_entropy_reduce(g, row_ent, heads_h, entropy_norm, st);
-    if (e != cudaSuccess) return e;
-    if (entropy) {
-        e = cudaMemcpyAsync(entropy, heads_h, static_cast<size_t>(g.B) * g.H * sizeof(float),
-                            cudaMemcpyDeviceToDevice, st);
-        if (e != cudaSuccess) return e;
-    }
-    route_kernel<<<g.B, 256, 0, st>>>(heads_h, g.H, low, low_heads, state);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorInvalidValue;
-    const long long pool_rows = static_cast<long long>(g.H / 2) * g.Cq;
-    const unsigned hx = static_cast<unsigned>(
-        max(1ll, min(static_cast<long long>(2 * sms) / max(g.B, 1), (pool_rows + 7) / 8)));
-    for (int level = 0; level < 3; ++level) {
-        const int nbits = kLevelBits[level];
-        const size_t smem = static_cast<size_t>(2) << nbits << 3;  // 2^nbits x 2 x 8 bytes
-        if ((e = cudaMemsetAsync(hist, 0,
-                                 static_cast<size_t>(g.B) * 2 * kMaxBins * sizeof(unsigned long long),
-                                 st)) != cudaSuccess)
-            return e;
-        if (smem > 48 * 1024 &&
-            (e = cudaFuncSetAttribute(pool_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      static_cast<int>(smem))) != cudaSuccess)
-            return e;
-        pool_hist_kernel<<<dim3(hx, g.B), 256, smem, st>>>(probs, vnorm, low, state, hist, g.H,
-                                                          g.Cq, g.Ck, nbits);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        pool_pick_kernel<<<g.B, 32, 0, st>>>(hist, state, pool_p, nbits, level == 0 ? 1 : 0);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-    tie_count_kernel<<<rgrid, 256, 0, st>>>(probs, vnorm, low, state, tiecnt, rows, g.H, g.Cq, g.Ck);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    tie_scan_kernel<<<g.B, 1024, 0, st>>>(tiecnt, state, g.H, g.Cq);
-    return cudaGetLastError();
+
+    EgArgs a;
+    a.probs = probs;
+    a.vnorm = vnorm;
+    a.ent_part = reinterpret_cast<double *>(workspace + w.ent_part);
+    a.heads_h = reinterpret_cast<float *>(workspace + w.heads_h);
+    a.entropy = entropy;
+    a.entropy_norm = entropy_norm;
+    a.low = workspace + w.low;
+    a.low_out = low_heads;
+    a.pool_heads = reinterpret_cast<int *>(workspace + w.pool_heads);
+    a.hist1 = reinterpret_cast<unsigned long long *>(workspace + w.hist1);
+    a.hist = reinterpret_cast<unsigned long long *>(workspace + w.hist);
+    a.tiecnt = reinterpret_cast<int *>(workspace + w.tiecnt);
+    a.state = reinterpret_cast<PoolState *>(workspace + w.state);
+    a.counter = reinterpret_cast<unsigned int *>(workspace + w.counters);
+    a.B = g.B;
+    a.H = g.H;
+    a.Cq = g.Cq;
+    a.Ck = g.Ck;
+    a.ctas = 0;
+    a.eps = eps;
+    a.inv_log_ck = g.Ck > 1 ? 1.0f / logf(static_cast<float>(g.Ck)) : 0.f;
+    a.pool_p = pool_p;
+
+    // level 1 with the row entropies: about two CTAs per SM, at least one row per
+    // warp, and few enough rows per warp that its 32-bit bins stay exact
+    const long long BH = static_cast<long long>(g.B) * g.H;
+    const long long rows_cap = static_cast<long long>(kBinCap / static_cast<uint32_t>(g.Ck)) * kWarps;
+    const long long c1 = max((static_cast<long long>(g.Cq) + rows_cap - 1) / rows_cap,
+                             min((2ll * sms + BH - 1) / BH, eg_level1_ctas_max(g.Cq)));
+    // later passes over the pooled rows: about two CTAs per SM in all, and at
+    // most kBinCap pairs per CTA (its warps share one histogram)
+    const long long prow = static_cast<long long>(g.H / 2) * g.Cq;
+    const long long prow_cap =
+        static_cast<long long>(kBinCap / (static_cast<uint32_t>(g.Ck) * kWarps)) * kWarps;
+    const long long c2 = max(max(1ll, (prow + prow_cap - 1) / prow_cap),
+                             min((2ll * sms + g.B - 1) / g.B, max(1ll, (prow + kWarps - 1) / kWarps)));
+    if (BH * c1 > 0x7FFFFFFFll || static_cast<long long>(g.B) * c2 > 0x7FFFFFFFll) return cudaErrorInvalidValue;
+    const int vpl = (g.Ck + 31) / 32;
+    if (vpl <= 4) return launch_eg_passes<4>(a, c1, c2, g.B, BH, st);
+    if (vpl <= 8) return launch_eg_passes<8>(a, c1, c2, g.B, BH, st);
+    if (vpl <= 16) return launch_eg_passes<16>(a, c1, c2, g.B, BH, st);
+    if (vpl <= 32) return launch_eg_passes<32>(a, c1, c2, g.B, BH, st);
+    return launch_eg_passes<64>(a, c1, c2, g.B, BH, st);
 }
 
 }  // namespace bsa

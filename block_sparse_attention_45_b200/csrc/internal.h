@@ -56,7 +56,7 @@ cudaError_t launch_entropy_reduce(const Geometry &g, const float *row_entropy, f
 struct PoolState {
     double target;                // pool_p * (total score of the pool)
     double above;                 // score mass of the pool above the current range
-    unsigned long long cnt_above; // number of pool pairs above the current range
+    unsigned long long pad2;
     uint32_t pre;                 // bit-pattern prefix of the current range
     int shift;                    // low bits below the prefix (0 once the cut value is found)
     int keep_all;                 // the pool never reaches target: every pair is kept
@@ -74,7 +74,9 @@ cudaError_t launch_value_norms(const Geometry &g, const void *v, float *vnorm, c
 
 // Workspace layout of bsa_build_mask_eg (byte offsets; all 256-aligned).
 struct EgWorkspace {
-    size_t row_entropy, heads_h, low, hist, state, tiecnt, bytes;
+    size_t ent_part, heads_h, low, pool_heads, state;
+    size_t zero_begin, zero_bytes;  // cleared at the start of every call
+    size_t hist1, hist, tiecnt, counters, bytes;
 };
 EgWorkspace eg_workspace(const Geometry &g);
 

@@ -128,6 +128,57 @@ def test_eg_overrides_and_per_row_heads(name):
     assert np.array_equal(g["mask"].cpu().numpy()[per_row], m0[per_row])
 
 
+@pytest.mark.parametrize("kind", ["uniform", "quantised"])
+@pytest.mark.parametrize("name", ["h3_b2", "h5_d128", "small"])
+def test_eg_many_ties(name, kind):
+    """Scores with many exact ties: the cut falls inside a run of equal scores
+    spread over many rows, so the kept ties follow the (h, i, j) order."""
+    w = CASES[name]
+    ora = oracle.default()
+    L = w.layout()
+    B, H = w.batch, w.heads
+    Cq, Ck = w.seq_pad // w.q_block, w.seq_pad // w.k_block
+    rng = np.random.default_rng(7)
+    if kind == "uniform":
+        probs = np.full((B, H, Cq, Ck), 1.0 / Ck, np.float32)
+        vn = np.ones((B, H, Ck), np.float32)
+        # distinct per-head entropies would all be equal here: the routing then
+        # follows the head index
+    else:
+        probs = (2.0 ** -rng.integers(3, 7, size=(B, H, Cq, Ck))).astype(np.float32)
+        vn = (2.0 ** rng.integers(0, 2, size=(B, H, Ck))).astype(np.float32)
+    tp = [0.8] * H
+    H_ora, _ = ora.entropy(L, probs)
+    for pool_p in (0.5, 0.9, 0.0):
+        g = bsa.build_mask_eg(w, torch.from_numpy(probs).cuda(), torch.from_numpy(vn).cuda(), tp,
+                              pool_p, 0)
+        torch.cuda.synchronize()
+        gpu_low = g["low_heads"].cpu().numpy()
+        low = ora.eg_route(L, H_ora)
+        exp = ora.eg_select(L, probs, vn, tp, pool_p, low)
+        got = g["mask"].cpu().numpy()
+        for b in range(B):
+            if np.array_equal(gpu_low[b], low[b]):
+                bad = np.argwhere((got[b] != exp[b]).any(-1))
+                assert bad.size == 0, (name, kind, pool_p, b, bad[:5].tolist())
+        checkers.check_lists(g["kv_index"].cpu().numpy(), g["kv_count"].cpu().numpy(), got)
+
+
+def test_eg_zero_eps_routes_every_batch_entry():
+    """eps = 0 (entropy terms of zero entries are 0 * log 0): the median split
+    still pools exactly floor(H/2) heads per batch entry."""
+    w, _, probs, _, vn = _oracle_inputs("h3_b2")
+    p = probs.copy()
+    p[..., ::3] = 0.0
+    g = bsa.build_mask_eg(w, torch.from_numpy(p).cuda(), torch.from_numpy(vn).cuda(),
+                          [0.8] * w.heads, 0.9, 0, eps=0.0)
+    torch.cuda.synchronize()
+    low = g["low_heads"].cpu().numpy()
+    assert np.array_equal(low.sum(-1), np.full(w.batch, w.heads // 2))
+    checkers.check_lists(g["kv_index"].cpu().numpy(), g["kv_count"].cpu().numpy(),
+                         g["mask"].cpu().numpy())
+
+
 def test_eg_single_head_is_the_per_row_rule():
     w, _, probs, _, vn = _oracle_inputs("h1")
     tp = [float(w.top_p)]
