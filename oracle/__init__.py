@@ -62,11 +62,16 @@ class Oracle:
         L.ora_topp.argtypes = [lp, vp, vp, vp, vp]
         L.ora_overrides.argtypes = [lp, ctypes.c_uint32, vp]
         L.ora_lists.argtypes = [lp, vp, vp, vp]
-        L.ora_attention.argtypes = [lp, vp, vp, vp, vp, ctypes.c_double, ctypes.c_long,
+        L.ora_attention.argtypes = [lp, vp, vp, vp, vp, vp, ctypes.c_double, ctypes.c_long,
                                     vp, vp, vp]
         L.ora_value_norms.argtypes = [lp, vp, vp]
         L.ora_eg_route.argtypes = [lp, vp, vp]
         L.ora_eg_select.argtypes = [lp, vp, vp, vp, ctypes.c_float, vp, vp]
+        L.ora_splitmix64.argtypes = [ctypes.c_uint64, ctypes.c_uint64]
+        L.ora_splitmix64.restype = ctypes.c_uint64
+        L.ora_inclusion.argtypes = [lp, vp, ctypes.c_float, ctypes.c_uint32, vp, vp]
+        L.ora_sample_select.argtypes = [lp, vp, ctypes.c_float, ctypes.c_uint64, ctypes.c_uint32,
+                                        vp, vp]
         L.ora_num_threads.restype = ctypes.c_int
         self.lib = L
 
@@ -138,18 +143,21 @@ class Oracle:
         self.lib.ora_lists(ctypes.byref(L), _ptr(mask), _ptr(idx), _ptr(cnt))
         return idx, cnt
 
-    def attention(self, L, q, k, v, mask=None, scale=None, rows=None):
+    def attention(self, L, q, k, v, mask=None, scale=None, rows=None, weight=None):
         """Exact softmax attention over the selected blocks (mask None = dense).
 
         rows: optional flat query-block ids (b*H*C_q + h*C_q + i).  Returns
         out fp32 [nrows, q_block, D] and lse fp32 [nrows, q_block]; with rows
         None the leading axis covers every query block in (b, h, i) order.
+        weight: optional fp32 [B,H,C_q,C_k], multiplying every exp term of a
+        key of block j (numerator and sum) by weight[b,h,i,j].
         """
         L = _layout(L)
         q, k, v = _u16(q), _u16(k), _u16(v)
         if scale is None:
             scale = 1.0 / math.sqrt(L.head_dim)
         m = None if mask is None else np.ascontiguousarray(mask, np.uint8)
+        wt = None if weight is None else np.ascontiguousarray(weight, np.float32)
         if rows is None:
             n = L.batch * L.heads * L.cq
             r = None
@@ -158,9 +166,33 @@ class Oracle:
             n = r.shape[0]
         out = np.empty((n, L.q_block, L.head_dim), np.float32)
         lse = np.empty((n, L.q_block), np.float32)
-        self.lib.ora_attention(ctypes.byref(L), _ptr(q), _ptr(k), _ptr(v), _ptr(m),
+        self.lib.ora_attention(ctypes.byref(L), _ptr(q), _ptr(k), _ptr(v), _ptr(m), _ptr(wt),
                                float(scale), n, _ptr(r), _ptr(out), _ptr(lse))
         return out, lse
+
+    def splitmix64(self, seed, idx):
+        """The idx-th output (from 0) of SplitMix64 started from state `seed`."""
+        return int(self.lib.ora_splitmix64(int(seed) & (2**64 - 1), int(idx) & (2**64 - 1)))
+
+    def inclusion(self, L, probs, budget, flags):
+        """Inclusion probability pi and weight 1/pi (fp32 [B,H,C_q,C_k]) of every pair."""
+        L = _layout(L)
+        probs = np.ascontiguousarray(probs, np.float32)
+        pi = np.empty(probs.shape, np.float32)
+        w = np.empty(probs.shape, np.float32)
+        self.lib.ora_inclusion(ctypes.byref(L), _ptr(probs), float(budget), int(flags), _ptr(pi),
+                               _ptr(w))
+        return pi, w
+
+    def sample_select(self, L, probs, budget, seed, flags):
+        """One draw of the importance sampler: mask u8 and weight fp32 [B,H,C_q,C_k]."""
+        L = _layout(L)
+        probs = np.ascontiguousarray(probs, np.float32)
+        mask = np.empty(probs.shape, np.uint8)
+        weight = np.empty(probs.shape, np.float32)
+        self.lib.ora_sample_select(ctypes.byref(L), _ptr(probs), float(budget),
+                                   int(seed) & (2**64 - 1), int(flags), _ptr(mask), _ptr(weight))
+        return mask, weight
 
     def value_norms(self, L, v):
         """||c^V_{h,j}||_2 of the value centroids, fp32 [B,H,C_k]."""

@@ -24,7 +24,10 @@
  *       cross-head" with the median split on H_h and the safeguard; s4 the
  *       value-aware score of the cross-head pool (EG-Sparse).
  *  [p5] "AB-Attention: accurate block-sparse attention for video diffusion"
- *       TL;DR: exact attention computed only on the selected K/V blocks.
+ *       TL;DR: exact attention computed only on the selected K/V blocks;
+ *       fix (2): blocks sampled in proportion to importance and reweighted
+ *       by the inverse inclusion probability (an unbiased one-pass estimate
+ *       of dense attention).
  *
  * Readings taken where the pages are silent or garbled (the equations of
  * [p3] are lost in the extracted text):
@@ -264,13 +267,16 @@ void ora_lists(const ora_layout *L, const uint8_t *mask, int32_t *kv_index, int3
  *   s_u = scale * (Q_t . K_u), two-pass softmax with the exact max,
  *   O_t = sum_u softmax_u V_u, lse_t = m + ln sum_u exp(s_u - m),
  * all in fp64, stored as fp32.  mask == NULL means every block (dense).
+ * weight (fp32 [B,H,C_q,C_k], or NULL for 1) multiplies every exp term of a
+ * key of block j by weight[row, j], in the sum z and in the numerator alike
+ * ([p5] fix (2): inverse-inclusion-probability reweighting).
  * Only the query blocks listed in `qrows` (flat b*H*C_q + h*C_q + i) are
  * computed; qrows == NULL means all of them.  out is fp32 [nrows, q_block, D]
  * and lse fp32 [nrows, q_block] (indexed by position in the row list).
  */
 void ora_attention(const ora_layout *L, const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                   const uint8_t *mask, double scale, long nrows, const int64_t *qrows,
-                   float *out, float *lse)
+                   const uint8_t *mask, const float *weight, double scale, long nrows,
+                   const int64_t *qrows, float *out, float *lse)
 {
     const int D = L->head_dim, bq = L->q_block, bk = L->k_block;
     const int Cq = L->seq_pad / bq, Ck = L->seq_pad / bk;
@@ -315,6 +321,7 @@ void ora_attention(const ora_layout *L, const uint16_t *q, const uint16_t *k, co
                 for (int d = 0; d < D; ++d) acc[d] = 0.0;
                 for (int a = 0; a < nu; ++a) {
                     double e = exp(s[a] - m);
+                    if (weight) e *= (double)weight[r * Ck + u_of[a] / bk];
                     const uint16_t *Vu = Vb + (long)u_of[a] * D;
                     z += e;
                     for (int d = 0; d < D; ++d) acc[d] += e * bf16_val(Vu[d]);
@@ -496,6 +503,77 @@ void ora_eg_select(const ora_layout *L, const float *probs, const float *vnorm,
             }
         }
     }
+}
+
+/*
+ * ---------------------------------------------------------------------------
+ * Importance sampling with inverse-inclusion-probability weights ([p5] TL;DR
+ * fix (2)).  The page gives no sampling law; the readings taken:
+ *  - importance is P'; every pair (b, h, i, j) is included independently of
+ *    the others (Poisson sampling) with probability
+ *    pi = min(1, fp32(K * P')), K the per-row budget: a row of P' sums to one,
+ *    so the expected number of blocks per row is at most K; a negative or NaN
+ *    P' counts as 0;
+ *  - the draw of pair idx = ((b*H + h)*C_q + i)*C_k + j is
+ *    u = (z >> 40) * 2^-24 with z the idx-th output (from 0) of SplitMix64
+ *    seeded with `seed`; the pair is included iff u < pi;
+ *  - an included pair carries w = fp32(1 / pi); the overrides (text columns,
+ *    frame-0 rows) are included with pi = 1 and w = 1;
+ *  - attention multiplies each included key's exp term by its block's w in
+ *    the numerator and in the sum alike (Horvitz-Thompson for both).
+ * ---------------------------------------------------------------------------
+ */
+
+/* The idx-th output (idx = 0 first) of SplitMix64 started from state `seed`
+ * (Steele, Lea and Flood, "Fast splittable pseudorandom number generators",
+ * OOPSLA 2014): the state advances by the golden-ratio increment, the output
+ * is the state passed through the two xor-shift-multiply rounds. */
+uint64_t ora_splitmix64(uint64_t seed, uint64_t idx)
+{
+    uint64_t z = seed + (idx + 1u) * 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+/* Inclusion probability and weight of every pair: pi fp32 and w = fp32(1/pi)
+ * (0 where pi = 0), both [B,H,C_q,C_k]; the overrides get pi = w = 1. */
+void ora_inclusion(const ora_layout *L, const float *probs, float budget, uint32_t flags,
+                   float *pi, float *w)
+{
+    const long n = (long)L->batch * L->heads * (L->seq_pad / L->q_block) * (L->seq_pad / L->k_block);
+    uint8_t *forced = (uint8_t *)calloc((size_t)n, 1);
+    ora_overrides(L, flags, forced);                     /* the pairs kept regardless */
+    for (long e = 0; e < n; ++e) {
+        float x = probs[e];
+        if (!(x > 0.0f)) x = 0.0f;
+        float prod = budget * x;                         /* fp32 product */
+        float p = prod < 1.0f ? prod : 1.0f;
+        if (!(p >= 0.0f)) p = 0.0f;
+        if (forced[e]) p = 1.0f;
+        pi[e] = p;
+        w[e] = p > 0.0f ? 1.0f / p : 0.0f;               /* fp32 division */
+    }
+    free(forced);
+}
+
+/* One draw of the sampler: mask u8 and weight fp32 (w of included pairs, 0
+ * elsewhere), [B,H,C_q,C_k]. */
+void ora_sample_select(const ora_layout *L, const float *probs, float budget, uint64_t seed,
+                       uint32_t flags, uint8_t *mask, float *weight)
+{
+    const long n = (long)L->batch * L->heads * (L->seq_pad / L->q_block) * (L->seq_pad / L->k_block);
+    float *pi = (float *)malloc(sizeof(float) * (size_t)n);
+    float *w = (float *)malloc(sizeof(float) * (size_t)n);
+    ora_inclusion(L, probs, budget, flags, pi, w);
+    for (long e = 0; e < n; ++e) {
+        double u = (double)(ora_splitmix64(seed, (uint64_t)e) >> 40) * (1.0 / 16777216.0);
+        int keep = u < (double)pi[e];
+        mask[e] = (uint8_t)keep;
+        weight[e] = keep ? w[e] : 0.0f;
+    }
+    free(pi);
+    free(w);
 }
 
 /* Threads OpenMP will use (reported next to oracle timings). */

@@ -46,6 +46,13 @@ MUTATIONS = [
     ("no safeguard", "m[best] = 1;", "(void)best;"),
     ("safeguard takes the last maximum", "if (x > bv) { bv = x; best = j; }",
      "if (x >= bv) { bv = x; best = j; }"),
+    ("weight pi instead of 1 / pi", "w[e] = p > 0.0f ? 1.0f / p : 0.0f;", "w[e] = p > 0.0f ? p : 0.0f;"),
+    ("sum of exp terms not reweighted", "z += e;",
+     "z += e / (weight ? (double)weight[r * Ck + u_of[a] / bk] : 1.0);"),
+    ("inclusion probability not capped at one", "float p = prod < 1.0f ? prod : 1.0f;", "float p = prod;"),
+    ("overrides sampled like the rest", "if (forced[e]) p = 1.0f;", "(void)forced;"),
+    ("draw ignores the seed", "uint64_t z = seed + (idx + 1u) * 0x9E3779B97F4A7C15ull;",
+     "uint64_t z = (idx + 1u) * 0x9E3779B97F4A7C15ull;"),
 ]
 
 

@@ -12,7 +12,8 @@ s4, s6, s7); "Competition Domains Matter: Selective Head Globalization ..." s3
 (centroids, cluster-size-weighted softmax P' whose rows sum to one, per-head
 entropy normalised by log C_k, per-row local top-p); "AB-Attention: accurate
 block-sparse attention for video diffusion" TL;DR (exact attention on the
-selected blocks).
+selected blocks; fix (2), blocks sampled in proportion to importance and
+reweighted by the inverse inclusion probability).
 """
 import itertools
 import json
@@ -514,6 +515,166 @@ def check_eg_select(ora):
     assert m[0, 0, 0, 1] == 1
 
 
+# --------------------------------------------------------------------------- sampling (p5 fix 2)
+
+def check_splitmix64(ora):
+    # the generator's published reference outputs
+    g = json.load(open(os.path.join(GOLDEN, "splitmix64_vectors.json")))
+    for vec in g["vectors"]:
+        outs = vec.get("outputs_hex")
+        exp = [int(x, 16) for x in outs] if outs else [int(x) for x in vec["outputs_dec"]]
+        got = [ora.splitmix64(vec["seed"], i) for i in range(len(exp))]
+        assert got == exp, (vec["seed"], [hex(x) for x in got])
+
+
+def _tiny_probs(rng, B, H, Cq, Ck):
+    P = rng.random((B, H, Cq, Ck)) ** 3
+    P /= P.sum(-1, keepdims=True)
+    return P.astype(np.float32)
+
+
+def check_inclusion_law(ora):
+    # "sampled in proportion to importance": pi proportional to P' below the cap, capped at 1,
+    # 0 for P' = 0; overrides always included with weight 1; w * pi = 1 up to fp32 rounding
+    rng = np.random.default_rng(11)
+    L = lay(seq_len=24, seq_pad=24, bq=4, bk=4, heads=2, text_len=4, tpf=8, frames=2)
+    P = _tiny_probs(rng, 1, 2, 6, 6)
+    P[0, 0, 3, 2] = 0.0
+    K = 2.5
+    pi, w = ora.inclusion(L, P, K, 0)
+    free = (pi < 1) & (P > 0)
+    r = pi[free] / P[free].astype(np.float64)
+    assert np.allclose(r, K, rtol=1e-6), r
+    assert (pi[P.astype(np.float64) * K >= 1] == 1).all()
+    assert pi[0, 0, 3, 2] == 0 and w[0, 0, 3, 2] == 0
+    pos = pi > 0
+    assert np.all(np.abs(w[pos].astype(np.float64) * pi[pos] - 1) <= 2 ** -23)
+    assert (pi <= 1).all() and (pi >= 0).all()
+    # expected count per row at most the budget (rows of P' sum to one)
+    assert (pi.astype(np.float64).sum(-1) <= K + 1e-6).all()
+    # overrides: text column 0 and frame-0 query blocks 1..2 always in, weight 1
+    pi2, w2 = ora.inclusion(L, P, K, 3)
+    assert (pi2[..., 0] == 1).all() and (w2[..., 0] == 1).all()
+    assert (pi2[:, :, 1:3, :] == 1).all() and (w2[:, :, 1:3, :] == 1).all()
+    np.testing.assert_array_equal(pi2[:, :, [0, 3, 4, 5], 1:], pi[:, :, [0, 3, 4, 5], 1:])
+
+
+def check_sample_frequencies(ora):
+    # over many seeds each pair is included with frequency pi (5 sigma), the draws of
+    # different pairs are independent (pairwise joint frequencies), and the weights of
+    # included pairs are the pair's 1 / pi
+    rng = np.random.default_rng(12)
+    L = lay(seq_len=24, seq_pad=24, bq=4, bk=4, heads=2)
+    P = _tiny_probs(rng, 1, 2, 6, 6)
+    K = 2.0
+    pi, w = ora.inclusion(L, P, K, 0)
+    n = 4000
+    hits = np.zeros(P.shape, np.float64)
+    joint = 0.0
+    for seed in range(n):
+        m, wt = ora.sample_select(L, P, K, seed, 0)
+        assert np.array_equal(wt, np.where(m == 1, w, 0).astype(np.float32))
+        hits += m
+        joint += float(m[0, 0, 0, 0] and m[0, 1, 5, 5])
+    f = hits / n
+    sd = np.sqrt(np.maximum(pi * (1 - pi), 1e-12) / n)
+    assert (np.abs(f - pi) <= 5 * sd + 1e-12).all(), np.abs(f - pi).max()
+    pj = float(pi[0, 0, 0, 0]) * float(pi[0, 1, 5, 5])
+    assert abs(joint / n - pj) <= 5 * math.sqrt(max(pj * (1 - pj), 1e-12) / n) + 1e-12
+    # the same seed gives the same draw; another seed another one
+    a, _ = ora.sample_select(L, P, K, 7, 0)
+    b, _ = ora.sample_select(L, P, K, 7, 0)
+    c, _ = ora.sample_select(L, P, K, 8, 0)
+    assert np.array_equal(a, b) and not np.array_equal(a, c)
+
+
+def check_sampled_attention_unbiased(ora):
+    # Horvitz-Thompson: over all inclusion patterns S of one row, weighted by
+    # P(S) = prod pi (1 - pi), the reweighted sum of exp terms and the reweighted
+    # numerator equal the dense ones exactly (up to rounding) -- "one pass is an
+    # unbiased estimate of dense attention".
+    rng = np.random.default_rng(13)
+    S, D = 22, 8
+    L = lay(seq_len=S, seq_pad=24, D=D, bq=4, bk=4, heads=1)
+    q = bits(rng.standard_normal((1, 1, 24, D)))
+    k = bits(rng.standard_normal((1, 1, 24, D)))
+    v = bits(rng.standard_normal((1, 1, 24, D)))
+    Cq, Ck = 6, 6
+    P = _tiny_probs(rng, 1, 1, Cq, Ck)
+    pi, w = ora.inclusion(L, P, 2.0, 1)       # text keep off (text_len 0), a mix of caps
+    dense_o, dense_l = ora.attention(L, q, k, v, None, 0.3)
+    for i in (0, 3, 5):
+        z_sum = np.zeros(4)
+        n_sum = np.zeros((4, D))
+        for bits_s in range(1 << Ck):
+            sel = np.array([(bits_s >> j) & 1 for j in range(Ck)], np.uint8)
+            prob = np.prod(np.where(sel == 1, pi[0, 0, i].astype(np.float64),
+                                    1 - pi[0, 0, i].astype(np.float64)))
+            if prob == 0 or not sel.any():
+                continue
+            m = np.zeros((1, 1, Cq, Ck), np.uint8)
+            m[0, 0, i] = sel
+            o, l = ora.attention(L, q, k, v, m, 0.3, rows=[i], weight=w)
+            ok = np.isfinite(dense_l[i])                  # padded query rows: -inf on both sides
+            rel = np.zeros(4)
+            rel[ok] = np.exp(l[0][ok].astype(np.float64) - dense_l[i][ok].astype(np.float64))
+            z_sum += prob * rel
+            n_sum += prob * rel[:, None] * o[0].astype(np.float64)
+        valid = np.arange(4) + 4 * i < S
+        np.testing.assert_allclose(z_sum[valid], 1.0, rtol=2e-6)
+        np.testing.assert_allclose(n_sum[valid], dense_o[i][valid].astype(np.float64), rtol=2e-5,
+                                   atol=2e-6)
+
+
+def check_sampled_degenerate(ora):
+    rng = np.random.default_rng(14)
+    L = lay(seq_len=22, seq_pad=24, D=8, bq=4, bk=4, heads=1, text_len=4, tpf=8, frames=2)
+    q = bits(rng.standard_normal((1, 1, 24, 8)))
+    k = bits(rng.standard_normal((1, 1, 24, 8)))
+    v = bits(rng.standard_normal((1, 1, 24, 8)))
+    P = _tiny_probs(rng, 1, 1, 6, 6)
+    # a budget above 1 / min P' includes every pair with weight 1: the dense result
+    m, wt = ora.sample_select(L, P, 1e9, 3, 0)
+    assert m.all() and (wt == 1).all()
+    o, l = ora.attention(L, q, k, v, m, 0.3, weight=wt)
+    od, ld = ora.attention(L, q, k, v, None, 0.3)
+    np.testing.assert_array_equal(o, od)
+    # budget 0: only the overrides (text column 0, frame-0 blocks 1..2), each with weight 1
+    m, wt = ora.sample_select(L, P, 0.0, 3, 3)
+    exp = ora.overrides(L, 3, np.zeros_like(m))
+    assert np.array_equal(m, exp) and (wt[m == 1] == 1).all()
+    m, wt = ora.sample_select(L, P, 0.0, 3, 0)
+    assert not m.any()
+    o, l = ora.attention(L, q, k, v, m, 0.3, weight=wt)
+    assert (o == 0).all() and np.isneginf(l).all()
+    # weights of one: the mask-only result
+    m = (rng.random((1, 1, 6, 6)) < 0.5).astype(np.uint8)
+    m[..., 0] = 1
+    o1, _ = ora.attention(L, q, k, v, m, 0.3, weight=np.ones(m.shape, np.float32))
+    o2, _ = ora.attention(L, q, k, v, m, 0.3)
+    np.testing.assert_array_equal(o1, o2)
+
+
+def test_splitmix64(ora):
+    check_splitmix64(ora)
+
+
+def test_inclusion_law(ora):
+    check_inclusion_law(ora)
+
+
+def test_sample_frequencies(ora):
+    check_sample_frequencies(ora)
+
+
+def test_sampled_attention_unbiased(ora):
+    check_sampled_attention_unbiased(ora)
+
+
+def test_sampled_degenerate(ora):
+    check_sampled_degenerate(ora)
+
+
 def test_eg_value_norms(ora):
     check_value_norms(ora)
 
@@ -528,4 +689,6 @@ def test_eg_select(ora):
 
 ALL_CHECKS = [check_geometry, check_pooling, check_scores, check_entropy, check_topp,
               check_overrides_lists, check_attention, check_pipeline, check_value_norms,
-              check_eg_route, check_eg_select]
+              check_eg_route, check_eg_select, check_splitmix64, check_inclusion_law,
+              check_sample_frequencies, check_sampled_attention_unbiased,
+              check_sampled_degenerate]
