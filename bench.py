@@ -50,9 +50,14 @@ def parse():
                     help="heads per group of the pipelined host-buffer call timed as e2e")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
-    ap.add_argument("--selection", default="top_p", choices=["top_p", "eg"],
-                    help="per-row top-p (bsa_build_mask) or entropy-guided grouped selection "
-                         "(bsa_value_norms + bsa_build_mask_eg) inside the step")
+    ap.add_argument("--selection", default="top_p", choices=["top_p", "eg", "sampled"],
+                    help="per-row top-p (bsa_build_mask), entropy-guided grouped selection "
+                         "(bsa_value_norms + bsa_build_mask_eg), or importance sampling with "
+                         "inverse-probability weights (bsa_build_mask_sampled + "
+                         "bsa_attention_fwd_weighted) inside the step")
+    ap.add_argument("--budget", type=float, default=None,
+                    help="per-row budget K of the sampler (default: calibrated so the expected "
+                         "density matches the per-row top-p selection)")
     ap.add_argument("--pool-p", type=float, default=None,
                     help="threshold of the low-entropy pool (default: the mean per-head top-p)")
     return ap.parse_args()
@@ -251,6 +256,10 @@ def our_arm(args, w):
     low = torch.empty((B, H), dtype=torch.uint8, device=dev)
     ws_eg = torch.empty(bsa.eg_workspace_bytes(w), dtype=torch.uint8, device=dev)
 
+    sampled = args.selection == "sampled"
+    kv_weight = torch.empty((B, H, Cq, Ck), **f32)
+    budget = args.budget
+
     def select_eg():
         bsa.value_norms(w, v, vnorm, stream=stream)
         bsa.build_mask_eg(w, probs, vnorm, top_p, pool_p, w.flags, 1e-8, mask, kv_index, kv_count,
@@ -269,19 +278,42 @@ def our_arm(args, w):
             marks[1].record(stream)
         if eg:
             select_eg()
+        elif sampled:
+            step.seed += 1
+            bsa.build_mask_sampled(w, probs, budget, step.seed, w.flags, mask, kv_index, kv_weight,
+                                   kv_count, stream=stream)
         else:
             bsa.build_mask(w, probs, top_p, w.flags, 1e-8, mask, kv_index, kv_count, ent, ent_n,
                            ws, stream=stream)
         if marks is not None:
             marks[2].record(stream)
-        bsa.attention_fwd(w, qq, kk, vv, kv_index, kv_count, None, out, lse, err, stream=stream)
+        if sampled:
+            bsa.attention_fwd_weighted(w, qq, kk, vv, kv_index, kv_weight, kv_count, None, out, lse,
+                                       err, stream=stream)
+        else:
+            bsa.attention_fwd(w, qq, kk, vv, kv_index, kv_count, None, out, lse, err, stream=stream)
         if marks is not None:
             marks[3].record(stream)
+    step.seed = 0
+
+    if sampled and budget is None:
+        # expected density of the sampler = mean of min(1, K P') (overrides aside), matched to
+        # the per-row top-p selection of the same P' by bisection (setup, not timed)
+        bsa.block_scores(w, q, k, qc, kc, probs, stream=stream)
+        bsa.build_mask(w, probs, top_p, w.flags, 1e-8, mask, kv_index, kv_count, ent, ent_n, ws,
+                       stream=stream)
+        target = float(kv_count.sum().item()) / float(B * H * Cq * Ck)
+        lo, hi = 0.0, float(Ck)
+        for _ in range(50):
+            mid = 0.5 * (lo + hi)
+            d = float(torch.clamp(probs * mid, max=1.0).mean().item())
+            lo, hi = (mid, hi) if d < target else (lo, mid)
+        budget = 0.5 * (lo + hi)
 
     # pool, score, mask, entropy reduce, attention; the entropy-guided selection runs
-    # value norms, row entropy, entropy reduce, route, 3 x (pool histogram, pick), tie count,
-    # tie scan and the mask kernel in place of mask + entropy reduce
-    launches_per_step = 15 if eg else 5
+    # value norms, entropy + level 1, two pool levels, the tie pass and the mask kernel in
+    # place of mask + entropy reduce; the sampler one kernel
+    launches_per_step = 9 if eg else (4 if sampled else 5)
     for _ in range(max(3, args.warmup)):
         step(q, k, v)
     torch.cuda.synchronize(dev)
@@ -320,7 +352,7 @@ def our_arm(args, w):
     # Q, K, V in and O (+ entropy) out per head group on two copy streams, overlapped
     # with the kernels of the neighbouring groups
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not eg and not sampled:   # the host-buffer call runs per-row top-p
         pin = {n: host[n].pin_memory() for n in ("q", "k", "v")}
         out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         ent_h = torch.empty((B, H), dtype=torch.float32).pin_memory()
@@ -417,7 +449,9 @@ def our_arm(args, w):
         config=dict(workload=w.name, batch=B, heads=H, seq_len=w.seq_len, seq_pad=Sp, head_dim=D,
                     q_block=w.q_block, k_block=w.k_block, text_len=w.text_len,
                     frames=w.num_frames, latent=[w.latent_h, w.latent_w],
-                    selection="entropy-guided grouped (pool_p %.4g)" % pool_p if eg
+                    selection=("entropy-guided grouped (pool_p %.4g)" % pool_p) if eg
+                              else ("importance-sampled, inverse-probability weights (budget K "
+                                    "%.4g per row, a new seed per step)" % budget) if sampled
                               else "per-row top-p",
                     density=density, skipped=1 - density, selected_pairs=pairs,
                     computed_tflop_per_step=step_flops / 1e12,

@@ -81,6 +81,12 @@ def load():
         L.bsa_build_mask_eg.argtypes = [lp, vp, vp, vp, ctypes.c_float, ctypes.c_uint32,
                                         ctypes.c_float, vp, vp, vp, vp, vp, vp, vp, vp]
         L.bsa_build_mask_eg.restype = ctypes.c_int
+        L.bsa_build_mask_sampled.argtypes = [lp, vp, ctypes.c_float, ctypes.c_uint64, ctypes.c_uint32,
+                                             vp, vp, vp, vp, vp]
+        L.bsa_build_mask_sampled.restype = ctypes.c_int
+        L.bsa_attention_fwd_weighted.argtypes = [lp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp,
+                                                 vp, vp, vp]
+        L.bsa_attention_fwd_weighted.restype = ctypes.c_int
         L.bsa_build_mask_eg_workspace_bytes.argtypes = [lp]
         L.bsa_build_mask_eg_workspace_bytes.restype = ctypes.c_size_t
         L.bsa_status_string.argtypes = [ctypes.c_int]
@@ -296,6 +302,61 @@ def attention_fwd(layout, q, k, v, kv_index, kv_count, softmax_scale=None, out=N
                                   _ptr(kv_count), float(softmax_scale), _ptr(out), _ptr(lse),
                                   _ptr(err_flag), _ptr(workspace), _stream(stream))
     _check("bsa_attention_fwd", rc)
+    return out, lse
+
+
+def build_mask_sampled(layout, probs, budget, seed, flags, mask=None, kv_index=None,
+                       kv_weight=None, kv_count=None, with_mask=True, stream=None):
+    """bsa_build_mask_sampled (importance sampling with inverse-inclusion-probability
+    weights): returns dict(mask, kv_index, kv_weight, kv_count)."""
+    L = make_layout(layout)
+    d = dims(L)
+    _need(probs, "probs", torch.float32, (d["B"], d["H"], d["Cq"], d["Ck"]))
+    dev = probs.device
+    shp = (d["B"], d["H"], d["Cq"], d["Ck"])
+    if mask is None and with_mask:
+        mask = torch.empty(shp, dtype=torch.uint8, device=dev)
+    if kv_index is None:
+        kv_index = torch.empty(shp, dtype=torch.int32, device=dev)
+    if kv_weight is None:
+        kv_weight = torch.empty(shp, dtype=torch.float32, device=dev)
+    if kv_count is None:
+        kv_count = torch.empty((d["B"], d["H"], d["Cq"]), dtype=torch.int32, device=dev)
+    _need(kv_index, "kv_index", torch.int32, shp)
+    _need(kv_weight, "kv_weight", torch.float32, shp)
+    _need(kv_count, "kv_count", torch.int32, (d["B"], d["H"], d["Cq"]))
+    rc = load().bsa_build_mask_sampled(ctypes.byref(L), _ptr(probs), float(budget),
+                                       int(seed) & (2**64 - 1), int(flags), _ptr(mask),
+                                       _ptr(kv_index), _ptr(kv_weight), _ptr(kv_count),
+                                       _stream(stream))
+    _check("bsa_build_mask_sampled", rc)
+    return dict(mask=mask, kv_index=kv_index, kv_weight=kv_weight, kv_count=kv_count)
+
+
+def attention_fwd_weighted(layout, q, k, v, kv_index, kv_weight, kv_count, softmax_scale=None,
+                           out=None, lse=None, err_flag=None, with_lse=True, workspace=None,
+                           stream=None):
+    """bsa_attention_fwd_weighted: returns (out, lse)."""
+    L = make_layout(layout)
+    d = dims(L)
+    qkv = (d["B"], d["H"], d["Sp"], d["D"])
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, qkv)
+    _need(kv_index, "kv_index", torch.int32, (d["B"], d["H"], d["Cq"], d["Ck"]))
+    _need(kv_weight, "kv_weight", torch.float32, (d["B"], d["H"], d["Cq"], d["Ck"]))
+    _need(kv_count, "kv_count", torch.int32, (d["B"], d["H"], d["Cq"]))
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d["D"])
+    if out is None:
+        out = torch.empty(qkv, dtype=torch.bfloat16, device=q.device)
+    if lse is None and with_lse:
+        lse = torch.empty((d["B"], d["H"], d["Sp"]), dtype=torch.float32, device=q.device)
+    workspace = _attn_workspace(L, q.device, workspace)
+    rc = load().bsa_attention_fwd_weighted(ctypes.byref(L), _ptr(q), _ptr(k), _ptr(v),
+                                           _ptr(kv_index), _ptr(kv_weight), _ptr(kv_count),
+                                           float(softmax_scale), _ptr(out), _ptr(lse),
+                                           _ptr(err_flag), _ptr(workspace), _stream(stream))
+    _check("bsa_attention_fwd_weighted", rc)
     return out, lse
 
 

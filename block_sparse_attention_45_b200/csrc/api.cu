@@ -221,8 +221,43 @@ int bsa_attention_fwd(const bsa_layout *layout, const void *q, const void *k, co
     if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return BSA_ERR_INVALID_ARG;
     if (workspace && !aligned(workspace, 16)) return BSA_ERR_INVALID_ARG;
     const Geometry g = bsa::make_geometry(*layout);
-    return bsa::launch_attention(g, q, k, v, kv_index, kv_count, softmax_scale, out, lse, err_flag,
+    return bsa::launch_attention(g, q, k, v, kv_index, nullptr, kv_count, softmax_scale, out, lse, err_flag,
                                  workspace, static_cast<cudaStream_t>(stream));
+}
+
+int bsa_attention_fwd_weighted(const bsa_layout *layout, const void *q, const void *k,
+                               const void *v, const int32_t *kv_index, const float *kv_weight,
+                               const int32_t *kv_count, float softmax_scale, void *out, float *lse,
+                               int32_t *err_flag, void *workspace, void *stream) {
+    int rc = check_layout(layout);
+    if (rc != BSA_OK) return rc;
+    if (!q || !k || !v || !out || !kv_index || !kv_weight || !kv_count) return BSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+        return BSA_ERR_INVALID_ARG;
+    if (!aligned(kv_index, 4) || !aligned(kv_weight, 4) || !aligned(kv_count, 4) ||
+        (lse && !aligned(lse, 4)) || (err_flag && !aligned(err_flag, 4)))
+        return BSA_ERR_INVALID_ARG;
+    if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return BSA_ERR_INVALID_ARG;
+    if (workspace && !aligned(workspace, 16)) return BSA_ERR_INVALID_ARG;
+    const Geometry g = bsa::make_geometry(*layout);
+    return bsa::launch_attention(g, q, k, v, kv_index, kv_weight, kv_count, softmax_scale, out, lse,
+                                 err_flag, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int bsa_build_mask_sampled(const bsa_layout *layout, const float *probs, float budget,
+                           uint64_t seed, uint32_t flags, uint8_t *mask, int32_t *kv_index,
+                           float *kv_weight, int32_t *kv_count, void *stream) {
+    int rc = check_layout(layout);
+    if (rc != BSA_OK) return rc;
+    if (!probs || !kv_index || !kv_weight || !kv_count) return BSA_ERR_INVALID_ARG;
+    if (flags & ~static_cast<uint32_t>(BSA_TEXT_KEEP | BSA_FRAME0_DENSE)) return BSA_ERR_INVALID_ARG;
+    if (!aligned(probs, 4) || !aligned(kv_index, 4) || !aligned(kv_weight, 4) || !aligned(kv_count, 4))
+        return BSA_ERR_INVALID_ARG;
+    if (!(budget >= 0.f) || !isfinite(budget)) return BSA_ERR_INVALID_ARG;
+    const Geometry g = bsa::make_geometry(*layout);
+    if (g.Ck > bsa::kMaxMaskCk) return BSA_ERR_UNSUPPORTED;
+    return launch_status(bsa::launch_sample(g, probs, budget, seed, flags, mask, kv_index, kv_weight,
+                                            kv_count, static_cast<cudaStream_t>(stream)));
 }
 
 int bsa_dense_fwd(const bsa_layout *layout, const void *q, const void *k, const void *v,
@@ -237,7 +272,7 @@ int bsa_dense_fwd(const bsa_layout *layout, const void *q, const void *k, const 
     if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return BSA_ERR_INVALID_ARG;
     if (workspace && !aligned(workspace, 16)) return BSA_ERR_INVALID_ARG;
     const Geometry g = bsa::make_geometry(*layout);
-    return bsa::launch_attention(g, q, k, v, nullptr, nullptr, softmax_scale, out, lse, err_flag,
+    return bsa::launch_attention(g, q, k, v, nullptr, nullptr, nullptr, softmax_scale, out, lse, err_flag,
                                  workspace, static_cast<cudaStream_t>(stream));
 }
 

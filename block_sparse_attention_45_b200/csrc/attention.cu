@@ -93,6 +93,7 @@ struct Cfg {
 
 struct AttnParams {
     const int32_t *kv_index;  // nullptr: dense (every key block)
+    const float *kv_weight;   // with W: the weight of every list entry (exp terms scaled by it)
     const int32_t *kv_count;
     __nv_bfloat16 *out;
     float *lse;
@@ -160,7 +161,7 @@ __device__ __forceinline__ void tile_block(const AttnParams &p, const int32_t *e
     if (valid) valid = min(BK, p.S - j * BK);
 }
 
-template <int D, int BK>
+template <int D, int BK, bool W>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
@@ -431,25 +432,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             int n_entries, n_tiles;
             bool bad_count;
             item_lists<BK>(p, item, entries, n_entries, n_tiles, bad_count);
+            const float *weights = (W && entries) ? p.kv_weight + item * p.Ck : nullptr;
             const int n_s = (n_tiles > s) ? (n_tiles - s + 1) / 2 : 0;
             float m_run = -INFINITY, l_run = 0.f;
-            // The list entries of this stream's next tile are read one tile ahead
-            // (raw block indices; -1 = no block) so their latency is hidden.
+            // The list entries (and weights) of this stream's next tile are read one
+            // tile ahead (raw block indices; -1 = no block) so their latency is hidden.
             int j_next0 = -1, j_next1 = -1;
+            float w_next0 = 1.f, w_next1 = 1.f;
             if (n_s > 0) {
                 const int e0 = (BK == 128) ? s : 2 * s;
                 j_next0 = entries ? __ldg(entries + e0) : e0;
-                if (BK != 128 && e0 + 1 < n_entries) j_next1 = entries ? __ldg(entries + e0 + 1) : e0 + 1;
+                if (W && weights) w_next0 = __ldg(weights + e0);
+                if (BK != 128 && e0 + 1 < n_entries) {
+                    j_next1 = entries ? __ldg(entries + e0 + 1) : e0 + 1;
+                    if (W && weights) w_next1 = __ldg(weights + e0 + 1);
+                }
             }
             for (int it = 0; ok && it < n_s; ++it) {
                 const int t = 2 * it + s;
                 const int j0 = j_next0, j1 = j_next1;
+                const float w0 = w_next0, w1 = w_next1;
                 if (t + 2 < n_tiles) {
                     const int e0 = (BK == 128) ? t + 2 : 2 * (t + 2);
                     j_next0 = entries ? __ldg(entries + e0) : e0;
+                    if (W && weights) w_next0 = __ldg(weights + e0);
                     j_next1 = -1;
-                    if (BK != 128 && e0 + 1 < n_entries)
+                    w_next1 = 1.f;
+                    if (BK != 128 && e0 + 1 < n_entries) {
                         j_next1 = entries ? __ldg(entries + e0 + 1) : e0 + 1;
+                        if (W && weights) w_next1 = __ldg(weights + e0 + 1);
+                    }
                 }
                 // tcgen05.ld/st below are warp-collective: leave together or not at all.
                 if (!__all_sync(0xffffffffu, mbar_wait(&hd.s_full[s], sc & 1, abort_flag))) {
@@ -505,14 +517,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
                 const float sl = p.scale_log2;
+                // Reweighting: w * 2^(s*sl - m) = 2^(s*sl - m + log2 w), one offset per half.
+                float nmh0 = nm, nmh1 = nm;
+                if (W) {
+                    nmh0 = nm + __log2f(w0);
+                    nmh1 = (kHalves > 1) ? nm + __log2f(w1) : nmh0;
+                }
                 float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t pk[16];
+                    const float off = (W && kHalves > 1 && c >= 2) ? nmh1 : nmh0;
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         float t0, t1, p0, p1;
-                        fma2(t0, t1, X(c * 32 + 2 * e), X(c * 32 + 2 * e + 1), sl, sl, nm, nm);
+                        fma2(t0, t1, X(c * 32 + 2 * e), X(c * 32 + 2 * e + 1), sl, sl, off, off);
                         p0 = ex2(t0);
                         p1 = ex2(t1);
                         pk[e] = pack_bf16x2(p0, p1);
@@ -637,15 +656,17 @@ bool make_map(CUtensorMap *m, const void *base, const Geometry &g, int box_rows)
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int BK>
+template <int D, int BK, bool W>
 int launch_t(const Geometry &g, const void *q, const void *k, const void *v,
-             const int32_t *kv_index, const int32_t *kv_count, float softmax_scale, void *out,
-             float *lse, int32_t *err, void *workspace, cudaStream_t st) {
+             const int32_t *kv_index, const float *kv_weight, const int32_t *kv_count,
+             float softmax_scale, void *out, float *lse, int32_t *err, void *workspace,
+             cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, q, g, g.bq) || !make_map(&mk, k, g, BK) || !make_map(&mv, v, g, BK))
         return BSA_ERR_DRIVER;
     AttnParams p;
     p.kv_index = kv_index;
+    p.kv_weight = kv_weight;
     p.kv_count = kv_count;
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.lse = lse;
@@ -659,7 +680,7 @@ int launch_t(const Geometry &g, const void *q, const void *k, const void *v,
     p.bq = g.bq;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
     const int smem = Cfg<D>::kSmemAlloc;
-    if (cudaFuncSetAttribute(attn_kernel<D, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(attn_kernel<D, BK, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
         return BSA_ERR_LAUNCH;
     const int sms = sm_count();
@@ -667,25 +688,38 @@ int launch_t(const Geometry &g, const void *q, const void *k, const void *v,
     const long long grid = p.n_items < sms ? p.n_items : sms;
     if (workspace && cudaMemsetAsync(workspace, 0, sizeof(int), st) != cudaSuccess)
         return BSA_ERR_LAUNCH;
-    attn_kernel<D, BK><<<static_cast<unsigned>(grid), kThreads, smem, st>>>(mq, mk, mv, p);
+    attn_kernel<D, BK, W><<<static_cast<unsigned>(grid), kThreads, smem, st>>>(mq, mk, mv, p);
     return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_LAUNCH;
 }
 
 }  // namespace
 
-int launch_attention(const Geometry &g, const void *q, const void *k, const void *v,
-                     const int32_t *kv_index, const int32_t *kv_count, float softmax_scale,
-                     void *out, float *lse, int32_t *err_flag, void *workspace, cudaStream_t st) {
+template <bool W>
+int launch_attention_w(const Geometry &g, const void *q, const void *k, const void *v,
+                       const int32_t *kv_index, const float *kv_weight, const int32_t *kv_count,
+                       float softmax_scale, void *out, float *lse, int32_t *err_flag,
+                       void *workspace, cudaStream_t st) {
     if (g.D == 128) {
-        return g.bk == 128 ? launch_t<128, 128>(g, q, k, v, kv_index, kv_count, softmax_scale, out,
-                                                lse, err_flag, workspace, st)
-                           : launch_t<128, 64>(g, q, k, v, kv_index, kv_count, softmax_scale, out,
-                                               lse, err_flag, workspace, st);
+        return g.bk == 128 ? launch_t<128, 128, W>(g, q, k, v, kv_index, kv_weight, kv_count,
+                                                   softmax_scale, out, lse, err_flag, workspace, st)
+                           : launch_t<128, 64, W>(g, q, k, v, kv_index, kv_weight, kv_count,
+                                                  softmax_scale, out, lse, err_flag, workspace, st);
     }
-    return g.bk == 128 ? launch_t<64, 128>(g, q, k, v, kv_index, kv_count, softmax_scale, out, lse,
-                                           err_flag, workspace, st)
-                       : launch_t<64, 64>(g, q, k, v, kv_index, kv_count, softmax_scale, out, lse,
-                                          err_flag, workspace, st);
+    return g.bk == 128 ? launch_t<64, 128, W>(g, q, k, v, kv_index, kv_weight, kv_count,
+                                              softmax_scale, out, lse, err_flag, workspace, st)
+                       : launch_t<64, 64, W>(g, q, k, v, kv_index, kv_weight, kv_count,
+                                             softmax_scale, out, lse, err_flag, workspace, st);
+}
+
+int launch_attention(const Geometry &g, const void *q, const void *k, const void *v,
+                     const int32_t *kv_index, const float *kv_weight, const int32_t *kv_count,
+                     float softmax_scale, void *out, float *lse, int32_t *err_flag,
+                     void *workspace, cudaStream_t st) {
+    if (kv_weight)
+        return launch_attention_w<true>(g, q, k, v, kv_index, kv_weight, kv_count, softmax_scale,
+                                        out, lse, err_flag, workspace, st);
+    return launch_attention_w<false>(g, q, k, v, kv_index, nullptr, kv_count, softmax_scale, out,
+                                     lse, err_flag, workspace, st);
 }
 
 }  // namespace bsa

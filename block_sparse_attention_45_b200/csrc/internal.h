@@ -94,9 +94,16 @@ cudaError_t launch_mask_eg(const Geometry &g, const float *probs, const float *v
                            cudaStream_t st);
 
 // Returns BSA_* status.
+// kv_weight (optional, with kv_index): every exp term of list entry e is scaled by kv_weight[e].
 int launch_attention(const Geometry &g, const void *q, const void *k, const void *v,
-                     const int32_t *kv_index, const int32_t *kv_count, float softmax_scale,
-                     void *out, float *lse, int32_t *err_flag, void *workspace, cudaStream_t st);
+                     const int32_t *kv_index, const float *kv_weight, const int32_t *kv_count,
+                     float softmax_scale, void *out, float *lse, int32_t *err_flag,
+                     void *workspace, cudaStream_t st);
+
+// Importance sampling of key blocks with inverse-inclusion-probability weights.
+cudaError_t launch_sample(const Geometry &g, const float *probs, float budget, uint64_t seed,
+                          uint32_t flags, uint8_t *mask, int32_t *kv_index, float *kv_weight,
+                          int32_t *kv_count, cudaStream_t st);
 
 constexpr size_t kAttnWorkspaceBytes = 256;
 

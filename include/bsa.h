@@ -220,6 +220,35 @@ int bsa_build_mask_eg(const bsa_layout *layout, const float *probs, const float 
 size_t bsa_build_mask_eg_workspace_bytes(const bsa_layout *layout);
 
 /*
+ * Importance sampling of key blocks ("AB-Attention: accurate block-sparse
+ * attention for video diffusion", TL;DR fix (2): blocks are sampled in
+ * proportion to importance and reweighted by the inverse inclusion
+ * probability, so that one pass is an unbiased estimate of dense attention).
+ * The page gives no sampling law; this one is used: every pair (b, h, i, j)
+ * is included independently with probability pi = min(1, fp32(budget * P'))
+ * (negative or NaN P' as 0; a row keeps at most `budget` blocks in
+ * expectation since its P' sums to one).  The draw of pair
+ * idx = ((b*H + h)*C_q + i)*C_k + j is u = (z >> 40) * 2^-24, z the idx-th
+ * output (from 0) of SplitMix64 started from state `seed`; the pair is
+ * included iff u < pi, and then carries the weight w = 1/pi (fp32, correctly
+ * rounded).  With BSA_TEXT_KEEP / BSA_FRAME0_DENSE the text key columns /
+ * frame-0 query blocks are included with pi = 1, w = 1.  Same seed, same
+ * draw, on any device.
+ *
+ * probs      fp32 [B,H,C_q,C_k] (read)
+ * budget     finite, >= 0 (else BSA_ERR_INVALID_ARG)
+ * mask       u8 [B,H,C_q,C_k] (written) or NULL
+ * kv_index   int32 [B,H,C_q,C_k]: included key blocks ascending in the first
+ *            kv_count entries (written)
+ * kv_weight  fp32 [B,H,C_q,C_k]: w of kv_index's entries, same positions (written)
+ * kv_count   int32 [B,H,C_q] (written)
+ * C_k above 2048: BSA_ERR_UNSUPPORTED.
+ */
+int bsa_build_mask_sampled(const bsa_layout *layout, const float *probs, float budget,
+                           uint64_t seed, uint32_t flags, uint8_t *mask, int32_t *kv_index,
+                           float *kv_weight, int32_t *kv_count, void *stream);
+
+/*
  * Block-sparse exact attention ("Attention matrix view ..." s2;
  * "AB-Attention ..." TL;DR).  For every valid query token t of query block i:
  *   U = tokens u < seq_len of the key blocks kv_index[b,h,i,0..kv_count-1]
@@ -250,6 +279,23 @@ size_t bsa_build_mask_eg_workspace_bytes(const bsa_layout *layout);
 int bsa_attention_fwd(const bsa_layout *layout, const void *q, const void *k, const void *v,
                       const int32_t *kv_index, const int32_t *kv_count, float softmax_scale,
                       void *out, float *lse, int32_t *err_flag, void *workspace, void *stream);
+
+/*
+ * bsa_attention_fwd with inverse-inclusion-probability weights
+ * ("AB-Attention ..." TL;DR fix (2)): every exp term of a key of list entry e
+ * is multiplied by kv_weight[b,h,i,e], in the numerator and in the sum alike:
+ *   O_t = sum_u w_u exp(s_u) V_u / sum_u w_u exp(s_u),
+ *   lse_t = ln sum_u w_u exp(s_u),  s_u = softmax_scale * Q_t . K_u,
+ * which with the weights of bsa_build_mask_sampled makes the numerator and the
+ * sum unbiased estimates of the dense ones.  Weights must be positive and
+ * finite.  Everything else as for bsa_attention_fwd.
+ *
+ * kv_weight  fp32 [B,H,C_q,C_k], entry e beside kv_index's entry e (read only)
+ */
+int bsa_attention_fwd_weighted(const bsa_layout *layout, const void *q, const void *k,
+                               const void *v, const int32_t *kv_index, const float *kv_weight,
+                               const int32_t *kv_count, float softmax_scale, void *out, float *lse,
+                               int32_t *err_flag, void *workspace, void *stream);
 
 /* Bytes of device workspace bsa_attention_fwd / bsa_dense_fwd can use. */
 size_t bsa_attention_workspace_bytes(const bsa_layout *layout);

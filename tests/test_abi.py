@@ -156,13 +156,44 @@ def test_eg_entry_points_validate_before_any_cuda_call():
     assert lib.bsa_value_norms(r, None, FAKE, None) == bsa.BSA_ERR_INVALID_ARG
     assert lib.bsa_value_norms(r, MISALIGNED, FAKE, None) == bsa.BSA_ERR_INVALID_ARG
     assert lib.bsa_value_norms(ctypes.byref(bad), FAKE, FAKE, None) == bsa.BSA_ERR_UNSUPPORTED
-    # workspace: row entropies + per-row tie counts + per-head values + one pool state and
+    # workspace: per-row tie counts + a 256-bin level-1 histogram per head + one pool state and
     # 4096-bin histogram per batch entry
     assert lib.bsa_build_mask_eg_workspace_bytes(ctypes.byref(bad)) == 0
     w = synth.WORKLOADS["hunyuan"]
     n = lib.bsa_build_mask_eg_workspace_bytes(ctypes.byref(bsa.make_layout(w)))
     rows = w.heads * (w.seq_pad // w.q_block)
-    assert n >= rows * 8 + 4096 * 16 and n % 256 == 0
+    assert n >= rows * 4 + w.heads * 256 * 16 + 4096 * 16 and n % 256 == 0
+
+
+def test_sampling_entry_points_validate_before_any_cuda_call():
+    lib = bsa.load()
+    L = _layout()
+    r = ctypes.byref(L)
+
+    def smp(probs=FAKE, budget=4.0, flags=3, idx=FAKE, wt=FAKE, cnt=FAKE):
+        return lib.bsa_build_mask_sampled(r, probs, budget, 7, flags, None, idx, wt, cnt, None)
+    assert smp(probs=None) == bsa.BSA_ERR_INVALID_ARG
+    assert smp(idx=None) == bsa.BSA_ERR_INVALID_ARG
+    assert smp(wt=None) == bsa.BSA_ERR_INVALID_ARG
+    assert smp(cnt=None) == bsa.BSA_ERR_INVALID_ARG
+    assert smp(wt=MISALIGNED) == bsa.BSA_ERR_INVALID_ARG
+    assert smp(flags=8) == bsa.BSA_ERR_INVALID_ARG
+    assert smp(budget=-1.0) == bsa.BSA_ERR_INVALID_ARG
+    assert smp(budget=float("nan")) == bsa.BSA_ERR_INVALID_ARG
+    assert smp(budget=float("inf")) == bsa.BSA_ERR_INVALID_ARG
+    bad = _layout(head_dim=96)
+    assert lib.bsa_build_mask_sampled(ctypes.byref(bad), FAKE, 4.0, 7, 0, None, FAKE, FAKE, FAKE,
+                                      None) == bsa.BSA_ERR_UNSUPPORTED
+
+    def wat(q=FAKE, idx=FAKE, wt=FAKE, cnt=FAKE, scale=0.125, out=FAKE):
+        return lib.bsa_attention_fwd_weighted(r, q, FAKE, FAKE, idx, wt, cnt, scale, out, None, None,
+                                              None, None)
+    assert wat(q=None) == bsa.BSA_ERR_INVALID_ARG
+    assert wat(wt=None) == bsa.BSA_ERR_INVALID_ARG
+    assert wat(idx=None) == bsa.BSA_ERR_INVALID_ARG
+    assert wat(wt=MISALIGNED) == bsa.BSA_ERR_INVALID_ARG
+    assert wat(scale=0.0) == bsa.BSA_ERR_INVALID_ARG
+    assert wat(out=MISALIGNED) == bsa.BSA_ERR_INVALID_ARG
 
 
 def test_calls_fail_loudly_without_the_library(monkeypatch):
