@@ -72,6 +72,8 @@ class Oracle:
         L.ora_inclusion.argtypes = [lp, vp, ctypes.c_float, ctypes.c_uint32, vp, vp]
         L.ora_sample_select.argtypes = [lp, vp, ctypes.c_float, ctypes.c_uint64, ctypes.c_uint32,
                                         vp, vp]
+        L.ora_subclusters.argtypes = [lp, vp, ctypes.c_int, ctypes.c_int, vp, vp]
+        L.ora_scores_clustered.argtypes = [lp, vp, vp, ctypes.c_int, vp, vp]
         L.ora_num_threads.restype = ctypes.c_int
         self.lib = L
 
@@ -106,6 +108,29 @@ class Oracle:
         kc = np.ascontiguousarray(kc, np.float32)
         out = np.empty((L.batch, L.heads, L.cq, L.ck), np.float32)
         self.lib.ora_scores(ctypes.byref(L), _ptr(qc), _ptr(kc), _ptr(out))
+        return out
+
+    def subclusters(self, L, q, nsub, iters):
+        """k-means sub-clusters of every query block: centroids fp32 [B,H,C_q,nsub,D] and
+        sizes int32 [B,H,C_q,nsub]."""
+        L = _layout(L)
+        q = _u16(q)
+        cent = np.empty((L.batch, L.heads, L.cq, nsub, L.head_dim), np.float32)
+        size = np.empty((L.batch, L.heads, L.cq, nsub), np.int32)
+        self.lib.ora_subclusters(ctypes.byref(L), _ptr(q), int(nsub), int(iters), _ptr(cent),
+                                 _ptr(size))
+        return cent, size
+
+    def scores_clustered(self, L, cent, size, kc):
+        """Block scores as the size-weighted mixture of the sub-centroid rows, fp32
+        [B,H,C_q,C_k]."""
+        L = _layout(L)
+        cent = np.ascontiguousarray(cent, np.float32)
+        size = np.ascontiguousarray(size, np.int32)
+        kc = np.ascontiguousarray(kc, np.float32)
+        out = np.empty((L.batch, L.heads, L.cq, L.ck), np.float32)
+        self.lib.ora_scores_clustered(ctypes.byref(L), _ptr(cent), _ptr(size), int(cent.shape[3]),
+                                      _ptr(kc), _ptr(out))
         return out
 
     def entropy(self, L, probs, eps=1e-8):

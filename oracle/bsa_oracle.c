@@ -27,7 +27,9 @@
  *       TL;DR: exact attention computed only on the selected K/V blocks;
  *       fix (2): blocks sampled in proportion to importance and reweighted
  *       by the inverse inclusion probability (an unbiased one-pass estimate
- *       of dense attention).
+ *       of dense attention); fix (1): the Intra-Block Clustering Selector
+ *       clusters queries only within each query block (no token permutation)
+ *       so the block importance estimate is faithful.
  *
  * Readings taken where the pages are silent or garbled (the equations of
  * [p3] are lost in the extracted text):
@@ -574,6 +576,131 @@ void ora_sample_select(const ora_layout *L, const float *probs, float budget, ui
     }
     free(pi);
     free(w);
+}
+
+/*
+ * ---------------------------------------------------------------------------
+ * Intra-block query clustering ([p5] TL;DR fix (1)).  The page names the idea
+ * (cluster the queries of each query block among themselves, tokens stay in
+ * place) but no procedure; the readings taken:
+ *  - k-means (Lloyd's iterations) on the block's valid query tokens, k = nsub
+ *    clusters, seeded with the tokens at positions floor(c * n / nsub),
+ *    c = 0 .. nsub-1 (n = valid tokens of the block); squared Euclidean
+ *    distance, ties to the lower cluster index; `iters` >= 1 rounds of
+ *    (assign every token, move every non-empty cluster to the mean of its
+ *    tokens); an empty cluster keeps its centroid and has size 0;
+ *  - the block's score row is the size-weighted mixture of its
+ *    sub-centroids' cluster-size-weighted softmax rows ([p3] Eq. 1 with the
+ *    sub-centroid in place of q_i):
+ *      P'_ij = sum_c (n_c / n_i) n_j exp(s_cj) / sum_j' n_j' exp(s_cj'),
+ *    s_cj = q_c . k_j / sqrt(D); rows still sum to one, and nsub = 1 is the
+ *    plain block centroid.
+ * ---------------------------------------------------------------------------
+ */
+
+/* Sub-cluster centroids fp32 [B,H,C_q,nsub,D] and sizes int32 [B,H,C_q,nsub]
+ * of every query block, in fp64 (sums in ascending token / dimension order). */
+void ora_subclusters(const ora_layout *L, const uint16_t *q, int nsub, int iters, float *cent,
+                     int32_t *size)
+{
+    const int D = L->head_dim, bq = L->q_block, Cq = L->seq_pad / bq;
+    const long BH = (long)L->batch * L->heads;
+    #pragma omp parallel
+    {
+        double *x = (double *)malloc(sizeof(double) * (size_t)bq * D);
+        double *c = (double *)malloc(sizeof(double) * (size_t)nsub * D);
+        double *acc = (double *)malloc(sizeof(double) * (size_t)nsub * D);
+        int *cnt = (int *)malloc(sizeof(int) * (size_t)nsub);
+        #pragma omp for schedule(static)
+        for (long r = 0; r < BH * Cq; ++r) {
+            long bh = r / Cq;
+            int i = (int)(r % Cq);
+            int n = ora_block_count(L->seq_len, bq, i);
+            const uint16_t *base = q + (bh * L->seq_pad + (long)i * bq) * D;
+            for (int t = 0; t < n; ++t)
+                for (int d = 0; d < D; ++d) x[(long)t * D + d] = bf16_val(base[(long)t * D + d]);
+            for (int k = 0; k < nsub; ++k) {
+                int t0 = n > 0 ? (int)(((long)k * n) / nsub) : 0;
+                for (int d = 0; d < D; ++d) c[(long)k * D + d] = n > 0 ? x[(long)t0 * D + d] : 0.0;
+                cnt[k] = 0;
+            }
+            for (int it = 0; it < iters; ++it) {
+                for (int k = 0; k < nsub; ++k) {
+                    cnt[k] = 0;
+                    for (int d = 0; d < D; ++d) acc[(long)k * D + d] = 0.0;
+                }
+                for (int t = 0; t < n; ++t) {
+                    int best = 0;
+                    double bd = INFINITY;
+                    for (int k = 0; k < nsub; ++k) {
+                        double dist = 0.0;
+                        for (int d = 0; d < D; ++d) {
+                            double e = x[(long)t * D + d] - c[(long)k * D + d];
+                            dist += e * e;
+                        }
+                        if (dist < bd) { bd = dist; best = k; }
+                    }
+                    cnt[best] += 1;
+                    for (int d = 0; d < D; ++d) acc[(long)best * D + d] += x[(long)t * D + d];
+                }
+                for (int k = 0; k < nsub; ++k)
+                    if (cnt[k] > 0)
+                        for (int d = 0; d < D; ++d) c[(long)k * D + d] = acc[(long)k * D + d] / cnt[k];
+            }
+            for (int k = 0; k < nsub; ++k) {
+                for (int d = 0; d < D; ++d) cent[(r * nsub + k) * D + d] = (float)c[(long)k * D + d];
+                size[r * nsub + k] = cnt[k];
+            }
+        }
+        free(x);
+        free(c);
+        free(acc);
+        free(cnt);
+    }
+}
+
+/* Block scores from sub-clusters: the size-weighted mixture of the
+ * sub-centroid rows, fp64, stored fp32 [B,H,C_q,C_k]. */
+void ora_scores_clustered(const ora_layout *L, const float *cent, const int32_t *size, int nsub,
+                          const float *kc, float *probs)
+{
+    const int D = L->head_dim;
+    const int Cq = L->seq_pad / L->q_block, Ck = L->seq_pad / L->k_block;
+    const long BH = (long)L->batch * L->heads;
+    const double inv_sqrt_d = 1.0 / sqrt((double)L->head_dim);
+    #pragma omp parallel
+    {
+        double *logit = (double *)malloc(sizeof(double) * Ck);
+        double *row = (double *)malloc(sizeof(double) * Ck);
+        #pragma omp for schedule(static)
+        for (long r = 0; r < BH * Cq; ++r) {
+            long bh = r / Cq;
+            long ntot = 0;
+            for (int k = 0; k < nsub; ++k) ntot += size[r * nsub + k];
+            for (int j = 0; j < Ck; ++j) row[j] = 0.0;
+            for (int k = 0; k < nsub; ++k) {
+                int nk = size[r * nsub + k];
+                if (nk <= 0) continue;
+                const float *qk = cent + (r * nsub + k) * D;
+                double m = -INFINITY;
+                for (int j = 0; j < Ck; ++j) {
+                    const float *kj = kc + (bh * Ck + j) * D;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += (double)qk[d] * (double)kj[d];
+                    int nj = ora_block_count(L->seq_len, L->k_block, j);
+                    logit[j] = nj > 0 ? log((double)nj) + dot * inv_sqrt_d : -INFINITY;
+                    if (logit[j] > m) m = logit[j];
+                }
+                double z = 0.0;
+                for (int j = 0; j < Ck; ++j) z += exp(logit[j] - m);
+                const double wk = (double)nk / (double)ntot;
+                for (int j = 0; j < Ck; ++j) row[j] += wk * (exp(logit[j] - m) / z);
+            }
+            for (int j = 0; j < Ck; ++j) probs[r * Ck + j] = (float)row[j];
+        }
+        free(logit);
+        free(row);
+    }
 }
 
 /* Threads OpenMP will use (reported next to oracle timings). */

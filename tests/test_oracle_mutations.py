@@ -53,6 +53,12 @@ MUTATIONS = [
     ("overrides sampled like the rest", "if (forced[e]) p = 1.0f;", "(void)forced;"),
     ("draw ignores the seed", "uint64_t z = seed + (idx + 1u) * 0x9E3779B97F4A7C15ull;",
      "uint64_t z = (idx + 1u) * 0x9E3779B97F4A7C15ull;"),
+    ("sub-clusters seeded from the first tokens", "int t0 = n > 0 ? (int)(((long)k * n) / nsub) : 0;",
+     "int t0 = n > 0 ? (k < n ? k : n - 1) : 0;"),
+    ("sub-cluster rows weighted equally", "const double wk = (double)nk / (double)ntot;",
+     "const double wk = 1.0 / (double)nsub;"),
+    ("sub-cluster ties to the higher index", "if (dist < bd) { bd = dist; best = k; }",
+     "if (dist <= bd) { bd = dist; best = k; }"),
 ]
 
 

@@ -655,6 +655,118 @@ def check_sampled_degenerate(ora):
     np.testing.assert_array_equal(o1, o2)
 
 
+# --------------------------------------------------------------------------- intra-block clustering
+
+def _np_assign(x, c):
+    """Nearest centroid of every token (squared distance, lower index on ties) and the SSE."""
+    d = ((x[:, None, :] - c[None, :, :]) ** 2).sum(-1)
+    a = d.argmin(1)
+    return a, float(d[np.arange(len(x)), a].sum())
+
+
+def check_subclusters(ora):
+    rng = np.random.default_rng(21)
+    D, bq = 8, 16
+    L = lay(seq_len=44, seq_pad=48, D=D, bq=bq, bk=8, heads=2)
+    q = bits(rng.standard_normal((1, 2, 48, D)) * 2)
+    x = val(q)
+    for nsub in (1, 2, 3, 5):
+        cent, size = ora.subclusters(L, q, nsub, 4)
+        for h in range(2):
+            for i in range(3):
+                n = min(bq, 44 - bq * i)
+                xs = x[0, h, bq * i:bq * i + n]
+                c = cent[0, h, i].astype(np.float64)
+                assert size[0, h, i].sum() == n
+                # the centroids are the means of their members under one more assignment
+                # step only at convergence; under the last assignment they are the means
+                # of the clusters that produced them: re-derive by running Lloyd here
+                cc = xs[[(k * n) // nsub for k in range(nsub)]].copy()
+                for _ in range(4):
+                    a, _ = _np_assign(xs, cc)
+                    cnt = np.bincount(a, minlength=nsub)
+                    for k in range(nsub):
+                        if cnt[k]:
+                            cc[k] = xs[a == k].mean(0)
+                np.testing.assert_allclose(c, cc, rtol=1e-6, atol=1e-6)
+                assert np.array_equal(size[0, h, i], cnt)
+    # more sub-clusters than tokens: repeated seeds tie, ties go to the lower index, the
+    # copies stay empty
+    L3 = lay(seq_len=19, seq_pad=32, D=D, bq=bq, bk=8, heads=1)
+    q3 = bits(rng.standard_normal((1, 1, 32, D)))
+    c3, s3 = ora.subclusters(L3, q3, 5, 3)
+    x3 = val(q3)[0, 0, 16:19]
+    assert s3[0, 0, 1].tolist() == [1, 0, 1, 0, 1], s3[0, 0, 1]
+    np.testing.assert_allclose(c3[0, 0, 1, [0, 2, 4]], x3, rtol=0, atol=0)
+    # one sub-cluster is the block centroid
+    cent, size = ora.subclusters(L, q, 1, 3)
+    np.testing.assert_array_equal(cent[:, :, :, 0], ora.pool(L, q, bq))
+    # Lloyd's objective never rises with more iterations
+    cent_prev = None
+    for it in range(1, 7):
+        c, _ = ora.subclusters(L, q, 3, it)
+        xs = x[0, 1, 16:32]
+        _, sse = _np_assign(xs, c[0, 1, 1].astype(np.float64))
+        if cent_prev is not None:
+            assert sse <= cent_prev + 1e-9
+        cent_prev = sse
+    # two separated groups of unequal size are found, with their sizes
+    g = np.zeros((1, 1, 16, D))
+    g[0, 0, :11] = 5.0 + 0.01 * rng.standard_normal((11, D))
+    g[0, 0, 11:] = -5.0 + 0.01 * rng.standard_normal((5, D))
+    L2 = lay(seq_len=16, seq_pad=16, D=D, bq=16, bk=8, heads=1)
+    c, sz = ora.subclusters(L2, bits(g), 2, 3)
+    gv = val(bits(g))[0, 0]
+    assert sorted(sz[0, 0, 0].tolist()) == [5, 11]
+    means = sorted([gv[:11].mean(0).sum(), gv[11:].mean(0).sum()])
+    assert np.allclose(sorted(c[0, 0, 0].astype(np.float64).sum(1)), means, atol=1e-5)
+
+
+def check_scores_clustered(ora):
+    rng = np.random.default_rng(22)
+    D, bq, bk = 8, 8, 8
+    L = lay(seq_len=38, seq_pad=40, D=D, bq=bq, bk=bk, heads=2)
+    q = bits(rng.standard_normal((1, 2, 40, D)) * 1.5)
+    k = bits(rng.standard_normal((1, 2, 40, D)) * 1.5)
+    kc = ora.pool(L, k, bk)
+    # nsub = 1: the plain cluster-size-weighted softmax of the block centroid
+    cent, size = ora.subclusters(L, q, 1, 2)
+    p1 = ora.scores_clustered(L, cent, size, kc)
+    p0 = ora.scores(L, ora.pool(L, q, bq), kc)
+    np.testing.assert_allclose(p1, p0, rtol=1e-6, atol=1e-8)
+    # every token its own cluster (distinct tokens): the mean over the block's tokens of the
+    # token-level cluster-size-weighted softmax over the key centroids -- a closed form
+    cent, size = ora.subclusters(L, q, bq, 2)
+    pk = ora.scores_clustered(L, cent, size, kc)
+    xq = val(q)
+    nj = np.array([min(bk, 38 - bk * j) for j in range(5)], np.float64)
+    for h in range(2):
+        for i in range(5):
+            n = min(bq, 38 - bq * i)
+            toks = xq[0, h, bq * i:bq * i + n]
+            lg = toks @ kc[0, h].astype(np.float64).T / math.sqrt(D) + np.log(nj)
+            e = np.exp(lg - lg.max(1, keepdims=True))
+            ref = (e / e.sum(1, keepdims=True)).mean(0)
+            np.testing.assert_allclose(pk[0, h, i], ref, rtol=1e-5, atol=1e-7)
+    # rows sum to one, and a mixture weighted by the sizes (unequal clusters)
+    cent, size = ora.subclusters(L, q, 3, 3)
+    p3 = ora.scores_clustered(L, cent, size, kc)
+    np.testing.assert_allclose(p3.sum(-1), 1.0, rtol=1e-6)
+    r = ora.scores(L, cent[:, :, :, 0], kc) * 0     # shape helper
+    for c in range(3):
+        pc = ora.scores(L, cent[:, :, :, c], kc)
+        r = r + pc.astype(np.float64) * (size[..., c:c + 1] / size.sum(-1, keepdims=True))
+    np.testing.assert_allclose(p3, r, rtol=1e-5, atol=1e-7)
+
+
+def test_subclusters(ora):
+    check_subclusters(ora)
+
+
+def test_scores_clustered(ora):
+    check_scores_clustered(ora)
+
+
 def test_splitmix64(ora):
     check_splitmix64(ora)
 
@@ -691,4 +803,4 @@ ALL_CHECKS = [check_geometry, check_pooling, check_scores, check_entropy, check_
               check_overrides_lists, check_attention, check_pipeline, check_value_norms,
               check_eg_route, check_eg_select, check_splitmix64, check_inclusion_law,
               check_sample_frequencies, check_sampled_attention_unbiased,
-              check_sampled_degenerate]
+              check_sampled_degenerate, check_subclusters, check_scores_clustered]
