@@ -55,6 +55,10 @@ def parse():
                          "(bsa_value_norms + bsa_build_mask_eg), or importance sampling with "
                          "inverse-probability weights (bsa_build_mask_sampled + "
                          "bsa_attention_fwd_weighted) inside the step")
+    ap.add_argument("--subclusters", type=int, default=1,
+                    help="query sub-clusters per block for the block scores (1: block centroids, "
+                         "bsa_block_scores; 2-16: bsa_block_scores_clustered)")
+    ap.add_argument("--kmeans-iters", type=int, default=3)
     ap.add_argument("--budget", type=float, default=None,
                     help="per-row budget K of the sampler (default: calibrated so the expected "
                          "density matches the per-row top-p selection)")
@@ -270,10 +274,23 @@ def our_arm(args, w):
     stream = torch.cuda.current_stream(dev)
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
 
+    nsub = args.subclusters
+    if nsub > 1:
+        sub_c = torch.empty((B, H, Cq, nsub, D), **f32)
+        sub_n = torch.empty((B, H, Cq, nsub), dtype=torch.int32, device=dev)
+        ws_cl = torch.empty(bsa.clustered_workspace_bytes(w, nsub), dtype=torch.uint8, device=dev)
+
+    def scores(qq, kk):
+        if nsub > 1:
+            bsa.block_scores_clustered(w, qq, kk, nsub, args.kmeans_iters, sub_c, sub_n, kc, probs,
+                                       ws_cl, stream=stream)
+        else:
+            bsa.block_scores(w, qq, kk, qc, kc, probs, stream=stream)
+
     def step(qq, kk, vv, marks=None):
         if marks is not None:
             marks[0].record(stream)
-        bsa.block_scores(w, qq, kk, qc, kc, probs, stream=stream)
+        scores(qq, kk)
         if marks is not None:
             marks[1].record(stream)
         if eg:
@@ -299,7 +316,7 @@ def our_arm(args, w):
     if sampled and budget is None:
         # expected density of the sampler = mean of min(1, K P') (overrides aside), matched to
         # the per-row top-p selection of the same P' by bisection (setup, not timed)
-        bsa.block_scores(w, q, k, qc, kc, probs, stream=stream)
+        scores(q, k)
         bsa.build_mask(w, probs, top_p, w.flags, 1e-8, mask, kv_index, kv_count, ent, ent_n, ws,
                        stream=stream)
         target = float(kv_count.sum().item()) / float(B * H * Cq * Ck)
@@ -314,6 +331,8 @@ def our_arm(args, w):
     # value norms, entropy + level 1, two pool levels, the tie pass and the mask kernel in
     # place of mask + entropy reduce; the sampler one kernel
     launches_per_step = 9 if eg else (4 if sampled else 5)
+    if nsub > 1:   # key pooling, k-means, score kernel, mix in place of pooling + score kernel
+        launches_per_step += 2
     for _ in range(max(3, args.warmup)):
         step(q, k, v)
     torch.cuda.synchronize(dev)
@@ -453,6 +472,8 @@ def our_arm(args, w):
                               else ("importance-sampled, inverse-probability weights (budget K "
                                     "%.4g per row, a new seed per step)" % budget) if sampled
                               else "per-row top-p",
+                    block_scores=("intra-block query clusters: %d per block, %d k-means rounds"
+                                  % (nsub, args.kmeans_iters)) if nsub > 1 else "block centroids",
                     density=density, skipped=1 - density, selected_pairs=pairs,
                     computed_tflop_per_step=step_flops / 1e12,
                     dense_equiv_tflop=4.0 * B * H * w.seq_len ** 2 * D / 1e12,

@@ -81,6 +81,11 @@ def load():
         L.bsa_build_mask_eg.argtypes = [lp, vp, vp, vp, ctypes.c_float, ctypes.c_uint32,
                                         ctypes.c_float, vp, vp, vp, vp, vp, vp, vp, vp]
         L.bsa_build_mask_eg.restype = ctypes.c_int
+        L.bsa_block_scores_clustered.argtypes = [lp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp, vp,
+                                                 vp, vp, vp]
+        L.bsa_block_scores_clustered.restype = ctypes.c_int
+        L.bsa_block_scores_clustered_workspace_bytes.argtypes = [lp, ctypes.c_int]
+        L.bsa_block_scores_clustered_workspace_bytes.restype = ctypes.c_size_t
         L.bsa_build_mask_sampled.argtypes = [lp, vp, ctypes.c_float, ctypes.c_uint64, ctypes.c_uint32,
                                              vp, vp, vp, vp, vp]
         L.bsa_build_mask_sampled.restype = ctypes.c_int
@@ -303,6 +308,39 @@ def attention_fwd(layout, q, k, v, kv_index, kv_count, softmax_scale=None, out=N
                                   _ptr(err_flag), _ptr(workspace), _stream(stream))
     _check("bsa_attention_fwd", rc)
     return out, lse
+
+
+def clustered_workspace_bytes(layout, n_sub):
+    L = make_layout(layout)
+    return int(load().bsa_block_scores_clustered_workspace_bytes(ctypes.byref(L), int(n_sub)))
+
+
+def block_scores_clustered(layout, q, k, n_sub, iters, sub_centroids=None, sub_sizes=None,
+                           k_centroids=None, probs=None, workspace=None, stream=None):
+    """bsa_block_scores_clustered: returns (sub_centroids, sub_sizes, k_centroids, probs)."""
+    L = make_layout(layout)
+    d = dims(L)
+    qkv = (d["B"], d["H"], d["Sp"], d["D"])
+    _need(q, "q", torch.bfloat16, qkv)
+    _need(k, "k", torch.bfloat16, qkv)
+    dev = q.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    if sub_centroids is None:
+        sub_centroids = torch.empty((d["B"], d["H"], d["Cq"], n_sub, d["D"]), **f32)
+    if sub_sizes is None:
+        sub_sizes = torch.empty((d["B"], d["H"], d["Cq"], n_sub), dtype=torch.int32, device=dev)
+    if k_centroids is None:
+        k_centroids = torch.empty((d["B"], d["H"], d["Ck"], d["D"]), **f32)
+    if probs is None:
+        probs = torch.empty((d["B"], d["H"], d["Cq"], d["Ck"]), **f32)
+    if workspace is None:
+        workspace = torch.empty(max(clustered_workspace_bytes(L, n_sub), 256), dtype=torch.uint8,
+                                device=dev)
+    rc = load().bsa_block_scores_clustered(ctypes.byref(L), _ptr(q), _ptr(k), int(n_sub), int(iters),
+                                           _ptr(sub_centroids), _ptr(sub_sizes), _ptr(k_centroids),
+                                           _ptr(probs), _ptr(workspace), _stream(stream))
+    _check("bsa_block_scores_clustered", rc)
+    return sub_centroids, sub_sizes, k_centroids, probs
 
 
 def build_mask_sampled(layout, probs, budget, seed, flags, mask=None, kv_index=None,

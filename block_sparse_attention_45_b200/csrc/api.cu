@@ -125,6 +125,33 @@ int bsa_block_scores(const bsa_layout *layout, const void *q, const void *k, flo
     return launch_status(bsa::launch_scores(g, q_centroids, k_centroids, probs, st));
 }
 
+size_t bsa_block_scores_clustered_workspace_bytes(const bsa_layout *layout, int n_sub) {
+    if (check_layout(layout) != BSA_OK) return 0;
+    if (n_sub < 1 || n_sub > bsa::kMaxSubclusters || (n_sub & (n_sub - 1))) return 0;
+    return ((bsa::cluster_workspace_bytes(bsa::make_geometry(*layout), n_sub) + 255) / 256) * 256;
+}
+
+int bsa_block_scores_clustered(const bsa_layout *layout, const void *q, const void *k, int n_sub,
+                               int iters, float *sub_centroids, int32_t *sub_sizes,
+                               float *k_centroids, float *probs, void *workspace, void *stream) {
+    int rc = check_layout(layout);
+    if (rc != BSA_OK) return rc;
+    if (!q || !k || !sub_centroids || !sub_sizes || !k_centroids || !probs || !workspace)
+        return BSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(sub_centroids, 16) ||
+        !aligned(k_centroids, 16) || !aligned(probs, 16) || !aligned(sub_sizes, 4) ||
+        !aligned(workspace, 256))
+        return BSA_ERR_INVALID_ARG;
+    if (iters < 1 || iters > 1000) return BSA_ERR_INVALID_ARG;
+    if (n_sub < 1 || n_sub > bsa::kMaxSubclusters || (n_sub & (n_sub - 1))) return BSA_ERR_UNSUPPORTED;
+    const Geometry g = bsa::make_geometry(*layout);
+    if (g.Ck > bsa::kMaxScoreCk) return BSA_ERR_UNSUPPORTED;
+    if (static_cast<long long>(g.B) * g.H * g.Cq * n_sub > 0x7FFFFFFFll) return BSA_ERR_UNSUPPORTED;
+    return launch_status(bsa::launch_scores_clustered(g, q, k, n_sub, iters, sub_centroids, sub_sizes,
+                                                      k_centroids, probs, workspace,
+                                                      static_cast<cudaStream_t>(stream)));
+}
+
 size_t bsa_build_mask_workspace_bytes(const bsa_layout *layout) {
     if (check_layout(layout) != BSA_OK) return 0;
     const size_t rows = static_cast<size_t>(layout->batch) * layout->heads *

@@ -100,6 +100,17 @@ int launch_attention(const Geometry &g, const void *q, const void *k, const void
                      float softmax_scale, void *out, float *lse, int32_t *err_flag,
                      void *workspace, cudaStream_t st);
 
+// Key centroids only (the pool kernel with no query blocks).
+cudaError_t launch_pool_keys(const Geometry &g, const void *k, float *kc, cudaStream_t st);
+
+// Intra-block clustering selector: sub-clusters per query block (n_sub in
+// {1, 2, 4, 8, 16}) and their size-weighted block scores.
+constexpr int kMaxSubclusters = 16;
+size_t cluster_workspace_bytes(const Geometry &g, int nsub);
+cudaError_t launch_scores_clustered(const Geometry &g, const void *q, const void *k, int nsub,
+                                    int iters, float *cent, int32_t *size, float *kc, float *probs,
+                                    void *workspace, cudaStream_t st);
+
 // Importance sampling of key blocks with inverse-inclusion-probability weights.
 cudaError_t launch_sample(const Geometry &g, const float *probs, float budget, uint64_t seed,
                           uint32_t flags, uint8_t *mask, int32_t *kv_index, float *kv_weight,

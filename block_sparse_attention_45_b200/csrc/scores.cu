@@ -554,6 +554,18 @@ cudaError_t launch_pool(const Geometry &g, const void *q, const void *k, float *
     return cudaGetLastError();
 }
 
+cudaError_t launch_pool_keys(const Geometry &g, const void *k, float *kc, cudaStream_t st) {
+    const long long nk = static_cast<long long>(g.B) * g.H * g.Ck;
+    const uint4 *k4 = static_cast<const uint4 *>(k);
+    if (g.D == 128)
+        pool_kernel<128><<<static_cast<unsigned>(nk), 256, 0, st>>>(
+            nullptr, k4, nullptr, kc, g.S, g.S_pad, g.bq, g.bk, g.Cq, g.Ck, 0);
+    else
+        pool_kernel<64><<<static_cast<unsigned>(nk), 256, 0, st>>>(
+            nullptr, k4, nullptr, kc, g.S, g.S_pad, g.bq, g.bk, g.Cq, g.Ck, 0);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_value_norms(const Geometry &g, const void *v, float *vnorm, cudaStream_t st) {
     const long long nk = static_cast<long long>(g.B) * g.H * g.Ck;
     const auto *v4 = static_cast<const uint4 *>(v);

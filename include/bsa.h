@@ -112,6 +112,40 @@ enum bsa_device_error {
 int bsa_block_scores(const bsa_layout *layout, const void *q, const void *k,
                      float *q_centroids, float *k_centroids, float *probs, void *stream);
 
+/*
+ * Block scores from intra-block query clusters ("AB-Attention: accurate
+ * block-sparse attention for video diffusion", TL;DR fix (1): the queries of
+ * each query block are clustered among themselves, tokens stay in place, so
+ * the importance estimate is finer than one block mean).  The page gives no
+ * procedure; this one is used.  Per query block: k-means (Lloyd) on its valid
+ * query tokens with n_sub clusters, seeded with the tokens at positions
+ * floor(c * n / n_sub) (n = valid tokens), squared Euclidean distance, ties
+ * to the lower cluster, `iters` rounds of (assign, move every non-empty
+ * cluster to its mean; an empty one keeps its centroid and has size 0), in
+ * fp32.  The block's row of P' is the size-weighted mixture of the
+ * sub-centroids' cluster-size-weighted softmax rows,
+ *   P'_ij = sum_c (n_c / n_i) n_j exp(s_cj) / sum_j' n_j' exp(s_cj'),
+ *   s_cj = q_c . k_j / sqrt(D),
+ * so rows sum to one and n_sub = 1 is bsa_block_scores.  P' then feeds
+ * bsa_build_mask / bsa_build_mask_eg / bsa_build_mask_sampled unchanged.
+ *
+ * n_sub          1, 2, 4, 8 or 16 (else BSA_ERR_UNSUPPORTED)
+ * iters          1 .. 1000
+ * sub_centroids  fp32 [B,H,C_q,n_sub,D], 16-byte aligned (written)
+ * sub_sizes      int32 [B,H,C_q,n_sub] (written)
+ * k_centroids    fp32 [B,H,C_k,D], 16-byte aligned (written)
+ * probs          fp32 [B,H,C_q,C_k], 16-byte aligned (written)
+ * workspace      device scratch of
+ *                bsa_block_scores_clustered_workspace_bytes(layout, n_sub)
+ *                bytes (the sub-centroid rows), 256-byte aligned
+ */
+int bsa_block_scores_clustered(const bsa_layout *layout, const void *q, const void *k, int n_sub,
+                               int iters, float *sub_centroids, int32_t *sub_sizes,
+                               float *k_centroids, float *probs, void *workspace, void *stream);
+
+/* Bytes of device workspace bsa_block_scores_clustered needs (0: invalid). */
+size_t bsa_block_scores_clustered_workspace_bytes(const bsa_layout *layout, int n_sub);
+
 /* Bytes of device workspace bsa_build_mask needs (per-row entropies). */
 size_t bsa_build_mask_workspace_bytes(const bsa_layout *layout);
 

@@ -165,6 +165,31 @@ def test_eg_entry_points_validate_before_any_cuda_call():
     assert n >= rows * 4 + w.heads * 256 * 16 + 4096 * 16 and n % 256 == 0
 
 
+def test_clustered_scores_validate_before_any_cuda_call():
+    lib = bsa.load()
+    L = _layout()
+    r = ctypes.byref(L)
+    ws = ctypes.c_void_p(0x100000)
+
+    def cl(q=FAKE, nsub=4, iters=3, cent=FAKE, size=FAKE, kc=FAKE, probs=FAKE, w=ws):
+        return lib.bsa_block_scores_clustered(r, q, FAKE, nsub, iters, cent, size, kc, probs, w, None)
+    assert cl(q=None) == bsa.BSA_ERR_INVALID_ARG
+    assert cl(cent=None) == bsa.BSA_ERR_INVALID_ARG
+    assert cl(size=None) == bsa.BSA_ERR_INVALID_ARG
+    assert cl(w=None) == bsa.BSA_ERR_INVALID_ARG
+    assert cl(w=ctypes.c_void_p(0x100010)) == bsa.BSA_ERR_INVALID_ARG
+    assert cl(cent=MISALIGNED) == bsa.BSA_ERR_INVALID_ARG
+    assert cl(iters=0) == bsa.BSA_ERR_INVALID_ARG
+    assert cl(nsub=3) == bsa.BSA_ERR_UNSUPPORTED
+    assert cl(nsub=32) == bsa.BSA_ERR_UNSUPPORTED
+    assert cl(nsub=0) == bsa.BSA_ERR_UNSUPPORTED
+    assert lib.bsa_block_scores_clustered_workspace_bytes(r, 3) == 0
+    w = synth.WORKLOADS["tiny"]
+    cq, ck = w.seq_pad // w.q_block, w.seq_pad // w.k_block
+    assert lib.bsa_block_scores_clustered_workspace_bytes(r, 4) >= \
+        w.batch * w.heads * cq * 4 * ck * 4
+
+
 def test_sampling_entry_points_validate_before_any_cuda_call():
     lib = bsa.load()
     L = _layout()
