@@ -74,6 +74,8 @@ class Oracle:
                                         vp, vp]
         L.ora_subclusters.argtypes = [lp, vp, ctypes.c_int, ctypes.c_int, vp, vp]
         L.ora_scores_clustered.argtypes = [lp, vp, vp, ctypes.c_int, vp, vp]
+        L.ora_frame_scores.argtypes = [lp, vp, vp, ctypes.c_double, ctypes.c_int, vp]
+        L.ora_dhp.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp]
         L.ora_num_threads.restype = ctypes.c_int
         self.lib = L
 
@@ -194,6 +196,26 @@ class Oracle:
         self.lib.ora_attention(ctypes.byref(L), _ptr(q), _ptr(k), _ptr(v), _ptr(m), _ptr(wt),
                                float(scale), n, _ptr(r), _ptr(out), _ptr(lse))
         return out, lse
+
+    def frame_scores(self, L, q, k, scale=None, query_stride=1):
+        """Per-head frame attention scores [alpha_sink, alpha_neighbor, alpha_current] of the
+        current frame's queries, fp64 [B,H,3]."""
+        L = _layout(L)
+        q, k = _u16(q), _u16(k)
+        if scale is None:
+            scale = 1.0 / math.sqrt(L.head_dim)
+        alpha = np.empty((L.batch, L.heads, 3), np.float64)
+        self.lib.ora_frame_scores(ctypes.byref(L), _ptr(q), _ptr(k), float(scale), int(query_stride),
+                                  _ptr(alpha))
+        return alpha
+
+    def dhp(self, alpha, n_dummy):
+        """Dynamic Head Programming labels (0 sink, 1 neighbor, 2 dummy) of the heads of alpha [H,3]."""
+        a = np.ascontiguousarray(alpha, np.float64)
+        H = a.shape[0]
+        label = np.empty(H, np.int32)
+        self.lib.ora_dhp(_ptr(a), H, int(n_dummy), _ptr(label))
+        return label
 
     def splitmix64(self, seed, idx):
         """The idx-th output (from 0) of SplitMix64 started from state `seed`."""

@@ -23,6 +23,10 @@
  *       domain 1 "per-row local" top-p (Eq. 2); domain 3 "grouped
  *       cross-head" with the median split on H_h and the safeguard; s4 the
  *       value-aware score of the cross-head pool (EG-Sparse).
+ *  [p2] "Efficient Autoregressive Video Diffusion with Dummy Head"
+ *       Step 0 frame attention score [alpha_sink, alpha_neighbor,
+ *       alpha_current] per head; Step 1 Dynamic Head Programming (the greedy
+ *       labelling into sink / neighbor / dummy heads).
  *  [p5] "AB-Attention: accurate block-sparse attention for video diffusion"
  *       TL;DR: exact attention computed only on the selected K/V blocks;
  *       fix (2): blocks sampled in proportion to importance and reweighted
@@ -701,6 +705,93 @@ void ora_scores_clustered(const ora_layout *L, const float *cent, const int32_t 
         free(logit);
         free(row);
     }
+}
+
+/*
+ * ---------------------------------------------------------------------------
+ * Head profiling for autoregressive generation ([p2] Step 0 and Step 1).
+ * Readings where the page is informal:
+ *  - the key window is num_frames frames of tokens_per_frame tokens (no text):
+ *    frame 0 the sink, frames 1 .. F-2 the neighbor window, frame F-1 the
+ *    current frame (the group of a key is its frame's);
+ *  - the queries are the current frame's tokens, every query_stride-th one
+ *    from the frame's first token ("a subset of queries for speed");
+ *  - a query's attention is the softmax of scale * q . k over the whole
+ *    window; alpha_g = the mean over the queries of the mass on group g
+ *    (so the three values sum to one: "normalize so they add up to 1");
+ *  - DHP: l_h = max(alpha_sink, alpha_neighbor); the n_dummy heads with the
+ *    smallest l_h (lower h on ties) are dummy; every other head is sink if
+ *    alpha_sink > alpha_neighbor, else neighbor.
+ * ---------------------------------------------------------------------------
+ */
+
+/* alpha fp64 [B,H,3] in the order sink, neighbor, current. */
+void ora_frame_scores(const ora_layout *L, const uint16_t *q, const uint16_t *k, double scale,
+                      int query_stride, double *alpha)
+{
+    const int D = L->head_dim, T = L->tokens_per_frame, F = L->num_frames;
+    const long BH = (long)L->batch * L->heads;
+    const int n_keys = F * T;
+    #pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)n_keys);
+        #pragma omp for schedule(static)
+        for (long bh = 0; bh < BH; ++bh) {
+            const uint16_t *Qb = q + bh * L->seq_pad * (long)D;
+            const uint16_t *Kb = k + bh * L->seq_pad * (long)D;
+            double acc[3] = {0.0, 0.0, 0.0};
+            long nq = 0;
+            for (int t = (F - 1) * T; t < F * T; t += query_stride) {
+                double m = -INFINITY;
+                for (int u = 0; u < n_keys; ++u) {
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d)
+                        dot += bf16_val(Qb[(long)t * D + d]) * bf16_val(Kb[(long)u * D + d]);
+                    s[u] = dot * scale;
+                    if (s[u] > m) m = s[u];
+                }
+                double z = 0.0, g[3] = {0.0, 0.0, 0.0};
+                for (int u = 0; u < n_keys; ++u) {
+                    double e = exp(s[u] - m);
+                    int f = u / T;
+                    int grp = f == 0 ? 0 : (f == F - 1 ? 2 : 1);
+                    z = z + e;
+                    g[grp] += e;
+                }
+                for (int c = 0; c < 3; ++c) acc[c] += g[c] / z;
+                ++nq;
+            }
+            for (int c = 0; c < 3; ++c) alpha[bh * 3 + c] = nq > 0 ? acc[c] / (double)nq : 0.0;
+        }
+        free(s);
+    }
+}
+
+static const double *ora_dhp_l;
+static int ora_dhp_cmp(const void *a, const void *b)
+{
+    int x = *(const int *)a, y = *(const int *)b;
+    if (ora_dhp_l[x] < ora_dhp_l[y]) return -1;
+    if (ora_dhp_l[x] > ora_dhp_l[y]) return 1;
+    return (x > y) - (x < y);
+}
+
+/* Dynamic Head Programming for one set of H heads: label[h] = 0 sink,
+ * 1 neighbor, 2 dummy, from alpha [H,3]. */
+void ora_dhp(const double *alpha, int H, int n_dummy, int *label)
+{
+    double *l = (double *)malloc(sizeof(double) * (size_t)H);
+    int *order = (int *)malloc(sizeof(int) * (size_t)H);
+    for (int h = 0; h < H; ++h) {
+        l[h] = alpha[h * 3] > alpha[h * 3 + 1] ? alpha[h * 3] : alpha[h * 3 + 1];
+        order[h] = h;
+    }
+    ora_dhp_l = l;
+    qsort(order, (size_t)H, sizeof(int), ora_dhp_cmp);
+    for (int h = 0; h < H; ++h) label[h] = alpha[h * 3] > alpha[h * 3 + 1] ? 0 : 1;
+    for (int r = 0; r < n_dummy && r < H; ++r) label[order[r]] = 2;
+    free(l);
+    free(order);
 }
 
 /* Threads OpenMP will use (reported next to oracle timings). */

@@ -59,6 +59,14 @@ MUTATIONS = [
      "const double wk = 1.0 / (double)nsub;"),
     ("sub-cluster ties to the higher index", "if (dist < bd) { bd = dist; best = k; }",
      "if (dist <= bd) { bd = dist; best = k; }"),
+    ("neighbor and current frames swapped", "int grp = f == 0 ? 0 : (f == F - 1 ? 2 : 1);",
+     "int grp = f == 0 ? 0 : (f == F - 1 ? 1 : 2);"),
+    ("dummy heads by the largest l", "if (ora_dhp_l[x] < ora_dhp_l[y]) return -1;",
+     "if (ora_dhp_l[x] < ora_dhp_l[y]) return 1;"),
+    ("opportunity cost from the sink alone",
+     "l[h] = alpha[h * 3] > alpha[h * 3 + 1] ? alpha[h * 3] : alpha[h * 3 + 1];", "l[h] = alpha[h * 3];"),
+    ("queries from the first frame", "for (int t = (F - 1) * T; t < F * T; t += query_stride) {",
+     "for (int t = 0; t < T; t += query_stride) {"),
 ]
 
 

@@ -767,6 +767,83 @@ def test_scores_clustered(ora):
     check_scores_clustered(ora)
 
 
+# --------------------------------------------------------------------------- head profiling (p2)
+
+def check_dhp(ora):
+    g = json.load(open(os.path.join(GOLDEN, "dhp_example.json")))
+    lv = np.array(g["l"])
+    # the page gives l_h = max(alpha_sink, alpha_neighbor); put it on sink for even heads and on
+    # neighbor for odd ones, the rest of the mass on the current frame
+    alpha = np.zeros((g["heads"], 3))
+    for h, x in enumerate(lv):
+        alpha[h, h % 2] = x
+        alpha[h, 1 - h % 2] = x / 3
+        alpha[h, 2] = 1 - x - x / 3
+    lab = ora.dhp(alpha, g["n_dummy"])
+    assert sorted(np.nonzero(lab == 2)[0].tolist()) == g["dummy_heads"], lab
+    for h in range(g["heads"]):
+        if lab[h] != 2:
+            assert lab[h] == h % 2, (h, lab)     # whichever of sink / neighbor is larger
+    # the step-0 examples: with one dummy slot the current-frame head is the dummy, the other
+    # keeps the neighbor window
+    ex = np.array([e["alpha"] for e in g["step0_examples"]])
+    assert ora.dhp(ex, 1).tolist() == [1, 2]
+    assert ora.dhp(ex, 0).tolist() == [1, 1]
+    # ties in l go to the lower head; n_dummy = H makes every head a dummy
+    tie = np.array([[0.2, 0.1, 0.7], [0.1, 0.2, 0.7], [0.5, 0.1, 0.4]])
+    assert ora.dhp(tie, 1).tolist() == [2, 1, 0]
+    assert ora.dhp(tie, 3).tolist() == [2, 2, 2]
+
+
+def _window(rng, F, T, D, H=2, scale_q=1.0):
+    S = F * T
+    L = lay(seq_len=S, seq_pad=S, D=D, bq=T, bk=T, heads=H, tpf=T, frames=F)
+    q = bits(rng.standard_normal((1, H, S, D)) * scale_q)
+    k = bits(rng.standard_normal((1, H, S, D)))
+    return L, q, k
+
+
+def check_frame_scores(ora):
+    rng = np.random.default_rng(31)
+    F, T, D = 4, 8, 16
+    # zero queries: uniform attention, alpha = group sizes / window size
+    L, q, k = _window(rng, F, T, D)
+    a0 = ora.frame_scores(L, np.zeros_like(q), k)
+    np.testing.assert_allclose(a0, np.broadcast_to([1 / F, (F - 2) / F, 1 / F], a0.shape), atol=1e-15)
+    # an independent matrix-form softmax over the window, every query and every 3rd one
+    x_q, x_k = val(q), val(k)
+    for stride in (1, 3):
+        a = ora.frame_scores(L, q, k, 0.25, stride)
+        for h in range(2):
+            rows = np.arange((F - 1) * T, F * T, stride)
+            lg = x_q[0, h, rows] @ x_k[0, h].T * 0.25
+            p = np.exp(lg - lg.max(1, keepdims=True))
+            p /= p.sum(1, keepdims=True)
+            ref = [p[:, :T].sum(1).mean(), p[:, T:(F - 1) * T].sum(1).mean(), p[:, (F - 1) * T:].sum(1).mean()]
+            np.testing.assert_allclose(a[0, h], ref, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(a.sum(-1), 1.0, rtol=1e-12)
+    # two frames: no neighbor window
+    L2, q2, k2 = _window(rng, 2, T, D)
+    a2 = ora.frame_scores(L2, q2, k2)
+    assert (a2[..., 1] == 0).all()
+    # keys of the current frame aligned with every query: the mass sits on the current frame
+    L3, q3, k3 = _window(rng, 3, T, D, H=1)
+    qa = np.zeros((1, 1, 3 * T, D), np.float32)
+    qa[..., 0] = 8.0
+    ka = np.zeros((1, 1, 3 * T, D), np.float32)
+    ka[0, 0, 2 * T:, 0] = 8.0
+    a3 = ora.frame_scores(L3, bits(qa), bits(ka))
+    assert a3[0, 0, 2] > 0.99 and a3[0, 0, 0] < 0.01
+
+
+def test_dhp(ora):
+    check_dhp(ora)
+
+
+def test_frame_scores(ora):
+    check_frame_scores(ora)
+
+
 def test_splitmix64(ora):
     check_splitmix64(ora)
 
@@ -803,4 +880,5 @@ ALL_CHECKS = [check_geometry, check_pooling, check_scores, check_entropy, check_
               check_overrides_lists, check_attention, check_pipeline, check_value_norms,
               check_eg_route, check_eg_select, check_splitmix64, check_inclusion_law,
               check_sample_frequencies, check_sampled_attention_unbiased,
-              check_sampled_degenerate, check_subclusters, check_scores_clustered]
+              check_sampled_degenerate, check_subclusters, check_scores_clustered, check_dhp,
+              check_frame_scores]
