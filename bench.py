@@ -50,6 +50,8 @@ def parse():
                     help="heads per group of the pipelined host-buffer call timed as e2e")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-profile", action="store_true",
+                    help="skip the head-profiling context measurement")
     ap.add_argument("--selection", default="top_p", choices=["top_p", "eg", "sampled"],
                     help="per-row top-p (bsa_build_mask), entropy-guided grouped selection "
                          "(bsa_value_norms + bsa_build_mask_eg), or importance sampling with "
@@ -439,6 +441,40 @@ def our_arm(args, w):
                       pooled_heads=int(low.sum().item()),
                       call="bsa_value_norms + bsa_build_mask_eg on the step's P'")
 
+    # head profiling of autoregressive generation for context (not part of the step): frame
+    # attention scores on a Self Forcing-shaped key window (sink + 3 neighbors + current frame),
+    # then Dynamic Head Programming on the host
+    prof = None
+    if not args.no_profile:
+        wv = synth.WINDOWS["selfforcing"]
+        xv = synth.generate(wv)
+        qv, kv = (torch.from_numpy(xv[n].view(np.int16)).view(torch.bfloat16).to(dev)
+                  for n in ("q", "k"))
+        alpha = torch.empty((wv.batch, wv.heads, 3), dtype=torch.float32, device=dev)
+        wsv = torch.empty(bsa.frame_scores_workspace_bytes(wv), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            bsa.frame_scores(wv, qv, kv, alpha=alpha, workspace=wsv, stream=stream)
+        a, b = ev(), ev()
+        a.record(stream)
+        npf = 10
+        for _ in range(npf):
+            bsa.frame_scores(wv, qv, kv, alpha=alpha, workspace=wsv, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        pms = a.elapsed_time(b) / npf
+        T, F = wv.tokens_per_frame, wv.num_frames
+        cq = wv.seq_pad // wv.q_block
+        i0, i1 = (F - 1) * T // wv.q_block, (F * T - 1) // wv.q_block
+        pflop = wv.batch * wv.heads * (i1 - i0 + 1) * cq * flops_per_pair(wv)
+        al = alpha.cpu().numpy()
+        labels = bsa.dhp_labels(al[0], wv.heads // 2)
+        prof = dict(workload="selfforcing: 12 heads, 5 frames x 1560 tokens, D 128", ms=pms,
+                    tflops=pflop / (pms * 1e-3) / 1e12,
+                    call="bsa_frame_scores (attention over a one-hot V) + bsa_dhp_labels (host)",
+                    dummy_heads=[int(h) for h in np.nonzero(labels == 2)[0]],
+                    alpha_mean=[float(v) for v in al.reshape(-1, 3).mean(0)])
+        del qv, kv, wsv
+
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -488,6 +524,7 @@ def our_arm(args, w):
                   frac_hbm=bytes_mask / (np.mean(ms_mask) * 1e-3) / 1e9 / hbm),
         dense=dense,
         eg_selection=eg_ctx,
+        head_profiling=prof,
         roofline=dict(bound="tensor", kernel="attn_kernel", achieved=achieved, peak=peak,
                       unit="TFLOP/s", frac=achieved / peak, peak_source=peak_note,
                       traffic=traffic, flop_per_launch=step_flops,

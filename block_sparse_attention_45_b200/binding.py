@@ -10,6 +10,7 @@ import math
 import os
 import re
 
+import numpy as np
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -86,6 +87,12 @@ def load():
         L.bsa_block_scores_clustered.restype = ctypes.c_int
         L.bsa_block_scores_clustered_workspace_bytes.argtypes = [lp, ctypes.c_int]
         L.bsa_block_scores_clustered_workspace_bytes.restype = ctypes.c_size_t
+        L.bsa_frame_scores.argtypes = [lp, vp, vp, ctypes.c_float, ctypes.c_int, vp, vp, vp]
+        L.bsa_frame_scores.restype = ctypes.c_int
+        L.bsa_frame_scores_workspace_bytes.argtypes = [lp]
+        L.bsa_frame_scores_workspace_bytes.restype = ctypes.c_size_t
+        L.bsa_dhp_labels.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp]
+        L.bsa_dhp_labels.restype = ctypes.c_int
         L.bsa_build_mask_sampled.argtypes = [lp, vp, ctypes.c_float, ctypes.c_uint64, ctypes.c_uint32,
                                              vp, vp, vp, vp, vp]
         L.bsa_build_mask_sampled.restype = ctypes.c_int
@@ -341,6 +348,44 @@ def block_scores_clustered(layout, q, k, n_sub, iters, sub_centroids=None, sub_s
                                            _ptr(probs), _ptr(workspace), _stream(stream))
     _check("bsa_block_scores_clustered", rc)
     return sub_centroids, sub_sizes, k_centroids, probs
+
+
+HEAD_SINK, HEAD_NEIGHBOR, HEAD_DUMMY = 0, 1, 2
+
+
+def frame_scores_workspace_bytes(layout):
+    L = make_layout(layout)
+    return int(load().bsa_frame_scores_workspace_bytes(ctypes.byref(L)))
+
+
+def frame_scores(layout, q, k, softmax_scale=None, query_stride=1, alpha=None, workspace=None,
+                 stream=None):
+    """bsa_frame_scores: [alpha_sink, alpha_neighbor, alpha_current] per head, fp32 [B,H,3]."""
+    L = make_layout(layout)
+    d = dims(L)
+    qkv = (d["B"], d["H"], d["Sp"], d["D"])
+    _need(q, "q", torch.bfloat16, qkv)
+    _need(k, "k", torch.bfloat16, qkv)
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d["D"])
+    if alpha is None:
+        alpha = torch.empty((d["B"], d["H"], 3), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(frame_scores_workspace_bytes(L), dtype=torch.uint8, device=q.device)
+    rc = load().bsa_frame_scores(ctypes.byref(L), _ptr(q), _ptr(k), float(softmax_scale),
+                                 int(query_stride), _ptr(alpha), _ptr(workspace), _stream(stream))
+    _check("bsa_frame_scores", rc)
+    return alpha
+
+
+def dhp_labels(alpha, n_dummy):
+    """bsa_dhp_labels (host): labels 0 sink, 1 neighbor, 2 dummy of the heads of alpha [H, 3]."""
+    a = np.ascontiguousarray(np.asarray(alpha, np.float32).reshape(-1, 3))
+    labels = np.empty(a.shape[0], np.int32)
+    rc = load().bsa_dhp_labels(a.ctypes.data_as(ctypes.c_void_p), a.shape[0], int(n_dummy),
+                               labels.ctypes.data_as(ctypes.c_void_p))
+    _check("bsa_dhp_labels", rc)
+    return labels
 
 
 def build_mask_sampled(layout, probs, budget, seed, flags, mask=None, kv_index=None,

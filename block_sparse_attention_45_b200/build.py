@@ -8,7 +8,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libbsa.so")
-SOURCES = ["api.cu", "scores.cu", "mask.cu", "eg.cu", "sample.cu", "cluster.cu", "attention.cu", "noalloc.cu", "pipeline.cu"]
+SOURCES = ["api.cu", "scores.cu", "mask.cu", "eg.cu", "sample.cu", "cluster.cu", "profile.cu", "attention.cu", "noalloc.cu", "pipeline.cu"]
 HEADERS = ["ptx.cuh", "internal.h"]
 
 NVCC_FLAGS = [

@@ -287,6 +287,54 @@ int bsa_build_mask_sampled(const bsa_layout *layout, const float *probs, float b
                                             kv_count, static_cast<cudaStream_t>(stream)));
 }
 
+size_t bsa_frame_scores_workspace_bytes(const bsa_layout *layout) {
+    if (check_layout(layout) != BSA_OK) return 0;
+    return bsa::profile_workspace(bsa::make_geometry(*layout)).bytes;
+}
+
+int bsa_frame_scores(const bsa_layout *layout, const void *q, const void *k, float softmax_scale,
+                     int query_stride, float *alpha, void *workspace, void *stream) {
+    int rc = check_layout(layout);
+    if (rc != BSA_OK) return rc;
+    if (!q || !k || !alpha || !workspace) return BSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(alpha, 4) || !aligned(workspace, 256))
+        return BSA_ERR_INVALID_ARG;
+    if (!(softmax_scale > 0.f) || !isfinite(softmax_scale) || query_stride < 1)
+        return BSA_ERR_INVALID_ARG;
+    const int T = layout->tokens_per_frame, F = layout->num_frames;
+    if (layout->text_len != 0 || F < 2 || T < 1 ||
+        static_cast<long long>(F) * T != static_cast<long long>(layout->seq_len))
+        return BSA_ERR_INVALID_ARG;
+    const Geometry g = bsa::make_geometry(*layout);
+    return bsa::launch_frame_scores(g, T, F, q, k, softmax_scale, query_stride, alpha,
+                                    static_cast<uint8_t *>(workspace),
+                                    static_cast<cudaStream_t>(stream));
+}
+
+int bsa_dhp_labels(const float *alpha, int heads, int n_dummy, int32_t *labels) {
+    if (!alpha || !labels || heads < 1 || n_dummy < 0 || n_dummy > heads) return BSA_ERR_INVALID_ARG;
+    // l_h = max(alpha_sink, alpha_neighbor); the n_dummy smallest (lower h on ties) are dummy
+    for (int h = 0; h < heads; ++h) {
+        const float s = alpha[3 * h], nb = alpha[3 * h + 1];
+        if (s != s || nb != nb) return BSA_ERR_INVALID_ARG;
+        labels[h] = s > nb ? BSA_HEAD_SINK : BSA_HEAD_NEIGHBOR;
+    }
+    for (int r = 0; r < n_dummy; ++r) {
+        int best = -1;
+        float bl = 0.f;
+        for (int h = 0; h < heads; ++h) {
+            if (labels[h] == BSA_HEAD_DUMMY) continue;
+            const float l = alpha[3 * h] > alpha[3 * h + 1] ? alpha[3 * h] : alpha[3 * h + 1];
+            if (best < 0 || l < bl) {
+                best = h;
+                bl = l;
+            }
+        }
+        labels[best] = BSA_HEAD_DUMMY;
+    }
+    return BSA_OK;
+}
+
 int bsa_dense_fwd(const bsa_layout *layout, const void *q, const void *k, const void *v,
                   float softmax_scale, void *out, float *lse, int32_t *err_flag, void *workspace,
                   void *stream) {

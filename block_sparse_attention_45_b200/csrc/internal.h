@@ -111,6 +111,17 @@ cudaError_t launch_scores_clustered(const Geometry &g, const void *q, const void
                                     int iters, float *cent, int32_t *size, float *kc, float *probs,
                                     void *workspace, cudaStream_t st);
 
+// Head profiling for autoregressive generation: frame attention scores over a
+// key window of F frames of T tokens (frame 0 sink, 1 .. F-2 neighbors, F-1
+// current), computed with the attention kernel and a one-hot V.
+struct ProfileWorkspace {
+    size_t v, out, kv_index, kv_count, sched, bytes;
+};
+ProfileWorkspace profile_workspace(const Geometry &g);
+int launch_frame_scores(const Geometry &g, int T, int F, const void *q, const void *k,
+                        float softmax_scale, int query_stride, float *alpha, uint8_t *workspace,
+                        cudaStream_t st);
+
 // Importance sampling of key blocks with inverse-inclusion-probability weights.
 cudaError_t launch_sample(const Geometry &g, const float *probs, float budget, uint64_t seed,
                           uint32_t flags, uint8_t *mask, int32_t *kv_index, float *kv_weight,

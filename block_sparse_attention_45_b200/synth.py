@@ -104,6 +104,18 @@ WORKLOADS = {
 }
 
 
+# Key windows of autoregressive generation for head profiling ("Efficient
+# Autoregressive Video Diffusion with Dummy Head", Step 0): a sink frame, a
+# neighbor window and the current frame, 832x480 video (30x52 latent tokens per
+# frame after 8x VAE and 2x2 patches), Wan2.1-1.3B heads.
+WINDOWS = {
+    "selfforcing": Workload("selfforcing", batch=1, heads=12, head_dim=128, text_len=0,
+                            num_frames=5, latent_h=30, latent_w=52, q_block=128, k_block=128,
+                            seed=5, kind="clustered", sigma_mean=2.0, top_p=0.9, text_keep=False,
+                            frame0_dense=False),
+}
+
+
 def custom(name="custom", **kw):
     """A workload with explicit fields (edge-case parity tests)."""
     base = dict(batch=1, heads=1, head_dim=128, text_len=0, num_frames=1, latent_h=8,

@@ -331,6 +331,45 @@ int bsa_attention_fwd_weighted(const bsa_layout *layout, const void *q, const vo
                                const int32_t *kv_count, float softmax_scale, void *out, float *lse,
                                int32_t *err_flag, void *workspace, void *stream);
 
+/*
+ * Head profiling for autoregressive video generation ("Efficient
+ * Autoregressive Video Diffusion with Dummy Head", Step 0 frame attention
+ * score).  The layout describes the key window: num_frames >= 2 frames of
+ * tokens_per_frame tokens, text_len 0, seq_len = num_frames *
+ * tokens_per_frame; frame 0 is the sink, frames 1 .. F-2 the neighbor window,
+ * frame F-1 the current frame.  For every (b, h) and every query_stride-th
+ * token t of the current frame (from its first token), the softmax of
+ * softmax_scale * Q_t . K_u over the whole window is summed per group, and
+ * alpha[b,h,:] = [alpha_sink, alpha_neighbor, alpha_current] is the mean over
+ * those queries (it sums to one).  Computed on the tensor cores as the
+ * attention of the current frame's query blocks over a one-hot V of the key
+ * groups (bf16 P: expect ~1e-3 absolute error).
+ *
+ * q, k       bf16 [B,H,seq_pad,D], 16-byte aligned (read)
+ * alpha      fp32 [B,H,3] device (written)
+ * workspace  device scratch of bsa_frame_scores_workspace_bytes(layout) bytes,
+ *            256-byte aligned
+ * A layout that is not such a window: BSA_ERR_INVALID_ARG.
+ */
+int bsa_frame_scores(const bsa_layout *layout, const void *q, const void *k, float softmax_scale,
+                     int query_stride, float *alpha, void *workspace, void *stream);
+
+/* Bytes of device workspace bsa_frame_scores needs (0: invalid layout). */
+size_t bsa_frame_scores_workspace_bytes(const bsa_layout *layout);
+
+enum { BSA_HEAD_SINK = 0, BSA_HEAD_NEIGHBOR = 1, BSA_HEAD_DUMMY = 2 };
+
+/*
+ * Dynamic Head Programming ("... Dummy Head", Step 1), on the HOST: from
+ * alpha [heads][3] (host memory, e.g. one (b) slice of bsa_frame_scores'
+ * output), the n_dummy heads with the smallest l_h = max(alpha_sink,
+ * alpha_neighbor) (lower h on ties) are labelled BSA_HEAD_DUMMY, every other
+ * head BSA_HEAD_SINK if alpha_sink > alpha_neighbor, else BSA_HEAD_NEIGHBOR.
+ * labels: int32 [heads] host memory (written).  NaN entries, n_dummy outside
+ * [0, heads]: BSA_ERR_INVALID_ARG.  No CUDA call is made.
+ */
+int bsa_dhp_labels(const float *alpha, int heads, int n_dummy, int32_t *labels);
+
 /* Bytes of device workspace bsa_attention_fwd / bsa_dense_fwd can use. */
 size_t bsa_attention_workspace_bytes(const bsa_layout *layout);
 

@@ -190,6 +190,32 @@ def test_clustered_scores_validate_before_any_cuda_call():
         w.batch * w.heads * cq * 4 * ck * 4
 
 
+def test_frame_scores_validate_before_any_cuda_call():
+    lib = bsa.load()
+    win = synth.WINDOWS["selfforcing"]
+    L = bsa.make_layout(win)
+    r = ctypes.byref(L)
+    ws = ctypes.c_void_p(0x100000)
+
+    def fs(lay=r, q=FAKE, alpha=FAKE, w=ws, scale=0.088, stride=1):
+        return lib.bsa_frame_scores(lay, q, FAKE, scale, stride, alpha, w, None)
+    assert fs(q=None) == bsa.BSA_ERR_INVALID_ARG
+    assert fs(alpha=None) == bsa.BSA_ERR_INVALID_ARG
+    assert fs(w=None) == bsa.BSA_ERR_INVALID_ARG
+    assert fs(w=ctypes.c_void_p(0x100010)) == bsa.BSA_ERR_INVALID_ARG
+    assert fs(stride=0) == bsa.BSA_ERR_INVALID_ARG
+    assert fs(scale=float("inf")) == bsa.BSA_ERR_INVALID_ARG
+    # not a key window: text tokens, one frame, or tokens outside the frames
+    for kw in (dict(text_len=64, seq_len=win.seq_len + 64, seq_pad=win.seq_pad + 128),
+               dict(num_frames=1, seq_len=win.tokens_per_frame, seq_pad=1664),
+               dict(seq_len=win.seq_len - 8, num_frames=4, seq_pad=win.seq_pad)):
+        d = win.layout()
+        d.update(kw)
+        assert fs(lay=ctypes.byref(bsa.make_layout(d))) == bsa.BSA_ERR_INVALID_ARG, kw
+    n = lib.bsa_frame_scores_workspace_bytes(r)
+    assert n >= 2 * 2 * win.heads * win.seq_pad * win.head_dim and n % 256 == 0
+
+
 def test_sampling_entry_points_validate_before_any_cuda_call():
     lib = bsa.load()
     L = _layout()
