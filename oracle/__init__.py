@@ -76,6 +76,7 @@ class Oracle:
         L.ora_scores_clustered.argtypes = [lp, vp, vp, ctypes.c_int, vp, vp]
         L.ora_frame_scores.argtypes = [lp, vp, vp, ctypes.c_double, ctypes.c_int, vp]
         L.ora_dhp.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp]
+        L.ora_centroid_distortion.argtypes = [lp, vp, vp, vp, vp]
         L.ora_num_threads.restype = ctypes.c_int
         self.lib = L
 
@@ -247,6 +248,18 @@ class Oracle:
         v = _u16(v)
         out = np.empty((L.batch, L.heads, L.ck), np.float32)
         self.lib.ora_value_norms(ctypes.byref(L), _ptr(v), _ptr(out))
+        return out
+
+    def centroid_distortion(self, L, probs, vcent, mask):
+        """Relative Frobenius error of the masked, row-renormalised centroid output
+        against the dense one, per head, fp64 [B,H]."""
+        L = _layout(L)
+        probs = np.ascontiguousarray(probs, np.float32)
+        vcent = np.ascontiguousarray(vcent, np.float32)
+        mask = np.ascontiguousarray(mask, np.uint8)
+        out = np.empty((L.batch, L.heads), np.float64)
+        self.lib.ora_centroid_distortion(ctypes.byref(L), _ptr(probs), _ptr(vcent), _ptr(mask),
+                                         _ptr(out))
         return out
 
     def eg_route(self, L, H):

@@ -386,6 +386,42 @@ void ora_value_norms(const ora_layout *L, const uint16_t *v, float *out)
     }
 }
 
+/* Centroid-output distortion ([p3] s3, the controlled diagnostic of the
+ * competition domains): per head the dense centroid output O_i = sum_j P'_ij
+ * c^V_j, the masked one renormalised per row, Om_i = sum_j M_ij P'_ij c^V_j /
+ * sum_j M_ij P'_ij (0 for an empty row), and the relative Frobenius error
+ * ||Om - O||_F / ||O||_F, fp64 [B,H].  vcent fp32 [B,H,C_k,D] (the value
+ * centroids, block means of V). */
+void ora_centroid_distortion(const ora_layout *L, const float *probs, const float *vcent,
+                             const uint8_t *mask, double *out)
+{
+    const int D = L->head_dim, Cq = L->seq_pad / L->q_block, Ck = L->seq_pad / L->k_block;
+    const long BH = (long)L->batch * L->heads;
+    #pragma omp parallel for schedule(static)
+    for (long bh = 0; bh < BH; ++bh) {
+        double num = 0.0, den = 0.0;
+        for (int i = 0; i < Cq; ++i) {
+            const float *p = probs + (bh * Cq + i) * (long)Ck;
+            const uint8_t *m = mask + (bh * Cq + i) * (long)Ck;
+            double z = 0.0;
+            for (int j = 0; j < Ck; ++j)
+                if (m[j]) z += (double)p[j];
+            for (int d = 0; d < D; ++d) {
+                double o = 0.0, om = 0.0;
+                for (int j = 0; j < Ck; ++j) {
+                    double c = (double)vcent[(bh * Ck + j) * D + d];
+                    o += (double)p[j] * c;
+                    if (m[j]) om += (double)p[j] * c;
+                }
+                om = z > 0.0 ? om / z : 0.0;
+                num += (om - o) * (om - o);
+                den += o * o;
+            }
+        }
+        out[bh] = den > 0.0 ? sqrt(num / den) : 0.0;
+    }
+}
+
 typedef struct { double H; int h; } ora_head;
 
 static int ora_head_cmp(const void *a, const void *b)

@@ -179,6 +179,31 @@ def test_eg_zero_eps_routes_every_batch_entry():
                          g["mask"].cpu().numpy())
 
 
+@pytest.mark.parametrize("name", ["small", "h3_b2", "h5_d128"])
+def test_eg_centroid_distortion(name):
+    """The competition-domain diagnostic ("Competition Domains Matter ..." s3: relative
+    Frobenius error of the masked, row-renormalised centroid output): the GPU's masks
+    give the oracle's distortion per head, every value in [0, 1), and keeping every block
+    gives zero."""
+    w, x, probs, H, vn = _oracle_inputs(name)
+    ora = oracle.default()
+    L = w.layout()
+    vcent = ora.pool(L, x["v"], w.k_block)
+    tp = [float(w.top_p)] * w.heads
+    g = bsa.build_mask_eg(w, torch.from_numpy(probs).cuda(), torch.from_numpy(vn).cuda(), tp, 0.9, 0)
+    r = bsa.build_mask(w, torch.from_numpy(probs).cuda(), tp, 0)
+    torch.cuda.synchronize()
+    low = ora.eg_route(L, H)
+    e_gpu = ora.centroid_distortion(L, probs, vcent, g["mask"].cpu().numpy())
+    e_ora = ora.centroid_distortion(L, probs, vcent, ora.eg_select(L, probs, vn, tp, 0.9, low))
+    same = (g["low_heads"].cpu().numpy() == low).all(-1)
+    np.testing.assert_allclose(e_gpu[same], e_ora[same], rtol=1e-12, atol=1e-15)
+    e_row = ora.centroid_distortion(L, probs, vcent, r["mask"].cpu().numpy())
+    assert ((e_gpu >= 0) & (e_gpu < 1)).all() and ((e_row >= 0) & (e_row < 1)).all()
+    full = np.ones_like(probs, dtype=np.uint8)
+    assert (ora.centroid_distortion(L, probs, vcent, full) == 0).all()
+
+
 def test_eg_single_head_is_the_per_row_rule():
     w, _, probs, _, vn = _oracle_inputs("h1")
     tp = [float(w.top_p)]

@@ -65,6 +65,8 @@ MUTATIONS = [
      "if (ora_dhp_l[x] < ora_dhp_l[y]) return 1;"),
     ("opportunity cost from the sink alone",
      "l[h] = alpha[h * 3] > alpha[h * 3 + 1] ? alpha[h * 3] : alpha[h * 3 + 1];", "l[h] = alpha[h * 3];"),
+    ("distortion without the row renormalisation", "om = z > 0.0 ? om / z : 0.0;",
+     "om = z > 0.0 ? om : 0.0;"),
     ("queries from the first frame", "for (int t = (F - 1) * T; t < F * T; t += query_stride) {",
      "for (int t = 0; t < T; t += query_stride) {"),
 ]

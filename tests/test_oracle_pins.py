@@ -864,6 +864,41 @@ def test_sampled_degenerate(ora):
     check_sampled_degenerate(ora)
 
 
+def check_centroid_distortion(ora):
+    # one row, two key blocks with P' = (3/4, 1/4) and orthonormal value centroids: keeping only
+    # the first gives O = (3/4, 1/4), Om = (1, 0), error sqrt(1/8 / 5/8) = sqrt(1/5)
+    L = lay(seq_len=8, seq_pad=8, D=4, bq=8, bk=4, heads=1)
+    P = np.array([[[[0.75, 0.25]]]], np.float32)
+    V = np.zeros((1, 1, 2, 4), np.float32)
+    V[0, 0, 0, 0] = 1.0
+    V[0, 0, 1, 1] = 1.0
+    e = ora.centroid_distortion(L, P, V, np.array([[[[1, 0]]]], np.uint8))
+    assert abs(e[0, 0] - math.sqrt(0.2)) < 1e-15
+    assert ora.centroid_distortion(L, P, V, np.ones((1, 1, 1, 2), np.uint8))[0, 0] == 0.0
+    # against a direct numpy evaluation on random inputs, invariant to scaling V, and an empty
+    # row counting as a zero output
+    rng = np.random.default_rng(51)
+    L = lay(seq_len=40, seq_pad=40, D=8, bq=8, bk=8, heads=2)
+    P = _tiny_probs(rng, 1, 2, 5, 5)
+    V = rng.standard_normal((1, 2, 5, 8)).astype(np.float32)
+    M = (rng.random((1, 2, 5, 5)) < 0.5).astype(np.uint8)
+    M[0, 1, 2] = 0
+    e = ora.centroid_distortion(L, P, V, M)
+    for h in range(2):
+        p64, v64 = P[0, h].astype(np.float64), V[0, h].astype(np.float64)
+        O = p64 @ v64
+        pm = p64 * M[0, h]
+        z = pm.sum(1, keepdims=True)
+        Om = np.where(z > 0, (pm @ v64) / np.where(z > 0, z, 1), 0)
+        ref = np.linalg.norm(Om - O) / np.linalg.norm(O)
+        assert abs(e[0, h] - ref) < 1e-12 * max(1.0, ref)
+    np.testing.assert_allclose(ora.centroid_distortion(L, P, 8 * V, M), e, rtol=1e-12)
+
+
+def test_centroid_distortion(ora):
+    check_centroid_distortion(ora)
+
+
 def test_eg_value_norms(ora):
     check_value_norms(ora)
 
@@ -881,4 +916,4 @@ ALL_CHECKS = [check_geometry, check_pooling, check_scores, check_entropy, check_
               check_eg_route, check_eg_select, check_splitmix64, check_inclusion_law,
               check_sample_frequencies, check_sampled_attention_unbiased,
               check_sampled_degenerate, check_subclusters, check_scores_clustered, check_dhp,
-              check_frame_scores]
+              check_frame_scores, check_centroid_distortion]
