@@ -184,7 +184,7 @@ def test_eg_centroid_distortion(name):
     """The competition-domain diagnostic ("Competition Domains Matter ..." s3: relative
     Frobenius error of the masked, row-renormalised centroid output): the GPU's masks
     give the oracle's distortion per head, every value in [0, 1), and keeping every block
-    gives zero."""
+    gives zero (up to the fp32 rows' rounding)."""
     w, x, probs, H, vn = _oracle_inputs(name)
     ora = oracle.default()
     L = w.layout()
@@ -200,8 +200,8 @@ def test_eg_centroid_distortion(name):
     np.testing.assert_allclose(e_gpu[same], e_ora[same], rtol=1e-12, atol=1e-15)
     e_row = ora.centroid_distortion(L, probs, vcent, r["mask"].cpu().numpy())
     assert ((e_gpu >= 0) & (e_gpu < 1)).all() and ((e_row >= 0) & (e_row < 1)).all()
-    full = np.ones_like(probs, dtype=np.uint8)
-    assert (ora.centroid_distortion(L, probs, vcent, full) == 0).all()
+    full = np.ones_like(probs, dtype=np.uint8)   # zero up to the fp32 rows' sum (1 +- 1e-7)
+    assert (ora.centroid_distortion(L, probs, vcent, full) < 1e-6).all()
 
 
 def test_eg_single_head_is_the_per_row_rule():
