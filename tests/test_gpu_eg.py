@@ -215,11 +215,13 @@ def test_eg_single_head_is_the_per_row_rule():
     assert torch.equal(g["mask"], r["mask"]) and torch.equal(g["kv_count"], r["kv_count"])
 
 
-def test_eg_full_pipeline_properties():
-    """GPU P' and value norms, wan1.3b shape: the pooled selection is the shortest
-    prefix reaching pool_p of the pool (checked on the GPU's own scores), every
-    pooled row is non-empty, and the lists match the mask."""
-    w = synth.WORKLOADS["wan1.3b"]
+@pytest.mark.parametrize("wname", ["wan1.3b", "wan14b"])
+def test_eg_full_pipeline_properties(wname):
+    """GPU P' and value norms at full size (Wan2.1-1.3B: 12 heads; Wan2.1-14B: 40 heads,
+    64-key blocks): the pooled selection is the shortest prefix reaching pool_p of the
+    pool (checked on the GPU's own scores), every pooled row is non-empty, and the lists
+    match the mask."""
+    w = synth.WORKLOADS[wname]
     x = synth.generate(w)
     q, k, v = _dev_bf16(x["q"]), _dev_bf16(x["k"]), _dev_bf16(x["v"])
     _, _, probs = bsa.block_scores(w, q, k)

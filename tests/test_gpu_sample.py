@@ -189,3 +189,44 @@ def test_reweighted_sum_is_unbiased_on_the_gpu():
     fin = torch.isfinite(l_plain[..., valid])
     diff = (l_w - l_plain)[..., valid][fin]
     assert float(diff.min()) > -1e-3 and float(diff.mean()) > 0.01
+
+
+def test_weighted_attention_full_size_sampled_rows():
+    """Wan2.1-14B at full size (40 heads, 64-key blocks gathered into 128-key tiles):
+    the GPU sampler's lists and weights feed the weighted kernel; 24 seeded query
+    blocks (frame-0 rows, the ragged last block, random ones) match the oracle's
+    weighted attention on the same lists."""
+    w = synth.WORKLOADS["wan14b"]
+    x = synth.generate(w)
+    ora = oracle.default()
+    L = w.layout()
+    q, k, v = _dev_bf16(x["q"]), _dev_bf16(x["k"]), _dev_bf16(x["v"])
+    _, _, probs = bsa.block_scores(w, q, k)
+    g = bsa.build_mask_sampled(w, probs, 40.0, 2024, w.flags)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = bsa.attention_fwd_weighted(w, q, k, v, g["kv_index"], g["kv_weight"], g["kv_count"],
+                                          err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    m_g = g["mask"].cpu().numpy()
+    wt = np.zeros(m_g.shape, np.float32)
+    idx, cnt, wts = g["kv_index"].cpu().numpy(), g["kv_count"].cpu().numpy(), g["kv_weight"].cpu().numpy()
+    B, H, Cq, Ck = m_g.shape
+    rng = np.random.default_rng(5)
+    rows = np.unique(np.concatenate([[0, 1, Cq - 1, 2 * Cq + 3, (H - 1) * Cq + Cq - 1],
+                                     rng.integers(0, B * H * Cq, 19)]))
+    for r in rows:
+        b, h, i = r // (H * Cq), (r // Cq) % H, r % Cq
+        n = cnt[b, h, i]
+        wt[b, h, i, idx[b, h, i, :n]] = wts[b, h, i, :n]
+    o_ora, l_ora = ora.attention(L, x["q"], x["k"], x["v"], m_g, rows=rows, weight=wt)
+    og = out.float().cpu().numpy().reshape(B * H, Cq, w.q_block, w.head_dim)
+    lg = lse.cpu().numpy().reshape(B * H, Cq, w.q_block)
+    for n_r, r in enumerate(rows):
+        bh, i = r // Cq, r % Cq
+        valid = np.arange(w.q_block) + i * w.q_block < w.seq_len
+        d = np.abs(og[bh, i][valid] - o_ora[n_r][valid])
+        assert d.max() <= checkers.MAX_ABS and d.mean() <= checkers.MEAN_ABS, (r, d.max(), d.mean())
+        fin = np.isfinite(l_ora[n_r][valid])
+        np.testing.assert_allclose(lg[bh, i][valid][fin], l_ora[n_r][valid][fin], rtol=1e-4,
+                                   atol=checkers.LSE_ABS)
