@@ -21,7 +21,6 @@ import argparse
 import glob
 import json
 import re
-import math
 import os
 import signal
 import subprocess

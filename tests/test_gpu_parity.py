@@ -14,7 +14,6 @@ import torch
 
 import oracle
 from block_sparse_attention_45_b200 import binding as bsa
-from block_sparse_attention_45_b200 import synth
 from tests import checkers
 from tests.gpu_util import (inputs, oracle_selection, sample_rows, to_dev, to_host_f32, top_p_of)
 

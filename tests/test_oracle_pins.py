@@ -21,7 +21,6 @@ import math
 import os
 
 import numpy as np
-import pytest
 import torch
 
 from block_sparse_attention_45_b200 import synth
