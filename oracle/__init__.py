@@ -77,6 +77,9 @@ class Oracle:
         L.ora_frame_scores.argtypes = [lp, vp, vp, ctypes.c_double, ctypes.c_int, vp]
         L.ora_dhp.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp]
         L.ora_centroid_distortion.argtypes = [lp, vp, vp, vp, vp]
+        L.ora_pool_select.argtypes = [lp, vp, vp, vp, ctypes.c_float, vp, ctypes.c_int, vp]
+        L.ora_domain_route.argtypes = [lp, vp, ctypes.c_int, vp]
+        L.ora_domain_route.restype = ctypes.c_int
         L.ora_num_threads.restype = ctypes.c_int
         self.lib = L
 
@@ -282,6 +285,27 @@ class Oracle:
         mask = np.empty((L.batch, L.heads, L.cq, L.ck), np.uint8)
         self.lib.ora_eg_select(ctypes.byref(L), _ptr(probs), _ptr(vn), _ptr(tp), float(pool_p),
                                _ptr(low), _ptr(mask))
+        return mask
+
+    def domain_route(self, L, H, domain):
+        """Pools of the competition domain (0 per-row, 1 per-head, 2 grouped, 3 all-head,
+        4 EG-Sparse): pool_of int8 [B,H] (-1 = per-row) and G, the pools per batch entry."""
+        L = _layout(L)
+        H = np.ascontiguousarray(H, np.float64)
+        pool_of = np.empty((L.batch, L.heads), np.int8)
+        G = self.lib.ora_domain_route(ctypes.byref(L), _ptr(H), int(domain), _ptr(pool_of))
+        return pool_of, int(G)
+
+    def pool_select(self, L, probs, vnorm, top_p, pool_p, pool_of, G):
+        """Pooled top-p over the pools of pool_of (-1 heads per-row), u8 [B,H,C_q,C_k]."""
+        L = _layout(L)
+        probs = np.ascontiguousarray(probs, np.float32)
+        vn = None if vnorm is None else np.ascontiguousarray(vnorm, np.float32)
+        tp = np.ascontiguousarray(np.broadcast_to(np.asarray(top_p, np.float32), (L.heads,)))
+        po = np.ascontiguousarray(pool_of, np.int8)
+        mask = np.empty((L.batch, L.heads, L.cq, L.ck), np.uint8)
+        self.lib.ora_pool_select(ctypes.byref(L), _ptr(probs), _ptr(vn), _ptr(tp), float(pool_p),
+                                 _ptr(po), int(G), _ptr(mask))
         return mask
 
     def eg_selection(self, L, q, k, v, top_p, pool_p, flags, eps=1e-8, value_aware=True):

@@ -483,22 +483,29 @@ static float ora_pool_score(const float *probs, const float *vnorm, long bh, int
  * every pair when no k qualifies.  Then every pool row (h,i) left without a
  * kept pair keeps its highest-scoring key block.  mask is u8 [B,H,C_q,C_k].
  */
-void ora_eg_select(const ora_layout *L, const float *probs, const float *vnorm,
-                   const float *top_p, float pool_p, const uint8_t *low, uint8_t *mask)
+/* Pooled top-p over competition domains: heads with pool_of[b,h] = g >= 0 form
+ * pool g of batch entry b (G pools per entry); the pairs (h, i, j) of one pool
+ * compete in (I desc, h, i, j asc) order for the shortest prefix reaching
+ * pool_p of the pool's total, then the safeguard; heads with pool_of = -1 keep
+ * the per-row rule with their top_p[h] ([p3] s3 the four domains). */
+void ora_pool_select(const ora_layout *L, const float *probs, const float *vnorm,
+                     const float *top_p, float pool_p, const int8_t *pool_of, int G, uint8_t *mask)
 {
     const int Cq = L->seq_pad / L->q_block, Ck = L->seq_pad / L->k_block;
     const int nh = L->heads;
     /* per-row heads: the domain-1 rule, whole layout at once */
     ora_topp(L, probs, top_p, mask, NULL);
-    for (int b = 0; b < L->batch; ++b) {
+    if (Cq <= 0 || Ck <= 0) return;
+    for (int b = 0; b < L->batch; ++b)
+      for (int g = 0; g < G; ++g) {
         long n = 0;
         for (int h = 0; h < nh; ++h)
-            if (low[(long)b * nh + h]) n += (long)Cq * Ck;
+            if (pool_of[(long)b * nh + h] == g) n += (long)Cq * Ck;
         if (n == 0) continue;
         ora_pair *e = (ora_pair *)malloc(sizeof(ora_pair) * (size_t)n);
         long k = 0;
         for (int h = 0; h < nh; ++h) {
-            if (!low[(long)b * nh + h]) continue;
+            if (pool_of[(long)b * nh + h] != g) continue;
             long bh = (long)b * nh + h;
             for (int i = 0; i < Cq; ++i) {
                 memset(mask + (bh * Cq + i) * (long)Ck, 0, (size_t)Ck);
@@ -528,7 +535,7 @@ void ora_eg_select(const ora_layout *L, const float *probs, const float *vnorm,
         free(e);
         /* safeguard: an empty pool row keeps its best key block */
         for (int h = 0; h < nh; ++h) {
-            if (!low[(long)b * nh + h]) continue;
+            if (pool_of[(long)b * nh + h] != g) continue;
             long bh = (long)b * nh + h;
             for (int i = 0; i < Cq; ++i) {
                 uint8_t *m = mask + (bh * Cq + i) * (long)Ck;
@@ -544,9 +551,45 @@ void ora_eg_select(const ora_layout *L, const float *probs, const float *vnorm,
                 m[best] = 1;
             }
         }
-    }
+      }
 }
 
+/* EG-Sparse: the low-entropy heads of every batch entry form one pool, the
+ * other heads stay per-row. */
+void ora_eg_select(const ora_layout *L, const float *probs, const float *vnorm,
+                   const float *top_p, float pool_p, const uint8_t *low, uint8_t *mask)
+{
+    const long BH = (long)L->batch * L->heads;
+    int8_t *pool_of = (int8_t *)malloc((size_t)BH);
+    for (long r = 0; r < BH; ++r) pool_of[r] = low[r] ? 0 : -1;
+    ora_pool_select(L, probs, vnorm, top_p, pool_p, pool_of, 1, mask);
+    free(pool_of);
+}
+
+/* The competition domains of [p3] s3 as pools: 0 per-row local (no pools),
+ * 1 per-head global (pool h = head h), 2 grouped cross-head (the low-entropy
+ * heads pool 0, the rest pool 1), 3 all-head global (one pool), 4 EG-Sparse
+ * (the low-entropy heads pool 0, the rest per-row).  pool_of int8 [B,H];
+ * returns G, the pools per batch entry. */
+int ora_domain_route(const ora_layout *L, const double *H, int domain, int8_t *pool_of)
+{
+    const long BH = (long)L->batch * L->heads;
+    uint8_t *low = (uint8_t *)malloc((size_t)BH);
+    ora_eg_route(L, H, low);
+    int G = 0;
+    for (long r = 0; r < BH; ++r) {
+        const int h = (int)(r % L->heads);
+        switch (domain) {
+            case 1: pool_of[r] = (int8_t)h; G = L->heads; break;
+            case 2: pool_of[r] = low[r] ? 0 : 1; G = 2; break;
+            case 3: pool_of[r] = 0; G = 1; break;
+            case 4: pool_of[r] = low[r] ? 0 : -1; G = 1; break;
+            default: pool_of[r] = -1; G = 0; break;
+        }
+    }
+    free(low);
+    return G;
+}
 /*
  * ---------------------------------------------------------------------------
  * Importance sampling with inverse-inclusion-probability weights ([p5] TL;DR

@@ -65,6 +65,10 @@ MUTATIONS = [
      "if (ora_dhp_l[x] < ora_dhp_l[y]) return 1;"),
     ("opportunity cost from the sink alone",
      "l[h] = alpha[h * 3] > alpha[h * 3 + 1] ? alpha[h * 3] : alpha[h * 3 + 1];", "l[h] = alpha[h * 3];"),
+    ("grouped domain pools swapped", "case 2: pool_of[r] = low[r] ? 0 : 1; G = 2; break;",
+     "case 2: pool_of[r] = low[r] ? 1 : 0; G = 2; break;"),
+    ("per-head domain in one pool", "case 1: pool_of[r] = (int8_t)h; G = L->heads; break;",
+     "case 1: pool_of[r] = 0; G = L->heads; break;"),
     ("distortion without the row renormalisation", "om = z > 0.0 ? om / z : 0.0;",
      "om = z > 0.0 ? om : 0.0;"),
     ("queries from the first frame", "for (int t = (F - 1) * T; t < F * T; t += query_stride) {",

@@ -899,6 +899,69 @@ def test_centroid_distortion(ora):
     check_centroid_distortion(ora)
 
 
+def check_domains(ora):
+    # routing of the four competition domains (and EG-Sparse) by the median split
+    L = lay(seq_len=16, seq_pad=16, bq=4, bk=4, heads=4, batch=2)
+    H = np.array([[0.3, 0.1, 0.5, 0.2], [0.9, 0.8, 0.1, 0.2]])
+    po, G = ora.domain_route(L, H, 0)
+    assert G == 0 and (po == -1).all()
+    po, G = ora.domain_route(L, H, 1)
+    assert G == 4 and po.tolist() == [[0, 1, 2, 3], [0, 1, 2, 3]]
+    po, G = ora.domain_route(L, H, 2)
+    assert G == 2 and po.tolist() == [[1, 0, 1, 0], [1, 1, 0, 0]]
+    po, G = ora.domain_route(L, H, 3)
+    assert G == 1 and (po == 0).all()
+    po, G = ora.domain_route(L, H, 4)
+    assert G == 1 and po.tolist() == [[-1, 0, -1, 0], [-1, -1, 0, 0]]
+    rng = np.random.default_rng(61)
+    # per-head global over a single query block is the per-row rule at p = pool_p (a dyadic
+    # row sums to exactly one, so the pool's target is pool_p itself)
+    L1 = lay(seq_len=16, seq_pad=16, bq=16, bk=4, heads=3)
+    P = (rng.integers(1, 9, size=(1, 3, 1, 4)).astype(np.float64))
+    P = (P / P.sum(-1, keepdims=True))
+    P = (np.round(P * 64) / 64)
+    P[..., -1] = 1 - P[..., :-1].sum(-1)
+    P = P.astype(np.float32)
+    for pp in (0.3, 0.5, 0.8, 1.0):
+        m = ora.pool_select(L1, P, None, [0.5] * 3, pp, np.array([[0, 1, 2]], np.int8), 3)
+        ref, _ = ora.topp(L1, P, [pp] * 3)
+        assert np.array_equal(m, ref), pp
+    # with one head, all-head global and per-head global are the same pool
+    L2 = lay(seq_len=16, seq_pad=16, bq=8, bk=4, heads=1)
+    assert ora.domain_route(L2, np.array([[0.4]]), 3) == (np.zeros((1, 1), np.int8), 1) or \
+        np.array_equal(ora.domain_route(L2, np.array([[0.4]]), 3)[0], ora.domain_route(L2, np.array([[0.4]]), 1)[0])
+    # brute force: every pool of the grouped domain keeps the heaviest shortest prefix of its
+    # own pairs (two pools of two heads, one query block of three key blocks each)
+    L3 = lay(seq_len=12, seq_pad=12, bq=12, bk=4, heads=4)
+    P3 = _tiny_probs(rng, 1, 4, 1, 3)
+    vn = (1 + rng.random((1, 4, 3))).astype(np.float32)
+    po = np.array([[0, 1, 1, 0]], np.int8)
+    for pp in (0.4, 0.75, 0.95):
+        m = ora.pool_select(L3, P3, vn, [0.5] * 4, pp, po, 2)
+        for g in (0, 1):
+            hs = [h for h in range(4) if po[0, h] == g]
+            I = np.array([np.float32(P3[0, h, 0, j] * vn[0, h, j]) for h in hs for j in range(3)])
+            keep = _brute_pool(I, np.float64(np.float32(pp)) * I.astype(np.float64).sum())
+            for r, h in enumerate(hs):   # the safeguard: an emptied row keeps its best block
+                if not any(3 * r + j in keep for j in range(3)):
+                    keep.add(3 * r + int(np.argmax(I[3 * r:3 * r + 3])))
+            got = {n for n, (h, j) in enumerate((h, j) for h in hs for j in range(3)) if m[0, h, 0, j]}
+            assert got == keep, (pp, g, got, keep)
+    # EG-Sparse is the grouped domain with the high-entropy pool left per-row
+    Hh = np.array([[0.2, 0.9, 0.7, 0.1]])
+    po_g, _ = ora.domain_route(L3, Hh, 2)
+    po_e, _ = ora.domain_route(L3, Hh, 4)
+    mg = ora.pool_select(L3, P3, vn, [0.5] * 4, 0.8, po_g, 2)
+    me = ora.pool_select(L3, P3, vn, [0.5] * 4, 0.8, po_e, 1)
+    low = po_e[0] == 0
+    assert np.array_equal(mg[0, low], me[0, low])
+    assert np.array_equal(me, ora.eg_select(L3, P3, vn, [0.5] * 4, 0.8, (po_e == 0).astype(np.uint8)))
+
+
+def test_domains(ora):
+    check_domains(ora)
+
+
 def test_eg_value_norms(ora):
     check_value_norms(ora)
 
@@ -916,4 +979,4 @@ ALL_CHECKS = [check_geometry, check_pooling, check_scores, check_entropy, check_
               check_eg_route, check_eg_select, check_splitmix64, check_inclusion_law,
               check_sample_frequencies, check_sampled_attention_unbiased,
               check_sampled_degenerate, check_subclusters, check_scores_clustered, check_dhp,
-              check_frame_scores, check_centroid_distortion]
+              check_frame_scores, check_centroid_distortion, check_domains]
