@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-profile", action="store_true",
                     help="skip the head-profiling context measurement")
+    ap.add_argument("--no-domains", action="store_true",
+                    help="skip the competition-domain context measurement")
     ap.add_argument("--selection", default="top_p", choices=["top_p", "eg", "sampled"],
                     help="per-row top-p (bsa_build_mask), entropy-guided grouped selection "
                          "(bsa_value_norms + bsa_build_mask_eg), or importance sampling with "
@@ -440,6 +442,38 @@ def our_arm(args, w):
                       pooled_heads=int(low.sum().item()),
                       call="bsa_value_norms + bsa_build_mask_eg on the step's P'")
 
+    # the pooled selection over each competition domain for context (not part of the step):
+    # bsa_build_mask_domain on the step's P' and value norms
+    domains_ctx = None
+    if not args.no_domains:
+        if not eg:
+            bsa.value_norms(w, v, vnorm, stream=stream)
+        domains_ctx = {}
+        pool_of = torch.empty((B, H), dtype=torch.int8, device=dev)
+        for dname, dom in (("per_row", bsa.DOMAIN_ROW), ("per_head", bsa.DOMAIN_HEAD),
+                           ("grouped", bsa.DOMAIN_GROUPED), ("all_head", bsa.DOMAIN_ALL),
+                           ("eg_sparse", bsa.DOMAIN_EG)):
+            ws_d = torch.empty(bsa.domain_workspace_bytes(w, dom), dtype=torch.uint8, device=dev)
+
+            def run_domain():
+                bsa.build_mask_domain(w, dom, probs, vnorm, top_p, pool_p, w.flags, 1e-8, mask,
+                                      kv_index, kv_count, ws_d, stream=stream, entropy=ent,
+                                      entropy_norm=ent_n, pool_of=pool_of)
+            for _ in range(2):
+                run_domain()
+            a, b = ev(), ev()
+            a.record(stream)
+            ne = max(3, args.steps)
+            for _ in range(ne):
+                run_domain()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            domains_ctx[dname] = dict(ms=a.elapsed_time(b) / ne,
+                                      density=int(kv_count.sum().item()) / float(B * H * Cq * Ck),
+                                      pooled_heads=int((pool_of >= 0).sum().item()))
+            del ws_d
+        domains_ctx["call"] = "bsa_build_mask_domain on the step's P' and value norms, pool_p %.4g" % pool_p
+
     # head profiling of autoregressive generation for context (not part of the step): frame
     # attention scores on a Self Forcing-shaped key window (sink + 3 neighbors + current frame),
     # then Dynamic Head Programming on the host
@@ -523,6 +557,7 @@ def our_arm(args, w):
                   frac_hbm=bytes_mask / (np.mean(ms_mask) * 1e-3) / 1e9 / hbm),
         dense=dense,
         eg_selection=eg_ctx,
+        competition_domains=domains_ctx,
         head_profiling=prof,
         roofline=dict(bound="tensor", kernel="attn_kernel", achieved=achieved, peak=peak,
                       unit="TFLOP/s", frac=achieved / peak, peak_source=peak_note,

@@ -101,6 +101,11 @@ def load():
         L.bsa_attention_fwd_weighted.restype = ctypes.c_int
         L.bsa_build_mask_eg_workspace_bytes.argtypes = [lp]
         L.bsa_build_mask_eg_workspace_bytes.restype = ctypes.c_size_t
+        L.bsa_build_mask_domain.argtypes = [lp, ctypes.c_int, vp, vp, vp, ctypes.c_float, ctypes.c_uint32,
+                                            ctypes.c_float, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.bsa_build_mask_domain.restype = ctypes.c_int
+        L.bsa_build_mask_domain_workspace_bytes.argtypes = [lp, ctypes.c_int]
+        L.bsa_build_mask_domain_workspace_bytes.restype = ctypes.c_size_t
         L.bsa_status_string.argtypes = [ctypes.c_int]
         L.bsa_status_string.restype = ctypes.c_char_p
         L.bsa_version.restype = ctypes.c_int
@@ -238,22 +243,16 @@ def eg_workspace_bytes(layout):
     return int(load().bsa_build_mask_eg_workspace_bytes(ctypes.byref(L)))
 
 
-def build_mask_eg(layout, probs, vnorm, top_p, pool_p, flags, eps=1e-8, mask=None,
-                  kv_index=None, kv_count=None, workspace=None, with_mask=True, stream=None,
-                  entropy=None, entropy_norm=None, low_heads=None):
-    """bsa_build_mask_eg (entropy-guided grouped cross-head selection): returns
-    dict(mask, kv_index, kv_count, entropy, entropy_norm, low_heads).  vnorm None
-    ranks the pools by P' alone."""
+# Competition domains (enum bsa_domain).
+DOMAIN_ROW, DOMAIN_HEAD, DOMAIN_GROUPED, DOMAIN_ALL, DOMAIN_EG = 0, 1, 2, 3, 4
+
+
+def domain_workspace_bytes(layout, domain):
     L = make_layout(layout)
-    d = dims(L)
-    _need(probs, "probs", torch.float32, (d["B"], d["H"], d["Cq"], d["Ck"]))
-    if vnorm is not None:
-        _need(vnorm, "vnorm", torch.float32, (d["B"], d["H"], d["Ck"]))
-    dev = probs.device
-    vals = list(top_p) if hasattr(top_p, "__len__") else [top_p] * d["H"]
-    if len(vals) != d["H"]:
-        raise ValueError("top_p needs one value per head")
-    tp = (ctypes.c_float * d["H"])(*[float(x) for x in vals])
+    return int(load().bsa_build_mask_domain_workspace_bytes(ctypes.byref(L), int(domain)))
+
+
+def _pooled_outputs(d, dev, mask, kv_index, kv_count, entropy, entropy_norm, with_mask):
     if mask is None and with_mask:
         mask = torch.empty((d["B"], d["H"], d["Cq"], d["Ck"]), dtype=torch.uint8, device=dev)
     if kv_index is None:
@@ -264,11 +263,36 @@ def build_mask_eg(layout, probs, vnorm, top_p, pool_p, flags, eps=1e-8, mask=Non
         entropy = torch.empty((d["B"], d["H"]), dtype=torch.float32, device=dev)
     if entropy_norm is None:
         entropy_norm = torch.empty((d["B"], d["H"]), dtype=torch.float32, device=dev)
+    _need(entropy, "entropy", torch.float32, (d["B"], d["H"]))
+    _need(entropy_norm, "entropy_norm", torch.float32, (d["B"], d["H"]))
+    return mask, kv_index, kv_count, entropy, entropy_norm
+
+
+def _pooled_inputs(L, probs, vnorm, top_p):
+    d = dims(L)
+    _need(probs, "probs", torch.float32, (d["B"], d["H"], d["Cq"], d["Ck"]))
+    if vnorm is not None:
+        _need(vnorm, "vnorm", torch.float32, (d["B"], d["H"], d["Ck"]))
+    vals = list(top_p) if hasattr(top_p, "__len__") else [top_p] * d["H"]
+    if len(vals) != d["H"]:
+        raise ValueError("top_p needs one value per head")
+    return d, (ctypes.c_float * d["H"])(*[float(x) for x in vals])
+
+
+def build_mask_eg(layout, probs, vnorm, top_p, pool_p, flags, eps=1e-8, mask=None,
+                  kv_index=None, kv_count=None, workspace=None, with_mask=True, stream=None,
+                  entropy=None, entropy_norm=None, low_heads=None):
+    """bsa_build_mask_eg (entropy-guided grouped cross-head selection): returns
+    dict(mask, kv_index, kv_count, entropy, entropy_norm, low_heads).  vnorm None
+    ranks the pools by P' alone."""
+    L = make_layout(layout)
+    d, tp = _pooled_inputs(L, probs, vnorm, top_p)
+    dev = probs.device
+    mask, kv_index, kv_count, entropy, entropy_norm = _pooled_outputs(
+        d, dev, mask, kv_index, kv_count, entropy, entropy_norm, with_mask)
     low = low_heads
     if low is None:
         low = torch.empty((d["B"], d["H"]), dtype=torch.uint8, device=dev)
-    _need(entropy, "entropy", torch.float32, (d["B"], d["H"]))
-    _need(entropy_norm, "entropy_norm", torch.float32, (d["B"], d["H"]))
     _need(low, "low_heads", torch.uint8, (d["B"], d["H"]))
     if workspace is None:
         workspace = torch.empty(eg_workspace_bytes(L), dtype=torch.uint8, device=dev)
@@ -280,6 +304,34 @@ def build_mask_eg(layout, probs, vnorm, top_p, pool_p, flags, eps=1e-8, mask=Non
     _check("bsa_build_mask_eg", rc)
     return dict(mask=mask, kv_index=kv_index, kv_count=kv_count, entropy=entropy,
                 entropy_norm=entropy_norm, low_heads=low)
+
+
+def build_mask_domain(layout, domain, probs, vnorm, top_p, pool_p, flags, eps=1e-8, mask=None,
+                      kv_index=None, kv_count=None, workspace=None, with_mask=True, stream=None,
+                      entropy=None, entropy_norm=None, pool_of=None):
+    """bsa_build_mask_domain (pooled top-p over a competition domain, DOMAIN_*):
+    returns dict(mask, kv_index, kv_count, entropy, entropy_norm, pool_of)."""
+    L = make_layout(layout)
+    d, tp = _pooled_inputs(L, probs, vnorm, top_p)
+    dev = probs.device
+    mask, kv_index, kv_count, entropy, entropy_norm = _pooled_outputs(
+        d, dev, mask, kv_index, kv_count, entropy, entropy_norm, with_mask)
+    if pool_of is None:
+        pool_of = torch.empty((d["B"], d["H"]), dtype=torch.int8, device=dev)
+    _need(pool_of, "pool_of", torch.int8, (d["B"], d["H"]))
+    if workspace is None:
+        n = domain_workspace_bytes(L, domain)
+        if n == 0:
+            raise BsaError("bsa_build_mask_domain", BSA_ERR_INVALID_ARG)
+        workspace = torch.empty(n, dtype=torch.uint8, device=dev)
+    rc = load().bsa_build_mask_domain(ctypes.byref(L), int(domain), _ptr(probs), _ptr(vnorm),
+                                      ctypes.cast(tp, ctypes.c_void_p), float(pool_p), int(flags),
+                                      float(eps), _ptr(mask), _ptr(kv_index), _ptr(kv_count),
+                                      _ptr(entropy), _ptr(entropy_norm), _ptr(pool_of),
+                                      _ptr(workspace), _stream(stream))
+    _check("bsa_build_mask_domain", rc)
+    return dict(mask=mask, kv_index=kv_index, kv_count=kv_count, entropy=entropy,
+                entropy_norm=entropy_norm, pool_of=pool_of)
 
 
 def attention_workspace_bytes(layout):

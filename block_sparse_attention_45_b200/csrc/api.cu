@@ -193,15 +193,12 @@ int bsa_value_norms(const bsa_layout *layout, const void *v, float *vnorm, void 
     return launch_status(bsa::launch_value_norms(g, v, vnorm, static_cast<cudaStream_t>(stream)));
 }
 
-size_t bsa_build_mask_eg_workspace_bytes(const bsa_layout *layout) {
-    if (check_layout(layout) != BSA_OK) return 0;
-    return bsa::eg_workspace(bsa::make_geometry(*layout)).bytes;
-}
-
-int bsa_build_mask_eg(const bsa_layout *layout, const float *probs, const float *vnorm,
-                      const float *top_p, float pool_p, uint32_t flags, float eps, uint8_t *mask,
-                      int32_t *kv_index, int32_t *kv_count, float *entropy, float *entropy_norm,
-                      uint8_t *low_heads, void *workspace, void *stream) {
+// The pooled selections: bsa_build_mask_eg and bsa_build_mask_domain.
+static int build_mask_pooled(const bsa_layout *layout, int domain, const float *probs,
+                             const float *vnorm, const float *top_p, float pool_p, uint32_t flags,
+                             float eps, uint8_t *mask, int32_t *kv_index, int32_t *kv_count,
+                             float *entropy, float *entropy_norm, uint8_t *low_heads, int8_t *pool_of,
+                             void *workspace, void *stream) {
     int rc = check_layout(layout);
     if (rc != BSA_OK) return rc;
     if (!probs || !top_p || !kv_index || !kv_count || !workspace) return BSA_ERR_INVALID_ARG;
@@ -220,13 +217,42 @@ int bsa_build_mask_eg(const bsa_layout *layout, const float *probs, const float 
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    rc = launch_status(bsa::launch_eg_prepare(g, probs, vnorm, pool_p, eps, entropy, entropy_norm,
-                                              low_heads, ws, st));
+    rc = launch_status(bsa::launch_eg_prepare(g, domain, probs, vnorm, pool_p, eps, entropy, entropy_norm,
+                                              low_heads, pool_of, ws, st));
     if (rc != BSA_OK) return rc;
-    const bsa::EgWorkspace w = bsa::eg_workspace(g);
+    const bsa::EgWorkspace w = bsa::eg_workspace(g, domain);
     return launch_status(bsa::launch_mask_eg(
-        g, probs, vnorm, tp, flags, mask, kv_index, kv_count, ws + w.low,
-        reinterpret_cast<const bsa::PoolState *>(ws + w.state), st));
+        g, probs, vnorm, tp, flags, mask, kv_index, kv_count, reinterpret_cast<const int8_t *>(ws + w.pool_of),
+        bsa::eg_pools(g.H, domain), reinterpret_cast<const bsa::PoolState *>(ws + w.state), st));
+}
+
+static bool valid_domain(int domain) { return domain >= BSA_DOMAIN_ROW && domain <= BSA_DOMAIN_EG; }
+
+size_t bsa_build_mask_eg_workspace_bytes(const bsa_layout *layout) {
+    return bsa_build_mask_domain_workspace_bytes(layout, BSA_DOMAIN_EG);
+}
+
+size_t bsa_build_mask_domain_workspace_bytes(const bsa_layout *layout, int domain) {
+    if (check_layout(layout) != BSA_OK || !valid_domain(domain)) return 0;
+    return bsa::eg_workspace(bsa::make_geometry(*layout), domain).bytes;
+}
+
+int bsa_build_mask_eg(const bsa_layout *layout, const float *probs, const float *vnorm,
+                      const float *top_p, float pool_p, uint32_t flags, float eps, uint8_t *mask,
+                      int32_t *kv_index, int32_t *kv_count, float *entropy, float *entropy_norm,
+                      uint8_t *low_heads, void *workspace, void *stream) {
+    return build_mask_pooled(layout, BSA_DOMAIN_EG, probs, vnorm, top_p, pool_p, flags, eps, mask, kv_index,
+                             kv_count, entropy, entropy_norm, low_heads, nullptr, workspace, stream);
+}
+
+int bsa_build_mask_domain(const bsa_layout *layout, int domain, const float *probs,
+                          const float *vnorm, const float *top_p, float pool_p, uint32_t flags,
+                          float eps, uint8_t *mask, int32_t *kv_index, int32_t *kv_count,
+                          float *entropy, float *entropy_norm, int8_t *pool_of, void *workspace,
+                          void *stream) {
+    if (!valid_domain(domain)) return BSA_ERR_INVALID_ARG;
+    return build_mask_pooled(layout, domain, probs, vnorm, top_p, pool_p, flags, eps, mask, kv_index,
+                             kv_count, entropy, entropy_norm, nullptr, pool_of, workspace, stream);
 }
 
 size_t bsa_attention_workspace_bytes(const bsa_layout *layout) {

@@ -117,12 +117,12 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // Called by every thread after its last global write: true in the one CTA of
-// the grid that finishes last, which then sees every other CTA's writes.
-__device__ bool last_cta(unsigned int *counter) {
+// the `total` that share `counter` to finish last, which then sees the others' writes.
+__device__ bool last_cta(unsigned int *counter, unsigned int total) {
     __shared__ int s_last;
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicAdd(counter, 1u) == gridDim.x - 1 ? 1 : 0;
+    if (threadIdx.x == 0) s_last = atomicAdd(counter, 1u) == total - 1 ? 1 : 0;
     __syncthreads();
     const bool last = s_last != 0;
     if (last) __threadfence();
@@ -281,13 +281,16 @@ struct EgArgs {
     float *heads_h;         // [B,H]
     float *entropy;         // [B,H] or nullptr (caller's)
     float *entropy_norm;    // [B,H] or nullptr (caller's)
-    uint8_t *low;           // [B,H]
-    uint8_t *low_out;       // [B,H] or nullptr (caller's)
-    int *pool_heads;        // [B,H]: the pooled heads of b in ascending order
+    int8_t *pool_of;        // [B,H]: the head's pool, -1 = per-row
+    uint8_t *low_out;       // [B,H] or nullptr (caller's): 1 for pooled heads
+    int8_t *pool_out;       // [B,H] or nullptr (caller's): copy of pool_of
+    int *pool_heads;        // [B,G,H]: the heads of pool (b, g) in ascending order
+    int *pool_nh;           // [B,G]: their number
+    int G, domain;          // pools per batch entry, competition domain
     unsigned long long *hist1;  // [B,H,256,2]
-    unsigned long long *hist;   // [B,4096,2]
+    unsigned long long *hist;   // [B,G,4096,2]
     int *tiecnt;            // [B,H,C_q]
-    PoolState *state;       // [B]
+    PoolState *state;       // [B,G]
     unsigned int *counter;  // this launch's finish counter
     int B, H, Cq, Ck;
     int ctas;               // CTAs per head (level 1) or per batch entry (later passes)
@@ -318,6 +321,7 @@ __global__ void __launch_bounds__(kThreads) entropy_level1_kernel(EgArgs a) {
     __shared__ double s_wsum[kWarps];
     __shared__ float s_h[kMaxHeads];
     __shared__ int s_heads[kMaxHeads];
+    __shared__ int s_np;
     const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
     __shared__ int s_zero;
     {
@@ -379,9 +383,9 @@ __global__ void __launch_bounds__(kThreads) entropy_level1_kernel(EgArgs a) {
             a.ent_part[bh * a.ctas + part] = cs;
         }
     }
-    if (!last_cta(a.counter)) return;
+    if (!last_cta(a.counter, gridDim.x)) return;
 
-    // ---- the last CTA: per-head means, median split, level-1 pick per batch entry
+    // ---- the last CTA: per-head means, the domain's pools, level-1 pick per pool
     const long long BH = static_cast<long long>(a.B) * a.H;
     for (long long bh = wid; bh < BH; bh += kWarps) {
         double s = 0.0;  // fixed order: part-strided per lane, then a butterfly; lane 0's sum
@@ -398,12 +402,13 @@ __global__ void __launch_bounds__(kThreads) entropy_level1_kernel(EgArgs a) {
     __syncthreads();
     uint32_t *cnt = sh;  // reuse: [256] counts, then [256] u64 sums
     unsigned long long *sum = reinterpret_cast<unsigned long long *>(sh + 2 * kL1Bins);
-    const int H = a.H, np = H / 2;
+    const int H = a.H, G = a.G;
     for (int b = 0; b < a.B; ++b) {
         for (int h = threadIdx.x; h < H; h += kThreads) s_h[h] = a.heads_h[static_cast<long long>(b) * H + h];
         __syncthreads();
-        // heads ordered by (H_h asc, h asc); the first floor(H/2) are pooled.  The
-        // ranks form a permutation even for NaN entropies (ordered last).
+        // The domain's pool of every head.  The grouped and entropy-guided domains split at
+        // the median: heads ordered by (H_h asc, h asc), the first floor(H/2) are the
+        // low-entropy ones; the ranks form a permutation even for NaN entropies.
         for (int h = threadIdx.x; h < H; h += kThreads) {
             const uint32_t x = order_key(s_h[h]);
             int rank = 0;
@@ -411,64 +416,77 @@ __global__ void __launch_bounds__(kThreads) entropy_level1_kernel(EgArgs a) {
                 const uint32_t y = order_key(s_h[o]);
                 rank += (y < x || (y == x && o < h)) ? 1 : 0;
             }
-            const uint8_t l = rank < np ? 1 : 0;
-            a.low[static_cast<long long>(b) * H + h] = l;
-            if (a.low_out) a.low_out[static_cast<long long>(b) * H + h] = l;
-            s_heads[h] = l;  // flag for now, list below
-        }
-        if (threadIdx.x == 0) {
-            PoolState z;
-            z.target = 0.0;
-            z.above = 0.0;
-            z.pad2 = 0;
-            z.pre = 0;
-            z.shift = 31;  // level 1 bins bits 30..23 of scores >= 0 (bit 31 is 0)
-            z.keep_all = 0;
-            z.empty = np == 0;
-            z.ucut = 0;
-            z.pad0 = 0;
-            z.need = 0;
-            z.cut_row = -1;
-            z.cut_rank = 0;
-            z.pad1 = 0;
-            s_st = z;
+            const bool lowh = rank < H / 2;
+            int pool;
+            switch (a.domain) {
+                case BSA_DOMAIN_HEAD: pool = h; break;
+                case BSA_DOMAIN_GROUPED: pool = lowh ? 0 : 1; break;
+                case BSA_DOMAIN_ALL: pool = 0; break;
+                case BSA_DOMAIN_EG: pool = lowh ? 0 : -1; break;
+                default: pool = -1; break;
+            }
+            const long long bh = static_cast<long long>(b) * H + h;
+            a.pool_of[bh] = static_cast<int8_t>(pool);
+            if (a.low_out) a.low_out[bh] = pool >= 0 ? 1 : 0;
+            if (a.pool_out) a.pool_out[bh] = static_cast<int8_t>(pool);
         }
         __syncthreads();
-        if (threadIdx.x == 0) {  // flags -> ascending list of pooled heads
-            int k = 0;
-            for (int h = 0; h < H; ++h)
-                if (s_heads[h]) s_heads[k++] = h;
-        }
-        __syncthreads();
-        for (int k = threadIdx.x; k < np; k += kThreads) a.pool_heads[static_cast<long long>(b) * H + k] = s_heads[k];
-        if (!s_st.empty) {
-            const int t = threadIdx.x;  // bin t over the pooled heads, loads 8 heads at a time
-            unsigned long long c = 0, s = 0;
-            for (int k0 = 0; k0 < np; k0 += 8) {
-                unsigned long long cc[8], ss[8];
+        for (int g = 0; g < G; ++g) {
+            const long long bp = static_cast<long long>(b) * G + g;
+            if (threadIdx.x == 0) {  // the pool's heads, ascending
+                int k = 0;
+                for (int h = 0; h < H; ++h)
+                    if (a.pool_of[static_cast<long long>(b) * H + h] == g) s_heads[k++] = h;
+                s_np = k;
+                PoolState z;
+                z.target = 0.0;
+                z.above = 0.0;
+                z.pad2 = 0;
+                z.pre = 0;
+                z.shift = 31;  // level 1 bins bits 30..23 of scores >= 0 (bit 31 is 0)
+                z.keep_all = 0;
+                z.empty = k == 0;
+                z.ucut = 0;
+                z.pad0 = 0;
+                z.need = 0;
+                z.cut_row = -1;
+                z.cut_rank = 0;
+                z.pad1 = 0;
+                s_st = z;
+                a.pool_nh[bp] = k;
+            }
+            __syncthreads();
+            const int np = s_np;
+            for (int k = threadIdx.x; k < np; k += kThreads) a.pool_heads[bp * H + k] = s_heads[k];
+            if (!s_st.empty) {
+                const int t = threadIdx.x;  // bin t over the pool's heads, loads 8 heads at a time
+                unsigned long long c = 0, s = 0;
+                for (int k0 = 0; k0 < np; k0 += 8) {
+                    unsigned long long cc[8], ss[8];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    cc[q] = ss[q] = 0ull;
-                    if (k0 + q < np) {
-                        const unsigned long long *g =
-                            a.hist1 + ((static_cast<long long>(b) * H + s_heads[k0 + q]) * kL1Bins + t) * 2;
-                        cc[q] = __ldcg(g);
-                        ss[q] = __ldcg(g + 1);
+                    for (int q = 0; q < 8; ++q) {
+                        cc[q] = ss[q] = 0ull;
+                        if (k0 + q < np) {
+                            const unsigned long long *gp =
+                                a.hist1 + ((static_cast<long long>(b) * H + s_heads[k0 + q]) * kL1Bins + t) * 2;
+                            cc[q] = __ldcg(gp);
+                            ss[q] = __ldcg(gp + 1);
+                        }
+                    }
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        c += cc[q];
+                        s += ss[q];
                     }
                 }
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    c += cc[q];
-                    s += ss[q];
-                }
+                cnt[t] = static_cast<uint32_t>(c);
+                sum[t] = s;
+                __syncthreads();
+                cta_pick(cnt, sum, 8, true, a.pool_p, s_st, sc);
             }
-            cnt[t] = static_cast<uint32_t>(c);
-            sum[t] = s;
+            if (threadIdx.x == 0) a.state[bp] = s_st;
             __syncthreads();
-            cta_pick(cnt, sum, 8, true, a.pool_p, s_st, sc);
         }
-        if (threadIdx.x == 0) a.state[b] = s_st;
-        __syncthreads();
     }
 }
 
@@ -493,21 +511,23 @@ __global__ void __launch_bounds__(kThreads) pool_level_kernel(EgArgs a) {
     __shared__ int s_heads[kMaxHeads];
     const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
     {
-        const int b = blockIdx.x / a.ctas, part = blockIdx.x % a.ctas;
-        const PoolState st = a.state[b];
+        const int bp = blockIdx.x / a.ctas, part = blockIdx.x % a.ctas;
+        const int b = bp / a.G;
+        const PoolState st = a.state[bp];
         if (pool_active(st) && st.shift >= NBITS) {
             uint32_t *c = sh, *lo = sh + nb, *hi = sh + 2 * nb;
             for (int k = threadIdx.x; k < 3 * nb; k += kThreads) sh[k] = 0u;
             if (threadIdx.x == 0) s_zero = 0;
             bool zero = false;
-            for (int k = threadIdx.x; k < a.H / 2; k += kThreads)
-                s_heads[k] = a.pool_heads[static_cast<long long>(b) * a.H + k];
+            const int np = a.pool_nh[bp];
+            for (int k = threadIdx.x; k < np; k += kThreads)
+                s_heads[k] = a.pool_heads[static_cast<long long>(bp) * a.H + k];
             __syncthreads();
             const int shift = st.shift, low_bits = st.shift - NBITS;
             const uint32_t pre = st.pre;
             const int Ck = a.Ck;
             long long r0, r1;
-            warp_rows(static_cast<long long>(a.H / 2) * a.Cq, static_cast<long long>(part) * kWarps + wid,
+            warp_rows(static_cast<long long>(np) * a.Cq, static_cast<long long>(part) * kWarps + wid,
                       static_cast<long long>(a.ctas) * kWarps, r0, r1);
             const bool va = a.vnorm != nullptr;
             float vn[VPL];
@@ -544,7 +564,7 @@ __global__ void __launch_bounds__(kThreads) pool_level_kernel(EgArgs a) {
             }
             if (!COUNTS && __any_sync(0xffffffffu, zero) && lane == 0) atomicOr(&s_zero, 1);
             __syncthreads();
-            unsigned long long *g = a.hist + static_cast<long long>(b) * 2 * kMaxBins;
+            unsigned long long *g = a.hist + static_cast<long long>(bp) * 2 * kMaxBins;
             for (int k = threadIdx.x; k < nb; k += kThreads) {
                 const unsigned long long sk = lo[k] + (static_cast<unsigned long long>(hi[k]) << 12);
                 const unsigned long long ck = COUNTS ? c[k] : ((sk || (k == 0 && s_zero)) ? 1ull : 0ull);
@@ -555,36 +575,33 @@ __global__ void __launch_bounds__(kThreads) pool_level_kernel(EgArgs a) {
             }
         }
     }
-    if (!last_cta(a.counter)) return;
-
-    // ---- the last CTA: the pick of every active batch entry
+    // ---- the last CTA of pool bp: its pick
+    const int bp = blockIdx.x / a.ctas;
+    if (!last_cta(a.counter + bp, static_cast<unsigned>(a.ctas))) return;
     uint32_t *cnt = sh;
     unsigned long long *sum = reinterpret_cast<unsigned long long *>(sh + nb);
-    for (int b = 0; b < a.B; ++b) {
-        if (threadIdx.x == 0) s_st = a.state[b];
-        __syncthreads();
-        if (pool_active(s_st) && s_st.shift >= NBITS) {
-            unsigned long long *g = a.hist + static_cast<long long>(b) * 2 * kMaxBins;
-            unsigned long long cc[per], ss[per];
+    if (threadIdx.x == 0) s_st = a.state[bp];
+    __syncthreads();
+    if (pool_active(s_st) && s_st.shift >= NBITS) {
+        unsigned long long *g = a.hist + static_cast<long long>(bp) * 2 * kMaxBins;
+        unsigned long long cc[per], ss[per];
 #pragma unroll
-            for (int q = 0; q < per; ++q) {
-                const int k = threadIdx.x + q * kThreads;
-                cc[q] = __ldcg(&g[2 * k]);
-                ss[q] = __ldcg(&g[2 * k + 1]);
-            }
+        for (int q = 0; q < per; ++q) {
+            const int k = threadIdx.x + q * kThreads;
+            cc[q] = __ldcg(&g[2 * k]);
+            ss[q] = __ldcg(&g[2 * k + 1]);
+        }
 #pragma unroll
-            for (int q = 0; q < per; ++q) {
-                const int k = threadIdx.x + q * kThreads;
-                cnt[k] = static_cast<uint32_t>(cc[q]);
-                sum[k] = ss[q];
-                g[2 * k] = 0ull;  // ready for the next level
-                g[2 * k + 1] = 0ull;
-            }
-            __syncthreads();
-            cta_pick(cnt, sum, NBITS, false, a.pool_p, s_st, sc);
-            if (threadIdx.x == 0) a.state[b] = s_st;
+        for (int q = 0; q < per; ++q) {
+            const int k = threadIdx.x + q * kThreads;
+            cnt[k] = static_cast<uint32_t>(cc[q]);
+            sum[k] = ss[q];
+            g[2 * k] = 0ull;  // ready for the next level
+            g[2 * k + 1] = 0ull;
         }
         __syncthreads();
+        cta_pick(cnt, sum, NBITS, false, a.pool_p, s_st, sc);
+        if (threadIdx.x == 0) a.state[bp] = s_st;
     }
 }
 
@@ -596,13 +613,15 @@ __global__ void __launch_bounds__(kThreads) tie_kernel(EgArgs a) {
     __shared__ ScanScratch sc;
     __shared__ int s_heads[kMaxHeads];
     const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
-    const long long rows = static_cast<long long>(a.H / 2) * a.Cq;
     {
-        const int b = blockIdx.x / a.ctas, part = blockIdx.x % a.ctas;
-        const PoolState st = a.state[b];
+        const int bp = blockIdx.x / a.ctas, part = blockIdx.x % a.ctas;
+        const int b = bp / a.G;
+        const PoolState st = a.state[bp];
+        const int np = a.pool_nh[bp];
+        const long long rows = static_cast<long long>(np) * a.Cq;
         if (pool_active(st) && st.cut_row == -1) {
-            for (int k = threadIdx.x; k < a.H / 2; k += kThreads)
-                s_heads[k] = a.pool_heads[static_cast<long long>(b) * a.H + k];
+            for (int k = threadIdx.x; k < np; k += kThreads)
+                s_heads[k] = a.pool_heads[static_cast<long long>(bp) * a.H + k];
             __syncthreads();
             const int Ck = a.Ck;
             long long r0, r1;
@@ -635,58 +654,58 @@ __global__ void __launch_bounds__(kThreads) tie_kernel(EgArgs a) {
             }
         }
     }
-    if (!last_cta(a.counter)) return;
-
-    // ---- the last CTA: a scan over the pooled rows of each batch entry that needs one
+    // ---- the last CTA of pool bp: a scan over its rows when it needs one
+    const int bp = blockIdx.x / a.ctas;
+    if (!last_cta(a.counter + bp, static_cast<unsigned>(a.ctas))) return;
     const int t = threadIdx.x;
-    for (int b = 0; b < a.B; ++b) {
-        const PoolState st = a.state[b];
-        if (!pool_active(st) || st.cut_row != -1) continue;  // uniform over the CTA
-        for (int k = t; k < a.H / 2; k += kThreads) s_heads[k] = a.pool_heads[static_cast<long long>(b) * a.H + k];
-        if (t == 0) sc.owner = INT_MAX;
-        __syncthreads();
-        const long long per = (rows + kThreads - 1) / kThreads;
-        const long long r0 = min(rows, t * per), r1 = min(rows, r0 + per);
-        unsigned long long n = 0;
-        for (long long r = r0; r < r1; r += 8) {  // 8 loads in flight
+    const int b = bp / a.G;
+    const PoolState st = a.state[bp];
+    if (!pool_active(st) || st.cut_row != -1) return;  // uniform over the CTA
+    const int np = a.pool_nh[bp];
+    const long long rows = static_cast<long long>(np) * a.Cq;
+    for (int k = t; k < np; k += kThreads) s_heads[k] = a.pool_heads[static_cast<long long>(bp) * a.H + k];
+    if (t == 0) sc.owner = INT_MAX;
+    __syncthreads();
+    const long long per = (rows + kThreads - 1) / kThreads;
+    const long long r0 = min(rows, t * per), r1 = min(rows, r0 + per);
+    unsigned long long n = 0;
+    for (long long r = r0; r < r1; r += 8) {  // 8 loads in flight
+        int v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = r + q < r1 ? __ldcg(a.tiecnt + pooled_row(a, s_heads, b, r + q)) : 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) n += static_cast<unsigned long long>(v[q]);
+    }
+    double dm = 0.0;
+    unsigned long long run = n;
+    cta_scan(dm, run, sc);  // inclusive tie counts in thread order
+    if (n > 0 && run >= st.need) atomicMin(&sc.owner, t);
+    __syncthreads();
+    if (t == sc.owner) {
+        unsigned long long acc = run - n;
+        long long cut_row = -1;
+        int cut_rank = 0;
+        for (long long r = r0; r < r1 && cut_row < 0; r += 8) {
             int v[8];
 #pragma unroll
             for (int q = 0; q < 8; ++q) v[q] = r + q < r1 ? __ldcg(a.tiecnt + pooled_row(a, s_heads, b, r + q)) : 0;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) n += static_cast<unsigned long long>(v[q]);
-        }
-        double dm = 0.0;
-        unsigned long long run = n;
-        cta_scan(dm, run, sc);  // inclusive tie counts in thread order
-        if (n > 0 && run >= st.need) atomicMin(&sc.owner, t);
-        __syncthreads();
-        if (t == sc.owner) {
-            unsigned long long acc = run - n;
-            long long cut_row = -1;
-            int cut_rank = 0;
-            for (long long r = r0; r < r1 && cut_row < 0; r += 8) {
-                int v[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) v[q] = r + q < r1 ? __ldcg(a.tiecnt + pooled_row(a, s_heads, b, r + q)) : 0;
-                for (int q = 0; q < 8 && r + q < r1; ++q) {
-                    const unsigned long long c = static_cast<unsigned long long>(v[q]);
-                    if (acc + c >= st.need) {
-                        cut_row = pooled_row(a, s_heads, b, r + q);
-                        cut_rank = static_cast<int>(st.need - acc);
-                        break;
-                    }
-                    acc += c;
+            for (int q = 0; q < 8 && r + q < r1; ++q) {
+                const unsigned long long c = static_cast<unsigned long long>(v[q]);
+                if (acc + c >= st.need) {
+                    cut_row = pooled_row(a, s_heads, b, r + q);
+                    cut_rank = static_cast<int>(st.need - acc);
+                    break;
                 }
+                acc += c;
             }
-            a.state[b].cut_row = cut_row;
-            a.state[b].cut_rank = cut_rank;
         }
-        __syncthreads();
+        a.state[bp].cut_row = cut_row;
+        a.state[bp].cut_rank = cut_rank;
     }
 }
 
 template <int VPL>
-cudaError_t launch_eg_passes(const EgArgs &base, long long c1, long long c2, int B, long long BH,
+cudaError_t launch_eg_passes(const EgArgs &base, long long c1, long long c2, long long pools, long long BH,
                              cudaStream_t st) {
     unsigned int *counters = base.counter;
     EgArgs a = base;
@@ -698,21 +717,22 @@ cudaError_t launch_eg_passes(const EgArgs &base, long long c1, long long c2, int
     if (e != cudaSuccess) return e;
     entropy_level1_kernel<VPL><<<static_cast<unsigned>(BH * c1), kThreads, kL1Smem, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (pools == 0) return cudaSuccess;  // every row per-row: no pool passes
     a.ctas = static_cast<int>(c2);
-    const unsigned grid2 = static_cast<unsigned>(B * c2);
+    const unsigned grid2 = static_cast<unsigned>(pools * c2);
     const size_t smem12 = 3 * (1 << kLevelBits[0]) * sizeof(uint32_t);
     const size_t smem11 = 3 * (1 << kLevelBits[1]) * sizeof(uint32_t);
     if ((e = cudaFuncSetAttribute(pool_level_kernel<VPL, kLevelBits[0], false>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(smem12))) != cudaSuccess)
         return e;
-    a.counter = counters + 1;
+    a.counter = counters + 1;  // then one counter per pool and pass
     pool_level_kernel<VPL, kLevelBits[0], false><<<grid2, kThreads, smem12, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    a.counter = counters + 2;
+    a.counter = counters + 1 + pools;
     pool_level_kernel<VPL, kLevelBits[1], true><<<grid2, kThreads, smem11, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    a.counter = counters + 3;
+    a.counter = counters + 1 + 2 * pools;
     tie_kernel<VPL><<<grid2, kThreads, 0, st>>>(a);
     return cudaGetLastError();
 }
@@ -727,44 +747,69 @@ static_assert(kMaxBins % kThreads == 0 && (1 << kLevelBits[1]) % kThreads == 0, 
 
 }  // namespace
 
-EgWorkspace eg_workspace(const Geometry &g) {
+int eg_pools(int H, int domain) {
+    switch (domain) {
+        case BSA_DOMAIN_HEAD: return H;
+        case BSA_DOMAIN_GROUPED: return 2;
+        case BSA_DOMAIN_ALL: return 1;
+        case BSA_DOMAIN_EG: return 1;
+        default: return 0;
+    }
+}
+
+// Heads in the largest pool of the domain.
+static int eg_max_pool_heads(int H, int domain) {
+    switch (domain) {
+        case BSA_DOMAIN_HEAD: return 1;
+        case BSA_DOMAIN_GROUPED: return H - H / 2;
+        case BSA_DOMAIN_ALL: return H;
+        case BSA_DOMAIN_EG: return H / 2;
+        default: return 0;
+    }
+}
+
+EgWorkspace eg_workspace(const Geometry &g, int domain) {
     const size_t rows = static_cast<size_t>(g.B) * g.H * g.Cq;
     const size_t bh = static_cast<size_t>(g.B) * g.H;
+    const size_t pools = static_cast<size_t>(g.B) * eg_pools(g.H, domain);
     EgWorkspace w;
     size_t off = 0;
     w.ent_part = off;
     off += round256(bh * static_cast<size_t>(eg_level1_ctas_max(g.Cq)) * sizeof(double));
     w.heads_h = off;
     off += round256(bh * sizeof(float));
-    w.low = off;
+    w.pool_of = off;
     off += round256(bh);
     w.pool_heads = off;
-    off += round256(bh * sizeof(int));
+    off += round256(pools * g.H * sizeof(int));
+    w.pool_nh = off;
+    off += round256(pools * sizeof(int));
     w.state = off;
-    off += round256(static_cast<size_t>(g.B) * sizeof(PoolState));
+    off += round256(pools * sizeof(PoolState));
     // zeroed once per call: histograms, tie counts, finish counters
     w.zero_begin = off;
     w.hist1 = off;
     off += round256(bh * kL1Bins * 2 * sizeof(unsigned long long));
     w.hist = off;
-    off += round256(static_cast<size_t>(g.B) * 2 * kMaxBins * sizeof(unsigned long long));
+    off += round256(pools * 2 * kMaxBins * sizeof(unsigned long long));
     w.tiecnt = off;
     off += round256(rows * sizeof(int));
     w.counters = off;
-    off += round256(4 * sizeof(unsigned int));
+    off += round256((1 + 3 * pools) * sizeof(unsigned int));
     w.zero_bytes = off - w.zero_begin;
     w.bytes = off;
     return w;
 }
 
-cudaError_t launch_eg_prepare(const Geometry &g, const float *probs, const float *vnorm,
+cudaError_t launch_eg_prepare(const Geometry &g, int domain, const float *probs, const float *vnorm,
                               float pool_p, float eps, float *entropy, float *entropy_norm,
-                              uint8_t *low_heads, uint8_t *workspace, cudaStream_t st) {
-    const EgWorkspace w = eg_workspace(g);
+                              uint8_t *low_heads, int8_t *pool_out, uint8_t *workspace, cudaStream_t st) {
+    const EgWorkspace w = eg_workspace(g, domain);
     cudaError_t e = cudaMemsetAsync(workspace + w.zero_begin, 0, w.zero_bytes, st);
     if (e != cudaSuccess) return e;
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorInvalidValue;
+    const int G = eg_pools(g.H, domain);
 
     EgArgs a;
     a.probs = probs;
@@ -773,9 +818,13 @@ cudaError_t launch_eg_prepare(const Geometry &g, const float *probs, const float
     a.heads_h = reinterpret_cast<float *>(workspace + w.heads_h);
     a.entropy = entropy;
     a.entropy_norm = entropy_norm;
-    a.low = workspace + w.low;
+    a.pool_of = reinterpret_cast<int8_t *>(workspace + w.pool_of);
     a.low_out = low_heads;
+    a.pool_out = pool_out;
     a.pool_heads = reinterpret_cast<int *>(workspace + w.pool_heads);
+    a.pool_nh = reinterpret_cast<int *>(workspace + w.pool_nh);
+    a.G = G;
+    a.domain = domain;
     a.hist1 = reinterpret_cast<unsigned long long *>(workspace + w.hist1);
     a.hist = reinterpret_cast<unsigned long long *>(workspace + w.hist);
     a.tiecnt = reinterpret_cast<int *>(workspace + w.tiecnt);
@@ -796,20 +845,23 @@ cudaError_t launch_eg_prepare(const Geometry &g, const float *probs, const float
     const long long rows_cap = static_cast<long long>(kBinCap / static_cast<uint32_t>(g.Ck)) * kWarps;
     const long long c1 = max((static_cast<long long>(g.Cq) + rows_cap - 1) / rows_cap,
                              min((2ll * sms + BH - 1) / BH, eg_level1_ctas_max(g.Cq)));
-    // later passes over the pooled rows: about two CTAs per SM in all, and at
-    // most kBinCap pairs per CTA (its warps share one histogram)
-    const long long prow = static_cast<long long>(g.H / 2) * g.Cq;
+    // later passes, c2 CTAs per pool: about two CTAs per SM in all, and at most
+    // kBinCap pairs per CTA (its warps share one histogram)
+    const long long pools = static_cast<long long>(g.B) * G;
+    const long long prow = static_cast<long long>(eg_max_pool_heads(g.H, domain)) * g.Cq;
     const long long prow_cap =
         static_cast<long long>(kBinCap / (static_cast<uint32_t>(g.Ck) * kWarps)) * kWarps;
-    const long long c2 = max(max(1ll, (prow + prow_cap - 1) / prow_cap),
-                             min((2ll * sms + g.B - 1) / g.B, max(1ll, (prow + kWarps - 1) / kWarps)));
-    if (BH * c1 > 0x7FFFFFFFll || static_cast<long long>(g.B) * c2 > 0x7FFFFFFFll) return cudaErrorInvalidValue;
+    const long long c2 =
+        pools == 0 ? 0
+                   : max(max(1ll, (prow + prow_cap - 1) / prow_cap),
+                         min((2ll * sms + pools - 1) / pools, max(1ll, (prow + kWarps - 1) / kWarps)));
+    if (BH * c1 > 0x7FFFFFFFll || pools * c2 > 0x7FFFFFFFll) return cudaErrorInvalidValue;
     const int vpl = (g.Ck + 31) / 32;
-    if (vpl <= 4) return launch_eg_passes<4>(a, c1, c2, g.B, BH, st);
-    if (vpl <= 8) return launch_eg_passes<8>(a, c1, c2, g.B, BH, st);
-    if (vpl <= 16) return launch_eg_passes<16>(a, c1, c2, g.B, BH, st);
-    if (vpl <= 32) return launch_eg_passes<32>(a, c1, c2, g.B, BH, st);
-    return launch_eg_passes<64>(a, c1, c2, g.B, BH, st);
+    if (vpl <= 4) return launch_eg_passes<4>(a, c1, c2, pools, BH, st);
+    if (vpl <= 8) return launch_eg_passes<8>(a, c1, c2, pools, BH, st);
+    if (vpl <= 16) return launch_eg_passes<16>(a, c1, c2, pools, BH, st);
+    if (vpl <= 32) return launch_eg_passes<32>(a, c1, c2, pools, BH, st);
+    return launch_eg_passes<64>(a, c1, c2, pools, BH, st);
 }
 
 }  // namespace bsa

@@ -49,10 +49,11 @@ cudaError_t launch_mask(const Geometry &g, const float *probs, const TopP &tp, u
 cudaError_t launch_entropy_reduce(const Geometry &g, const float *row_entropy, float *entropy,
                                   float *entropy_norm, cudaStream_t st);
 
-// ---- entropy-guided grouped cross-head selection ("Competition Domains Matter
-// ..." s3.3 domain 3, s4 value-aware score): the shared state of one batch
-// entry's cross-head pool, written by the radix-select kernels of eg.cu and
-// read by the final per-row pass of mask.cu.
+// ---- pooled top-p over a competition domain ("Competition Domains Matter ..."
+// s3: per-row, per-head, grouped cross-head, all-head, and the entropy-guided
+// EG-Sparse of s3.3 with the s4 value-aware score): the shared state of one
+// pool, written by the radix-select kernels of eg.cu and read by the final
+// per-row pass of mask.cu.
 struct PoolState {
     double target;                // pool_p * (total score of the pool)
     double above;                 // score mass of the pool above the current range
@@ -60,7 +61,7 @@ struct PoolState {
     uint32_t pre;                 // bit-pattern prefix of the current range
     int shift;                    // low bits below the prefix (0 once the cut value is found)
     int keep_all;                 // the pool never reaches target: every pair is kept
-    int empty;                    // the batch entry has no pooled head
+    int empty;                    // the pool has no head
     uint32_t ucut;                // the cut score's bit pattern
     int pad0;
     unsigned long long need;      // pairs with score == ucut to keep, in (h, i, j) order
@@ -72,25 +73,30 @@ struct PoolState {
 // Value-centroid norms ||c^V_{h,j}||_2, fp32 [B,H,C_k].
 cudaError_t launch_value_norms(const Geometry &g, const void *v, float *vnorm, cudaStream_t st);
 
-// Workspace layout of bsa_build_mask_eg (byte offsets; all 256-aligned).
+// Pools per batch entry of a BSA_DOMAIN_* value (0 for per-row).
+int eg_pools(int H, int domain);
+
+// Workspace layout of the pooled selection (byte offsets; all 256-aligned).
 struct EgWorkspace {
-    size_t ent_part, heads_h, low, pool_heads, state;
+    size_t ent_part, heads_h, pool_of, pool_heads, pool_nh, state;
     size_t zero_begin, zero_bytes;  // cleared at the start of every call
     size_t hist1, hist, tiecnt, counters, bytes;
 };
-EgWorkspace eg_workspace(const Geometry &g);
+EgWorkspace eg_workspace(const Geometry &g, int domain);
 
-// Entropy-guided selection up to the final pass: row entropies, per-head
-// entropy (into `entropy` / `entropy_norm` when given, always into the
-// workspace), the median split (into `low_heads` when given) and the pool cut.
-cudaError_t launch_eg_prepare(const Geometry &g, const float *probs, const float *vnorm,
+// Pooled selection up to the final pass: row entropies, per-head entropy (into
+// `entropy` / `entropy_norm` when given, always into the workspace), the
+// domain's pools (into `low_heads` as pooled-or-not and `pool_out` as the pool
+// id, when given) and every pool's cut.
+cudaError_t launch_eg_prepare(const Geometry &g, int domain, const float *probs, const float *vnorm,
                               float pool_p, float eps, float *entropy, float *entropy_norm,
-                              uint8_t *low_heads, uint8_t *workspace, cudaStream_t st);
-// The final pass: per-row top-p for the other heads, the pool cut and the
+                              uint8_t *low_heads, int8_t *pool_out, uint8_t *workspace, cudaStream_t st);
+// The final pass: per-row top-p for the per-row heads, the pool cut and the
 // one-key-per-row safeguard for the pooled heads, overrides and lists.
+// pool_of [B,H] (-1 = per-row), state [B,G].
 cudaError_t launch_mask_eg(const Geometry &g, const float *probs, const float *vnorm,
                            const TopP &tp, uint32_t flags, uint8_t *mask, int32_t *kv_index,
-                           int32_t *kv_count, const uint8_t *low, const PoolState *state,
+                           int32_t *kv_count, const int8_t *pool_of, int G, const PoolState *state,
                            cudaStream_t st);
 
 // Returns BSA_* status.

@@ -41,8 +41,9 @@ struct MaskArgs {
     int text_kblocks, f0_first, f0_last;
     // entropy-guided mode: pooled heads take the batch entry's pool cut
     const float *vnorm;           // value-centroid norms [B,H,C_k], or nullptr
-    const uint8_t *low;           // [B,H]: 1 = pooled head
-    const PoolState *state;       // [B]
+    const int8_t *pool_of;        // [B,H]: the head's pool, -1 = per-row
+    const PoolState *state;       // [B,G]
+    int G;                        // pools per batch entry
 };
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -429,7 +430,8 @@ mask_kernel(MaskArgs a, TopP tp) {
         v[s] = (j < Ck) ? __ldg(src + j) : 0.f;
     }
     const long long bh = row / a.Cq;
-    const bool pooled = EG && a.low[bh];
+    const int pool = EG ? a.pool_of[bh] : -1;
+    const bool pooled = pool >= 0;
     float ent = 0.f;
     uint32_t umax = 0;
 #pragma unroll
@@ -459,7 +461,7 @@ mask_kernel(MaskArgs a, TopP tp) {
         if (!pooled) {
             find_cut<VPL>(v, src, Ck, p, umax, lane, ws, ucut, jcut);
         } else {
-            const PoolState st = a.state[bh / a.H];
+            const PoolState st = a.state[(bh / a.H) * a.G + pool];
             if (!st.keep_all) {
                 ucut = st.ucut;
                 jcut = row < st.cut_row ? 0x7FFFFFFF
@@ -556,14 +558,15 @@ cudaError_t launch_mask(const Geometry &g, const float *probs, const TopP &tp, u
     a.f0_first = g.f0_first;
     a.f0_last = g.f0_last;
     a.vnorm = nullptr;
-    a.low = nullptr;
+    a.pool_of = nullptr;
     a.state = nullptr;
+    a.G = 0;
     return launch_mask_vpl<false>(a, tp, g.Ck, st);
 }
 
 cudaError_t launch_mask_eg(const Geometry &g, const float *probs, const float *vnorm,
                            const TopP &tp, uint32_t flags, uint8_t *mask, int32_t *kv_index,
-                           int32_t *kv_count, const uint8_t *low, const PoolState *state,
+                           int32_t *kv_count, const int8_t *pool_of, int G, const PoolState *state,
                            cudaStream_t st) {
     MaskArgs a;
     a.probs = probs;
@@ -581,8 +584,9 @@ cudaError_t launch_mask_eg(const Geometry &g, const float *probs, const float *v
     a.f0_first = g.f0_first;
     a.f0_last = g.f0_last;
     a.vnorm = vnorm;
-    a.low = low;
+    a.pool_of = pool_of;
     a.state = state;
+    a.G = G;
     return launch_mask_vpl<true>(a, tp, g.Ck, st);
 }
 

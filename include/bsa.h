@@ -250,6 +250,50 @@ int bsa_build_mask_eg(const bsa_layout *layout, const float *probs, const float 
                       int32_t *kv_index, int32_t *kv_count, float *entropy, float *entropy_norm,
                       uint8_t *low_heads, void *workspace, void *stream);
 
+/*
+ * Competition domains ("Competition Domains Matter ..." s3): which pairs
+ * (h, i, j) of one batch entry compete for one top-p budget.
+ *   BSA_DOMAIN_ROW      per-row local: no pools, every row the rule of bsa_build_mask
+ *   BSA_DOMAIN_HEAD     per-head global: pool g = head g (G = H pools)
+ *   BSA_DOMAIN_GROUPED  grouped cross-head with both groups pooled: the floor(H/2)
+ *                       lowest-entropy heads form pool 0, the rest pool 1 (G = 2)
+ *   BSA_DOMAIN_ALL      all-head global: one pool of every head (G = 1)
+ *   BSA_DOMAIN_EG       EG-Sparse: the low-entropy half pooled (pool 0), the
+ *                       rest per-row (G = 1); bsa_build_mask_eg
+ * The entropy split is the one of bsa_build_mask_eg.
+ */
+enum bsa_domain {
+    BSA_DOMAIN_ROW = 0,
+    BSA_DOMAIN_HEAD = 1,
+    BSA_DOMAIN_GROUPED = 2,
+    BSA_DOMAIN_ALL = 3,
+    BSA_DOMAIN_EG = 4
+};
+
+/* Bytes of device scratch bsa_build_mask_domain needs for `domain` (0 on a bad
+ * layout or domain). */
+size_t bsa_build_mask_domain_workspace_bytes(const bsa_layout *layout, int domain);
+
+/*
+ * Pooled top-p over a competition domain: as bsa_build_mask_eg, with the pools
+ * of `domain` (enum bsa_domain).  Every pool ranks its pairs by the score I of
+ * bsa_build_mask_eg in (I descending, h, i, j ascending) order, keeps the
+ * shortest prefix reaching pool_p times its total score, and then gives a row
+ * it left empty its best key block; rows of unpooled heads keep their per-row
+ * top_p[h].  BSA_DOMAIN_EG gives exactly bsa_build_mask_eg.
+ *
+ * pool_of       i8 [B,H]: each head's pool (-1 = per-row), or NULL
+ * workspace     device scratch of bsa_build_mask_domain_workspace_bytes(layout,
+ *               domain) bytes, 256-byte aligned
+ * other arguments as for bsa_build_mask_eg.  Returns BSA_ERR_INVALID_ARG for a
+ * domain outside the enum.
+ */
+int bsa_build_mask_domain(const bsa_layout *layout, int domain, const float *probs,
+                          const float *vnorm, const float *top_p, float pool_p, uint32_t flags,
+                          float eps, uint8_t *mask, int32_t *kv_index, int32_t *kv_count,
+                          float *entropy, float *entropy_norm, int8_t *pool_of, void *workspace,
+                          void *stream);
+
 /* Bytes of device workspace bsa_build_mask_eg needs (0: invalid layout). */
 size_t bsa_build_mask_eg_workspace_bytes(const bsa_layout *layout);
 

@@ -163,6 +163,24 @@ def test_eg_entry_points_validate_before_any_cuda_call():
     n = lib.bsa_build_mask_eg_workspace_bytes(ctypes.byref(bsa.make_layout(w)))
     rows = w.heads * (w.seq_pad // w.q_block)
     assert n >= rows * 4 + w.heads * 256 * 16 + 4096 * 16 and n % 256 == 0
+    # the domain entry: the same checks, plus the domain; the EG domain's workspace is EG's,
+    # per-head pools need one 4096-bin histogram per head
+    assert lib.bsa_build_mask_domain_workspace_bytes(ctypes.byref(bsa.make_layout(w)), bsa.DOMAIN_EG) == n
+    assert lib.bsa_build_mask_domain_workspace_bytes(ctypes.byref(bsa.make_layout(w)), 5) == 0
+    assert lib.bsa_build_mask_domain_workspace_bytes(ctypes.byref(bsa.make_layout(w)), -1) == 0
+    assert lib.bsa_build_mask_domain_workspace_bytes(ctypes.byref(bad), bsa.DOMAIN_ALL) == 0
+    nh = lib.bsa_build_mask_domain_workspace_bytes(ctypes.byref(bsa.make_layout(w)), bsa.DOMAIN_HEAD)
+    assert nh >= n + (w.heads - 1) * 4096 * 16
+
+    def dom(domain=bsa.DOMAIN_GROUPED, probs=FAKE, top=tpv, idx=FAKE, w=ws):
+        return lib.bsa_build_mask_domain(r, domain, probs, None, top, 0.9, 3, 1e-8, None, idx, FAKE,
+                                         None, None, None, w, None)
+    for d in (-1, 5, 100):
+        assert dom(domain=d) == bsa.BSA_ERR_INVALID_ARG
+    assert dom(probs=None) == bsa.BSA_ERR_INVALID_ARG
+    assert dom(top=None) == bsa.BSA_ERR_INVALID_ARG
+    assert dom(idx=None) == bsa.BSA_ERR_INVALID_ARG
+    assert dom(w=ctypes.c_void_p(0x100010)) == bsa.BSA_ERR_INVALID_ARG
 
 
 def test_clustered_scores_validate_before_any_cuda_call():
