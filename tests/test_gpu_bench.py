@@ -32,3 +32,8 @@ def test_bench_line(selection):
     assert line["gpu_launches"] == 2 * {"top_p": 5, "eg": 9, "sampled": 4}[selection]
     if selection == "top_p":
         assert line["e2e"]["value"] > 0 and line["e2e"]["h2d_bytes_per_step"] > 0
+    doms = line["competition_domains"]
+    assert set(doms) == {"per_row", "per_head", "grouped", "all_head", "eg_sparse", "call"}
+    for name in ("per_row", "per_head", "grouped", "all_head", "eg_sparse"):
+        assert doms[name]["ms"] > 0 and 0 < doms[name]["density"] <= 1
+    assert doms["per_row"]["pooled_heads"] == 0 and doms["all_head"]["pooled_heads"] == line["config"]["heads"]
