@@ -1,15 +1,17 @@
-// eg.cu -- entropy-guided grouped cross-head selection, up to the final pass.
+// eg.cu -- pooled top-p over a competition domain, up to the final pass.
 //
 // "Competition Domains Matter: Selective Head Globalization for Training-Free
 // Sparse Attention in Video Diffusion Transformers", s3.3 domain 3 ("grouped
 // cross-head": heads split by the median of their entropy H_h; low-entropy
 // heads compete in one shared pool, the others keep per-row local top-p), the
 // one-key-per-row safeguard, and s4 (the pool ranks pairs by the value-aware
-// score P'_{h,i,j} * ||c^V_{h,j}||).
+// score P'_{h,i,j} * ||c^V_{h,j}||); s3's other domains route the heads of a
+// batch entry into other pools: one per head, one per entropy half, one for
+// all heads (BSA_DOMAIN_*), G pools per batch entry.
 //
-// Per batch entry b the pool holds every pair (h, i, j) of its low-entropy
-// heads, ordered by (score desc, h, i, j asc), and keeps the shortest prefix
-// whose running sum reaches pool_p times the pool total.  The cut is found
+// Pool (b, g) holds every pair (h, i, j) of its heads, ordered by (score desc,
+// h, i, j asc), and keeps the shortest prefix whose running sum reaches pool_p
+// times the pool total.  The cut is found
 // without sorting by an exact radix select over the fp32 bit patterns of the
 // scores (scores >= 0 order like their bit patterns): a histogram of the
 // exponent field, then of mantissa bits 22..11, then 10..0, each bin holding
@@ -22,12 +24,15 @@
 // does that launch's serial step, so no launch waits on another's CTAs):
 //   entropy_level1_kernel  -sum_j P' ln(P' + eps) per row and a per-head
 //                          histogram of the scores' exponent fields; its last
-//                          CTA takes the per-head means, the median split and
-//                          the level-1 pick of every batch entry
+//                          CTA takes the per-head means, routes the heads to
+//                          the domain's pools and takes the level-1 pick of
+//                          every pool
 //   pool_level_kernel x2   mantissa bits 22..11, then 10..0, over the pooled
-//                          heads only; the last CTA picks the bin
+//                          heads only, c2 CTAs per pool; the last CTA of each
+//                          pool picks that pool's bin
 //   tie_kernel             pairs equal to the cut pattern per pooled row; the
-//                          last CTA finds the row and rank of the last kept tie
+//                          last CTA of each pool finds the row and rank of the
+//                          last kept tie
 #include <cuda_runtime.h>
 #include <limits.h>
 #include <math.h>
@@ -171,7 +176,7 @@ __device__ void cta_scan(double &m, unsigned long long &c, ScanScratch &sc) {
     __syncthreads();
 }
 
-// One radix level of one batch entry, by the whole CTA, on its histogram in
+// One radix level of one pool, by the whole CTA, on its histogram in
 // shared memory (sum[k] = significand sum of bin k; cnt[k] = its count at the
 // last level, before it only zero or not as the bin is empty or not).  The
 // level's bin holding the cut: scanning bins from the largest value down, the
@@ -293,7 +298,7 @@ struct EgArgs {
     PoolState *state;       // [B,G]
     unsigned int *counter;  // this launch's finish counter
     int B, H, Cq, Ck;
-    int ctas;               // CTAs per head (level 1) or per batch entry (later passes)
+    int ctas;               // CTAs per head (level 1) or per pool (later passes)
     float eps, inv_log_ck, pool_p;
 };
 
@@ -490,14 +495,14 @@ __global__ void __launch_bounds__(kThreads) entropy_level1_kernel(EgArgs a) {
     }
 }
 
-// Pooled rows of batch entry b in (h, i) order: row r is row r % C_q of the
-// (r / C_q)-th pooled head.
+// Rows of a pool of batch entry b in (h, i) order: row r is row r % C_q of the
+// (r / C_q)-th head of the pool.
 __device__ __forceinline__ long long pooled_row(const EgArgs &a, const int *heads, int b, long long r) {
     const long long kk = r / a.Cq;
     return (static_cast<long long>(b) * a.H + heads[kk]) * a.Cq + (r - kk * a.Cq);
 }
 
-// One later radix level over the pooled rows of batch entry blockIdx.x / ctas:
+// One later radix level over the rows of pool blockIdx.x / ctas:
 // every score in the current range (bits above `shift` equal to `pre`) adds
 // (1, significand) to bin (u >> (shift - NBITS)) & (2^NBITS - 1).
 template <int VPL, int NBITS, bool COUNTS>

@@ -39,7 +39,7 @@ struct MaskArgs {
     uint32_t flags;
     float eps;
     int text_kblocks, f0_first, f0_last;
-    // entropy-guided mode: pooled heads take the batch entry's pool cut
+    // pooled mode: pooled heads take their pool's cut
     const float *vnorm;           // value-centroid norms [B,H,C_k], or nullptr
     const int8_t *pool_of;        // [B,H]: the head's pool, -1 = per-row
     const PoolState *state;       // [B,G]
@@ -397,8 +397,8 @@ __device__ __forceinline__ float lg2_approx(float y) {
 }
 
 // EG = false: every row takes its per-row top-p.  EG = true ("Competition
-// Domains Matter ..." s3.3 domain 3): rows of pooled heads keep the pairs of the
-// batch entry's pool cut (scores P' * ||c^V|| above the cut pattern, ties at
+// Domains Matter ..." s3.3 domain 3 and s3's other pooled domains): rows of
+// pooled heads keep the pairs of their pool's cut (scores P' * ||c^V|| above the cut pattern, ties at
 // it up to the cut row's rank) and, if that leaves them empty, their single
 // best key block (the one-key-per-row safeguard); the other rows keep their
 // per-row top-p.  Entropies are not computed in that mode.
