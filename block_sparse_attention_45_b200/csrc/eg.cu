@@ -25,11 +25,12 @@
 //   entropy_level1_kernel  -sum_j P' ln(P' + eps) per row and a per-head
 //                          histogram of the scores' exponent fields; its last
 //                          CTA takes the per-head means, routes the heads to
-//                          the domain's pools and takes the level-1 pick of
-//                          every pool
+//                          the domain's pools and lists each pool's heads
 //   pool_level_kernel x2   mantissa bits 22..11, then 10..0, over the pooled
-//                          heads only, c2 CTAs per pool; the last CTA of each
-//                          pool picks that pool's bin
+//                          heads only, c2 CTAs per pool; each CTA of the first
+//                          takes its pool's level-1 pick (the same in all of
+//                          them), and the last CTA of each pool picks that
+//                          pool's bin
 //   tie_kernel             pairs equal to the cut pattern per pooled row; the
 //                          last CTA of each pool finds the row and rank of the
 //                          last kept tie
@@ -321,12 +322,9 @@ __global__ void __launch_bounds__(kThreads) entropy_level1_kernel(EgArgs a) {
     // per warp kL1Copies histograms (count, lo, hi), lane l bins into copy l % kL1Copies;
     // copies kL1Stride words apart so that one bin's copies sit in different banks
     extern __shared__ __align__(16) uint32_t sh[];
-    __shared__ ScanScratch sc;
-    __shared__ PoolState s_st;
     __shared__ double s_wsum[kWarps];
     __shared__ float s_h[kMaxHeads];
-    __shared__ int s_heads[kMaxHeads];
-    __shared__ int s_np;
+    __shared__ int s_pool[kMaxHeads];
     const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
     __shared__ int s_zero;
     {
@@ -390,7 +388,7 @@ __global__ void __launch_bounds__(kThreads) entropy_level1_kernel(EgArgs a) {
     }
     if (!last_cta(a.counter, gridDim.x)) return;
 
-    // ---- the last CTA: per-head means, the domain's pools, level-1 pick per pool
+    // ---- the last CTA: per-head means, the domain's pools and their heads
     const long long BH = static_cast<long long>(a.B) * a.H;
     for (long long bh = wid; bh < BH; bh += kWarps) {
         double s = 0.0;  // fixed order: part-strided per lane, then a butterfly; lane 0's sum
@@ -405,8 +403,6 @@ __global__ void __launch_bounds__(kThreads) entropy_level1_kernel(EgArgs a) {
         }
     }
     __syncthreads();
-    uint32_t *cnt = sh;  // reuse: [256] counts, then [256] u64 sums
-    unsigned long long *sum = reinterpret_cast<unsigned long long *>(sh + 2 * kL1Bins);
     const int H = a.H, G = a.G;
     for (int b = 0; b < a.B; ++b) {
         for (int h = threadIdx.x; h < H; h += kThreads) s_h[h] = a.heads_h[static_cast<long long>(b) * H + h];
@@ -431,68 +427,73 @@ __global__ void __launch_bounds__(kThreads) entropy_level1_kernel(EgArgs a) {
                 default: pool = -1; break;
             }
             const long long bh = static_cast<long long>(b) * H + h;
+            s_pool[h] = pool;
             a.pool_of[bh] = static_cast<int8_t>(pool);
             if (a.low_out) a.low_out[bh] = pool >= 0 ? 1 : 0;
             if (a.pool_out) a.pool_out[bh] = static_cast<int8_t>(pool);
         }
         __syncthreads();
-        for (int g = 0; g < G; ++g) {
+        // each pool's heads in ascending order, one thread per pool
+        for (int g = threadIdx.x; g < G; g += kThreads) {
             const long long bp = static_cast<long long>(b) * G + g;
-            if (threadIdx.x == 0) {  // the pool's heads, ascending
-                int k = 0;
-                for (int h = 0; h < H; ++h)
-                    if (a.pool_of[static_cast<long long>(b) * H + h] == g) s_heads[k++] = h;
-                s_np = k;
-                PoolState z;
-                z.target = 0.0;
-                z.above = 0.0;
-                z.pad2 = 0;
-                z.pre = 0;
-                z.shift = 31;  // level 1 bins bits 30..23 of scores >= 0 (bit 31 is 0)
-                z.keep_all = 0;
-                z.empty = k == 0;
-                z.ucut = 0;
-                z.pad0 = 0;
-                z.need = 0;
-                z.cut_row = -1;
-                z.cut_rank = 0;
-                z.pad1 = 0;
-                s_st = z;
-                a.pool_nh[bp] = k;
-            }
-            __syncthreads();
-            const int np = s_np;
-            for (int k = threadIdx.x; k < np; k += kThreads) a.pool_heads[bp * H + k] = s_heads[k];
-            if (!s_st.empty) {
-                const int t = threadIdx.x;  // bin t over the pool's heads, loads 8 heads at a time
-                unsigned long long c = 0, s = 0;
-                for (int k0 = 0; k0 < np; k0 += 8) {
-                    unsigned long long cc[8], ss[8];
+            int k = 0;
+            for (int h = 0; h < H; ++h)
+                if (s_pool[h] == g) a.pool_heads[bp * H + k++] = h;
+            a.pool_nh[bp] = k;
+        }
+        __syncthreads();
+    }
+}
+
+// The level-1 pick of a pool of batch entry b (its np heads in `heads`) into
+// `st`, by the whole CTA: the pool's exponent histogram is the sum of its
+// heads' histograms.  Every CTA
+// of the pool takes it from the same complete histograms, so all agree.
+__device__ __noinline__ void level1_pick(const EgArgs &a, int b, int np, const int *heads, uint32_t *cnt,
+                            unsigned long long *sum, PoolState &st, ScanScratch &sc) {
+    if (threadIdx.x == 0) {
+        PoolState z;
+        z.target = 0.0;
+        z.above = 0.0;
+        z.pad2 = 0;
+        z.pre = 0;
+        z.shift = 31;  // level 1 bins bits 30..23 of scores >= 0 (bit 31 is 0)
+        z.keep_all = 0;
+        z.empty = np == 0;
+        z.ucut = 0;
+        z.pad0 = 0;
+        z.need = 0;
+        z.cut_row = -1;
+        z.cut_rank = 0;
+        z.pad1 = 0;
+        st = z;
+    }
+    __syncthreads();
+    if (np == 0) return;
+    const int t = threadIdx.x;  // bin t over the pool's heads, loads 8 heads at a time
+    unsigned long long c = 0, s = 0;
+    for (int k0 = 0; k0 < np; k0 += 8) {
+        unsigned long long cc[8], ss[8];
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        cc[q] = ss[q] = 0ull;
-                        if (k0 + q < np) {
-                            const unsigned long long *gp =
-                                a.hist1 + ((static_cast<long long>(b) * H + s_heads[k0 + q]) * kL1Bins + t) * 2;
-                            cc[q] = __ldcg(gp);
-                            ss[q] = __ldcg(gp + 1);
-                        }
-                    }
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        c += cc[q];
-                        s += ss[q];
-                    }
-                }
-                cnt[t] = static_cast<uint32_t>(c);
-                sum[t] = s;
-                __syncthreads();
-                cta_pick(cnt, sum, 8, true, a.pool_p, s_st, sc);
+        for (int q = 0; q < 8; ++q) {
+            cc[q] = ss[q] = 0ull;
+            if (k0 + q < np) {
+                const unsigned long long *gp =
+                    a.hist1 + ((static_cast<long long>(b) * a.H + heads[k0 + q]) * kL1Bins + t) * 2;
+                cc[q] = __ldcg(gp);
+                ss[q] = __ldcg(gp + 1);
             }
-            if (threadIdx.x == 0) a.state[bp] = s_st;
-            __syncthreads();
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            c += cc[q];
+            s += ss[q];
         }
     }
+    cnt[t] = static_cast<uint32_t>(c);
+    sum[t] = s;
+    __syncthreads();
+    cta_pick(cnt, sum, 8, true, a.pool_p, st, sc);
 }
 
 // Rows of a pool of batch entry b in (h, i) order: row r is row r % C_q of the
@@ -504,29 +505,38 @@ __device__ __forceinline__ long long pooled_row(const EgArgs &a, const int *head
 
 // One later radix level over the rows of pool blockIdx.x / ctas:
 // every score in the current range (bits above `shift` equal to `pre`) adds
-// (1, significand) to bin (u >> (shift - NBITS)) & (2^NBITS - 1).
+// (1, significand) to bin (u >> (shift - NBITS)) & (2^NBITS - 1).  The first
+// of them (no counts) starts from the level-1 pick, which each of its CTAs
+// takes itself; the second from the state the first one's last CTA wrote.
 template <int VPL, int NBITS, bool COUNTS>
 __global__ void __launch_bounds__(kThreads) pool_level_kernel(EgArgs a) {
     constexpr int nb = 1 << NBITS;
     constexpr int per = nb / kThreads;
+    constexpr bool kFirst = !COUNTS;
     __shared__ int s_zero;
     extern __shared__ __align__(16) uint32_t sh[];  // [3 * nb]: count, lo, hi; then count + u64 sum
     __shared__ ScanScratch sc;
     __shared__ PoolState s_st;
     __shared__ int s_heads[kMaxHeads];
     const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
+    const int bp = blockIdx.x / a.ctas, part = blockIdx.x % a.ctas;
+    const int b = bp / a.G;
+    const int np = a.pool_nh[bp];
+    for (int k = threadIdx.x; k < np; k += kThreads) s_heads[k] = a.pool_heads[static_cast<long long>(bp) * a.H + k];
+    if (kFirst) {
+        __syncthreads();
+        level1_pick(a, b, np, s_heads, sh, reinterpret_cast<unsigned long long *>(sh + 2 * kL1Bins), s_st, sc);
+    } else {
+        if (threadIdx.x == 0) s_st = a.state[bp];
+        __syncthreads();
+    }
     {
-        const int bp = blockIdx.x / a.ctas, part = blockIdx.x % a.ctas;
-        const int b = bp / a.G;
-        const PoolState st = a.state[bp];
+        const PoolState st = s_st;
         if (pool_active(st) && st.shift >= NBITS) {
             uint32_t *c = sh, *lo = sh + nb, *hi = sh + 2 * nb;
             for (int k = threadIdx.x; k < 3 * nb; k += kThreads) sh[k] = 0u;
             if (threadIdx.x == 0) s_zero = 0;
             bool zero = false;
-            const int np = a.pool_nh[bp];
-            for (int k = threadIdx.x; k < np; k += kThreads)
-                s_heads[k] = a.pool_heads[static_cast<long long>(bp) * a.H + k];
             __syncthreads();
             const int shift = st.shift, low_bits = st.shift - NBITS;
             const uint32_t pre = st.pre;
@@ -580,13 +590,10 @@ __global__ void __launch_bounds__(kThreads) pool_level_kernel(EgArgs a) {
             }
         }
     }
-    // ---- the last CTA of pool bp: its pick
-    const int bp = blockIdx.x / a.ctas;
+    // ---- the last CTA of pool bp: its pick (s_st still holds the state this launch started from)
     if (!last_cta(a.counter + bp, static_cast<unsigned>(a.ctas))) return;
     uint32_t *cnt = sh;
     unsigned long long *sum = reinterpret_cast<unsigned long long *>(sh + nb);
-    if (threadIdx.x == 0) s_st = a.state[bp];
-    __syncthreads();
     if (pool_active(s_st) && s_st.shift >= NBITS) {
         unsigned long long *g = a.hist + static_cast<long long>(bp) * 2 * kMaxBins;
         unsigned long long cc[per], ss[per];
@@ -606,8 +613,8 @@ __global__ void __launch_bounds__(kThreads) pool_level_kernel(EgArgs a) {
         }
         __syncthreads();
         cta_pick(cnt, sum, NBITS, false, a.pool_p, s_st, sc);
-        if (threadIdx.x == 0) a.state[bp] = s_st;
     }
+    if (threadIdx.x == 0) a.state[bp] = s_st;
 }
 
 // Needed only when some but not all pairs equal to the cut pattern are kept:
