@@ -15,15 +15,18 @@
 //       P'_ij = sum_c (n_c / n_i) softmax_j(q_c . k_j / sqrt(D) + ln n_j).
 //
 // Launches: pool_kernel (key centroids only), subcluster_kernel (one CTA per
-// query block, the block's tokens in shared memory), score_kernel of
+// query block, the block's tokens in shared memory, each k-means round two
+// tcgen05 products), score_kernel of
 // scores.cu on the C_q * n_sub sub-centroid rows (split-tf32 tcgen05 GEMM with
 // the fused row softmax) into a workspace, mix_kernel (one warp per block row:
 // the size-weighted sum of its n_sub rows).
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace bsa {
 
@@ -31,137 +34,272 @@ namespace {
 
 constexpr int kClusterThreads = 128;
 
-// k-means of one query block.  Thread t holds token t in registers and picks
-// its cluster by the smallest ||c_k||^2 - 2 x.c_k (the distance without the
-// token's own ||x||^2; one independent FMA chain per centroid, centroids read
-// as broadcast float4).  Ballots then group the tokens by cluster into a
-// permutation (ascending token order inside a cluster), and thread d sums
-// dimension d over each cluster's segment from a dimension-major copy of the
-// tokens (row stride odd, so a column read is conflict-free).
+constexpr int kPanel = 128 * 128;   // one 128-byte swizzle panel: 128 rows x 64 bf16
+constexpr int kOhPanel = 16 * 128;  // one-hot operand panel: 16 rows x 64 tokens
+constexpr uint32_t kTmemCols = 64;  // one accumulator, reused by the two products
+
+// Byte offset of bf16 element (row r, column c < 64) in a 128-byte-swizzled
+// panel: row r at r * 128, its 16-byte chunk c / 8 stored at chunk (c / 8) ^ (r % 8)
+// (the layout TMA's 128-byte swizzle writes, read by the tensor core).
+__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
+    return static_cast<uint32_t>(r * 128 + ((((c >> 3) ^ r) & 7) << 4) + (c & 7) * 2);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
+    return __uint_as_float(static_cast<uint32_t>(h) << 16);
+}
+
+// x = hi + mid + lo with each part a bf16 (round to nearest; x - hi and the
+// next remainder are exact in fp32), so the three parts carry 24 bits of x.
+__device__ __forceinline__ void split3(float x, uint32_t &hi, uint32_t &mid, uint32_t &lo) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    const float r1 = x - __bfloat162float(h);
+    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(m);
+    const __nv_bfloat16 l = __float2bfloat16_rn(r2);
+    hi = __bfloat16_as_ushort(h);
+    mid = __bfloat16_as_ushort(m);
+    lo = __bfloat16_as_ushort(l);
+}
+
+// ||c_k||^2 of every centroid: warp w takes clusters w, w + 4, ..., each lane a
+// strided run of dimensions, then a butterfly sum.  Called by every thread.
+template <int D, int NSUB>
+__device__ __forceinline__ void centroid_norms(const float *c, float *cn, int lane, int wid) {
+    constexpr int kWarps = kClusterThreads / 32;
+    for (int k = wid; k < NSUB; k += kWarps) {
+        float s2 = 0.f;
+#pragma unroll
+        for (int d = lane; d < D; d += 32) s2 = fmaf(c[k * D + d], c[k * D + d], s2);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+        if (lane == 0) cn[k] = s2;
+    }
+}
+
+// k-means of one query block on the tensor cores, one CTA of 128 threads per
+// block, thread t owning token t.  The block's tokens X (bf16, exact) sit in
+// shared memory once, 128 x 128 (dimensions past D and tokens past n zero).
+// Each round is two tcgen05 products into one TMEM accumulator:
+//   distances   X (128 tokens x D) . [C_hi; C_mid; C_lo]^T, the centroids split
+//               into three bf16 parts, so x . c_k = sum of the three columns
+//               to fp32 accuracy; thread t takes argmin_k ||c_k||^2 - 2 x_t . c_k
+//               (ties to the lower k);
+//   sums        X^T (D x 128 tokens, the same tile read dimension-major) .
+//               OneHot (128 tokens x 16), OneHot[t][k] = 1 iff token t joined
+//               cluster k; thread d reads the 16 cluster sums of dimension d.
+// One thread issues the MMAs; every wait on their completion is bounded, and a
+// CTA whose wait gives up writes NaN centroids and zero sizes.
 template <int D, int NSUB>
 __global__ void __launch_bounds__(kClusterThreads) subcluster_kernel(
     const uint16_t *__restrict__ q, float *__restrict__ cent, int32_t *__restrict__ size, int S,
     int S_pad, int bq, int Cq, int iters) {
-    constexpr int LDT = kClusterThreads + 1;
     constexpr int kWarps = kClusterThreads / 32;
+    constexpr int ND = (3 * NSUB + 15) / 16 * 16;  // distance product N: hi, mid, lo rows
+    constexpr uint32_t kIdescDist = idesc_bf16_f32(128, ND, false);
+    constexpr uint32_t kIdescSum = idesc_bf16_f32(128, 16, false) | (1u << 15);  // A = X^T, MN-major
+    static_assert(NSUB <= 16, "one-hot operand holds 16 clusters");
+    extern __shared__ uint8_t dyn[];
     __shared__ __align__(16) float c[NSUB * D];
-    __shared__ float cn[NSUB];                 // ||c_k||^2
-    __shared__ int perm[kClusterThreads];      // tokens grouped by cluster
-    __shared__ int seg[NSUB + 1];              // cluster k = perm[seg[k] .. seg[k+1])
+    __shared__ float cn[NSUB];
     __shared__ int wcnt[kWarps][NSUB];
-    extern __shared__ float xt[];              // [D][LDT]: xt[d][t]
+    __shared__ int csize[NSUB];
+    __shared__ __align__(8) uint64_t bar, drain;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_v;
+
+    uint8_t *sX = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn) + 1023) & ~uintptr_t(1023));
+    uint8_t *sOH = sX + 2 * kPanel;     // 2 panels (tokens 0-63, 64-127) x 16 rows
+    uint8_t *sBD = sOH + 2 * kOhPanel;  // 2 panels (dimensions 0-63, 64-127) x ND rows
 
     const long long blk = blockIdx.x;
     const long long bh = blk / Cq;
     const int i = static_cast<int>(blk % Cq);
     const int n = max(0, min(bq, S - i * bq));
     const int tid = threadIdx.x, lane = tid % 32, wid = tid / 32;
-    float xr[D];
-    {
+
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        mbar_init(&drain, 1);
+        abort_v = 0;
+        fence_mbar_init();
+    }
+    if (wid == 0) {
+        tmem_alloc(&tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    if (tid < NSUB) csize[tid] = 0;
+    // the one-hot and split operands start zero (their rows past the live ones stay so)
+    for (int e = tid * 16; e < 2 * kOhPanel + 2 * ND * 128; e += kClusterThreads * 16)
+        *reinterpret_cast<uint4 *>(sOH + e) = make_uint4(0u, 0u, 0u, 0u);
+    {  // token tid -> row tid of X
         const uint4 *src = reinterpret_cast<const uint4 *>(
             q + (bh * S_pad + static_cast<long long>(i) * bq + min(tid, max(n - 1, 0))) * D);
 #pragma unroll
-        for (int v8 = 0; v8 < D / 8; ++v8) {
-            const uint4 v = tid < n ? __ldg(src + v8) : make_uint4(0u, 0u, 0u, 0u);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                xr[v8 * 8 + 2 * m] = __uint_as_float(w[m] << 16);
-                xr[v8 * 8 + 2 * m + 1] = __uint_as_float(w[m] & 0xFFFF0000u);
-            }
+        for (int j = 0; j < 16; ++j) {
+            const uint4 v = (tid < n && j < D / 8) ? __ldg(src + j) : make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4 *>(sX + (j / 8) * kPanel + tid * 128 + (((j & 7) ^ (tid & 7)) << 4)) = v;
         }
-#pragma unroll
-        for (int d = 0; d < D; ++d) xt[d * LDT + tid] = xr[d];
     }
+    fence_proxy_async_smem();
+    tc_fence_before();
     __syncthreads();
-    // seeds: the tokens at floor(c * n / NSUB); their squared norms
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(wid * 32) << 16);
+    // seeds: the tokens at floor(k * n / NSUB)
     for (int e = tid; e < NSUB * D; e += kClusterThreads) {
         const int k = e / D, d = e % D;
         const int t0 = n > 0 ? static_cast<int>((static_cast<long long>(k) * n) / NSUB) : 0;
-        c[e] = n > 0 ? xt[d * LDT + t0] : 0.f;
+        const uint16_t h = *reinterpret_cast<const uint16_t *>(sX + (d / 64) * kPanel + sw128_off(t0, d % 64));
+        c[e] = n > 0 ? bf16_bits_to_float(h) : 0.f;
     }
     __syncthreads();
-    if (tid < NSUB) {
-        float s2 = 0.f;
-        for (int d = 0; d < D; ++d) s2 = fmaf(c[tid * D + d], c[tid * D + d], s2);
-        cn[tid] = s2;
-    }
+    centroid_norms<D, NSUB>(c, cn, lane, wid);
     __syncthreads();
-    int best = 0;
+
+    uint32_t phase = 0;
+    bool ok = true;
     for (int it = 0; it < iters; ++it) {
-        best = 0;
-        if (NSUB > 1 && tid < n) {  // nearest centroid, ties to the lower index
-            float dot[NSUB];
+        int best = 0;
+        if (NSUB > 1) {
+            // split operand: row k = hi, NSUB + k = mid, 2 NSUB + k = lo of centroid k
+            for (int e = tid; e < NSUB * (D / 8); e += kClusterThreads) {
+                const int k = e / (D / 8), j = e % (D / 8);
+                const float4 v0 = reinterpret_cast<const float4 *>(c + k * D)[2 * j];
+                const float4 v1 = reinterpret_cast<const float4 *>(c + k * D)[2 * j + 1];
+                const float xs[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                uint32_t hw[4], mw[4], lw[4];
 #pragma unroll
-            for (int k = 0; k < NSUB; ++k) dot[k] = 0.f;
+                for (int p2 = 0; p2 < 4; ++p2) {
+                    uint32_t h0, m0, l0, h1, m1, l1;
+                    split3(xs[2 * p2], h0, m0, l0);
+                    split3(xs[2 * p2 + 1], h1, m1, l1);
+                    hw[p2] = h0 | (h1 << 16);
+                    mw[p2] = m0 | (m1 << 16);
+                    lw[p2] = l0 | (l1 << 16);
+                }
+                uint8_t *pb = sBD + (j / 8) * (ND * 128);
+                const int jj = j & 7;
+                const int rows[3] = {k, NSUB + k, 2 * NSUB + k};
+                const uint32_t *parts[3] = {hw, mw, lw};
 #pragma unroll
-            for (int d4 = 0; d4 < D / 4; ++d4) {
+                for (int m3 = 0; m3 < 3; ++m3) {
+                    const int r = rows[m3];
+                    *reinterpret_cast<uint4 *>(pb + r * 128 + ((jj ^ (r & 7)) << 4)) =
+                        make_uint4(parts[m3][0], parts[m3][1], parts[m3][2], parts[m3][3]);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t a_off = (kk / 4) * kPanel + (kk % 4) * 32;
+                    const uint32_t b_off = (kk / 4) * (ND * 128) + (kk % 4) * 32;
+                    mma_ss(tmem, sw128_desc(smem_u32(sX) + a_off, 16, 1024),
+                           sw128_desc(smem_u32(sBD) + b_off, 16, 1024), kIdescDist, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&bar);
+            }
+            ok = mbar_wait(&bar, phase, &abort_v);
+            phase ^= 1u;
+            if (!__syncthreads_and(ok)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t r[ND];
+#pragma unroll
+            for (int q16 = 0; q16 < ND / 16; ++q16) {
+                uint32_t part[16];
+                tmem_ld16(t_lane + static_cast<uint32_t>(q16 * 16), part);
+                tmem_ld_wait();
+                reg_fence(part);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) r[q16 * 16 + e] = part[e];
+            }
+            if (tid < n) {
+                float bd = INFINITY;
 #pragma unroll
                 for (int k = 0; k < NSUB; ++k) {
-                    const float4 cv = reinterpret_cast<const float4 *>(c + k * D)[d4];
-                    dot[k] = fmaf(xr[4 * d4], cv.x, dot[k]);
-                    dot[k] = fmaf(xr[4 * d4 + 1], cv.y, dot[k]);
-                    dot[k] = fmaf(xr[4 * d4 + 2], cv.z, dot[k]);
-                    dot[k] = fmaf(xr[4 * d4 + 3], cv.w, dot[k]);
+                    const float dot = (__uint_as_float(r[k]) + __uint_as_float(r[NSUB + k])) +
+                                      __uint_as_float(r[2 * NSUB + k]);
+                    const float dist = fmaf(-2.f, dot, cn[k]);
+                    if (dist < bd) {
+                        bd = dist;
+                        best = k;
+                    }
                 }
             }
-            float bd = INFINITY;
-#pragma unroll
-            for (int k = 0; k < NSUB; ++k) {
-                const float dist = fmaf(-2.f, dot[k], cn[k]);
-                if (dist < bd) {
-                    bd = dist;
-                    best = k;
-                }
-            }
+            tc_fence_before();
         }
-        // group by cluster: per-warp counts, then each token's slot
+        // cluster sizes by ballots; column tid of the one-hot operand
         const bool live = tid < n;
-        int rank_in_warp = 0;
 #pragma unroll
         for (int k = 0; k < NSUB; ++k) {
             const unsigned bal = __ballot_sync(0xffffffffu, live && best == k);
-            if (best == k) rank_in_warp = __popc(bal & ((1u << lane) - 1u));
             if (lane == 0) wcnt[wid][k] = __popc(bal);
+            *reinterpret_cast<uint16_t *>(sOH + (tid / 64) * kOhPanel + sw128_off(k, tid % 64)) =
+                (live && best == k) ? static_cast<uint16_t>(0x3F80u) : static_cast<uint16_t>(0u);
         }
-        __syncthreads();
-        if (tid == 0) {
-            int off = 0;
-            for (int k = 0; k < NSUB; ++k) {
-                seg[k] = off;
-                for (int w = 0; w < kWarps; ++w) {
-                    const int m = wcnt[w][k];
-                    wcnt[w][k] = off;  // now the warp's first slot in cluster k
-                    off += m;
-                }
-            }
-            seg[NSUB] = off;
-        }
-        __syncthreads();
-        if (live) perm[wcnt[wid][best] + rank_in_warp] = tid;
-        __syncthreads();
-        // move the centroids: thread d sums dimension d over each cluster
-        if (tid < D) {
-#pragma unroll
-            for (int k = 0; k < NSUB; ++k) {
-                const int a = seg[k], b = seg[k + 1];
-                if (b > a) {
-                    float s = 0.f;
-                    for (int idx = a; idx < b; ++idx) s += xt[tid * LDT + perm[idx]];
-                    c[k * D + tid] = s / static_cast<float>(b - a);
-                }
-            }
-        }
+        fence_proxy_async_smem();
         __syncthreads();
         if (tid < NSUB) {
-            float s2 = 0.f;
-            for (int d = 0; d < D; ++d) s2 = fmaf(c[tid * D + d], c[tid * D + d], s2);
-            cn[tid] = s2;
+            int sz = 0;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) sz += wcnt[w][tid];
+            csize[tid] = sz;
         }
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t a_off = kk * 2048;  // tokens 16 kk .. 16 kk + 15 of X^T
+                const uint32_t b_off = (kk / 4) * kOhPanel + (kk % 4) * 32;
+                mma_ss(tmem, sw128_desc(smem_u32(sX) + a_off, kPanel, 1024),
+                       sw128_desc(smem_u32(sOH) + b_off, 16, 1024), kIdescSum, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&bar);
+        }
+        ok = mbar_wait(&bar, phase, &abort_v);
+        phase ^= 1u;
+        if (!__syncthreads_and(ok)) {  // also publishes csize
+            ok = false;
+            break;
+        }
+        tc_fence_after();
+        {  // move the centroids: thread d reads the 16 cluster sums of dimension d
+            uint32_t u[16];
+            tmem_ld16(t_lane, u);
+            tmem_ld_wait();
+            reg_fence(u);
+            if (tid < D) {
+#pragma unroll
+                for (int k = 0; k < NSUB; ++k)
+                    if (csize[k] > 0) c[k * D + tid] = __uint_as_float(u[k]) / static_cast<float>(csize[k]);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        centroid_norms<D, NSUB>(c, cn, lane, wid);
         __syncthreads();
     }
-    for (int e = tid; e < NSUB * D; e += kClusterThreads) cent[blk * NSUB * D + e] = c[e];
-    if (tid < NSUB) size[blk * NSUB + tid] = iters > 0 ? seg[tid + 1] - seg[tid] : 0;
+    if (!ok) {  // let whatever was issued finish before TMEM is freed
+        if (tid == 0) {
+            mma_commit(&drain);
+            volatile int no_abort = 0;
+            mbar_wait(&drain, 0, &no_abort);
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < NSUB * D; e += kClusterThreads) cent[blk * NSUB * D + e] = ok ? c[e] : NAN;
+    if (tid < NSUB) size[blk * NSUB + tid] = ok ? csize[tid] : 0;
+    if (wid == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
 }
 
 // P'[r, :] = sum_c (n_c / n) P_sub[r * NSUB + c, :], one warp per row, in
@@ -195,7 +333,8 @@ __global__ void __launch_bounds__(256) mix_kernel(const float *__restrict__ psub
 template <int D, int NSUB>
 cudaError_t launch_sub_t(const uint16_t *q, float *cent, int32_t *size, const Geometry &g,
                          long long blocks, int iters, cudaStream_t st) {
-    const size_t smem = static_cast<size_t>(D) * (kClusterThreads + 1) * sizeof(float);
+    constexpr int ND = (3 * NSUB + 15) / 16 * 16;
+    const size_t smem = 1024 + 2 * kPanel + 2 * kOhPanel + 2 * ND * 128;
     cudaError_t e = cudaFuncSetAttribute(subcluster_kernel<D, NSUB>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
