@@ -27,6 +27,13 @@ CASES = {
     "h5_d128": synth.custom("h5_d128", heads=5, head_dim=128, q_block=64, k_block=128,
                             text_len=40, num_frames=3, latent_h=10, latent_w=10, top_p=0.7,
                             seed=32),
+    # last query blocks of 5 and 3 tokens: fewer tokens than clusters (repeated seeds,
+    # empty clusters of size 0)
+    "tail5": synth.custom("tail5", heads=2, head_dim=64, q_block=64, k_block=64, text_len=69,
+                          num_frames=2, latent_h=8, latent_w=8, top_p=0.8, seed=34),
+    "tail3_d128": synth.custom("tail3_d128", heads=3, head_dim=128, q_block=128, k_block=128,
+                               text_len=3, num_frames=2, latent_h=8, latent_w=16, top_p=0.8,
+                               seed=35),
 }
 
 _CACHE = {}
