@@ -62,36 +62,24 @@ __device__ __forceinline__ void split3(float x, uint32_t &hi, uint32_t &mid, uin
     lo = __bfloat16_as_ushort(l);
 }
 
-// ||c_k||^2 of every centroid: warp w takes clusters w, w + 4, ..., each lane a
-// strided run of dimensions, then a butterfly sum.  Called by every thread.
-template <int D, int NSUB>
-__device__ __forceinline__ void centroid_norms(const float *c, float *cn, int lane, int wid) {
-    constexpr int kWarps = kClusterThreads / 32;
-    for (int k = wid; k < NSUB; k += kWarps) {
-        float s2 = 0.f;
-#pragma unroll
-        for (int d = lane; d < D; d += 32) s2 = fmaf(c[k * D + d], c[k * D + d], s2);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-        if (lane == 0) cn[k] = s2;
-    }
-}
-
 // k-means of one query block on the tensor cores, one CTA of 128 threads per
-// block, thread t owning token t.  The block's tokens X (bf16, exact) sit in
-// shared memory once, 128 x 128 (dimensions past D and tokens past n zero).
-// Each round is two tcgen05 products into one TMEM accumulator:
+// block.  The block's tokens X (bf16, exact) sit in shared memory once,
+// 128 x 128 (dimensions past D and tokens past n zero); thread t owns token t
+// for the assignment and dimension t of every centroid (in registers) for the
+// update.  Each round is two tcgen05 products into one TMEM accumulator:
 //   distances   X (128 tokens x D) . [C_hi; C_mid; C_lo]^T, the centroids split
-//               into three bf16 parts, so x . c_k = sum of the three columns
+//               into three bf16 parts, so x . c_k is the sum of three columns
 //               to fp32 accuracy; thread t takes argmin_k ||c_k||^2 - 2 x_t . c_k
 //               (ties to the lower k);
 //   sums        X^T (D x 128 tokens, the same tile read dimension-major) .
 //               OneHot (128 tokens x 16), OneHot[t][k] = 1 iff token t joined
-//               cluster k; thread d reads the 16 cluster sums of dimension d.
+//               cluster k; thread d reads the 16 cluster sums of dimension d,
+//               moves its coordinate of every non-empty centroid, and writes the
+//               three parts of it and its share of ||c_k||^2 for the next round.
 // One thread issues the MMAs; every wait on their completion is bounded, and a
 // CTA whose wait gives up writes NaN centroids and zero sizes.
 template <int D, int NSUB>
-__global__ void __launch_bounds__(kClusterThreads) subcluster_kernel(
+__global__ void __launch_bounds__(kClusterThreads, 3) subcluster_kernel(
     const uint16_t *__restrict__ q, float *__restrict__ cent, int32_t *__restrict__ size, int S,
     int S_pad, int bq, int Cq, int iters) {
     constexpr int kWarps = kClusterThreads / 32;
@@ -99,11 +87,10 @@ __global__ void __launch_bounds__(kClusterThreads) subcluster_kernel(
     constexpr uint32_t kIdescDist = idesc_bf16_f32(128, ND, false);
     constexpr uint32_t kIdescSum = idesc_bf16_f32(128, 16, false) | (1u << 15);  // A = X^T, MN-major
     static_assert(NSUB <= 16, "one-hot operand holds 16 clusters");
+    static_assert(D <= kClusterThreads, "one thread per dimension");
     extern __shared__ uint8_t dyn[];
-    __shared__ __align__(16) float c[NSUB * D];
-    __shared__ float cn[NSUB];
+    __shared__ float cnp[kWarps][NSUB];  // per-warp shares of ||c_k||^2
     __shared__ int wcnt[kWarps][NSUB];
-    __shared__ int csize[NSUB];
     __shared__ __align__(8) uint64_t bar, drain;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_v;
@@ -117,6 +104,7 @@ __global__ void __launch_bounds__(kClusterThreads) subcluster_kernel(
     const int i = static_cast<int>(blk % Cq);
     const int n = max(0, min(bq, S - i * bq));
     const int tid = threadIdx.x, lane = tid % 32, wid = tid / 32;
+    const bool owns_dim = tid < D;
 
     if (tid == 0) {
         mbar_init(&bar, 1);
@@ -128,7 +116,6 @@ __global__ void __launch_bounds__(kClusterThreads) subcluster_kernel(
         tmem_alloc(&tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    if (tid < NSUB) csize[tid] = 0;
     // the one-hot and split operands start zero (their rows past the live ones stay so)
     for (int e = tid * 16; e < 2 * kOhPanel + 2 * ND * 128; e += kClusterThreads * 16)
         *reinterpret_cast<uint4 *>(sOH + e) = make_uint4(0u, 0u, 0u, 0u);
@@ -141,57 +128,55 @@ __global__ void __launch_bounds__(kClusterThreads) subcluster_kernel(
             *reinterpret_cast<uint4 *>(sX + (j / 8) * kPanel + tid * 128 + (((j & 7) ^ (tid & 7)) << 4)) = v;
         }
     }
+    __syncthreads();
+
+    // Coordinate tid of every centroid, its three bf16 parts into the distance
+    // operand (rows k, NSUB + k, 2 NSUB + k) and the warp's share of ||c_k||^2.
+    float cd[NSUB];
+    auto publish = [&]() {
+#pragma unroll
+        for (int k = 0; k < NSUB; ++k) {
+            float sq = 0.f;
+            if (owns_dim) {
+                uint32_t h, m, l;
+                split3(cd[k], h, m, l);
+                uint8_t *pb = sBD + (tid / 64) * (ND * 128);
+                *reinterpret_cast<uint16_t *>(pb + sw128_off(k, tid % 64)) = static_cast<uint16_t>(h);
+                *reinterpret_cast<uint16_t *>(pb + sw128_off(NSUB + k, tid % 64)) = static_cast<uint16_t>(m);
+                *reinterpret_cast<uint16_t *>(pb + sw128_off(2 * NSUB + k, tid % 64)) = static_cast<uint16_t>(l);
+                sq = cd[k] * cd[k];
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+            if (lane == 0) cnp[wid][k] = sq;
+        }
+        fence_proxy_async_smem();
+    };
+    // seeds: the tokens at floor(k * n / NSUB)
+#pragma unroll
+    for (int k = 0; k < NSUB; ++k) {
+        const int t0 = n > 0 ? static_cast<int>((static_cast<long long>(k) * n) / NSUB) : 0;
+        cd[k] = 0.f;
+        if (owns_dim && n > 0)
+            cd[k] = bf16_bits_to_float(
+                *reinterpret_cast<const uint16_t *>(sX + (tid / 64) * kPanel + sw128_off(t0, tid % 64)));
+    }
+    publish();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wid * 32) << 16);
-    // seeds: the tokens at floor(k * n / NSUB)
-    for (int e = tid; e < NSUB * D; e += kClusterThreads) {
-        const int k = e / D, d = e % D;
-        const int t0 = n > 0 ? static_cast<int>((static_cast<long long>(k) * n) / NSUB) : 0;
-        const uint16_t h = *reinterpret_cast<const uint16_t *>(sX + (d / 64) * kPanel + sw128_off(t0, d % 64));
-        c[e] = n > 0 ? bf16_bits_to_float(h) : 0.f;
-    }
-    __syncthreads();
-    centroid_norms<D, NSUB>(c, cn, lane, wid);
-    __syncthreads();
 
     uint32_t phase = 0;
     bool ok = true;
+    int sz[NSUB];
+#pragma unroll
+    for (int k = 0; k < NSUB; ++k) sz[k] = 0;
     for (int it = 0; it < iters; ++it) {
         int best = 0;
         if (NSUB > 1) {
-            // split operand: row k = hi, NSUB + k = mid, 2 NSUB + k = lo of centroid k
-            for (int e = tid; e < NSUB * (D / 8); e += kClusterThreads) {
-                const int k = e / (D / 8), j = e % (D / 8);
-                const float4 v0 = reinterpret_cast<const float4 *>(c + k * D)[2 * j];
-                const float4 v1 = reinterpret_cast<const float4 *>(c + k * D)[2 * j + 1];
-                const float xs[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-                uint32_t hw[4], mw[4], lw[4];
-#pragma unroll
-                for (int p2 = 0; p2 < 4; ++p2) {
-                    uint32_t h0, m0, l0, h1, m1, l1;
-                    split3(xs[2 * p2], h0, m0, l0);
-                    split3(xs[2 * p2 + 1], h1, m1, l1);
-                    hw[p2] = h0 | (h1 << 16);
-                    mw[p2] = m0 | (m1 << 16);
-                    lw[p2] = l0 | (l1 << 16);
-                }
-                uint8_t *pb = sBD + (j / 8) * (ND * 128);
-                const int jj = j & 7;
-                const int rows[3] = {k, NSUB + k, 2 * NSUB + k};
-                const uint32_t *parts[3] = {hw, mw, lw};
-#pragma unroll
-                for (int m3 = 0; m3 < 3; ++m3) {
-                    const int r = rows[m3];
-                    *reinterpret_cast<uint4 *>(pb + r * 128 + ((jj ^ (r & 7)) << 4)) =
-                        make_uint4(parts[m3][0], parts[m3][1], parts[m3][2], parts[m3][3]);
-                }
-            }
-            fence_proxy_async_smem();
-            __syncthreads();
             if (tid == 0) {
                 tc_fence_after();
 #pragma unroll
@@ -224,16 +209,18 @@ __global__ void __launch_bounds__(kClusterThreads) subcluster_kernel(
                 float bd = INFINITY;
 #pragma unroll
                 for (int k = 0; k < NSUB; ++k) {
+                    float cn = cnp[0][k];
+#pragma unroll
+                    for (int w = 1; w < kWarps; ++w) cn += cnp[w][k];
                     const float dot = (__uint_as_float(r[k]) + __uint_as_float(r[NSUB + k])) +
                                       __uint_as_float(r[2 * NSUB + k]);
-                    const float dist = fmaf(-2.f, dot, cn[k]);
+                    const float dist = fmaf(-2.f, dot, cn);
                     if (dist < bd) {
                         bd = dist;
                         best = k;
                     }
                 }
             }
-            tc_fence_before();
         }
         // cluster sizes by ballots; column tid of the one-hot operand
         const bool live = tid < n;
@@ -245,13 +232,8 @@ __global__ void __launch_bounds__(kClusterThreads) subcluster_kernel(
                 (live && best == k) ? static_cast<uint16_t>(0x3F80u) : static_cast<uint16_t>(0u);
         }
         fence_proxy_async_smem();
+        tc_fence_before();
         __syncthreads();
-        if (tid < NSUB) {
-            int sz = 0;
-#pragma unroll
-            for (int w = 0; w < kWarps; ++w) sz += wcnt[w][tid];
-            csize[tid] = sz;
-        }
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
@@ -263,9 +245,16 @@ __global__ void __launch_bounds__(kClusterThreads) subcluster_kernel(
             }
             mma_commit(&bar);
         }
+#pragma unroll
+        for (int k = 0; k < NSUB; ++k) {
+            int s2 = 0;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) s2 += wcnt[w][k];
+            sz[k] = s2;
+        }
         ok = mbar_wait(&bar, phase, &abort_v);
         phase ^= 1u;
-        if (!__syncthreads_and(ok)) {  // also publishes csize
+        if (!__syncthreads_and(ok)) {
             ok = false;
             break;
         }
@@ -275,15 +264,12 @@ __global__ void __launch_bounds__(kClusterThreads) subcluster_kernel(
             tmem_ld16(t_lane, u);
             tmem_ld_wait();
             reg_fence(u);
-            if (tid < D) {
 #pragma unroll
-                for (int k = 0; k < NSUB; ++k)
-                    if (csize[k] > 0) c[k * D + tid] = __uint_as_float(u[k]) / static_cast<float>(csize[k]);
-            }
+            for (int k = 0; k < NSUB; ++k)
+                if (sz[k] > 0) cd[k] = __uint_as_float(u[k]) / static_cast<float>(sz[k]);
         }
+        publish();
         tc_fence_before();
-        __syncthreads();
-        centroid_norms<D, NSUB>(c, cn, lane, wid);
         __syncthreads();
     }
     if (!ok) {  // let whatever was issued finish before TMEM is freed
@@ -294,8 +280,14 @@ __global__ void __launch_bounds__(kClusterThreads) subcluster_kernel(
         }
     }
     __syncthreads();
-    for (int e = tid; e < NSUB * D; e += kClusterThreads) cent[blk * NSUB * D + e] = ok ? c[e] : NAN;
-    if (tid < NSUB) size[blk * NSUB + tid] = ok ? csize[tid] : 0;
+    if (owns_dim) {
+#pragma unroll
+        for (int k = 0; k < NSUB; ++k) cent[(blk * NSUB + k) * D + tid] = ok ? cd[k] : NAN;
+    }
+    if (tid == 0) {
+#pragma unroll
+        for (int k = 0; k < NSUB; ++k) size[blk * NSUB + k] = ok ? sz[k] : 0;
+    }
     if (wid == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
