@@ -119,14 +119,20 @@ __global__ void __launch_bounds__(kClusterThreads, 3) subcluster_kernel(
     // the one-hot and split operands start zero (their rows past the live ones stay so)
     for (int e = tid * 16; e < 2 * kOhPanel + 2 * ND * 128; e += kClusterThreads * 16)
         *reinterpret_cast<uint4 *>(sOH + e) = make_uint4(0u, 0u, 0u, 0u);
-    {  // token tid -> row tid of X
-        const uint4 *src = reinterpret_cast<const uint4 *>(
-            q + (bh * S_pad + static_cast<long long>(i) * bq + min(tid, max(n - 1, 0))) * D);
+    {  // tokens -> X: warp w copies tokens 32w .. 32w + 31, each load 32 consecutive 16-byte
+       // chunks of their rows (coalesced); chunks of tokens past n are zero
+        constexpr int CH = D / 8;  // 16-byte chunks per token row
+        const uint4 *src = reinterpret_cast<const uint4 *>(q + (bh * S_pad + static_cast<long long>(i) * bq) * D);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const uint4 v = (tid < n && j < D / 8) ? __ldg(src + j) : make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4 *>(sX + (j / 8) * kPanel + tid * 128 + (((j & 7) ^ (tid & 7)) << 4)) = v;
+        for (int it2 = 0; it2 < CH; ++it2) {
+            const int idx = it2 * 32 + lane;
+            const int t = 32 * wid + idx / CH, j = idx % CH;
+            const uint4 v = t < n ? __ldg(src + t * CH + j) : make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4 *>(sX + (j / 8) * kPanel + t * 128 + (((j & 7) ^ (t & 7)) << 4)) = v;
         }
+        if (D < 128)  // dimensions past D: the second panel is zero
+            for (int e = tid * 16; e < kPanel; e += kClusterThreads * 16)
+                *reinterpret_cast<uint4 *>(sX + kPanel + e) = make_uint4(0u, 0u, 0u, 0u);
     }
     __syncthreads();
 
