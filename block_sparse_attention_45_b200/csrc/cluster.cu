@@ -14,12 +14,11 @@
 //     sub-centroids' cluster-size-weighted softmax rows:
 //       P'_ij = sum_c (n_c / n_i) softmax_j(q_c . k_j / sqrt(D) + ln n_j).
 //
-// Launches: pool_kernel (key centroids only), subcluster_kernel (one CTA per
+// Launches: pool_kernel (key centroids only); subcluster_kernel (one CTA per
 // query block, the block's tokens in shared memory, each k-means round two
-// tcgen05 products), score_kernel of
-// scores.cu on the C_q * n_sub sub-centroid rows (split-tf32 tcgen05 GEMM with
-// the fused row softmax) into a workspace, mix_kernel (one warp per block row:
-// the size-weighted sum of its n_sub rows).
+// tcgen05 products); score_kernel of scores.cu on the C_q * n_sub sub-centroid
+// rows (split-tf32 tcgen05 GEMM with the fused row softmax) into a workspace;
+// mix_kernel (one warp per block row: the size-weighted sum of its n_sub rows).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
