@@ -334,8 +334,8 @@ def our_arm(args, w):
     # value norms, entropy + level 1, two pool levels, the tie pass and the mask kernel in
     # place of mask + entropy reduce; the sampler one kernel
     launches_per_step = 9 if eg else (4 if sampled else 5)
-    if nsub > 1:   # key pooling, k-means, score kernel, mix in place of pooling + score kernel
-        launches_per_step += 2
+    if nsub > 1:   # key pooling, k-means, the mixing score kernel in place of pooling + score kernel
+        launches_per_step += 1
     for _ in range(max(3, args.warmup)):
         step(q, k, v)
     torch.cuda.synchronize(dev)

@@ -17,8 +17,8 @@
 // Launches: pool_kernel (key centroids only); subcluster_kernel (one CTA per
 // query block, the block's tokens in shared memory, each k-means round two
 // tcgen05 products); score_kernel of scores.cu on the C_q * n_sub sub-centroid
-// rows (split-tf32 tcgen05 GEMM with the fused row softmax) into a workspace;
-// mix_kernel (one warp per block row: the size-weighted sum of its n_sub rows).
+// rows (split-tf32 tcgen05 GEMM with the fused row softmax; the logits go to a
+// workspace and its last pass writes each block's size-weighted mixture).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -299,34 +299,6 @@ __global__ void __launch_bounds__(kClusterThreads, 3) subcluster_kernel(
     }
 }
 
-// P'[r, :] = sum_c (n_c / n) P_sub[r * NSUB + c, :], one warp per row, in
-// ascending c; the weights are fixed per row, the column loop keeps several
-// rows' loads in flight.
-template <int NSUB>
-__global__ void __launch_bounds__(256) mix_kernel(const float *__restrict__ psub,
-                                                  const int32_t *__restrict__ size,
-                                                  float *__restrict__ probs, long long rows, int Ck) {
-    const int lane = threadIdx.x % 32;
-    const long long r = static_cast<long long>(blockIdx.x) * 8 + threadIdx.x / 32;
-    if (r >= rows) return;
-    float wk[NSUB];
-    int ntot = 0;
-#pragma unroll
-    for (int k = 0; k < NSUB; ++k) ntot += __ldg(size + r * NSUB + k);
-    const float inv = ntot > 0 ? 1.f / static_cast<float>(ntot) : 0.f;
-#pragma unroll
-    for (int k = 0; k < NSUB; ++k) wk[k] = static_cast<float>(__ldg(size + r * NSUB + k)) * inv;
-    const float *src = psub + r * NSUB * Ck;
-#pragma unroll 4
-    for (int j = lane; j < Ck; j += 32) {
-        float acc = 0.f;
-#pragma unroll
-        for (int k = 0; k < NSUB; ++k)
-            if (wk[k] > 0.f) acc = fmaf(wk[k], __ldg(src + k * Ck + j), acc);
-        probs[r * Ck + j] = acc;
-    }
-}
-
 template <int D, int NSUB>
 cudaError_t launch_sub_t(const uint16_t *q, float *cent, int32_t *size, const Geometry &g,
                          long long blocks, int iters, cudaStream_t st) {
@@ -373,20 +345,12 @@ cudaError_t launch_scores_clustered(const Geometry &g, const void *q, const void
         e = launch_subclusters<64>(q16, cent, size, g, blocks, nsub, iters, st);
     if (e != cudaSuccess) return e;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // the sub-centroid rows as C_q * nsub query rows of the score kernel
+    // the sub-centroid rows as C_q * nsub query rows of the score kernel, which mixes
+    // each block's rows into its P' row
     Geometry gs = g;
     gs.Cq = g.Cq * nsub;
     float *psub = static_cast<float *>(workspace);
-    if ((e = launch_scores(gs, cent, kc, psub, st)) != cudaSuccess) return e;
-    const unsigned grid = static_cast<unsigned>((blocks + 7) / 8);
-    switch (nsub) {
-        case 1: mix_kernel<1><<<grid, 256, 0, st>>>(psub, size, probs, blocks, g.Ck); break;
-        case 2: mix_kernel<2><<<grid, 256, 0, st>>>(psub, size, probs, blocks, g.Ck); break;
-        case 4: mix_kernel<4><<<grid, 256, 0, st>>>(psub, size, probs, blocks, g.Ck); break;
-        case 8: mix_kernel<8><<<grid, 256, 0, st>>>(psub, size, probs, blocks, g.Ck); break;
-        default: mix_kernel<16><<<grid, 256, 0, st>>>(psub, size, probs, blocks, g.Ck); break;
-    }
-    return cudaGetLastError();
+    return launch_scores(gs, cent, kc, psub, st, size, nsub, probs);
 }
 
 }  // namespace bsa

@@ -36,8 +36,13 @@ int check_layout(const bsa_layout *L);
 
 cudaError_t launch_pool(const Geometry &g, const void *q, const void *k, float *qc, float *kc,
                         cudaStream_t st);
+// P' rows of the centroid rows qc.  With mix_out: qc holds nsub sub-centroid
+// rows per query block (g.Cq = blocks * nsub) and the block's mixed row
+// sum_c (n_c / n) P'_c (sizes n_c in mix_size) goes to mix_out; probs then
+// only holds intermediate values.
 cudaError_t launch_scores(const Geometry &g, const float *qc, const float *kc, float *probs,
-                          cudaStream_t st);
+                          cudaStream_t st, const int32_t *mix_size = nullptr, int nsub = 1,
+                          float *mix_out = nullptr);
 
 struct TopP {
     float p[kMaxHeads];

@@ -202,6 +202,12 @@ struct Params {
     float *probs;
     int Cq, Ck, S, bk, n_rt, n_items;
     float scale2;  // log2(e) / sqrt(D)
+    // Mixing (the rows are nsub sub-centroid rows per query block): instead of
+    // normalising its rows in place, the last pass writes each block's row
+    // sum_c (n_c / n) P'_c into mix_out; nullptr = plain rows.
+    const int32_t *mix_size;  // [blocks, nsub] cluster sizes
+    float *mix_out;           // [blocks, C_k]
+    int nsub;
 };
 
 // Clear the low 13 mantissa bits: an exact tf32 value, and x - hi is exact.
@@ -457,6 +463,46 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
             hd.m2[rl] = m2;
             hd.inv_z[rl] = 1.0f / z;
             __syncwarp();
+            if (p.mix_out) {
+                // A block's nsub rows are consecutive and never straddle a warp's 32 rows
+                // (nsub divides 32): its P' row is sum_c w_c 2^(s2_c - m2_c) / z_c with
+                // w_c = n_c / n, the terms added in ascending c (fused multiply-add), the
+                // same arithmetic as normalising the rows and then mixing them.
+                const int ns = p.nsub;
+                for (int i = 0; i < my_rows; i += ns) {
+                    const long long brow = (static_cast<long long>(bh) * p.Cq + r0 + ew * 32 + i) / ns;
+                    int ntot = 0;
+                    for (int c = 0; c < ns; ++c) ntot += __ldg(p.mix_size + brow * ns + c);
+                    const float inv = ntot > 0 ? 1.f / static_cast<float>(ntot) : 0.f;
+                    float *out = p.mix_out + brow * p.Ck;
+                    for (int c0 = 0; c0 < p.Ck; c0 += 1024) {
+                        float acc[32];
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) acc[k] = 0.f;
+                        for (int c = 0; c < ns; ++c) {
+                            const float wc = static_cast<float>(__ldg(p.mix_size + brow * ns + c)) * inv;
+                            if (!(wc > 0.f)) continue;
+                            const float mc = hd.m2[ew * 32 + i + c], izc = hd.inv_z[ew * 32 + i + c];
+                            const float *rc = wtile + static_cast<long long>(i + c) * p.Ck;
+                            float v[32];
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) {
+                                const int col = c0 + lane + 32 * k;
+                                v[k] = col < p.Ck ? rc[col] : 0.f;
+                            }
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) acc[k] = fmaf(wc, ex2(v[k] - mc) * izc, acc[k]);
+                        }
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) {
+                            const int col = c0 + lane + 32 * k;
+                            if (col < p.Ck) out[col] = acc[k];
+                        }
+                    }
+                }
+                __syncwarp();  // m2 / inv_z of this warp's rows are reused by the next item
+                continue;
+            }
             for (int i = 0; i < my_rows; i += 2) {
                 const bool two = i + 1 < my_rows;
                 const float ma = hd.m2[ew * 32 + i], iza = hd.inv_z[ew * 32 + i];
@@ -511,7 +557,7 @@ bool make_f32_map(CUtensorMap *m, const float *base, long long BH, int rows, int
 
 template <int D>
 cudaError_t launch_scores_t(const Geometry &g, const float *qc, const float *kc, float *probs,
-                            cudaStream_t st) {
+                            cudaStream_t st, const int32_t *mix_size, int nsub, float *mix_out) {
     const long long BH = static_cast<long long>(g.B) * g.H;
     CUtensorMap mq, mk;
     if (!make_f32_map(&mq, qc, BH, g.Cq, D, sc::kRows) || !make_f32_map(&mk, kc, BH, g.Ck, D, sc::kCols))
@@ -527,6 +573,10 @@ cudaError_t launch_scores_t(const Geometry &g, const float *qc, const float *kc,
     if (items > 0x7FFFFFFFll) return cudaErrorInvalidValue;
     p.n_items = static_cast<int>(items);
     p.scale2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+    p.mix_size = mix_size;
+    p.mix_out = mix_out;
+    p.nsub = nsub;
+    if (mix_out && (!mix_size || nsub < 1 || 32 % nsub != 0 || g.Cq % nsub != 0)) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          sc::kSmemAlloc);
     if (e != cudaSuccess) return e;
@@ -577,9 +627,9 @@ cudaError_t launch_value_norms(const Geometry &g, const void *v, float *vnorm, c
 }
 
 cudaError_t launch_scores(const Geometry &g, const float *qc, const float *kc, float *probs,
-                          cudaStream_t st) {
-    return g.D == 128 ? launch_scores_t<128>(g, qc, kc, probs, st)
-                      : launch_scores_t<64>(g, qc, kc, probs, st);
+                          cudaStream_t st, const int32_t *mix_size, int nsub, float *mix_out) {
+    return g.D == 128 ? launch_scores_t<128>(g, qc, kc, probs, st, mix_size, nsub, mix_out)
+                      : launch_scores_t<64>(g, qc, kc, probs, st, mix_size, nsub, mix_out);
 }
 
 }  // namespace bsa
