@@ -9,7 +9,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libbsa.so")
 SOURCES = ["api.cu", "scores.cu", "mask.cu", "eg.cu", "sample.cu", "cluster.cu", "profile.cu", "attention.cu", "noalloc.cu", "pipeline.cu"]
-HEADERS = ["ptx.cuh", "internal.h"]
+HEADERS = ["ptx.cuh", "internal.h", "bits.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -39,6 +39,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include "bits.cuh"
 #include "internal.h"
 
 namespace bsa {
@@ -55,23 +56,7 @@ constexpr int kMaxBins = 4096;                // widest later level
 constexpr int kLevelBits[2] = {12, 11};       // mantissa 22..11, 10..0
 constexpr uint32_t kBinCap = (1u << 20) - 1;  // pairs one 32-bit shared bin may take (12-bit halves)
 
-__device__ __forceinline__ float lg2_fast(float y) {
-    float r;
-    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(y));
-    return r;
-}
-
 __device__ __forceinline__ uint32_t pos_bits(float y) { return __float_as_uint(y > 0.f ? y : 0.f); }
-
-__device__ __forceinline__ uint32_t significand(uint32_t u) {
-    return (u & 0x7FFFFFu) | ((u >> 23) ? 0x800000u : 0u);
-}
-
-// 2^(max(e, 1) - 150): the weight of one significand unit in binade e.
-__device__ __forceinline__ double unit_of_binade(uint32_t e) {
-    const int k = static_cast<int>(e > 1u ? e : 1u) - 150;
-    return __longlong_as_double(static_cast<long long>(k + 1023) << 52);
-}
 
 // Score of a pooled pair as a bit pattern: P' (negatives and NaN as +0) times
 // ||c^V|| (vn), rounded to fp32; P' alone without value norms.
@@ -114,12 +99,6 @@ __device__ __forceinline__ void bin_add_sum(uint32_t *lo, uint32_t *hi, uint32_t
     const uint32_t s = significand(u);
     atomicAdd(lo + bin, s & 0xFFFu);
     atomicAdd(hi + bin, s >> 12);
-}
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
 }
 
 // Called by every thread after its last global write: true in the one CTA of
@@ -358,7 +337,7 @@ __global__ void __launch_bounds__(kThreads) entropy_level1_kernel(EgArgs a) {
                 const int j = lane + 32 * s;
                 if (j < Ck) {
                     const float x = y[s] > 0.f ? y[s] : 0.f;
-                    ent = fmaf(x, lg2_fast(x + a.eps), ent);
+                    ent = fmaf(x, lg2_approx(x + a.eps), ent);
                     const uint32_t u = score_bits(x, va, vn[s]);
                     bin_add_sum(wl, wh, u >> 23, u);
                     zero |= u == 0u;

@@ -22,6 +22,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include "bits.cuh"
 #include "internal.h"
 
 namespace bsa {
@@ -45,12 +46,6 @@ struct MaskArgs {
     const PoolState *state;       // [B,G]
     int G;                        // pools per batch entry
 };
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
 
 __device__ __forceinline__ int warp_sum_i(int v) {
 #pragma unroll
@@ -104,16 +99,6 @@ struct WarpScratch {
     uint32_t cand_u[32];
     int cand_j[32];
 };
-
-__device__ __forceinline__ uint32_t significand(uint32_t u) {
-    return (u & 0x7FFFFFu) | ((u >> 23) ? 0x800000u : 0u);
-}
-
-// 2^(max(e, 1) - 150): the weight of one significand unit in binade e.
-__device__ __forceinline__ double unit_of_binade(uint32_t e) {
-    const int k = static_cast<int>(e > 1u ? e : 1u) - 150;
-    return __longlong_as_double(static_cast<long long>(k + 1023) << 52);
-}
 
 // Lane r < kRowsTab returns the sum of row r and clears it (other lanes 0).
 // Quarter-warps read 8 distinct bank groups thanks to the rotation.
@@ -390,12 +375,6 @@ __device__ __forceinline__ void find_cut(const float (&v)[VPL], const float *__r
 }
 
 // Hardware base-2 logarithm (MUFU approximation, relative error ~2^-22).
-__device__ __forceinline__ float lg2_approx(float y) {
-    float r;
-    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(y));
-    return r;
-}
-
 // EG = false: every row takes its per-row top-p.  EG = true ("Competition
 // Domains Matter ..." s3.3 domain 3 and s3's other pooled domains): rows of
 // pooled heads keep the pairs of their pool's cut (scores P' * ||c^V|| above the cut pattern, ties at
