@@ -108,6 +108,7 @@ def load():
         L.bsa_build_mask_domain_workspace_bytes.restype = ctypes.c_size_t
         L.bsa_status_string.argtypes = [ctypes.c_int]
         L.bsa_status_string.restype = ctypes.c_char_p
+        L.bsa_version.argtypes = []
         L.bsa_version.restype = ctypes.c_int
         _LIB = L
     return _LIB

@@ -270,3 +270,13 @@ def test_calls_fail_loudly_without_the_library(monkeypatch):
     monkeypatch.setattr(bsa, "LIB_PATH", "/nonexistent/libbsa.so")
     with pytest.raises(RuntimeError, match="not built"):
         bsa.load()
+
+
+def test_binding_types_every_declared_entry_point():
+    """Every function of include/bsa.h gets argtypes and restype in the binding,
+    so no pointer or size crosses the boundary as a default C int."""
+    lib = bsa.load()
+    for name in sorted(bsa.declared_symbols()):
+        fn = getattr(lib, name)
+        assert fn.argtypes is not None, name
+        assert fn.restype is not None, name
