@@ -40,8 +40,8 @@
  *     legacy default stream) and never synchronises.
  *   - Arguments are validated on the host before anything is launched; a
  *     failed check returns BSA_ERR_INVALID_ARG (or BSA_ERR_UNSUPPORTED for a
- *     valid shape this build has no kernel for) and launches nothing.
- *   - A launch failure returns BSA_ERR_LAUNCH; a failure of the driver's
+ *     valid shape the library has no kernel for) and launches nothing.
+ *   - A launch failure returns BSA_ERR_LAUNCH; a failure of the CUDA driver's
  *     tensor-map encoder returns BSA_ERR_DRIVER.
  *   - Bad data found on the device (a list entry outside [0, C_k), a count
  *     outside [0, C_k], a wait that timed out) never traps: the kernel skips
