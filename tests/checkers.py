@@ -11,6 +11,8 @@ Attention: given identical masks, the bf16 output must be within MAX_ABS of
 the fp64-computed fp32 oracle at every element and MEAN_ABS on average; the
 log-sum-exp within LSE_ABS.  Entropy within ENTROPY_REL relative.
 """
+import itertools
+
 import numpy as np
 
 MARGIN = 1e-4            # end to end (GPU P' vs oracle P'): all three margin terms
@@ -119,3 +121,37 @@ def check_attention(out_gpu, out_ora, lse_gpu=None, lse_ora=None, what="", max_a
             e = np.abs(lg[fin] - lo[fin]).max()
             assert e <= LSE_ABS, "%s: lse err %.3g" % (what, e)
     return float(err.max()), float(err.mean())
+
+
+def kmeans_end_states(x, n_sub, iters, rel=1e-4, cap=4096):
+    """(centroids, sizes) of every end state of the k-means rounds on the block's
+    tokens x [n, D] (fp64) when a token whose squared distance to a centroid is
+    within rel * (|x|^2 + max |c|^2) of its nearest may be assigned to it.  Seeds,
+    the move step and empty clusters follow the oracle's k-means."""
+    n, D = x.shape
+    xx = (x * x).sum(1)
+    c0 = np.stack([x[(k * n) // n_sub] if n > 0 else np.zeros(D) for k in range(n_sub)])
+    states = [(c0, np.zeros(n_sub, np.int64))]
+    for _ in range(iters):
+        nxt = {}
+        for c, _sizes in states:
+            d = ((x[:, None, :] - c[None, :, :]) ** 2).sum(-1)
+            dmin = d.min(1)
+            tol = rel * (xx + (c * c).sum(1).max())
+            cands = [np.nonzero(d[t] <= dmin[t] + tol[t])[0] for t in range(n)]
+            amb = [t for t in range(n) if len(cands[t]) > 1]
+            n_combos = int(np.prod([len(cands[t]) for t in amb])) if amb else 1
+            assert n_combos <= cap, "too many near-equidistant tokens to replay (%d)" % n_combos
+            base = d.argmin(1)
+            for combo in itertools.product(*[cands[t] for t in amb]):
+                a = base.copy()
+                a[amb] = combo
+                sizes = np.bincount(a, minlength=n_sub)
+                cn = c.copy()
+                for k in range(n_sub):
+                    if sizes[k] > 0:
+                        cn[k] = x[a == k].mean(0)
+                nxt[a.tobytes() + cn[sizes == 0].tobytes()] = (cn, sizes)
+        states = list(nxt.values())
+        assert len(states) <= cap, "too many branches to replay (%d)" % len(states)
+    return states

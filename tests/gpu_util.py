@@ -44,8 +44,11 @@ def oracle_selection(name):
     return oracle.select(w.layout(), x["q"], x["k"], top_p_of(w), w.flags)
 
 
-def sample_rows(w, n_random=3, seed=0):
-    """Flat query-block ids to check at full size: frame-0, text, last (ragged), random."""
+def sample_rows(w, n_random=64, seed=0, frame0_head=0):
+    """Flat query-block ids to check at full size: the first frame-0 block, a text
+    block, the ragged last block, every frame-0 block of head `frame0_head` (None:
+    skip), and n_random random blocks spread over every head (random block of
+    head r mod B*H for r = 0 .. n_random-1)."""
     cq = w.seq_pad // w.q_block
     L = w.layout()
     f0, f1 = oracle.frame0_qblocks(L)
@@ -53,6 +56,12 @@ def sample_rows(w, n_random=3, seed=0):
     rows = {0 * cq + f0, (w.heads - 1) * cq + cq - 1, (w.heads // 2) * cq + min(f1 + 1, cq - 1)}
     if w.text_len > 0:
         rows.add((w.heads // 3) * cq + 0)
-    while len(rows) < 4 + n_random:
-        rows.add(int(rng.integers(w.batch * w.heads * cq)))
+    if frame0_head is not None and f1 >= f0:
+        rows.update(frame0_head * cq + i for i in range(f0, f1 + 1))
+    bh = w.batch * w.heads
+    fixed = len(rows)
+    r = 0
+    while len(rows) < fixed + n_random:
+        rows.add(int((r % bh) * cq + rng.integers(cq)))
+        r += 1
     return np.array(sorted(rows), np.int64)

@@ -4,10 +4,15 @@
 fix (1): queries clustered within each query block; the block's score row is
 the size-weighted mixture of its sub-centroids' rows.  k-means assignments are
 decisions taken in floating point (fp32 on the GPU, fp64 in the oracle), so
-near-equidistant tokens may land differently: blocks whose cluster sizes agree
-(nearly all) must agree in centroids and score rows; the rest must still be a
-valid clustering (sizes summing to the block's tokens, rows summing to one).
+near-equidistant tokens may land differently.  Blocks whose cluster sizes agree
+(nearly all) must agree in centroids and score rows.  Every other block must be
+a clustering that Lloyd's rounds reach when each token whose nearest centroids
+are within 1e-4 (relative) of each other may take any of them: its sizes and
+centroids must equal one of the end states of that branching replay.  Every
+block's score row must equal the oracle's mixture fed the GPU's own
+sub-centroids and sizes.
 """
+
 import numpy as np
 import pytest
 import torch
@@ -15,6 +20,7 @@ import torch
 import oracle
 from block_sparse_attention_45_b200 import binding as bsa
 from block_sparse_attention_45_b200 import synth
+from tests import checkers
 
 pytestmark = pytest.mark.gpu
 
@@ -50,6 +56,14 @@ def _dev_bf16(a):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
 
 
+def _check_differing_block(x, n_sub, iters, c_g, s_g):
+    for c, sizes in checkers.kmeans_end_states(x.astype(np.float64), n_sub, iters):
+        if np.array_equal(sizes, s_g) and np.allclose(c_g, c, rtol=1e-4, atol=1e-4):
+            return
+    raise AssertionError("GPU clustering (sizes %s) is not reachable by the k-means rounds" %
+                         s_g.tolist())
+
+
 def _valid_tokens(w):
     cq = w.seq_pad // w.q_block
     return np.array([min(w.q_block, w.seq_len - i * w.q_block) for i in range(cq)])
@@ -81,6 +95,21 @@ def test_clustered_scores_match_the_oracle(name, n_sub, iters):
     np.testing.assert_allclose(c_g[same][live], c_o[same][live], rtol=1e-4, atol=1e-4)
     d = np.abs(p_g[same] - p_o[same])
     assert d.max() <= 1e-4, d.max()
+    # every block's row: the oracle's mixture fed the GPU's own sub-centroids and sizes
+    p_own = ora.scores_clustered(L, c_g, s_g, kc_o)
+    d = np.abs(p_g - p_own)
+    assert d.max() <= 1e-4, d.max()
+    # blocks whose sizes differ: a clustering the rounds reach with near-ties taken either way
+    cq = w.seq_pad // w.q_block
+    xq = synth.bf16_bits_to_f32(x["q"]).reshape(w.batch * w.heads, w.seq_pad, w.head_dim)
+    nvalid = _valid_tokens(w)
+    for flat in np.nonzero(~same.reshape(-1))[0]:
+        bh, i = flat // cq, flat % cq
+        toks = xq[bh, i * w.q_block:i * w.q_block + nvalid[i]]
+        _check_differing_block(toks, n_sub, iters, c_g.reshape(-1, n_sub, w.head_dim)[flat],
+                               s_g.reshape(-1, n_sub)[flat])
+    print("%s n_sub=%d iters=%d: %d blocks differ from the oracle's sizes, all reachable"
+          % (name, n_sub, iters, int((~same).sum())))
 
 
 @pytest.mark.parametrize("name", ["small", "h5_d128"])

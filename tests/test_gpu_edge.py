@@ -14,6 +14,7 @@ from block_sparse_attention_45_b200 import binding as bsa
 from block_sparse_attention_45_b200 import synth
 from tests import checkers
 from tests.gpu_util import to_dev, to_host_f32
+from tests.guard import Guard
 
 pytestmark = pytest.mark.gpu
 
@@ -48,12 +49,20 @@ def _data(w):
     return x, {k: to_dev(v) for k, v in x.items()}
 
 
-def _attn_vs_oracle(w, x, xd, mask, idx, cnt, what):
+def _attn_vs_oracle(w, x, xd, mask, idx, cnt, what, gd=None):
     L = w.layout()
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    outs = {}
+    if gd is not None:
+        B, H, Sp, D = w.batch, w.heads, w.seq_pad, w.head_dim
+        outs = dict(out=gd.alloc((B, H, Sp, D), torch.bfloat16, what + " out"),
+                    lse=gd.alloc((B, H, Sp), torch.float32, what + " lse"),
+                    workspace=gd.bytes(bsa.attention_workspace_bytes(w), what + " workspace"))
     out, lse = bsa.attention_fwd(w, xd["q"], xd["k"], xd["v"], torch.from_numpy(idx).cuda(),
-                                 torch.from_numpy(cnt).cuda(), err_flag=err)
+                                 torch.from_numpy(cnt).cuda(), err_flag=err, **outs)
     torch.cuda.synchronize()
+    if gd is not None:
+        gd.check()
     o_ora, l_ora = oracle.attention(L, x["q"], x["k"], x["v"], mask)
     cq = w.seq_pad // w.q_block
     og = to_host_f32(out).reshape(o_ora.shape)
@@ -64,27 +73,53 @@ def _attn_vs_oracle(w, x, xd, mask, idx, cnt, what):
     return out, lse, int(err.item())
 
 
+def _mask_outputs(gd, w, tag):
+    B, H = w.batch, w.heads
+    cq, ck = w.seq_pad // w.q_block, w.seq_pad // w.k_block
+    return dict(mask=gd.alloc((B, H, cq, ck), torch.uint8, tag + " mask"),
+                kv_index=gd.alloc((B, H, cq, ck), torch.int32, tag + " kv_index"),
+                kv_count=gd.alloc((B, H, cq), torch.int32, tag + " kv_count"),
+                entropy=gd.alloc((B, H), torch.float32, tag + " entropy"),
+                entropy_norm=gd.alloc((B, H), torch.float32, tag + " entropy_norm"),
+                workspace=gd.bytes(bsa.workspace_bytes(w), tag + " workspace"))
+
+
 @pytest.mark.parametrize("name", sorted(EDGE))
 def test_pipeline_edge_shapes(name):
+    """Every stage on a ragged shape, each output and workspace between guard canaries."""
     w = EDGE[name]
     x, xd = _data(w)
     L = w.layout()
     tp = [w.top_p] * w.heads
+    B, H, Sp, D = w.batch, w.heads, w.seq_pad, w.head_dim
+    cq, ck = Sp // w.q_block, Sp // w.k_block
+    gd = Guard()
     sel = oracle.select(L, x["q"], x["k"], tp, w.flags)
-    qc, kc, probs = bsa.block_scores(w, xd["q"], xd["k"])
+    qc, kc, probs = bsa.block_scores(w, xd["q"], xd["k"],
+                                     gd.alloc((B, H, cq, D), torch.float32, "q_centroids"),
+                                     gd.alloc((B, H, ck, D), torch.float32, "k_centroids"),
+                                     gd.alloc((B, H, cq, ck), torch.float32, "probs"))
+    gd.check()
     np.testing.assert_allclose(to_host_f32(qc), sel["q_centroids"], rtol=1e-5, atol=2e-6)
     np.testing.assert_allclose(to_host_f32(kc), sel["k_centroids"], rtol=1e-5, atol=2e-6)
     assert np.abs(to_host_f32(probs) - sel["probs"]).max() <= 1e-4
-    g0 = bsa.build_mask(w, torch.from_numpy(sel["probs"]).cuda(), tp, 0)
+    g0 = bsa.build_mask(w, torch.from_numpy(sel["probs"]).cuda(), tp, 0, **_mask_outputs(gd, w, "top-p"))
+    gd.check()
     checkers.check_topp_masks(g0["mask"].cpu().numpy(), sel["topp_mask"], sel["probs"], tp,
                               same_probs=True)
-    g = bsa.build_mask(w, torch.from_numpy(sel["probs"]).cuda(), tp, w.flags)
+    g = bsa.build_mask(w, torch.from_numpy(sel["probs"]).cuda(), tp, w.flags,
+                       **_mask_outputs(gd, w, "overrides"))
+    gd.check()
     m = g["mask"].cpu().numpy()
     assert np.array_equal(m, oracle.overrides(L, w.flags, g0["mask"].cpu().numpy()))
     checkers.check_lists(g["kv_index"].cpu().numpy(), g["kv_count"].cpu().numpy(), m)
     np.testing.assert_allclose(g["entropy"].cpu().numpy(), sel["entropy"], rtol=checkers.ENTROPY_REL)
-    _attn_vs_oracle(w, x, xd, sel["mask"], sel["kv_index"], sel["kv_count"], name)
-    out, lse = bsa.dense_fwd(w, xd["q"], xd["k"], xd["v"])
+    _attn_vs_oracle(w, x, xd, sel["mask"], sel["kv_index"], sel["kv_count"], name, gd)
+    out, lse = bsa.dense_fwd(w, xd["q"], xd["k"], xd["v"],
+                             out=gd.alloc((B, H, Sp, D), torch.bfloat16, "dense out"),
+                             lse=gd.alloc((B, H, Sp), torch.float32, "dense lse"),
+                             workspace=gd.bytes(bsa.attention_workspace_bytes(w), "dense workspace"))
+    gd.check()
     o_ora, l_ora = oracle.attention(L, x["q"], x["k"], x["v"], None)
     vmax = np.abs(synth.bf16_bits_to_f32(x["v"])).max()
     checkers.check_attention(to_host_f32(out).reshape(o_ora.shape), o_ora,

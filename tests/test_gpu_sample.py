@@ -18,6 +18,7 @@ import oracle
 from block_sparse_attention_45_b200 import binding as bsa
 from block_sparse_attention_45_b200 import synth
 from tests import checkers
+from tests.gpu_util import sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -193,9 +194,9 @@ def test_reweighted_sum_is_unbiased_on_the_gpu():
 
 def test_weighted_attention_full_size_sampled_rows():
     """Wan2.1-14B at full size (40 heads, 64-key blocks gathered into 128-key tiles):
-    the GPU sampler's lists and weights feed the weighted kernel; 24 seeded query
-    blocks (frame-0 rows, the ragged last block, random ones) match the oracle's
-    weighted attention on the same lists."""
+    the GPU sampler's lists and weights feed the weighted kernel; the sampled query
+    blocks (every frame-0 block of head 0, the ragged last block, 64 random ones
+    spread over every head) match the oracle's weighted attention on the same lists."""
     w = synth.WORKLOADS["wan14b"]
     x = synth.generate(w)
     ora = oracle.default()
@@ -212,9 +213,7 @@ def test_weighted_attention_full_size_sampled_rows():
     wt = np.zeros(m_g.shape, np.float32)
     idx, cnt, wts = g["kv_index"].cpu().numpy(), g["kv_count"].cpu().numpy(), g["kv_weight"].cpu().numpy()
     B, H, Cq, Ck = m_g.shape
-    rng = np.random.default_rng(5)
-    rows = np.unique(np.concatenate([[0, 1, Cq - 1, 2 * Cq + 3, (H - 1) * Cq + Cq - 1],
-                                     rng.integers(0, B * H * Cq, 19)]))
+    rows = sample_rows(w, seed=5)
     for r in rows:
         b, h, i = r // (H * Cq), (r // Cq) % H, r % Cq
         n = cnt[b, h, i]
