@@ -110,6 +110,8 @@ def load():
         L.bsa_status_string.restype = ctypes.c_char_p
         L.bsa_version.argtypes = []
         L.bsa_version.restype = ctypes.c_int
+        L.bsa_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+        L.bsa_set_wait_limit_ns.restype = ctypes.c_int
         _LIB = L
     return _LIB
 
@@ -119,6 +121,11 @@ def declared_symbols():
     text = open(HEADER).read()
     return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(bsa_[a-z_0-9]+)\s*\(",
                                  text, re.M)))
+
+
+def set_wait_limit_ns(ns):
+    """bsa_set_wait_limit_ns: limit of the attention kernel's pipeline waits (0: default 2 s)."""
+    _check("bsa_set_wait_limit_ns", load().bsa_set_wait_limit_ns(int(ns)))
 
 
 def status_string(status):

@@ -49,6 +49,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "internal.h"
@@ -100,6 +101,7 @@ struct AttnParams {
     int32_t *err;
     int *sched;               // work-queue counter (zeroed before launch), or nullptr: static
     long long n_items;
+    unsigned long long wait_ns;  // limit of every pipeline wait (the drains keep kWaitTimeoutNs)
     int S, S_pad, Cq, Ck, bq;
     float scale_log2;
 };
@@ -113,10 +115,13 @@ struct Header {
     uint64_t o_full, o_free;
     uint64_t item_full[4], item_empty[4];  // work-item ring: producer -> MMA + softmax warps
     uint64_t stats_full;                   // both streams' (m, l) of an item are in smem
+    uint64_t mma_drain;                    // every product issued has completed (at exit)
     int item_ring[4];
     uint32_t tmem_base;
     int abort;
 };
+static_assert(sizeof(Header<64>) <= Cfg<64>::kHeader && sizeof(Header<128>) <= Cfg<128>::kHeader,
+              "barrier header fits its slot");
 constexpr int kItemConsumers = 1 + 8;  // the MMA thread + one arrival per softmax warp
 
 // List entries of a work item, clamped to [0, C_k], and its number of tiles.
@@ -202,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&hd.item_empty[s], kItemConsumers);
         }
         mbar_init(&hd.stats_full, 256);
+        mbar_init(&hd.mma_drain, 1);
         hd.abort = 0;
         fence_mbar_init();
     }
@@ -234,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (;; ++qn) {
                 // Claim the next item and publish it (an index >= n_items ends the loop).
                 const int slot = qn & 3;
-                if (!mbar_wait(&hd.item_empty[slot], ((qn >> 2) & 1) ^ 1, abort_flag)) break;
+                if (!mbar_wait(&hd.item_empty[slot], ((qn >> 2) & 1) ^ 1, abort_flag, p.wait_ns)) break;
                 long long item = p.sched ? static_cast<long long>(atomicAdd(p.sched, 1))
                                          : blockIdx.x + static_cast<long long>(qn) * gridDim.x;
                 if (stop || item > p.n_items) item = p.n_items;
@@ -247,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bool bad_count;
                 item_lists<BK>(p, item, entries, n_entries, n_tiles, bad_count);
                 any_bad_count |= bad_count;
-                if (!mbar_wait(&hd.q_empty, (qn & 1) ^ 1, abort_flag)) {
+                if (!mbar_wait(&hd.q_empty, (qn & 1) ^ 1, abort_flag, p.wait_ns)) {
                     stop = true;
                     continue;   // publishes the end marker next
                 }
@@ -265,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         any_bad |= bad;
                     }
                     const int ks = kt % NK;
-                    if (!mbar_wait(&hd.k_empty[ks], ((kt / NK) & 1) ^ 1, abort_flag)) {
+                    if (!mbar_wait(&hd.k_empty[ks], ((kt / NK) & 1) ^ 1, abort_flag, p.wait_ns)) {
                         stop = true;
                         break;
                     }
@@ -278,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         &tmK, &hd.k_full[ks], pn * 64, jl[hf] * BK, bh);
                     ++kt;
                     const int vs = vt % NV;
-                    if (!mbar_wait(&hd.v_empty[vs], ((vt / NV) & 1) ^ 1, abort_flag)) {
+                    if (!mbar_wait(&hd.v_empty[vs], ((vt / NV) & 1) ^ 1, abort_flag, p.wait_ns)) {
                         stop = true;
                         break;
                     }
@@ -323,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (; ok; ++qn) {
                 const int slot = qn & 3;
-                if (!mbar_wait(&hd.item_full[slot], (qn >> 2) & 1, abort_flag)) {
+                if (!mbar_wait(&hd.item_full[slot], (qn >> 2) & 1, abort_flag, p.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -337,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // S_s(t) = Q K_t^T; frees the K stage, and Q once t is the item's last tile.
                 auto issue_s = [&](int t, bool k_ready) -> bool {
                     const int ks = kt % NK;
-                    if (!k_ready && !mbar_wait(&hd.k_full[ks], (kt / NK) & 1, abort_flag))
+                    if (!k_ready && !mbar_wait(&hd.k_full[ks], (kt / NK) & 1, abort_flag, p.wait_ns))
                         return false;
                     tc_fence_after();
                     const uint32_t k_lo = static_cast<uint32_t>(k_desc0) +
@@ -355,29 +361,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ++kt;
                     return true;
                 };
-                ok = mbar_wait(&hd.q_full, qn & 1, abort_flag);
+                ok = mbar_wait(&hd.q_full, qn & 1, abort_flag, p.wait_ns);
                 if (ok && n_tiles == 0) mma_commit(&hd.q_empty);
                 if (ok && n_tiles > 0) ok = issue_s(0, false);
                 if (ok && n_tiles > 1) ok = issue_s(1, false);
                 // O_a / O_b still hold the previous item until its epilogue has read them.
                 // Waited for every item (even one without tiles) so that the wait never
                 // runs two phases ahead of the epilogues.
-                if (ok && qn > 0) ok = mbar_wait(&hd.o_free, (qn - 1) & 1, abort_flag);
+                if (ok && qn > 0) ok = mbar_wait(&hd.o_free, (qn - 1) & 1, abort_flag, p.wait_ns);
                 for (int t = 0; ok && t < n_tiles; ++t) {
                     const int s = t & 1;
                     // V(t) and K(t+2) normally landed long ago; checking them before P(t)
                     // keeps those barrier round trips off the softmax -> PV path.
                     const int vs = vt % NV;
-                    if (!mbar_wait(&hd.v_full[vs], (vt / NV) & 1, abort_flag)) {
+                    if (!mbar_wait(&hd.v_full[vs], (vt / NV) & 1, abort_flag, p.wait_ns)) {
                         ok = false;
                         break;
                     }
                     if (t + 2 < n_tiles &&
-                        !mbar_wait(&hd.k_full[kt % NK], (kt / NK) & 1, abort_flag)) {
+                        !mbar_wait(&hd.k_full[kt % NK], (kt / NK) & 1, abort_flag, p.wait_ns)) {
                         ok = false;
                         break;
                     }
-                    if (!mbar_wait(&hd.p_full[s], pc[s] & 1, abort_flag)) {
+                    if (!mbar_wait(&hd.p_full[s], pc[s] & 1, abort_flag, p.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -401,11 +407,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 mma_commit(&hd.o_full);
             }
-            if (!ok) {  // let whatever was issued finish before TMEM is freed
-                mma_commit(&hd.o_full);
-                volatile int no_abort = 0;
-                mbar_wait(&hd.o_full, qn & 1, &no_abort);
-            }
+            // Let whatever was issued finish before TMEM is freed, on every exit: after an
+            // abort the epilogue may have skipped its wait for the last item's products.
+            // A barrier of its own, so that no role waiting on o_full sees an extra phase.
+            mma_commit(&hd.mma_drain);
+            volatile int no_abort = 0;
+            mbar_wait(&hd.mma_drain, 0, &no_abort);
         }
     }
     } else {
@@ -421,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (;; ++qn) {
             const int slot = qn & 3;
-            if (!__all_sync(0xffffffffu, mbar_wait(&hd.item_full[slot], (qn >> 2) & 1, abort_flag)))
+            if (!__all_sync(0xffffffffu, mbar_wait(&hd.item_full[slot], (qn >> 2) & 1, abort_flag, p.wait_ns)))
                 break;
             const long long item = *reinterpret_cast<volatile int *>(&hd.item_ring[slot]);
             __syncwarp();
@@ -464,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 // tcgen05.ld/st below are warp-collective: leave together or not at all.
-                if (!__all_sync(0xffffffffu, mbar_wait(&hd.s_full[s], sc & 1, abort_flag))) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&hd.s_full[s], sc & 1, abort_flag, p.wait_ns))) {
                     ok = false;
                     break;
                 }
@@ -567,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
 
             // -------------------------------------------------------- epilogue
-            ok = ok && !*abort_flag && mbar_wait(&hd.o_full, qn & 1, abort_flag);
+            ok = ok && !*abort_flag && mbar_wait(&hd.o_full, qn & 1, abort_flag, p.wait_ns);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
             // Exchange (m, l) between the streams.  Double-buffered by item parity: a
@@ -577,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             st[s * 128 + r] = m_run;
             st[256 + s * 128 + r] = l_run;
             mbar_arrive(&hd.stats_full);
-            ok = __all_sync(0xffffffffu, mbar_wait(&hd.stats_full, qn & 1, abort_flag) && ok);
+            ok = __all_sync(0xffffffffu, mbar_wait(&hd.stats_full, qn & 1, abort_flag, p.wait_ns) && ok);
             const float ma = st[r], mb = st[128 + r];
             const float la = st[256 + r], lb = st[384 + r];
             const float m = fmaxf(ma, mb);
@@ -641,6 +648,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------ host side
 
+std::atomic<unsigned long long> g_wait_limit_ns{kWaitTimeoutNs};
+
+unsigned long long attention_wait_limit_ns() { return g_wait_limit_ns.load(); }
+
 // [B*H, S, D] bf16 view with rows >= S out of bounds (loads read zero).
 bool make_map(CUtensorMap *m, const void *base, const Geometry &g, int box_rows) {
     TensorMapEncoder enc = tensor_map_encoder();
@@ -673,6 +684,7 @@ int launch_t(const Geometry &g, const void *q, const void *k, const void *v,
     p.err = err;
     p.sched = static_cast<int *>(workspace);
     p.n_items = static_cast<long long>(g.B) * g.H * g.Cq;
+    p.wait_ns = attention_wait_limit_ns();
     p.S = g.S;
     p.S_pad = g.S_pad;
     p.Cq = g.Cq;
@@ -723,3 +735,8 @@ int launch_attention(const Geometry &g, const void *q, const void *k, const void
 }
 
 }  // namespace bsa
+
+extern "C" int bsa_set_wait_limit_ns(unsigned long long ns) {
+    bsa::g_wait_limit_ns.store(ns == 0 ? bsa::kWaitTimeoutNs : ns);
+    return BSA_OK;
+}

@@ -57,9 +57,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity of *bar has completed.  Returns
-// false if *abort was raised by another role or if the wait outlived
-// kWaitTimeoutNs (then it raises *abort itself).
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+// false if *abort was raised by another role or if the wait outlived limit_ns
+// (then it raises *abort itself).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          uint64_t limit_ns = kWaitTimeoutNs) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer();
@@ -67,7 +68,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
         if (mbar_try_wait(a, parity)) return true;
         if ((it & 63u) == 0) {
             if (*abort) return false;
-            if (globaltimer() - t0 > kWaitTimeoutNs) {
+            if (globaltimer() - t0 > limit_ns) {
                 *abort = 1;
                 return false;
             }
@@ -90,6 +91,21 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, uin
         : "memory");
 }
 
+// Untiled bulk copy global -> this CTA's shared memory, completing on *bar (no
+// multicast): dst and src 16-byte aligned, bytes a non-zero multiple of 16.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// *p += v in shared memory, no result returned (so no dependency on the old value).
+__device__ __forceinline__ void red_add_shared(unsigned long long *p, unsigned long long v) {
+    asm volatile("red.shared.add.u64 [%0], %1;" ::"r"(smem_u32(p)), "l"(v) : "memory");
+}
+
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *m, const void *src, int x, int y,
                                              int z) {
     asm volatile(
@@ -110,6 +126,21 @@ __device__ __forceinline__ void tma_store_wait_all() {
 // Generic-proxy shared-memory writes -> visible to the async proxy (TMA, MMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Barrier `id` over nthreads threads that also ANDs a predicate across them: every
+// participant learns whether all of them passed `pred`.
+__device__ __forceinline__ bool bar_and(uint32_t id, uint32_t nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred q, r;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred r, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, r;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
 }
 
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {

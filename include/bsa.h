@@ -192,14 +192,20 @@ int bsa_build_mask(const bsa_layout *layout, const float *probs, const float *to
  * Same arguments and results as bsa_build_mask minus `workspace`: the
  * per-row entropies go to a fixed array inside the library (4 bytes per row,
  * BSA_NOALLOC_MAX_MASK_ROWS rows, resident on every GPU that loads the
- * library until the process exits).  Returns BSA_ERR_UNSUPPORTED when
- * batch * heads * (seq_pad / q_block) exceeds BSA_NOALLOC_MAX_MASK_ROWS and
- * BSA_ERR_LAUNCH if the array's device address cannot be obtained.  The call
- * allocates and frees nothing.  All calls on a device share the array (it
- * keeps the last call's contents; nothing in it needs clearing), so calls that
- * overlap on the GPU race.  The first call on each device looks the array up
- * (cudaGetSymbolAddress) with that device current; make it before any stream
- * capture.
+ * library until the process exits).  When entropy or entropy_norm is given,
+ * returns BSA_ERR_UNSUPPORTED if batch * heads * (seq_pad / q_block) exceeds
+ * BSA_NOALLOC_MAX_MASK_ROWS and BSA_ERR_LAUNCH if the array's device address
+ * cannot be obtained; a call that asks for neither uses no workspace, so the
+ * array neither caps it nor is touched.  The call allocates and frees nothing.
+ * All calls on a device share the array (it keeps the last call's contents;
+ * nothing in it needs clearing), so calls that overlap on the GPU race.
+ * The first call on each device that asks for entropies looks the array up
+ * (cudaGetSymbolAddress) with that device current.  Under CUDA's default lazy
+ * module loading that lookup also loads the module holding the array, so the
+ * array's 1 MB is reserved by that first call: make it before reserving the
+ * rest of device memory and before any stream capture.  The address is cached
+ * per device with the current context's id; after a device reset (a new
+ * context) the next call looks it up again.
  */
 #define BSA_NOALLOC_MAX_MASK_ROWS 262144
 int bsa_build_mask_noalloc(const bsa_layout *layout, const float *probs, const float *top_p,
@@ -470,6 +476,21 @@ int bsa_sparse_attention_host(const bsa_layout *layout, int heads_per_group, con
 
 /* Device workspace bytes bsa_sparse_attention_host needs (0: invalid layout). */
 size_t bsa_pipeline_workspace_bytes(const bsa_layout *layout, int heads_per_group);
+
+/*
+ * Limit of every internal pipeline wait (mbarrier) of the attention kernel
+ * (bsa_attention_fwd, bsa_attention_fwd_weighted, bsa_dense_fwd,
+ * bsa_frame_scores, and the attention launches of bsa_sparse_attention_host),
+ * in nanoseconds, for the launches made after the call; ns = 0 restores the
+ * default of 2 s.  A wait that outlives the limit makes the kernel stop: every
+ * copy and product already started is waited for (under the default limit),
+ * the tensor memory is released, the outputs of the rows not finished are
+ * undefined (lse NaN where the row had started) and BSA_DEVERR_TIMEOUT is ORed
+ * into err_flag; the stream and the context stay usable.  The pages have no counterpart: this is a diagnostic
+ * setting, process-wide, meant for tests of that stop path (a limit far below
+ * the kernel's own latency makes it fire).  Always returns BSA_OK.
+ */
+int bsa_set_wait_limit_ns(unsigned long long ns);
 
 /* Human-readable name of a bsa_status value (static storage). */
 const char *bsa_status_string(int status);
