@@ -59,9 +59,9 @@ def sample_rows(w, n_random=64, seed=0, frame0_head=0):
     if frame0_head is not None and f1 >= f0:
         rows.update(frame0_head * cq + i for i in range(f0, f1 + 1))
     bh = w.batch * w.heads
-    fixed = len(rows)
+    want = min(len(rows) + n_random, bh * cq)   # a small workload has fewer blocks than asked for
     r = 0
-    while len(rows) < fixed + n_random:
+    while len(rows) < want:
         rows.add(int((r % bh) * cq + rng.integers(cq)))
         r += 1
     return np.array(sorted(rows), np.int64)
