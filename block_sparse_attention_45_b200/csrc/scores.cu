@@ -142,10 +142,10 @@ __global__ void __launch_bounds__(256) vnorm_kernel(const uint4 *__restrict__ v,
 // ---------------------------------------------------------------------------
 // score_kernel: the centroid GEMM on the tensor cores, row softmax fused.
 //
-// Work item = (b*h, 128 query-block rows).  For each chunk of 256 key-block
-// columns the item's logits accumulate in TMEM (two chunk buffers of 256
+// Work item = (b*h, 128 query-block rows).  For each chunk of 128 key-block
+// columns the item's logits accumulate in TMEM (two chunk buffers of 128
 // columns), fed by 2 shared-memory stages that each hold one 32-wide slice of
-// D ("panel") of q-bar (128 x 32 fp32) and k-bar (256 x 32 fp32).
+// D ("panel") of q-bar (128 x 32 fp32) and k-bar (128 x 32 fp32).
 //
 // Precision: plain tf32 keeps ~11 significant bits, far too coarse for logits
 // of magnitude ~50 (P' must stay within 1e-4).  Each operand x is split
@@ -156,20 +156,23 @@ __global__ void __launch_bounds__(256) vnorm_kernel(const uint4 *__restrict__ v,
 // Warp roles (384 threads):
 //   warp 0      TMA producer: q-bar and k-bar panels into the stage's hi halves
 //   warp 1      TMEM owner; lane 0 issues the tcgen05.mma (kind::tf32)
-//   warps 4-7   split workers: hi/lo in place for each landed stage
-//   warps 8-11  epilogue: thread = query-block row (TMEM lane); per 32-column
-//               slice s2 = acc * log2(e)/sqrt(D) + log2 n_j, a running row
-//               max m2 and sum z of 2^(s2 - m2); each warp transposes its own
-//               32 x 32 slice through shared memory so it writes one row's 32
-//               values contiguously.  After the last chunk the warp rewrites its
-//               rows s2 -> 2^(s2 - m2) / z, a row at a time across the warp.
+//   warps 2-3   split workers: hi/lo in place for each landed stage
+//   warps 4-11  epilogue, two groups of four: thread = query-block row (TMEM
+//               lane); group g takes 32-column slices 2g, 2g+1 of every chunk:
+//               s2 = acc * log2(e)/sqrt(D) + log2 n_j, a running row max m2 and
+//               sum z of 2^(s2 - m2); each warp transposes its own 32 x 32 slice
+//               through shared memory so it writes one row's 32 values
+//               contiguously.  After the last chunk the groups' (m2, z) are
+//               merged and the eight warps rewrite 16 rows each,
+//               s2 -> 2^(s2 - m2) / z, a row at a time across the warp.
 namespace sc {
 
 constexpr int kThreads = 384;
+constexpr int kSplitThreads = 64;                    // warps 2-3
 constexpr int kRows = 128;                           // MMA M
-constexpr int kCols = 256;                           // MMA N: key-block columns per chunk
+constexpr int kCols = 128;                           // MMA N: key-block columns per chunk
 constexpr int kAPanelBytes = kRows * 128;            // 128 rows x 32 fp32
-constexpr int kBPanelBytes = kCols * 128;            // 256 rows x 32 fp32
+constexpr int kBPanelBytes = kCols * 128;            // 128 rows x 32 fp32
 constexpr int kStageBytes = 2 * (kAPanelBytes + kBPanelBytes);  // A, A_lo, B, B_lo
 constexpr int kStages = 2;
 constexpr int kTmemCols = 2 * kCols;
@@ -180,20 +183,21 @@ constexpr int kPitch = 36;
 
 struct Header {
     uint64_t full[kStages];    // TMA landed (expect_tx)
-    uint64_t split[kStages];   // hi / lo written (128 arrivals)
+    uint64_t split[kStages];   // hi / lo written (kSplitThreads arrivals)
     uint64_t empty[kStages];   // MMAs done with the stage (commit)
     uint64_t acc_full[2];      // chunk accumulated (commit)
-    uint64_t acc_empty[2];     // epilogue read the chunk (128 arrivals)
+    uint64_t acc_empty[2];     // epilogue read the chunk (256 arrivals)
     uint64_t mma_done;         // every issued MMA finished (commit)
     uint32_t tmem_base;
     int abort;
-    float m2[kRows], inv_z[kRows];
+    float m2[2][kRows], z[2][kRows];  // per epilogue group: running max and sum of each row
 };
-constexpr int kHeaderBytes = 2048;
+constexpr int kHeaderBytes = 3072;
 static_assert(sizeof(Header) <= kHeaderBytes, "header");
 constexpr int kOffLog2n = kHeaderBytes;
 constexpr int kOffStaging = kOffLog2n + kMaxScoreCk * 4;
-constexpr int kOffStages = ((kOffStaging + kRows * kPitch * 4) + 1023) / 1024 * 1024;
+constexpr int kEpiWarps = 8;
+constexpr int kOffStages = ((kOffStaging + kEpiWarps * 32 * kPitch * 4) + 1023) / 1024 * 1024;
 constexpr int kSmemBytes = kOffStages + kStages * kStageBytes;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
 static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
@@ -243,12 +247,12 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&hd.full[s], 1);
-            mbar_init(&hd.split[s], 128);
+            mbar_init(&hd.split[s], kSplitThreads);
             mbar_init(&hd.empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&hd.acc_full[b], 1);
-            mbar_init(&hd.acc_empty[b], 128);
+            mbar_init(&hd.acc_empty[b], 256);
         }
         mbar_init(&hd.mma_done, 1);
         hd.abort = 0;
@@ -341,9 +345,9 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
             volatile int no_abort = 0;
             mbar_wait(&hd.mma_done, 0, &no_abort);
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp == 2 || warp == 3) {
         // ------------------------------------------------------------ split workers
-        const int tid = threadIdx.x - 128;
+        const int tid = threadIdx.x - 64;
         int it = 0;
         bool ok = true;
         for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
@@ -361,14 +365,14 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
                     // same byte offset in the lo half: the 128-byte swizzle depends only
                     // on the address bits inside the 1024-byte-aligned atom
 #pragma unroll 4
-                    for (int i = tid; i < kAPanelBytes / 16; i += 128) {
+                    for (int i = tid; i < kAPanelBytes / 16; i += kSplitThreads) {
                         uint4 x = a[i], lo;
                         split4(x, lo);
                         a[i] = x;
                         a_lo[i] = lo;
                     }
 #pragma unroll 4
-                    for (int i = tid; i < kBPanelBytes / 16; i += 128) {
+                    for (int i = tid; i < kBPanelBytes / 16; i += kSplitThreads) {
                         uint4 x = b[i], lo;
                         split4(x, lo);
                         b[i] = x;
@@ -379,22 +383,29 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
                 }
             }
         }
-    } else if (warp >= 8) {
+    } else if (warp >= 4) {
         // ------------------------------------------------------------ epilogue
-        // Warp ew owns rows 32*ew .. 32*ew+31 of the tile (its TMEM lanes) for the
-        // whole item: it transposes its own 32 x 32 slices in a private staging
-        // block and normalises its own rows, so the four warps never wait for one
-        // another.
-        const int ew = warp - 8;
-        const int rl = ew * 32 + lane;  // row within the tile = TMEM lane
+        // Two warpgroups: group eg takes slices 4*eg .. 4*eg+3 (32 columns each) of
+        // every 256-column chunk; warp quarter ew of a group owns TMEM lanes
+        // 32*ew .. 32*ew+31, i.e. tile rows, and keeps their running max m2 and sum z
+        // over its own slices.  Each warp transposes its own 32 x 32 slices in a
+        // private staging block, so the warps never wait for one another inside a
+        // chunk.  At the end of an item the two groups' (m2, z) are merged through
+        // shared memory and the eight warps rewrite 16 rows each:
+        // s2 -> 2^(s2 - m2) / z.  The two named-barrier steps are votes
+        // (bar.red.and), so an aborted wait makes all eight warps stop together.
+        const int eg = (warp - 4) >> 2;
+        const int ew = warp & 3;
+        const int ewarp = warp - 4;        // 0 .. 7
+        const int rl = ew * 32 + lane;     // row within the tile = TMEM lane
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(ew * 32) << 16);
-        float *wst = stg + ew * 32 * kPitch;  // this warp's 32 x kPitch staging block
+        float *wst = stg + ewarp * 32 * kPitch;  // this warp's 32 x kPitch staging block
         int ch = 0;
         bool ok = true;
         for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
             const int bh = item / p.n_rt, r0 = (item % p.n_rt) * kRows;
             const int nrows = min(kRows, p.Cq - r0);
-            const int my_rows = max(0, min(32, nrows - ew * 32));  // rows of this warp
+            const int my_rows = max(0, min(32, nrows - ew * 32));  // rows of this warp's quarter
             float *wtile = p.probs + (static_cast<long long>(bh) * p.Cq + r0 + ew * 32) * p.Ck;
             float m2 = -INFINITY, z = 0.f;
             for (int c = 0; c < nch; ++c, ++ch) {
@@ -406,18 +417,21 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
                 }
                 tc_fence_after();
                 const int n_sl = min(kCols / 32, (p.Ck - c * kCols + 31) / 32);
+                const int s_lo = 2 * eg, s_hi = min(s_lo + 2, n_sl);
                 uint32_t nxt[32];
-                tmem_ld32(t_lane + static_cast<uint32_t>(buf * kCols), nxt);
-                tmem_ld_wait();
-                reg_fence(nxt);  // no read of nxt may move above the wait
-                for (int s = 0; s < n_sl; ++s) {
+                if (s_lo < s_hi) {
+                    tmem_ld32(t_lane + static_cast<uint32_t>(buf * kCols + s_lo * 32), nxt);
+                    tmem_ld_wait();
+                    reg_fence(nxt);  // no read of nxt may move above the wait
+                }
+                for (int s = s_lo; s < s_hi; ++s) {
                     const int col0 = c * kCols + s * 32;
                     uint32_t r[32];
 #pragma unroll
                     for (int j = 0; j < 32; ++j) r[j] = nxt[j];
                     reg_fence(r);
                     // the next slice's TMEM load runs while this one is processed
-                    if (s + 1 < n_sl)
+                    if (s + 1 < s_hi)
                         tmem_ld32(t_lane + static_cast<uint32_t>(buf * kCols + (s + 1) * 32), nxt);
                     float mx = -INFINITY;
 #pragma unroll
@@ -451,26 +465,40 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
                             if (i < my_rows) wtile[static_cast<long long>(i) * p.Ck + col] = v[i];
                     }
                     __syncwarp();
-                    tmem_ld_wait();  // the prefetched slice has landed
-                    reg_fence(nxt);
+                    if (s + 1 < s_hi) {
+                        tmem_ld_wait();  // the prefetched slice has landed
+                        reg_fence(nxt);
+                    }
                 }
                 tc_fence_before();
                 mbar_arrive(&hd.acc_empty[buf]);
             }
+            // merge the two groups' statistics of every row (all eight warps vote, so an
+            // abort in any of them ends the item in all of them)
+            hd.m2[eg][rl] = m2;
+            hd.z[eg][rl] = z;
+            ok = bar_and(1, 256, ok);
             if (!ok) break;
-            // P' = 2^(s2 - m2) / z for this warp's rows, one row at a time across the
+            // P' = 2^(s2 - m2) / z for 16 rows per warp, one row at a time across the
             // warp (coalesced), two rows in flight
-            hd.m2[rl] = m2;
-            hd.inv_z[rl] = 1.0f / z;
-            __syncwarp();
+            const int w0 = ewarp * 16;                                  // first tile row
+            const int w_rows = max(0, min(16, nrows - w0));
+            float *wrows = p.probs + (static_cast<long long>(bh) * p.Cq + r0 + w0) * p.Ck;
+            auto merged = [&](int tr, float &m, float &iz) {
+                const float ma = hd.m2[0][tr], mb = hd.m2[1][tr];
+                m = fmaxf(ma, mb);
+                const float za = ma == -INFINITY ? 0.f : hd.z[0][tr] * ex2(ma - m);
+                const float zb = mb == -INFINITY ? 0.f : hd.z[1][tr] * ex2(mb - m);
+                iz = 1.0f / (za + zb);
+            };
             if (p.mix_out) {
-                // A block's nsub rows are consecutive and never straddle a warp's 32 rows
-                // (nsub divides 32): its P' row is sum_c w_c 2^(s2_c - m2_c) / z_c with
+                // A block's nsub rows are consecutive and never straddle a warp's 16 rows
+                // (nsub divides 16): its P' row is sum_c w_c 2^(s2_c - m2_c) / z_c with
                 // w_c = n_c / n, the terms added in ascending c (fused multiply-add), the
                 // same arithmetic as normalising the rows and then mixing them.
                 const int ns = p.nsub;
-                for (int i = 0; i < my_rows; i += ns) {
-                    const long long brow = (static_cast<long long>(bh) * p.Cq + r0 + ew * 32 + i) / ns;
+                for (int i = 0; i < w_rows; i += ns) {
+                    const long long brow = (static_cast<long long>(bh) * p.Cq + r0 + w0 + i) / ns;
                     int ntot = 0;
                     for (int c = 0; c < ns; ++c) ntot += __ldg(p.mix_size + brow * ns + c);
                     const float inv = ntot > 0 ? 1.f / static_cast<float>(ntot) : 0.f;
@@ -482,8 +510,9 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
                         for (int c = 0; c < ns; ++c) {
                             const float wc = static_cast<float>(__ldg(p.mix_size + brow * ns + c)) * inv;
                             if (!(wc > 0.f)) continue;
-                            const float mc = hd.m2[ew * 32 + i + c], izc = hd.inv_z[ew * 32 + i + c];
-                            const float *rc = wtile + static_cast<long long>(i + c) * p.Ck;
+                            float mc, izc;
+                            merged(w0 + i + c, mc, izc);
+                            const float *rc = wrows + static_cast<long long>(i + c) * p.Ck;
                             float v[32];
 #pragma unroll
                             for (int k = 0; k < 32; ++k) {
@@ -500,35 +529,36 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
                         }
                     }
                 }
-                __syncwarp();  // m2 / inv_z of this warp's rows are reused by the next item
-                continue;
-            }
-            for (int i = 0; i < my_rows; i += 2) {
-                const bool two = i + 1 < my_rows;
-                const float ma = hd.m2[ew * 32 + i], iza = hd.inv_z[ew * 32 + i];
-                const float mb = two ? hd.m2[ew * 32 + i + 1] : 0.f;
-                const float izb = two ? hd.inv_z[ew * 32 + i + 1] : 0.f;
-                float *ra = wtile + static_cast<long long>(i) * p.Ck;
-                float *rb = ra + p.Ck;
-                for (int c0 = 0; c0 < p.Ck; c0 += 1024) {
-                    float va[32], vb[32];
+            } else {
+                for (int i = 0; i < w_rows; i += 2) {
+                    const bool two = i + 1 < w_rows;
+                    float ma, iza, mb = 0.f, izb = 0.f;
+                    merged(w0 + i, ma, iza);
+                    if (two) merged(w0 + i + 1, mb, izb);
+                    float *ra = wrows + static_cast<long long>(i) * p.Ck;
+                    float *rb = ra + p.Ck;
+                    for (int c0 = 0; c0 < p.Ck; c0 += 1024) {
+                        float va[32], vb[32];
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        const int col = c0 + lane + 32 * k;
-                        va[k] = col < p.Ck ? ra[col] : 0.f;
-                        vb[k] = (two && col < p.Ck) ? rb[col] : 0.f;
-                    }
+                        for (int k = 0; k < 32; ++k) {
+                            const int col = c0 + lane + 32 * k;
+                            va[k] = col < p.Ck ? ra[col] : 0.f;
+                            vb[k] = (two && col < p.Ck) ? rb[col] : 0.f;
+                        }
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        const int col = c0 + lane + 32 * k;
-                        if (col < p.Ck) {
-                            ra[col] = ex2(va[k] - ma) * iza;
-                            if (two) rb[col] = ex2(vb[k] - mb) * izb;
+                        for (int k = 0; k < 32; ++k) {
+                            const int col = c0 + lane + 32 * k;
+                            if (col < p.Ck) {
+                                ra[col] = ex2(va[k] - ma) * iza;
+                                if (two) rb[col] = ex2(vb[k] - mb) * izb;
+                            }
                         }
                     }
                 }
             }
-            __syncwarp();  // m2 / inv_z of this warp's rows are reused by the next item
+            // the statistics are reused by the next item; its first-pass stores must
+            // also come after this pass's reads of the same rows
+            ok = bar_and(1, 256, ok);
         }
     }
     __syncthreads();
@@ -576,7 +606,7 @@ cudaError_t launch_scores_t(const Geometry &g, const float *qc, const float *kc,
     p.mix_size = mix_size;
     p.mix_out = mix_out;
     p.nsub = nsub;
-    if (mix_out && (!mix_size || nsub < 1 || 32 % nsub != 0 || g.Cq % nsub != 0)) return cudaErrorInvalidValue;
+    if (mix_out && (!mix_size || nsub < 1 || 16 % nsub != 0 || g.Cq % nsub != 0)) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          sc::kSmemAlloc);
     if (e != cudaSuccess) return e;
