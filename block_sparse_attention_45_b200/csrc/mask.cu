@@ -24,6 +24,7 @@
 
 #include "bits.cuh"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace bsa {
 
@@ -374,6 +375,402 @@ __device__ __forceinline__ void find_cut(const float (&v)[VPL], const float *__r
     jcut = n_keep == 0 ? -1 : nth_tie<VPL>(v, Ck, uc, n_keep, lane);
 }
 
+// ---------------------------------------------------------------------------
+// Per-row top-p, streaming form (the path of bsa_build_mask).
+//
+// The same selection as find_cut above, organised for throughput:
+//   * each warp walks rows blockIdx*4+warp, + 4*gridDim, ...; the next row's P'
+//     is copied into shared memory by one bulk TMA copy (double buffered) while
+//     the current row is processed, so DRAM latency hides behind the compute;
+//   * level 1 bins the binades below the row maximum in windows of kWin
+//     binades (per-lane columns, fire-and-forget shared reductions), moving the
+//     window down only when the cut lies deeper;
+//   * inside the cut binade, 5-bit digit levels (shared reductions into 32
+//     bins) narrow the range until at most 32 entries remain;
+//   * those candidates are resolved by a warp loop over register shuffles: each
+//     knows the exact significand sum of the candidates before it in (P' desc,
+//     j asc) order.
+// Masses inside one binade are exact integers; binades are summed in fp64,
+// exactly while the cut is within ~2^-29 of the row total (as in the oracle's
+// own fp64 running sum).  Zero entries (and padding) carry no mass and are
+// never the cut except in an all-zero row, so they are left out of the bins.
+constexpr int kTpWarps = 4;              // rows in flight per CTA (one per warp)
+constexpr int kL1Rows = 16;              // level-1 table rows
+constexpr int kWin = kL1Rows - 1;        // binades per level-1 window; row kWin: deeper
+
+struct alignas(16) TpWarp {
+    unsigned long long l1[kL1Rows][kLanes];  // level-1 bins, one column per lane
+    unsigned long long dig[32];              // digit bins (shared by the lanes)
+    uint32_t cand_u[32];
+    int cand_j[32];
+    uint64_t bar[2];                         // row-buffer barriers
+};
+
+__host__ __device__ constexpr int tp_row_bytes(int vpl) { return 16 + 128 * vpl; }
+__host__ __device__ constexpr int tp_smem_bytes(int vpl) {
+    return kTpWarps * (static_cast<int>(sizeof(TpWarp)) + 2 * tp_row_bytes(vpl));
+}
+
+// Level-1 pass over one window: ranks [off, off + kWin) below the maximum's
+// binade go to rows 0 .. kWin-1, deeper ones to row kWin; ranks above the
+// window are skipped (their mass is already known).  NONZERO: leave out zero
+// entries (needed once the window reaches exponent field 0).
+template <int VPL, bool NONZERO>
+__device__ __forceinline__ void tp_bin_window(const float (&v)[VPL], uint32_t emax, int off,
+                                              unsigned long long *col) {
+#pragma unroll
+    for (int s = 0; s < VPL; ++s) {
+        const uint32_t u = __float_as_uint(v[s]);
+        const int r = static_cast<int>(emax - (u >> 23)) - off;
+        const bool in = r >= 0 && (!NONZERO || u != 0u);
+        if (in) red_add_shared(col + min(r, kWin) * kLanes, kCountOne | (u & 0x7FFFFFu));
+    }
+}
+
+// The cut of one row held as v[s] = max(P'[lane + 32 s], 0) (padding 0):
+// the row keeps the entries with pattern > ucut, or == ucut and j <= jcut.
+template <int VPL>
+__device__ __forceinline__ void tp_cut(const float (&v)[VPL], int Ck, float p, uint32_t umax,
+                                       int lane, TpWarp &ws, uint32_t &ucut, int &jcut) {
+    const double pd = static_cast<double>(p);
+    if (umax == 0u) {  // every entry is zero: nothing ever reaches p > 0
+        ucut = 0u;
+        jcut = pd <= 0.0 ? 0 : 0x7FFFFFFF;
+        return;
+    }
+    const uint32_t emax = umax >> 23;
+    double above = 0.0;  // mass of the binades above the current range
+    int cnt_above = 0;
+    int cnt = 0;
+    uint32_t e = 0;
+    unsigned long long *col = &ws.l1[0][lane];
+    // lane L sums half (L & 1) of level-1 row L >> 1
+    const int prow = lane >> 1, phalf = lane & 1;
+    for (int off = 0;; off += kWin) {
+        if (static_cast<int>(emax) < off + kWin) tp_bin_window<VPL, true>(v, emax, off, col);
+        else tp_bin_window<VPL, false>(v, emax, off, col);
+        __syncwarp();
+        unsigned long long half = 0;
+        {
+            ulonglong2 *rw = reinterpret_cast<ulonglong2 *>(&ws.l1[prow][16 * phalf]);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int kk = (k + lane) & 7;
+                const ulonglong2 x = rw[kk];
+                half += x.x + x.y;
+                rw[kk] = make_ulonglong2(0ull, 0ull);
+            }
+        }
+        __syncwarp();
+        const unsigned long long tot2 = half + __shfl_xor_sync(0xffffffffu, half, 1);
+        const unsigned long long tot = __shfl_sync(0xffffffffu, tot2, (2 * lane) & 31);
+        const int e_r = static_cast<int>(emax) - off - lane;  // exponent field of row `lane`
+        const bool real = lane < kWin && e_r >= 0;
+        const int cnt_r = real ? static_cast<int>(tot >> 40) : 0;
+        double mass_r = 0.0;
+        if (real) {
+            const unsigned long long sig = (tot & kSigMask) +
+                (e_r > 0 ? kImplicit * static_cast<unsigned long long>(cnt_r) : 0ull);
+            mass_r = static_cast<double>(sig) * unit_of_binade(static_cast<uint32_t>(e_r));
+        }
+        const double incl = scan_incl_d(mass_r, lane);
+        const int cincl = static_cast<int>(scan_incl_u64(static_cast<unsigned long long>(cnt_r), lane));
+        const uint32_t hit = __ballot_sync(0xffffffffu, cnt_r > 0 && above + incl >= pd);
+        if (hit) {
+            const int b = __ffs(hit) - 1;
+            above += __shfl_sync(0xffffffffu, incl - mass_r, b);
+            cnt_above += __shfl_sync(0xffffffffu, cincl - cnt_r, b);
+            cnt = __shfl_sync(0xffffffffu, cnt_r, b);
+            e = emax - static_cast<uint32_t>(off + b);
+            break;
+        }
+        // Not in this window: move below it, or keep the whole row if nothing is left.
+        above += __shfl_sync(0xffffffffu, incl, kWin - 1);
+        cnt_above += __shfl_sync(0xffffffffu, cincl, kWin - 1);
+        const int deeper = static_cast<int>(__shfl_sync(0xffffffffu, tot2, 2 * kWin) >> 40);
+        if (deeper == 0 || static_cast<int>(emax) < off + kWin) {
+            ucut = 0u;
+            jcut = 0x7FFFFFFF;
+            return;
+        }
+    }
+    // ---- digit levels inside binade e: the range is [lo, hi] = prefix `pre` above bit sh
+    const double unit = unit_of_binade(e);
+    const unsigned long long implicit = e > 0u ? kImplicit : 0ull;
+    unsigned long long s_above = 0;  // significands of the binade's entries above the range
+    uint32_t pre = e;
+    int sh = 23;
+    uint32_t lo = e > 0u ? (e << 23) : 1u, span = (e << 23 | 0x7FFFFFu) - lo;
+    while (cnt > 32 && sh > 0) {
+        const int w = sh >= 5 ? 5 : sh;
+        sh -= w;
+        const uint32_t top = (1u << w) - 1u;
+#pragma unroll
+        for (int s = 0; s < VPL; ++s) {
+            const uint32_t u = __float_as_uint(v[s]);
+            if (u - lo <= span)
+                red_add_shared(&ws.dig[top - ((u >> sh) & top)], kCountOne | (u & 0x7FFFFFu));
+        }
+        __syncwarp();
+        unsigned long long acc = 0;
+        if (lane <= static_cast<int>(top)) {
+            acc = ws.dig[lane];
+            ws.dig[lane] = 0ull;
+        }
+        __syncwarp();
+        const int c_r = static_cast<int>(acc >> 40);
+        const unsigned long long sg_r = (acc & kSigMask) + implicit * static_cast<unsigned long long>(c_r);
+        const unsigned long long sg_incl = scan_incl_u64(sg_r, lane);
+        const int c_incl = static_cast<int>(scan_incl_u64(static_cast<unsigned long long>(c_r), lane));
+        const bool reaches = above + static_cast<double>(s_above + sg_incl) * unit >= pd;
+        const int r = pick_row(c_r > 0, reaches);
+        s_above += __shfl_sync(0xffffffffu, sg_incl - sg_r, r);
+        cnt_above += __shfl_sync(0xffffffffu, c_incl - c_r, r);
+        cnt = __shfl_sync(0xffffffffu, c_r, r);
+        pre = (pre << w) | (top - static_cast<uint32_t>(r));
+        const uint32_t lo_new = pre << sh;
+        lo = lo_new > 0u ? lo_new : 1u;
+        span = (lo_new | ((1u << sh) - 1u)) - lo;
+    }
+    if (cnt <= 32) {
+        // ---- at most 32 candidates: compact them, then each learns the exact mass before it
+        const uint32_t lt_mask = (1u << lane) - 1u;
+        int c = 0;
+#pragma unroll
+        for (int s = 0; s < VPL; ++s) {
+            const uint32_t u = __float_as_uint(v[s]);
+            const bool is_c = u - lo <= span;
+            const uint32_t bal = __ballot_sync(0xffffffffu, is_c);
+            if (is_c) {
+                const int pos = c + __popc(bal & lt_mask);
+                ws.cand_u[pos] = u;
+                ws.cand_j[pos] = lane + 32 * s;
+            }
+            c += __popc(bal);
+        }
+        __syncwarp();
+        const bool mine = lane < cnt;
+        const uint32_t um = mine ? ws.cand_u[lane] : 0u;
+        const int jm = mine ? ws.cand_j[lane] : 0;
+        __syncwarp();
+        const uint32_t imp32 = e > 0u ? 0x800000u : 0u;
+        uint32_t s_before = 0;  // < 32 * 2^24
+        int n_before = 0;
+        for (int n = 0; n < cnt; ++n) {
+            const uint32_t un = __shfl_sync(0xffffffffu, um, n);
+            const int jn = __shfl_sync(0xffffffffu, jm, n);
+            if (un > um || (un == um && jn < jm)) {
+                s_before += (un & 0x7FFFFFu) | imp32;
+                ++n_before;
+            }
+        }
+        const double before = above + static_cast<double>(s_above + s_before) * unit;
+        const bool kept = mine && (before < pd || (cnt_above == 0 && n_before == 0));
+        const uint64_t key = kept ? ((static_cast<uint64_t>(um) << 32) |
+                                     (0xFFFFFFFFu - static_cast<uint32_t>(jm)))
+                                  : ~0ull;
+        const uint64_t best = warp_min_u64(key);
+        if (best == ~0ull) {  // the range starts past p (rounding): keep only what is above it
+            uint32_t mx = mine ? um : 0u;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            ucut = mx;
+            jcut = -1;
+        } else {
+            ucut = static_cast<uint32_t>(best >> 32);
+            jcut = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(best));
+        }
+        return;
+    }
+    // ---- more than 32 entries with one bit pattern: ties in ascending j
+    const uint32_t uc = pre;
+    const unsigned long long sg = significand(uc);
+    int n_keep = 0;
+    for (int k = lane; k < cnt; k += 32)
+        n_keep += (above + static_cast<double>(s_above + sg * static_cast<unsigned long long>(k)) *
+                               unit < pd) ? 1 : 0;
+    n_keep = warp_sum_i(n_keep);
+    if (n_keep == 0 && cnt_above == 0) n_keep = 1;
+    ucut = uc;
+    jcut = n_keep == 0 ? -1 : nth_tie<VPL>(v, Ck, uc, n_keep, lane);
+}
+
+// One warp per row at a time; rows blockIdx.x * 4 + warp, then + 4 * gridDim.x.
+// KFULL: slots that are never padding (the launcher guarantees Ck > 32 * KFULL).
+template <int VPL, int KFULL>
+__global__ void __launch_bounds__(128, 4) topp_kernel(MaskArgs a, TopP tp) {
+    extern __shared__ __align__(128) uint8_t tp_smem[];
+    constexpr int RB = tp_row_bytes(VPL);
+    const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
+    TpWarp &ws = *reinterpret_cast<TpWarp *>(tp_smem + wid * sizeof(TpWarp));
+    uint8_t *rbuf = tp_smem + kTpWarps * sizeof(TpWarp) + wid * 2 * RB;
+    {
+        ulonglong2 *t = reinterpret_cast<ulonglong2 *>(&ws.l1[0][0]);
+        for (int k = lane; k < kL1Rows * kLanes / 2; k += 32) t[k] = make_ulonglong2(0ull, 0ull);
+        ws.dig[lane] = 0ull;
+        if (lane == 0) {
+            mbar_init(&ws.bar[0], 1);
+            mbar_init(&ws.bar[1], 1);
+            fence_mbar_init();
+        }
+        __syncwarp();
+    }
+    const int Ck = a.Ck;
+    const long long stride = static_cast<long long>(gridDim.x) * kTpWarps;
+    long long row = static_cast<long long>(blockIdx.x) * kTpWarps + wid;
+    // Buffer b holds row r from the 16-byte boundary a0 at or below its start: the
+    // 16-byte aligned whole lines [c0, a1) inside the row come by one bulk copy,
+    // the head [start, c0) and tail [a1, end) (< 16 bytes each) by plain loads,
+    // so nothing outside the row is read.
+    auto issue = [&](long long r, int b) {
+        if (lane == 0) {
+            const uintptr_t gs = reinterpret_cast<uintptr_t>(a.probs + r * Ck);
+            const uintptr_t a0 = gs & ~static_cast<uintptr_t>(15);
+            const uintptr_t c0 = (gs + 15u) & ~static_cast<uintptr_t>(15);
+            const uintptr_t a1 = (gs + 4u * static_cast<uintptr_t>(Ck)) & ~static_cast<uintptr_t>(15);
+            if (a1 > c0) {
+                const uint32_t n = static_cast<uint32_t>(a1 - c0);
+                mbar_arrive_expect_tx(&ws.bar[b], n);
+                bulk_load(rbuf + b * RB + (c0 - a0), reinterpret_cast<const void *>(c0), n, &ws.bar[b]);
+            } else {
+                mbar_arrive(&ws.bar[b]);
+            }
+        }
+    };
+    int issued[2] = {0, 0}, waited[2] = {0, 0};
+    bool tma = true;
+    if (row < a.rows) {
+        issue(row, 0);
+        issued[0] = 1;
+    }
+    volatile int no_abort = 0;
+    for (int n = 0; row < a.rows; ++n, row += stride) {
+        const int b = n & 1;
+        const long long nxt = row + stride;
+        if (tma && nxt < a.rows) {
+            fence_proxy_async_smem();  // this warp's reads of buffer b^1 come before the copy
+            issue(nxt, b ^ 1);
+            ++issued[b ^ 1];
+        }
+        const float *src = a.probs + row * Ck;
+        const uintptr_t gs = reinterpret_cast<uintptr_t>(src);
+        const uintptr_t a0 = gs & ~static_cast<uintptr_t>(15);
+        float *sv = reinterpret_cast<float *>(rbuf + b * RB + (gs - a0));  // sv[j] = P'[row, j]
+        bool from_smem = false;
+        if (tma) {
+            from_smem = __all_sync(0xffffffffu, mbar_wait(&ws.bar[b], waited[b] & 1, &no_abort));
+            if (from_smem) ++waited[b];
+            tma = from_smem;  // a copy that never landed: read global memory from here on
+        }
+        float v[VPL];
+        if (from_smem) {
+            // the unaligned head and tail (< 16 bytes each) and the padding slots, then
+            // the row from shared memory
+            const uintptr_t c0 = (gs + 15u) & ~static_cast<uintptr_t>(15);
+            const uintptr_t a1 = (gs + 4u * static_cast<uintptr_t>(Ck)) & ~static_cast<uintptr_t>(15);
+            if (a1 > c0) {
+                const int jh = static_cast<int>((c0 - gs) / 4), jt = static_cast<int>((a1 - gs) / 4);
+                if (lane < jh) sv[lane] = __ldg(src + lane);
+                if (lane < 4 && jt + lane < Ck) sv[jt + lane] = __ldg(src + jt + lane);
+            } else if (lane < Ck) {  // a row of fewer than 8 entries: no whole line inside it
+                sv[lane] = __ldg(src + lane);
+            }
+            for (int j = Ck + lane; j < 32 * VPL; j += 32) sv[j] = 0.f;
+            __syncwarp();
+#pragma unroll
+            for (int s = 0; s < VPL; ++s) v[s] = sv[lane + 32 * s];
+            __syncwarp();
+        } else {
+#pragma unroll
+            for (int s = 0; s < VPL; ++s) {
+                const int j = lane + 32 * s;
+                v[s] = (s < KFULL || j < Ck) ? __ldg(src + j) : 0.f;
+            }
+        }
+        const int row32 = static_cast<int>(row);  // rows < 2^31 (checked on the host)
+        const int i = row32 % a.Cq;
+        const int h = (row32 / a.Cq) % a.H;
+        float ent = 0.f;
+        uint32_t umax = 0;
+        const bool want_ent = a.row_entropy != nullptr;
+#pragma unroll
+        for (int s = 0; s < VPL; ++s) {
+            const float x = v[s] > 0.f ? v[s] : 0.f;  // -0.0 and NaN become +0.0
+            if (want_ent && (s < KFULL || lane + 32 * s < Ck)) ent = fmaf(x, lg2_approx(x + a.eps), ent);
+            v[s] = x;
+            umax = max(umax, __float_as_uint(x));
+        }
+        if (want_ent) {
+            ent = -warp_sum(ent) * 0.6931471805599453f;  // ln 2
+            if (lane == 0) a.row_entropy[row] = ent;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) umax = max(umax, __shfl_xor_sync(0xffffffffu, umax, o));
+
+        const bool dense_row = (a.flags & BSA_FRAME0_DENSE) && i >= a.f0_first && i <= a.f0_last;
+        uint32_t ucut = 0;
+        int jcut = 0x7FFFFFFF;  // keep every entry
+        if (!dense_row) tp_cut<VPL>(v, Ck, tp.p[h], umax, lane, ws, ucut, jcut);
+
+        const int text_k = (a.flags & BSA_TEXT_KEEP) ? a.text_kblocks : 0;
+        uint8_t *mrow = a.mask ? a.mask + row * Ck : nullptr;
+        int32_t *irow = a.kv_index + row * Ck;
+        const uint32_t lt_mask = (1u << lane) - 1u;
+        int base = 0;
+#pragma unroll
+        for (int s = 0; s < VPL; ++s) {
+            const int j = lane + 32 * s;
+            const bool real = s < KFULL || j < Ck;
+            const uint32_t us = __float_as_uint(v[s]);
+            const bool sel = real && (us > ucut || (us == ucut && j <= jcut) || j < text_k);
+            if (mrow && real) mrow[j] = sel ? 1 : 0;
+            const uint32_t bal = __ballot_sync(0xffffffffu, sel);
+            if (sel) irow[base + __popc(bal & lt_mask)] = j;
+            base += __popc(bal);
+        }
+        if (lane == 0) a.kv_count[row] = base;
+    }
+    // every copy started must land before the CTA ends
+    for (int b = 0; b < 2; ++b)
+        while (waited[b] < issued[b]) {
+            mbar_wait(&ws.bar[b], waited[b] & 1, &no_abort);
+            ++waited[b];
+        }
+}
+
+template <int VPL>
+cudaError_t launch_topp_t(const MaskArgs &a, const TopP &tp, cudaStream_t st) {
+    constexpr int kStep = VPL <= 32 ? 2 : 8;  // the dispatcher's VPL granularity
+    constexpr int kFull = VPL - kStep;         // so Ck > 32 * kFull
+    constexpr int smem = tp_smem_bytes(VPL);
+    auto kern = topp_kernel<VPL, kFull>;
+    // the attribute is per device context: set it on every call
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return cudaErrorInvalidValue;
+    static int blocks_per_sm = 0;  // the same on every device this library runs on
+    if (blocks_per_sm == 0) {
+        int nb = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, 128, smem) != cudaSuccess)
+            return cudaErrorInvalidValue;
+        blocks_per_sm = nb > 0 ? nb : 1;
+    }
+    const int sms = sm_count();
+    if (sms <= 0) return cudaErrorInvalidValue;
+    const long long want = (a.rows + kTpWarps - 1) / kTpWarps;
+    const long long cap = static_cast<long long>(sms) * blocks_per_sm;
+    const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
+    kern<<<grid, 128, smem, st>>>(a, tp);
+    return cudaGetLastError();
+}
+
+template <int VPL>
+cudaError_t launch_topp_upto(const MaskArgs &a, const TopP &tp, int vpl, cudaStream_t st) {
+    if constexpr (VPL < 64) {
+        if (vpl > VPL) return launch_topp_upto<VPL < 32 ? VPL + 2 : VPL + 8>(a, tp, vpl, st);
+    }
+    return launch_topp_t<VPL>(a, tp, st);
+}
+
 // Hardware base-2 logarithm (MUFU approximation, relative error ~2^-22).
 // EG = false: every row takes its per-row top-p.  EG = true ("Competition
 // Domains Matter ..." s3.3 domain 3 and s3's other pooled domains): rows of
@@ -540,7 +937,7 @@ cudaError_t launch_mask(const Geometry &g, const float *probs, const TopP &tp, u
     a.pool_of = nullptr;
     a.state = nullptr;
     a.G = 0;
-    return launch_mask_vpl<false>(a, tp, g.Ck, st);
+    return launch_topp_upto<2>(a, tp, (g.Ck + 31) / 32, st);
 }
 
 cudaError_t launch_mask_eg(const Geometry &g, const float *probs, const float *vnorm,

@@ -66,7 +66,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(a, parity)) return true;
-        if ((it & 63u) == 0) {
+        // the clock is read on the first retry and then every 64th, so a limit shorter
+        // than 64 polls still takes effect
+        if (it == 1u || (it & 63u) == 0) {
             if (*abort) return false;
             if (globaltimer() - t0 > limit_ns) {
                 *abort = 1;
