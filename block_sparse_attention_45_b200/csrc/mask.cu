@@ -10,21 +10,25 @@
 // One warp per row; element j of the row lives in lane j % 32, slot j / 32.
 // Top-p without sorting: P' >= 0, so fp32 bit patterns order like the values,
 // and the kept set is every entry whose key (bits, -j) is at least the cut's.
-// The cut is found by an exact radix selection (below): histograms of integer
-// significand sums pick the binade, then 4 mantissa bits at a time, until at
-// most 32 candidates remain; candidate m is kept iff it is the first of the
+// The cut is found by an exact radix selection: histograms of integer
+// significand sums pick the binade, then mantissa digits, until at most 32
+// candidates remain; candidate m is kept iff it is the first of the
 // (P' desc, j asc) order or the mass strictly before it is below p -- the
 // shortest prefix of the sorted row whose running sum reaches p (at least one
 // entry, also for p <= 0).  Masses inside one binade are exact integers; the
 // binades above it are summed in fp64.  Row entropies go to a workspace; a
 // second kernel sums them per head in a fixed order.
+//
+// Two kernels: topp_kernel (per-row top-p for every head: bsa_build_mask) and
+// mask_kernel<VPL, true> (the pooled domains of bsa_build_mask_eg /
+// bsa_build_mask_domain, whose per-row heads take find_cut).
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
 
 #include "bits.cuh"
 #include "internal.h"
-#include "ptx.cuh"
+#include "ptx.cuh"  // red_add_shared
 
 namespace bsa {
 
@@ -376,12 +380,11 @@ __device__ __forceinline__ void find_cut(const float (&v)[VPL], const float *__r
 }
 
 // ---------------------------------------------------------------------------
-// Per-row top-p, streaming form (the path of bsa_build_mask).
+// Per-row top-p, the path of bsa_build_mask.
 //
 // The same selection as find_cut above, organised for throughput:
-//   * each warp walks rows blockIdx*4+warp, + 4*gridDim, ...; the next row's P'
-//     is copied into shared memory by one bulk TMA copy (double buffered) while
-//     the current row is processed, so DRAM latency hides behind the compute;
+//   * each warp walks rows blockIdx*4+warp, + 4*gridDim, ... (7 CTAs of 4 warps
+//     per SM at 72 registers), so its tables are cleared once, not per row;
 //   * level 1 bins the binades below the row maximum in windows of kWin
 //     binades (per-lane columns, fire-and-forget shared reductions), moving the
 //     window down only when the cut lies deeper;
@@ -394,7 +397,7 @@ __device__ __forceinline__ void find_cut(const float (&v)[VPL], const float *__r
 // exactly while the cut is within ~2^-29 of the row total (as in the oracle's
 // own fp64 running sum).  Zero entries (and padding) carry no mass and are
 // never the cut except in an all-zero row, so they are left out of the bins.
-constexpr int kTpWarps = 4;              // rows in flight per CTA (one per warp)
+constexpr int kTpWarps = 4;              // warps per CTA, one row at a time each
 constexpr int kL1Rows = 16;              // level-1 table rows
 constexpr int kWin = kL1Rows - 1;        // binades per level-1 window; row kWin: deeper
 
@@ -403,13 +406,7 @@ struct alignas(16) TpWarp {
     unsigned long long dig[32];              // digit bins (shared by the lanes)
     uint32_t cand_u[32];
     int cand_j[32];
-    uint64_t bar[2];                         // row-buffer barriers
 };
-
-__host__ __device__ constexpr int tp_row_bytes(int vpl) { return 16 + 128 * vpl; }
-__host__ __device__ constexpr int tp_smem_bytes(int vpl) {
-    return kTpWarps * (static_cast<int>(sizeof(TpWarp)) + 2 * tp_row_bytes(vpl));
-}
 
 // Level-1 pass over one window: ranks [off, off + kWin) below the maximum's
 // binade go to rows 0 .. kWin-1, deeper ones to row kWin; ranks above the
@@ -598,94 +595,25 @@ __device__ __forceinline__ void tp_cut(const float (&v)[VPL], int Ck, float p, u
 // One warp per row at a time; rows blockIdx.x * 4 + warp, then + 4 * gridDim.x.
 // KFULL: slots that are never padding (the launcher guarantees Ck > 32 * KFULL).
 template <int VPL, int KFULL>
-__global__ void __launch_bounds__(128, 4) topp_kernel(MaskArgs a, TopP tp) {
-    extern __shared__ __align__(128) uint8_t tp_smem[];
-    constexpr int RB = tp_row_bytes(VPL);
+__global__ void __launch_bounds__(128, 7) topp_kernel(MaskArgs a, TopP tp) {
+    __shared__ TpWarp s_tp[kTpWarps];
     const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
-    TpWarp &ws = *reinterpret_cast<TpWarp *>(tp_smem + wid * sizeof(TpWarp));
-    uint8_t *rbuf = tp_smem + kTpWarps * sizeof(TpWarp) + wid * 2 * RB;
+    TpWarp &ws = s_tp[wid];
     {
         ulonglong2 *t = reinterpret_cast<ulonglong2 *>(&ws.l1[0][0]);
         for (int k = lane; k < kL1Rows * kLanes / 2; k += 32) t[k] = make_ulonglong2(0ull, 0ull);
         ws.dig[lane] = 0ull;
-        if (lane == 0) {
-            mbar_init(&ws.bar[0], 1);
-            mbar_init(&ws.bar[1], 1);
-            fence_mbar_init();
-        }
         __syncwarp();
     }
     const int Ck = a.Ck;
     const long long stride = static_cast<long long>(gridDim.x) * kTpWarps;
-    long long row = static_cast<long long>(blockIdx.x) * kTpWarps + wid;
-    // Buffer b holds row r from the 16-byte boundary a0 at or below its start: the
-    // 16-byte aligned whole lines [c0, a1) inside the row come by one bulk copy,
-    // the head [start, c0) and tail [a1, end) (< 16 bytes each) by plain loads,
-    // so nothing outside the row is read.
-    auto issue = [&](long long r, int b) {
-        if (lane == 0) {
-            const uintptr_t gs = reinterpret_cast<uintptr_t>(a.probs + r * Ck);
-            const uintptr_t a0 = gs & ~static_cast<uintptr_t>(15);
-            const uintptr_t c0 = (gs + 15u) & ~static_cast<uintptr_t>(15);
-            const uintptr_t a1 = (gs + 4u * static_cast<uintptr_t>(Ck)) & ~static_cast<uintptr_t>(15);
-            if (a1 > c0) {
-                const uint32_t n = static_cast<uint32_t>(a1 - c0);
-                mbar_arrive_expect_tx(&ws.bar[b], n);
-                bulk_load(rbuf + b * RB + (c0 - a0), reinterpret_cast<const void *>(c0), n, &ws.bar[b]);
-            } else {
-                mbar_arrive(&ws.bar[b]);
-            }
-        }
-    };
-    int issued[2] = {0, 0}, waited[2] = {0, 0};
-    bool tma = true;
-    if (row < a.rows) {
-        issue(row, 0);
-        issued[0] = 1;
-    }
-    volatile int no_abort = 0;
-    for (int n = 0; row < a.rows; ++n, row += stride) {
-        const int b = n & 1;
-        const long long nxt = row + stride;
-        if (tma && nxt < a.rows) {
-            fence_proxy_async_smem();  // this warp's reads of buffer b^1 come before the copy
-            issue(nxt, b ^ 1);
-            ++issued[b ^ 1];
-        }
+    for (long long row = static_cast<long long>(blockIdx.x) * kTpWarps + wid; row < a.rows; row += stride) {
         const float *src = a.probs + row * Ck;
-        const uintptr_t gs = reinterpret_cast<uintptr_t>(src);
-        const uintptr_t a0 = gs & ~static_cast<uintptr_t>(15);
-        float *sv = reinterpret_cast<float *>(rbuf + b * RB + (gs - a0));  // sv[j] = P'[row, j]
-        bool from_smem = false;
-        if (tma) {
-            from_smem = __all_sync(0xffffffffu, mbar_wait(&ws.bar[b], waited[b] & 1, &no_abort));
-            if (from_smem) ++waited[b];
-            tma = from_smem;  // a copy that never landed: read global memory from here on
-        }
         float v[VPL];
-        if (from_smem) {
-            // the unaligned head and tail (< 16 bytes each) and the padding slots, then
-            // the row from shared memory
-            const uintptr_t c0 = (gs + 15u) & ~static_cast<uintptr_t>(15);
-            const uintptr_t a1 = (gs + 4u * static_cast<uintptr_t>(Ck)) & ~static_cast<uintptr_t>(15);
-            if (a1 > c0) {
-                const int jh = static_cast<int>((c0 - gs) / 4), jt = static_cast<int>((a1 - gs) / 4);
-                if (lane < jh) sv[lane] = __ldg(src + lane);
-                if (lane < 4 && jt + lane < Ck) sv[jt + lane] = __ldg(src + jt + lane);
-            } else if (lane < Ck) {  // a row of fewer than 8 entries: no whole line inside it
-                sv[lane] = __ldg(src + lane);
-            }
-            for (int j = Ck + lane; j < 32 * VPL; j += 32) sv[j] = 0.f;
-            __syncwarp();
 #pragma unroll
-            for (int s = 0; s < VPL; ++s) v[s] = sv[lane + 32 * s];
-            __syncwarp();
-        } else {
-#pragma unroll
-            for (int s = 0; s < VPL; ++s) {
-                const int j = lane + 32 * s;
-                v[s] = (s < KFULL || j < Ck) ? __ldg(src + j) : 0.f;
-            }
+        for (int s = 0; s < VPL; ++s) {
+            const int j = lane + 32 * s;
+            v[s] = (s < KFULL || j < Ck) ? __ldg(src + j) : 0.f;
         }
         const int row32 = static_cast<int>(row);  // rows < 2^31 (checked on the host)
         const int i = row32 % a.Cq;
@@ -730,27 +658,17 @@ __global__ void __launch_bounds__(128, 4) topp_kernel(MaskArgs a, TopP tp) {
         }
         if (lane == 0) a.kv_count[row] = base;
     }
-    // every copy started must land before the CTA ends
-    for (int b = 0; b < 2; ++b)
-        while (waited[b] < issued[b]) {
-            mbar_wait(&ws.bar[b], waited[b] & 1, &no_abort);
-            ++waited[b];
-        }
 }
 
 template <int VPL>
 cudaError_t launch_topp_t(const MaskArgs &a, const TopP &tp, cudaStream_t st) {
     constexpr int kStep = VPL <= 32 ? 2 : 8;  // the dispatcher's VPL granularity
     constexpr int kFull = VPL - kStep;         // so Ck > 32 * kFull
-    constexpr int smem = tp_smem_bytes(VPL);
     auto kern = topp_kernel<VPL, kFull>;
-    // the attribute is per device context: set it on every call
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return cudaErrorInvalidValue;
     static int blocks_per_sm = 0;  // the same on every device this library runs on
     if (blocks_per_sm == 0) {
         int nb = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, 128, smem) != cudaSuccess)
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, 128, 0) != cudaSuccess)
             return cudaErrorInvalidValue;
         blocks_per_sm = nb > 0 ? nb : 1;
     }
@@ -759,7 +677,7 @@ cudaError_t launch_topp_t(const MaskArgs &a, const TopP &tp, cudaStream_t st) {
     const long long want = (a.rows + kTpWarps - 1) / kTpWarps;
     const long long cap = static_cast<long long>(sms) * blocks_per_sm;
     const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
-    kern<<<grid, 128, smem, st>>>(a, tp);
+    kern<<<grid, 128, 0, st>>>(a, tp);
     return cudaGetLastError();
 }
 

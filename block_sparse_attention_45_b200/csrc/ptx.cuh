@@ -93,16 +93,6 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, uin
         : "memory");
 }
 
-// Untiled bulk copy global -> this CTA's shared memory, completing on *bar (no
-// multicast): dst and src 16-byte aligned, bytes a non-zero multiple of 16.
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
 // *p += v in shared memory, no result returned (so no dependency on the old value).
 __device__ __forceinline__ void red_add_shared(unsigned long long *p, unsigned long long v) {
     asm volatile("red.shared.add.u64 [%0], %1;" ::"r"(smem_u32(p)), "l"(v) : "memory");

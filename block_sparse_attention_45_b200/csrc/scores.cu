@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(256) vnorm_kernel(const uint4 *__restrict__ v,
 //   warps 2-3   split workers: hi/lo in place for each landed stage
 //   warps 4-11  epilogue, two groups of four: thread = query-block row (TMEM
 //               lane); group g takes 32-column slices 2g, 2g+1 of every chunk:
-//               s2 = acc * log2(e)/sqrt(D) + log2 n_j, a running row max m2 and
+//               s2 = acc * log2(e)/sqrt(D) + log2(n_j/k_block), a running row max m2 and
 //               sum z of 2^(s2 - m2); each warp transposes its own 32 x 32 slice
 //               through shared memory so it writes one row's 32 values
 //               contiguously.  After the last chunk the groups' (m2, z) are
@@ -194,8 +194,7 @@ struct Header {
 };
 constexpr int kHeaderBytes = 3072;
 static_assert(sizeof(Header) <= kHeaderBytes, "header");
-constexpr int kOffLog2n = kHeaderBytes;
-constexpr int kOffStaging = kOffLog2n + kMaxScoreCk * 4;
+constexpr int kOffStaging = kHeaderBytes;
 constexpr int kEpiWarps = 8;
 constexpr int kOffStages = ((kOffStaging + kEpiWarps * 32 * kPitch * 4) + 1023) / 1024 * 1024;
 constexpr int kSmemBytes = kOffStages + kStages * kStageBytes;
@@ -206,6 +205,7 @@ struct Params {
     float *probs;
     int Cq, Ck, S, bk, n_rt, n_items;
     float scale2;  // log2(e) / sqrt(D)
+    float last_log2n;  // log2(n / k_block) of the last key block (the others hold k_block tokens)
     // Mixing (the rows are nsub sub-centroid rows per query block): instead of
     // normalising its rows in place, the last pass writes each block's row
     // sum_c (n_c / n) P'_c into mix_out; nullptr = plain rows.
@@ -237,7 +237,6 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     Header &hd = *reinterpret_cast<Header *>(smem);
-    float *log2n = reinterpret_cast<float *>(smem + kOffLog2n);
     float *stg = reinterpret_cast<float *>(smem + kOffStaging);
     uint8_t *stages = smem + kOffStages;
     volatile int *abort_flag = &hd.abort;
@@ -258,9 +257,6 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
         hd.abort = 0;
         fence_mbar_init();
     }
-    // log2 of the key-block sizes n_j (every block holds at least one token)
-    for (int j = threadIdx.x; j < p.Ck; j += kThreads)
-        log2n[j] = log2f(static_cast<float>(min(p.bk, p.S - j * p.bk)));
     if (warp == 1) {
         tmem_alloc(&hd.tmem_base, kTmemCols);
         tmem_relinquish();
@@ -433,15 +429,27 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
                     // the next slice's TMEM load runs while this one is processed
                     if (s + 1 < s_hi)
                         tmem_ld32(t_lane + static_cast<uint32_t>(buf * kCols + (s + 1) * 32), nxt);
+                    // s2 = acc * log2(e)/sqrt(D) + log2(n_j / k_block): every key block but
+                    // the last holds k_block tokens, so the offset is 0 except in the last
+                    // column (a common shift of a row leaves its softmax unchanged)
                     float mx = -INFINITY;
+                    if (col0 + 32 < p.Ck) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int col = col0 + j;
-                        const float t = col < p.Ck
-                                            ? fmaf(__uint_as_float(r[j]), p.scale2, log2n[col])
-                                            : -INFINITY;
-                        r[j] = __float_as_uint(t);
-                        mx = fmaxf(mx, t);
+                        for (int j = 0; j < 32; ++j) {
+                            const float t = __uint_as_float(r[j]) * p.scale2;
+                            r[j] = __float_as_uint(t);
+                            mx = fmaxf(mx, t);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int col = col0 + j;
+                            const float t = col < p.Ck ? fmaf(__uint_as_float(r[j]), p.scale2,
+                                                              col == p.Ck - 1 ? p.last_log2n : 0.f)
+                                                       : -INFINITY;
+                            r[j] = __float_as_uint(t);
+                            mx = fmaxf(mx, t);
+                        }
                     }
                     const float mn = fmaxf(m2, mx);
                     float sum = 0.f;
@@ -603,6 +611,7 @@ cudaError_t launch_scores_t(const Geometry &g, const float *qc, const float *kc,
     if (items > 0x7FFFFFFFll) return cudaErrorInvalidValue;
     p.n_items = static_cast<int>(items);
     p.scale2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+    p.last_log2n = log2f(static_cast<float>(g.S - (g.Ck - 1) * g.bk) / static_cast<float>(g.bk));
     p.mix_size = mix_size;
     p.mix_out = mix_out;
     p.nsub = nsub;
