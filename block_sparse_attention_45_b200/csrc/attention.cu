@@ -235,6 +235,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
+            // Q tiles and O rows are used once: evict them first, so that L2 keeps the K and
+            // V blocks that the head's other query blocks fetch again
+            const uint64_t pol_q = policy_evict_first(), pol_kv = policy_evict_last();
             int kt = 0, vt = 0, qn = 0, q_loads = 0;
             bool any_bad = false, any_bad_count = false, stop = false;
             for (;; ++qn) {
@@ -259,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 mbar_arrive_expect_tx(&hd.q_full, static_cast<uint32_t>(p.bq * D * 2));
                 for (int pn = 0; pn < C::kPanels; ++pn)
-                    tma_load_3d(sQ + pn * kPanelBytes, &tmQ, &hd.q_full, pn * 64, qi * p.bq, bh);
+                    tma_load_3d_hint(sQ + pn * kPanelBytes, &tmQ, &hd.q_full, pn * 64, qi * p.bq, bh, pol_q);
                 ++q_loads;
                 for (int t = 0; t < n_tiles; ++t) {
                     int jl[kHalves];
@@ -280,8 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int hf = 0; hf < kHalves; ++hf)
                         for (int pn = 0; pn < C::kPanels; ++pn)
-                            tma_load_3d(sK + ks * C::kTileBytes + pn * kPanelBytes + hf * BK * 128,
-                                        &tmK, &hd.k_full[ks], pn * 64, jl[hf] * BK, bh);
+                            tma_load_3d_hint(sK + ks * C::kTileBytes + pn * kPanelBytes + hf * BK * 128,
+                                             &tmK, &hd.k_full[ks], pn * 64, jl[hf] * BK, bh, pol_kv);
                     ++kt;
                     const int vs = vt % NV;
                     if (!mbar_wait(&hd.v_empty[vs], ((vt / NV) & 1) ^ 1, abort_flag, p.wait_ns)) {
@@ -292,8 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int hf = 0; hf < kHalves; ++hf)
                         for (int pn = 0; pn < C::kPanels; ++pn)
-                            tma_load_3d(sV + vs * C::kTileBytes + pn * kPanelBytes + hf * BK * 128,
-                                        &tmV, &hd.v_full[vs], pn * 64, jl[hf] * BK, bh);
+                            tma_load_3d_hint(sV + vs * C::kTileBytes + pn * kPanelBytes + hf * BK * 128,
+                                             &tmV, &hd.v_full[vs], pn * 64, jl[hf] * BK, bh, pol_kv);
                     ++vt;
                 }
             }
@@ -623,9 +626,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (row_out && ok) {
                     uint4 *dst = reinterpret_cast<uint4 *>(p.out + grow * D + col);
+                    const uint64_t pol_o = policy_evict_first();
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4)
-                        dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+                        st_v4_hint(dst + q4, make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]), pol_o);
                 }
             }
             tc_fence_before();
