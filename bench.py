@@ -222,6 +222,20 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def wait_first_sample(self, timeout=5.0):
+        """Block until nvidia-smi has written its first sample (its start-up takes a
+        while), so that a short timed region still falls between samples."""
+        if self.proc is None:
+            return
+        t0 = time.time()
+        while time.time() - t0 < timeout and self.proc.poll() is None:
+            try:
+                if os.path.getsize(self.path) > 0:
+                    return
+            except OSError:
+                return
+            time.sleep(0.02)
+
     def stop(self):
         if self.proc is None:
             return None
@@ -386,7 +400,7 @@ def our_arm(args, w):
     marks = [[ev() for _ in range(4)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     clocks.start()
-    time.sleep(0.3)
+    clocks.wait_first_sample()
     barrier()
     torch.cuda.synchronize(dev)
     t_start, t_end = ev(), ev()
@@ -396,6 +410,7 @@ def our_arm(args, w):
     t_end.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
+    time.sleep(0.25)   # one more sample after the timed region
     clk = clocks.stop()
     ms_total = t_start.elapsed_time(t_end)
     ms_attn = [m[2].elapsed_time(m[3]) for m in marks]
