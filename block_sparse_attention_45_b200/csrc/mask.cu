@@ -384,7 +384,8 @@ __device__ __forceinline__ void find_cut(const float (&v)[VPL], const float *__r
 //
 // The same selection as find_cut above, organised for throughput:
 //   * each warp walks rows blockIdx*4+warp, + 4*gridDim, ... (7 CTAs of 4 warps
-//     per SM at 72 registers), so its tables are cleared once, not per row;
+//     per SM at 72 registers up to C_k = 1024, 3 beyond), so its tables are
+//     cleared once, not per row;
 //   * level 1 bins the binades below the row maximum in windows of kWin
 //     binades (per-lane columns, fire-and-forget shared reductions), moving the
 //     window down only when the cut lies deeper;
@@ -595,7 +596,7 @@ __device__ __forceinline__ void tp_cut(const float (&v)[VPL], int Ck, float p, u
 // One warp per row at a time; rows blockIdx.x * 4 + warp, then + 4 * gridDim.x.
 // KFULL: slots that are never padding (the launcher guarantees Ck > 32 * KFULL).
 template <int VPL, int KFULL>
-__global__ void __launch_bounds__(128, 7) topp_kernel(MaskArgs a, TopP tp) {
+__global__ void __launch_bounds__(128, VPL <= 32 ? 7 : 3) topp_kernel(MaskArgs a, TopP tp) {
     __shared__ TpWarp s_tp[kTpWarps];
     const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
     TpWarp &ws = s_tp[wid];

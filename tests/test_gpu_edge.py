@@ -251,7 +251,7 @@ def _crafted_probs(rng, rows, ck):
     return np.stack(out)
 
 
-@pytest.mark.parametrize("ck_blocks", [5, 64, 300, 931])
+@pytest.mark.parametrize("ck_blocks", [5, 64, 300, 931, 1500, 2048])
 def test_topp_crafted_rows_exact(ck_blocks):
     """On identical fp32 P' the GPU top-p must equal the oracle's row for row:
     both sum in fp64 in the same order-independent way at the cut."""
