@@ -143,8 +143,9 @@ __global__ void __launch_bounds__(256) vnorm_kernel(const uint4 *__restrict__ v,
 // score_kernel: the centroid GEMM on the tensor cores, row softmax fused.
 //
 // Work item = (b*h, 128 query-block rows).  For each chunk of 128 key-block
-// columns the item's logits accumulate in TMEM (two chunk buffers of 128
-// columns), fed by 2 shared-memory stages that each hold one 32-wide slice of
+// columns the item's logits accumulate in TMEM (four chunk buffers of 128
+// columns, so the products run ahead while the epilogue normalises the
+// previous item), fed by 2 shared-memory stages that each hold one 32-wide slice of
 // D ("panel") of q-bar (128 x 32 fp32) and k-bar (128 x 32 fp32).
 //
 // Precision: plain tf32 keeps ~11 significant bits, far too coarse for logits
@@ -175,7 +176,8 @@ constexpr int kAPanelBytes = kRows * 128;            // 128 rows x 32 fp32
 constexpr int kBPanelBytes = kCols * 128;            // 128 rows x 32 fp32
 constexpr int kStageBytes = 2 * (kAPanelBytes + kBPanelBytes);  // A, A_lo, B, B_lo
 constexpr int kStages = 2;
-constexpr int kTmemCols = 2 * kCols;
+constexpr int kAccBufs = 4;                          // chunk accumulators in TMEM
+constexpr int kTmemCols = kAccBufs * kCols;
 // Staging row pitch (floats): a multiple of 4, so a lane writes its row with
 // 16-byte stores (conflict-free per quarter-warp), and 4i + lane keeps the
 // column reads of one row conflict-free.
@@ -185,8 +187,8 @@ struct Header {
     uint64_t full[kStages];    // TMA landed (expect_tx)
     uint64_t split[kStages];   // hi / lo written (kSplitThreads arrivals)
     uint64_t empty[kStages];   // MMAs done with the stage (commit)
-    uint64_t acc_full[2];      // chunk accumulated (commit)
-    uint64_t acc_empty[2];     // epilogue read the chunk (256 arrivals)
+    uint64_t acc_full[kAccBufs];   // chunk accumulated (commit)
+    uint64_t acc_empty[kAccBufs];  // epilogue read the chunk (256 arrivals)
     uint64_t mma_done;         // every issued MMA finished (commit)
     uint32_t tmem_base;
     int abort;
@@ -249,7 +251,7 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
             mbar_init(&hd.split[s], kSplitThreads);
             mbar_init(&hd.empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kAccBufs; ++b) {
             mbar_init(&hd.acc_full[b], 1);
             mbar_init(&hd.acc_empty[b], 256);
         }
@@ -303,8 +305,9 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
             bool ok = true;
             for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
                 for (int c = 0; ok && c < nch; ++c, ++ch) {
-                    const int buf = ch & 1;
-                    if (ch >= 2 && !mbar_wait(&hd.acc_empty[buf], ((ch >> 1) - 1) & 1, abort_flag)) {
+                    const int buf = ch % kAccBufs;
+                    if (ch >= kAccBufs &&
+                        !mbar_wait(&hd.acc_empty[buf], ((ch / kAccBufs) - 1) & 1, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -359,21 +362,27 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
                     uint4 *b = a_lo + kAPanelBytes / 16;
                     uint4 *b_lo = b + kBPanelBytes / 16;
                     // same byte offset in the lo half: the 128-byte swizzle depends only
-                    // on the address bits inside the 1024-byte-aligned atom
-#pragma unroll 4
-                    for (int i = tid; i < kAPanelBytes / 16; i += kSplitThreads) {
-                        uint4 x = a[i], lo;
-                        split4(x, lo);
-                        a[i] = x;
-                        a_lo[i] = lo;
-                    }
-#pragma unroll 4
-                    for (int i = tid; i < kBPanelBytes / 16; i += kSplitThreads) {
-                        uint4 x = b[i], lo;
-                        split4(x, lo);
-                        b[i] = x;
-                        b_lo[i] = lo;
-                    }
+                    // on the address bits inside the 1024-byte-aligned atom.  Eight 16-byte
+                    // loads are in flight per thread before any is split.
+                    auto split_panel = [&](uint4 *hi, uint4 *lo_out) {
+                        constexpr int kPer = kAPanelBytes / 16 / kSplitThreads;
+                        static_assert(kAPanelBytes == kBPanelBytes && kPer % 8 == 0, "split batches");
+#pragma unroll
+                        for (int b0 = 0; b0 < kPer; b0 += 8) {
+                            uint4 x[8];
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) x[u] = hi[tid + (b0 + u) * kSplitThreads];
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                uint4 lo;
+                                split4(x[u], lo);
+                                hi[tid + (b0 + u) * kSplitThreads] = x[u];
+                                lo_out[tid + (b0 + u) * kSplitThreads] = lo;
+                            }
+                        }
+                    };
+                    split_panel(a, a_lo);
+                    split_panel(b, b_lo);
                     fence_proxy_async_smem();
                     mbar_arrive(&hd.split[st]);
                 }
@@ -405,9 +414,9 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
             float *wtile = p.probs + (static_cast<long long>(bh) * p.Cq + r0 + ew * 32) * p.Ck;
             float m2 = -INFINITY, z = 0.f;
             for (int c = 0; c < nch; ++c, ++ch) {
-                const int buf = ch & 1;
+                const int buf = ch % kAccBufs;
                 if (!__all_sync(0xffffffffu,
-                                mbar_wait(&hd.acc_full[buf], (ch >> 1) & 1, abort_flag))) {
+                                mbar_wait(&hd.acc_full[buf], (ch / kAccBufs) & 1, abort_flag))) {
                     ok = false;
                     break;
                 }
