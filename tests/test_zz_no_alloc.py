@@ -107,3 +107,27 @@ def test_noalloc_without_entropy_is_not_capped():
     for _ in range(2):
         got = _noalloc(layout, probs, tp, 0, with_entropy=False)
         _same(got, ref)
+
+
+def test_noalloc_writes_only_inside_its_buffers():
+    """Every output sits between guard canaries that must stay intact."""
+    from tests.guard import Guard
+    w, probs = _probs("small")
+    B, H = w.batch, w.heads
+    cq, ck = w.seq_pad // w.q_block, w.seq_pad // w.k_block
+    gd = Guard()
+    outs = dict(mask=gd.alloc((B, H, cq, ck), torch.uint8, "mask"),
+                kv_index=gd.alloc((B, H, cq, ck), torch.int32, "kv_index"),
+                kv_count=gd.alloc((B, H, cq), torch.int32, "kv_count"),
+                entropy=gd.alloc((B, H), torch.float32, "entropy"),
+                entropy_norm=gd.alloc((B, H), torch.float32, "entropy_norm"))
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    tp = [float(w.top_p)] * H
+    tpc = (ctypes.c_float * H)(*tp)
+    rc = bsa.load().bsa_build_mask_noalloc(
+        ctypes.byref(bsa.make_layout(w)), ptr(probs), ctypes.cast(tpc, ctypes.c_void_p), w.flags,
+        1e-8, ptr(outs["mask"]), ptr(outs["kv_index"]), ptr(outs["kv_count"]), ptr(outs["entropy"]),
+        ptr(outs["entropy_norm"]), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == bsa.BSA_OK, bsa.status_string(rc)
+    gd.check()
+    _same(outs, bsa.build_mask(w, probs, tp, w.flags))
