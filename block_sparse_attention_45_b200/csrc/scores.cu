@@ -152,12 +152,17 @@ __global__ void __launch_bounds__(256) vnorm_kernel(const uint4 *__restrict__ v,
 // of magnitude ~50 (P' must stay within 1e-4).  Each operand x is split
 // exactly into hi = x with the low 13 mantissa bits cleared (a tf32 value)
 // and lo = x - hi, and the product is hi_a hi_b + hi_a lo_b + lo_a hi_b
-// (three tf32 MMAs), which leaves an error near 2^-21 relative.
+// (three tf32 MMAs), which leaves an error near 2^-21 relative.  The kind::tf32
+// MMA reads only the upper 19 bits of each 32-bit operand, so the fp32 panel as
+// loaded serves as hi and only lo is written.  q-bar is the same for all chunks of
+// an item: its lo panels are made once per item into a resident region; per
+// stage only k-bar's lo is made.
 //
 // Warp roles (384 threads):
-//   warp 0      TMA producer: q-bar and k-bar panels into the stage's hi halves
+//   warp 0      TMA producer: q-bar and k-bar panels into the stage
 //   warp 1      TMEM owner; lane 0 issues the tcgen05.mma (kind::tf32)
-//   warps 2-3   split workers: hi/lo in place for each landed stage
+//   warps 2-3   split workers: k-bar lo for each landed stage, and at an item's
+//               first chunk also the q-bar lo panels of the item
 //   warps 4-11  epilogue, two groups of four: thread = query-block row (TMEM
 //               lane); group g takes 32-column slices 2g, 2g+1 of every chunk:
 //               s2 = acc * log2(e)/sqrt(D) + log2(n_j/k_block), a running row max m2 and
@@ -174,7 +179,8 @@ constexpr int kRows = 128;                           // MMA M
 constexpr int kCols = 128;                           // MMA N: key-block columns per chunk
 constexpr int kAPanelBytes = kRows * 128;            // 128 rows x 32 fp32
 constexpr int kBPanelBytes = kCols * 128;            // 128 rows x 32 fp32
-constexpr int kStageBytes = 2 * (kAPanelBytes + kBPanelBytes);  // A, A_lo, B, B_lo
+constexpr int kStageBytes = kAPanelBytes + 2 * kBPanelBytes;  // A, B, B_lo
+constexpr int kMaxPanels = 4;                        // D / 32 for D <= 128
 constexpr int kStages = 2;
 constexpr int kAccBufs = 4;                          // chunk accumulators in TMEM
 constexpr int kTmemCols = kAccBufs * kCols;
@@ -199,7 +205,8 @@ static_assert(sizeof(Header) <= kHeaderBytes, "header");
 constexpr int kOffStaging = kHeaderBytes;
 constexpr int kEpiWarps = 8;
 constexpr int kOffStages = ((kOffStaging + kEpiWarps * 32 * kPitch * 4) + 1023) / 1024 * 1024;
-constexpr int kSmemBytes = kOffStages + kStages * kStageBytes;
+constexpr int kOffALo = kOffStages + kStages * kStageBytes;  // the item's q-bar lo panels
+constexpr int kSmemBytes = kOffALo + kMaxPanels * kAPanelBytes;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
 static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
 
@@ -241,6 +248,8 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
     Header &hd = *reinterpret_cast<Header *>(smem);
     float *stg = reinterpret_cast<float *>(smem + kOffStaging);
     uint8_t *stages = smem + kOffStages;
+    uint8_t *a_lo_res = smem + kOffALo;
+    static_assert(NP <= kMaxPanels, "resident q-bar lo panels");
     volatile int *abort_flag = &hd.abort;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int nch = (p.Ck + kCols - 1) / kCols;
@@ -287,8 +296,7 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
                         uint8_t *sb = stages + st * kStageBytes;
                         mbar_arrive_expect_tx(&hd.full[st], kAPanelBytes + kBPanelBytes);
                         tma_load_3d(sb, &mq, &hd.full[st], pn * 32, r0, bh);
-                        tma_load_3d(sb + 2 * kAPanelBytes, &mk, &hd.full[st], pn * 32, c * kCols,
-                                    bh);
+                        tma_load_3d(sb + kAPanelBytes, &mk, &hd.full[st], pn * 32, c * kCols, bh);
                     }
                 }
             }
@@ -322,10 +330,10 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
                         tc_fence_after();
                         const uint32_t sb = smem_u32(stages + st * kStageBytes);
                         const uint64_t a_hi = sw128_desc(sb, 16, 1024);
-                        const uint64_t a_lo = sw128_desc(sb + kAPanelBytes, 16, 1024);
-                        const uint64_t b_hi = sw128_desc(sb + 2 * kAPanelBytes, 16, 1024);
-                        const uint64_t b_lo =
-                            sw128_desc(sb + 2 * kAPanelBytes + kBPanelBytes, 16, 1024);
+                        const uint64_t a_lo =
+                            sw128_desc(smem_u32(a_lo_res + pn * kAPanelBytes), 16, 1024);
+                        const uint64_t b_hi = sw128_desc(sb + kAPanelBytes, 16, 1024);
+                        const uint64_t b_lo = sw128_desc(sb + kAPanelBytes + kBPanelBytes, 16, 1024);
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {  // K = 8 tf32 = 32 bytes per MMA
                             const uint64_t o = static_cast<uint64_t>(k * 2);
@@ -358,30 +366,39 @@ __global__ void __launch_bounds__(sc::kThreads, 1)
                         break;
                     }
                     uint4 *a = reinterpret_cast<uint4 *>(stages + st * kStageBytes);
-                    uint4 *a_lo = a + kAPanelBytes / 16;
-                    uint4 *b = a_lo + kAPanelBytes / 16;
+                    uint4 *b = a + kAPanelBytes / 16;
                     uint4 *b_lo = b + kBPanelBytes / 16;
-                    // same byte offset in the lo half: the 128-byte swizzle depends only
-                    // on the address bits inside the 1024-byte-aligned atom.  Eight 16-byte
-                    // loads are in flight per thread before any is split.
-                    auto split_panel = [&](uint4 *hi, uint4 *lo_out) {
+                    // lo at the same byte offset as its source: the 128-byte swizzle depends
+                    // only on the address bits inside the 1024-byte-aligned atom.  Eight
+                    // 16-byte loads are in flight per thread before any is split.
+                    auto split_panel = [&](const uint4 *src, uint4 *lo_out) {
                         constexpr int kPer = kAPanelBytes / 16 / kSplitThreads;
                         static_assert(kAPanelBytes == kBPanelBytes && kPer % 8 == 0, "split batches");
 #pragma unroll
                         for (int b0 = 0; b0 < kPer; b0 += 8) {
                             uint4 x[8];
 #pragma unroll
-                            for (int u = 0; u < 8; ++u) x[u] = hi[tid + (b0 + u) * kSplitThreads];
+                            for (int u = 0; u < 8; ++u) x[u] = src[tid + (b0 + u) * kSplitThreads];
 #pragma unroll
                             for (int u = 0; u < 8; ++u) {
                                 uint4 lo;
                                 split4(x[u], lo);
-                                hi[tid + (b0 + u) * kSplitThreads] = x[u];
                                 lo_out[tid + (b0 + u) * kSplitThreads] = lo;
                             }
                         }
                     };
-                    split_panel(a, a_lo);
+                    if (c == 0) {
+                        // The item's q-bar lo panel pn is made from its first chunk.  Before
+                        // the first one is overwritten, every product of the previous item
+                        // (the last readers of the region) must have completed: the commit
+                        // after stage use it-1 covers them all.
+                        if (pn == 0 && it > 0 &&
+                            !mbar_wait(&hd.empty[(it - 1) % kStages], ((it - 1) / kStages) & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        split_panel(a, reinterpret_cast<uint4 *>(a_lo_res + pn * kAPanelBytes));
+                    }
                     split_panel(b, b_lo);
                     fence_proxy_async_smem();
                     mbar_arrive(&hd.split[st]);
